@@ -1,0 +1,216 @@
+"""fp64 CPU oracle for MLA attention over the compressed KV cache.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package. The CUDA library never loads it, and it shares no code with that
+library: the two meet only through the seeded input generators.
+
+The arithmetic lives in ``mla_oracle.c`` (plain C, fp64, OpenMP over query
+rows). This module compiles it with gcc on first use and wraps it with ctypes.
+What it computes and which page passage each part follows is written at the
+top of ``mla_oracle.c``.
+
+Parity pins (checked by ``tests/test_oracle_pins.py`` against closed forms,
+brute force and invariants, never against the oracle itself):
+  attention / attention_online / attention_split / compact / dequant_q8_0.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mla_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+
+DK = 576
+DV = 512
+Q8_ROW_BYTES = 612
+KV_F16 = 0
+KV_Q8_0 = 1
+
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile mla_oracle.c into oracle/_build/liboracle.so (gcc, OpenMP)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+    cmd = ["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
+           _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        L = ctypes.c_long
+        I = ctypes.c_int
+        D = ctypes.c_double
+        lib.oracle_init.restype = None
+        lib.oracle_max_threads.restype = I
+        lib.oracle_set_threads.argtypes = [I]
+        lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
+        lib.oracle_half_to_double.restype = D
+        common = [P, P, I, P, P, L, I, I, L, D, P, L]
+        lib.oracle_attention.argtypes = common + [P]
+        lib.oracle_attention.restype = I
+        lib.oracle_attention_online.argtypes = common + [L, P]
+        lib.oracle_attention_online.restype = I
+        lib.oracle_attention_split.argtypes = common + [P, I, P]
+        lib.oracle_attention_split.restype = I
+        lib.oracle_compact.argtypes = [P, L, P]
+        lib.oracle_compact.restype = L
+        lib.oracle_dequant_q8_0.argtypes = [P, L, P]
+        lib.oracle_dequant_q8_0.restype = None
+        lib.oracle_init()
+        _lib = lib
+        return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits16(a):
+    """f16 array (or its uint16 bit view) as a C-contiguous uint16 array."""
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        return a.view(np.uint16)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected float16/uint16, got {a.dtype}")
+    return a
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def half_to_double(bits: int) -> float:
+    return float(_load().oracle_half_to_double(int(bits)))
+
+
+def _prep(q, kcache, kv_type, mask, idx, rows):
+    q = _bits16(q)
+    if q.ndim != 3 or q.shape[2] != DK:
+        raise ValueError("q must be [n_q][n_head][576]")
+    n_q, n_head, _ = q.shape
+    if kv_type == KV_F16:
+        kc = _bits16(kcache)
+        if kc.ndim != 2 or kc.shape[1] != DK:
+            raise ValueError("f16 kcache must be [n_kv][576]")
+    elif kv_type == KV_Q8_0:
+        kc = np.ascontiguousarray(kcache, dtype=np.uint8)
+        if kc.ndim != 2 or kc.shape[1] != Q8_ROW_BYTES:
+            raise ValueError("q8_0 kcache must be [n_kv][612] bytes")
+    else:
+        raise ValueError("unknown kv_type")
+    n_kv = kc.shape[0]
+    m = None
+    if mask is not None:
+        m = _bits16(mask)
+        if m.shape != (n_q, n_kv):
+            raise ValueError("mask must be [n_q][n_kv]")
+    ix = None if idx is None else np.ascontiguousarray(idx, dtype=np.int32)
+    rw = None if rows is None else np.ascontiguousarray(rows, dtype=np.int32)
+    n_out = n_q * n_head if rw is None else len(rw)
+    out = np.zeros((n_out, DV), dtype=np.float64)
+    return q, kc, m, ix, rw, n_q, n_head, n_kv, out
+
+
+def attention(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None, idx=None):
+    """Two-pass fp64 softmax(scale*Q.K^T + mask).V with V = K[:, :512].
+
+    q: f16 [n_q][n_head][576]; kcache: f16 [n_kv][576] or q8_0 bytes [n_kv][612];
+    mask: f16 [n_q][n_kv] or None; idx: optional int32 kept rows (sparse);
+    rows: optional row ids t*n_head+h to compute. Returns float64 [rows][512].
+    """
+    q, kc, m, ix, rw, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, rows)
+    rc = _load().oracle_attention(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
+                                  0 if ix is None else len(ix), n_q, n_head, n_kv, float(scale),
+                                  _ptr(rw), 0 if rw is None else len(rw), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_attention rejected its arguments")
+    return out
+
+
+def attention_online(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, tile=64, rows=None,
+                     idx=None):
+    """One-pass tiled online-softmax variant (running max m, running sum l)."""
+    q, kc, m, ix, rw, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, rows)
+    rc = _load().oracle_attention_online(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
+                                         0 if ix is None else len(ix), n_q, n_head, n_kv,
+                                         float(scale), _ptr(rw), 0 if rw is None else len(rw),
+                                         int(tile), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_attention_online rejected its arguments")
+    return out
+
+
+def attention_split(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, bounds=None, rows=None,
+                    idx=None):
+    """Split-KV variant: per-part (acc, m, l) merged by the log-sum-exp rule."""
+    q, kc, m, ix, rw, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, rows)
+    b = np.ascontiguousarray(bounds, dtype=np.int32)
+    rc = _load().oracle_attention_split(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
+                                        0 if ix is None else len(ix), n_q, n_head, n_kv,
+                                        float(scale), _ptr(rw), 0 if rw is None else len(rw),
+                                        _ptr(b), len(b) - 1, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_attention_split rejected its arguments")
+    return out
+
+
+def compact(mask_row):
+    """Ascending int32 indices of the cells whose f16 bits are not -inf."""
+    m = _bits16(mask_row).ravel()
+    idx = np.empty(max(len(m), 1), dtype=np.int32)
+    n = _load().oracle_compact(_ptr(m), len(m), _ptr(idx))
+    return idx[:n].copy()
+
+
+def dequant_q8_0(rows_bytes):
+    """q8_0 rows [n][612] -> float64 [n][576], value = d * q per 32-block."""
+    r = np.ascontiguousarray(rows_bytes, dtype=np.uint8)
+    if r.ndim != 2 or r.shape[1] != Q8_ROW_BYTES:
+        raise ValueError("q8_0 rows must be [n][612]")
+    out = np.empty((r.shape[0], DK), dtype=np.float64)
+    _load().oracle_dequant_q8_0(_ptr(r), r.shape[0], _ptr(out))
+    return out
+
+
+def attention_batched(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None, idx=None,
+                      counts=None):
+    """Per-sequence loop for batched inputs.
+
+    q [n_seq][n_q][n_head][576]; kcache [n_seq][n_kv][...]; mask [n_seq][n_q][n_kv] or None;
+    rows: optional list (one array or None per sequence); idx/counts for sparse.
+    Returns a list of float64 arrays, one per sequence.
+    """
+    outs = []
+    for b in range(q.shape[0]):
+        ib = None
+        if idx is not None:
+            ib = idx[b][: counts[b]] if counts is not None else idx[b]
+        outs.append(attention(q[b], kcache[b], kv_type, None if mask is None else mask[b],
+                              scale, None if rows is None else rows[b], ib))
+    return outs

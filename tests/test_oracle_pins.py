@@ -1,0 +1,346 @@
+"""Pins for the fp64 oracle (CPU only).
+
+Each test checks the oracle against something other than itself: a closed form,
+an explicit numpy float64 matrix route written here, an invariant of softmax
+attention, or brute force on tiny inputs. The pages print no worked example for
+this computation (see tests/golden/README.md), so these are the pins.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from mla_flash_attention_attn_b200 import workloads as W
+
+DK, DV = 576, 512
+NEG = np.float16(-np.inf)
+
+
+def rand_f16(rng, shape, std=1.0):
+    return (rng.standard_normal(shape) * std).astype(np.float16)
+
+
+def brute_force(q, k, mask, scale):
+    """softmax(scale * Q K^T + mask) V with explicit float64 matrices.
+
+    q [n_q][H][576] f16, k [n][576] f16, mask [n_q][n] f16 or None."""
+    qd = q.astype(np.float64)
+    kd = k.astype(np.float64)
+    n_q, H, _ = q.shape
+    out = np.zeros((n_q, H, DV))
+    for t in range(n_q):
+        S = scale * (qd[t] @ kd.T)  # [H][n]
+        if mask is not None:
+            S = S + mask[t].astype(np.float64)[None, :]
+        mx = S.max(axis=1, keepdims=True)
+        P = np.where(np.isneginf(S), 0.0, np.exp(S - np.where(np.isneginf(mx), 0.0, mx)))
+        den = P.sum(axis=1, keepdims=True)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            O = np.where(den > 0, (P @ kd[:, :DV]) / np.where(den > 0, den, 1.0), 0.0)
+        out[t] = O
+    return out.reshape(n_q * H, DV)
+
+
+def test_half_conversion_matches_numpy_on_all_finite_patterns():
+    bits = np.arange(65536, dtype=np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits[::97]])
+    r = ref[::97]
+    fin = np.isfinite(r)
+    assert np.array_equal(got[fin], r[fin])
+    assert oracle.half_to_double(0xFC00) == -math.inf
+    assert oracle.half_to_double(0x7C00) == math.inf
+    assert oracle.half_to_double(0x0001) == 2.0 ** -24
+
+
+def test_single_key_gives_its_value_row_exactly():
+    rng = np.random.default_rng(1)
+    q = rand_f16(rng, (2, 3, DK))
+    k = rand_f16(rng, (1, DK))
+    for mask in (None, np.array([[1.5], [-7.0]], np.float16)):
+        out = oracle.attention(q, k, mask=mask, scale=0.3)
+        expect = np.broadcast_to(k[0, :DV].astype(np.float64), out.shape)
+        assert np.array_equal(out, expect)
+
+
+def test_zero_query_gives_mean_of_kept_values():
+    rng = np.random.default_rng(2)
+    n = 37
+    q = np.zeros((1, 4, DK), np.float16)
+    k = rand_f16(rng, (n, DK))
+    keep = rng.random(n) < 0.6
+    keep[0] = True
+    mask = np.where(keep, np.float16(0), NEG).astype(np.float16)[None]
+    out = oracle.attention(q, k, mask=mask, scale=1.0 / math.sqrt(192))
+    mean = k[keep, :DV].astype(np.float64).mean(axis=0)
+    np.testing.assert_allclose(out, np.broadcast_to(mean, out.shape), rtol=0, atol=1e-14)
+
+
+def test_two_key_closed_form_and_mask_is_added_after_scaling():
+    # Q = e_0 so the dot with key j is k[j][0]; scores s_j = scale*k_j0 + m_j.
+    q = np.zeros((1, 1, DK), np.float16)
+    q[0, 0, 0] = 1.0
+    k = np.zeros((2, DK), np.float16)
+    k[0, 0], k[1, 0] = 2.0, -1.0
+    k[0, 1:DV] = 0.25
+    k[1, 1:DV] = -0.5
+    k[:, DV:] = 3.0  # rope columns take part in the dot product only through c=0 here
+    scale = 0.5
+    m = np.array([[0.75, 2.0]], np.float16)
+    out = oracle.attention(q, k, mask=m, scale=scale)[0]
+    s0 = scale * 2.0 + 0.75
+    s1 = scale * -1.0 + 2.0
+    delta = s1 - s0
+    v0, v1 = k[0, :DV].astype(np.float64), k[1, :DV].astype(np.float64)
+    expect = (v0 + math.exp(delta) * v1) / (1.0 + math.exp(delta))
+    np.testing.assert_allclose(out, expect, rtol=1e-15, atol=1e-15)
+
+
+def test_rope_columns_enter_the_score_but_not_the_value():
+    # Q nonzero only on a rope column: the score must see it.
+    q = np.zeros((1, 1, DK), np.float16)
+    q[0, 0, 540] = 1.0
+    k = np.zeros((2, DK), np.float16)
+    k[0, 540] = 4.0
+    k[0, :DV] = 1.0
+    k[1, :DV] = -1.0
+    out = oracle.attention(q, k, scale=1.0)[0]
+    w1 = 1.0 / (1.0 + math.exp(4.0))
+    expect = (1.0 - w1) * 1.0 + w1 * -1.0
+    np.testing.assert_allclose(out, expect, rtol=1e-14)
+
+
+@pytest.mark.parametrize("n_q,H,n", [(1, 1, 1), (1, 2, 5), (3, 2, 8), (2, 1, 7)])
+def test_brute_force_tiny(n_q, H, n):
+    rng = np.random.default_rng(100 + n_q * 10 + n)
+    q = rand_f16(rng, (n_q, H, DK))
+    k = rand_f16(rng, (n, DK))
+    mask = rand_f16(rng, (n_q, n), std=2.0)
+    mask[rng.random((n_q, n)) < 0.3] = NEG
+    scale = 1.0 / math.sqrt(192)
+    got = oracle.attention(q, k, mask=mask, scale=scale)
+    np.testing.assert_allclose(got, brute_force(q, k, mask, scale), rtol=1e-12, atol=1e-13)
+
+
+def test_brute_force_per_token_mask_rows_and_heads_distinct():
+    # Distinct masks per token and distinct queries per head catch transposed indices.
+    rng = np.random.default_rng(7)
+    q = rand_f16(rng, (4, 3, DK))
+    k = rand_f16(rng, (6, DK))
+    mask = np.zeros((4, 6), np.float16)
+    for t in range(4):
+        mask[t, t + 1:] = NEG  # causal-like, different per token
+    got = oracle.attention(q, k, mask=mask, scale=0.1)
+    np.testing.assert_allclose(got, brute_force(q, k, mask, 0.1), rtol=1e-12, atol=1e-13)
+
+
+def test_shift_invariance_of_mask():
+    rng = np.random.default_rng(3)
+    q = rand_f16(rng, (2, 2, DK))
+    k = rand_f16(rng, (40, DK))
+    mask = np.zeros((2, 40), np.float16)
+    mask[:, 30:] = NEG
+    base = oracle.attention(q, k, mask=mask, scale=0.07)
+    shifted = np.where(np.isneginf(mask), mask, mask + np.float16(6.0)).astype(np.float16)
+    np.testing.assert_allclose(oracle.attention(q, k, mask=shifted, scale=0.07), base,
+                               rtol=1e-13, atol=1e-14)
+
+
+def test_masked_garbage_rows_contribute_nothing_bit_identical():
+    rng = np.random.default_rng(4)
+    q = rand_f16(rng, (1, 3, DK))
+    k = rand_f16(rng, (20, DK))
+    mask = np.zeros((1, 20), np.float16)
+    base = oracle.attention(q, k, mask=mask, scale=0.05)
+    garbage = np.full((9, DK), np.float16(60000.0))
+    garbage[::2] = np.float16(-60000.0)
+    k2 = np.concatenate([k, garbage])
+    mask2 = np.concatenate([mask, np.full((1, 9), NEG, np.float16)], axis=1)
+    assert np.array_equal(oracle.attention(q, k2, mask=mask2, scale=0.05), base)
+
+
+def test_fully_masked_row_is_zero():
+    rng = np.random.default_rng(5)
+    q = rand_f16(rng, (2, 2, DK))
+    k = rand_f16(rng, (10, DK))
+    mask = np.zeros((2, 10), np.float16)
+    mask[1, :] = NEG
+    out = oracle.attention(q, k, mask=mask, scale=0.1).reshape(2, 2, DV)
+    assert np.all(out[1] == 0.0)
+    assert np.all(np.abs(out[0]) > 0.0)
+
+
+def test_permutation_invariance():
+    rng = np.random.default_rng(6)
+    q = rand_f16(rng, (2, 2, DK))
+    k = rand_f16(rng, (33, DK))
+    mask = rand_f16(rng, (2, 33))
+    mask[:, ::5] = NEG
+    perm = rng.permutation(33)
+    a = oracle.attention(q, k, mask=mask, scale=0.06)
+    b = oracle.attention(q, k[perm], mask=mask[:, perm], scale=0.06)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("tile", [1, 7, 64, 1000])
+def test_online_matches_two_pass(tile):
+    rng = np.random.default_rng(8)
+    n = 150
+    q = rand_f16(rng, (2, 2, DK))
+    k = rand_f16(rng, (n, DK))
+    mask = np.zeros((2, n), np.float16)
+    mask[0, :40] = NEG  # first tiles fully masked for one row
+    mask[1, 100:] = NEG
+    a = oracle.attention(q, k, mask=mask, scale=0.09)
+    b = oracle.attention_online(q, k, mask=mask, scale=0.09, tile=tile)
+    np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-14)
+
+
+def test_online_with_growing_scores_has_no_positional_bias():
+    # Scores increase along the sequence, so the running max grows every tile: a broken
+    # rescale would bias the late keys (the failure mode the article warns about).
+    q = np.zeros((1, 1, DK), np.float16)
+    q[0, 0, 0] = 1.0
+    n = 64
+    k = np.zeros((n, DK), np.float16)
+    k[:, 0] = np.linspace(-8, 8, n).astype(np.float16)
+    k[:, 1] = np.arange(n).astype(np.float16)
+    a = oracle.attention(q, k, scale=1.0)
+    b = oracle.attention_online(q, k, scale=1.0, tile=3)
+    np.testing.assert_allclose(b, a, rtol=1e-12)
+    np.testing.assert_allclose(a, brute_force(q, k, None, 1.0), rtol=1e-12)
+
+
+@pytest.mark.parametrize("bounds", [[0, 50], [0, 1, 50], [0, 13, 13, 40, 50], [0, 20, 30, 49, 50]])
+def test_split_combine_matches_unsplit(bounds):
+    rng = np.random.default_rng(9)
+    q = rand_f16(rng, (1, 3, DK))
+    k = rand_f16(rng, (50, DK))
+    mask = np.zeros((1, 50), np.float16)
+    mask[0, 13:40] = NEG  # some parts fully masked (l_s = 0 parts are skipped)
+    a = oracle.attention(q, k, mask=mask, scale=0.08)
+    b = oracle.attention_split(q, k, mask=mask, scale=0.08, bounds=bounds)
+    np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-14)
+
+
+def test_rows_subset_matches_full():
+    rng = np.random.default_rng(10)
+    q = rand_f16(rng, (3, 4, DK))
+    k = rand_f16(rng, (12, DK))
+    full = oracle.attention(q, k, scale=0.1)
+    rows = np.array([11, 0, 5], np.int32)
+    assert np.array_equal(oracle.attention(q, k, scale=0.1, rows=rows), full[rows])
+
+
+def test_compaction_brute_force_all_16_cell_masks():
+    pats = np.arange(1 << 16, dtype=np.uint32)
+    bits = ((pats[:, None] >> np.arange(16, dtype=np.uint32)[None, :]) & 1).astype(bool)
+    for i in range(0, 1 << 16, 1):
+        keep = bits[i]
+        row = np.where(keep, np.float16(0), NEG).astype(np.float16)
+        got = oracle.compact(row)
+        if i % 4096 == 0 or i in (1, 2, 3, 0xFFFF):
+            assert np.array_equal(got, np.nonzero(keep)[0].astype(np.int32))
+        assert len(got) == int(keep.sum())
+
+
+def test_compaction_keep_rule_only_minus_inf_dropped():
+    row = np.array([0, -np.inf, -60000.0, np.inf, -0.0, 1e-7, -np.inf], np.float16)
+    assert oracle.compact(row).tolist() == [0, 2, 3, 4, 5]
+    row2 = np.full(1000, NEG, np.float16)
+    assert len(oracle.compact(row2)) == 0
+
+
+def test_compaction_random_long_rows_equal_numpy_filter():
+    rng = np.random.default_rng(11)
+    for n in (1, 31, 32, 33, 1023, 4097):
+        keep = rng.random(n) < 0.3
+        row = np.where(keep, rng.standard_normal(n), -np.inf).astype(np.float16)
+        assert np.array_equal(oracle.compact(row), np.nonzero(keep)[0].astype(np.int32))
+
+
+def test_q8_0_dequant_hand_built_blocks():
+    n = 2
+    d = np.ones((n, 18), np.float16)
+    d[1] = np.float16(0.5)
+    qv = np.zeros((n, 18, 32), np.int8)
+    ramp = np.arange(-16, 16, dtype=np.int8)
+    qv[0] = ramp[None, :]
+    qv[1] = np.int8(-127)
+    qv[1, 17, 31] = 127
+    rows = W.q8_0_pack(d, qv)
+    assert rows.shape == (2, 612)
+    deq = oracle.dequant_q8_0(rows)
+    assert np.array_equal(deq[0], np.tile(ramp.astype(np.float64), 18))
+    expect1 = np.full(DK, -63.5)
+    expect1[-1] = 63.5
+    assert np.array_equal(deq[1], expect1)
+
+
+def test_q8_0_attention_equals_f16_attention_on_exactly_representable_values():
+    # d = 1/64 (a power of two) and |q| <= 127: d*q is exact in f16, so the q8_0 path must
+    # equal the f16 path on the same values bit for bit.
+    rng = np.random.default_rng(12)
+    n = 45
+    qv = rng.integers(-127, 128, size=(n, 18, 32)).astype(np.int8)
+    d = np.full((n, 18), np.float16(1.0 / 64))
+    rows = W.q8_0_pack(d, qv)
+    kf16 = (qv.reshape(n, DK).astype(np.float32) / 64.0).astype(np.float16)
+    q = rand_f16(rng, (1, 4, DK))
+    mask = np.zeros((1, n), np.float16)
+    mask[0, 7] = NEG
+    a = oracle.attention(q, rows, kv_type=oracle.KV_Q8_0, mask=mask, scale=0.05)
+    b = oracle.attention(q, kf16, kv_type=oracle.KV_F16, mask=mask, scale=0.05)
+    assert np.array_equal(a, b)
+
+
+def test_sparse_index_path_equals_dense_masked_path():
+    rng = np.random.default_rng(13)
+    n = 300
+    q = rand_f16(rng, (1, 3, DK))
+    k = rand_f16(rng, (n, DK))
+    keep = rng.random(n) < 0.2
+    mask = np.where(keep, np.float16(0), NEG).astype(np.float16)[None]
+    idx = np.nonzero(keep)[0].astype(np.int32)
+    dense = oracle.attention(q, k, mask=mask, scale=0.07)
+    sparse = oracle.attention(q, k, mask=mask, scale=0.07, idx=idx)
+    np.testing.assert_allclose(sparse, dense, rtol=1e-12, atol=1e-14)
+
+
+def test_oracle_rejects_out_of_range_index():
+    q = np.zeros((1, 1, DK), np.float16)
+    k = np.zeros((4, DK), np.float16)
+    with pytest.raises(ValueError):
+        oracle.attention(q, k, idx=np.array([0, 4], np.int32))
+
+
+def test_planted_mistakes_are_caught():
+    """The checks above must fail on plausible oracle mistakes; emulate three of them on
+    the CPU in numpy (wrong V columns, mask scaled, rope dropped) and confirm that the
+    brute-force pin separates each from the oracle's answer."""
+    rng = np.random.default_rng(14)
+    q = rand_f16(rng, (2, 2, DK))
+    k = rand_f16(rng, (9, DK))
+    mask = rand_f16(rng, (2, 9), std=3.0)
+    scale = 0.2
+    ref = oracle.attention(q, k, mask=mask, scale=scale)
+
+    def route(qq, kk, vv, mm):
+        S = scale * np.einsum("thc,nc->thn", qq.astype(np.float64), kk.astype(np.float64))
+        S = S + mm
+        P = np.exp(S - S.max(-1, keepdims=True))
+        P /= P.sum(-1, keepdims=True)
+        return np.einsum("thn,nd->thd", P, vv.astype(np.float64)).reshape(-1, DV)
+
+    m64 = mask.astype(np.float64)[:, None, :]
+    good = route(q, k, k[:, :DV], m64)
+    np.testing.assert_allclose(ref, good, rtol=1e-12, atol=1e-13)
+    wrong_v = route(q, k, k[:, DK - DV:], m64)
+    scaled_mask = route(q, k, k[:, :DV], scale * m64)
+    q_norope = q.copy()
+    q_norope[..., DV:] = 0
+    no_rope = route(q_norope, k, k[:, :DV], m64)
+    for bad in (wrong_v, scaled_mask, no_rope):
+        assert np.max(np.abs(bad - ref)) > 1e-3
