@@ -1,0 +1,463 @@
+"""Benchmark of the MLA attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the workload's whole hot path through the C ABI
+(attention kernel, split-KV combine, and for the sparse workload the mask
+compaction first) over one batch of synthetic inputs resident in HBM. Between
+timed steps L2 is flushed by writing a 256 MiB buffer (outside the timed
+events). Each step is timed with CUDA events on the launching stream; with N
+ranks every rank runs its own replica of the batch (weak scaling, no
+collective on the data path) and the time is the max over ranks.
+
+Printed (rank 0): one JSON line with the metric, whole-job KV-cache GB/s,
+us/call, the roofline of the dominant kernel (live CUDA-event duration of its
+launches), an end-to-end figure through the same C ABI with host buffers
+(pinned host -> device copies of the inputs and device -> host copy of the
+output inside the timed region), the oracle's CPU throughput on a bounded
+sample, SM clocks sampled during the timed region, and the launch count.
+
+--impl reference times the fp64 CPU oracle as the reference arm (there is no
+runnable reference implementation of this path), on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mla_flash_attention_attn_b200 import workloads as W  # noqa: E402
+
+METRIC = ("MLA attention µs/call & KV-cache GB/s (DK576/DV512), "
+          "% of HBM/tensor roofline")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+DEFAULT_WORKLOAD = "v3_batched_decode"
+
+
+# ----------------------------------------------------------------------------- accounting
+def algorithmic(w, kept_cells=None):
+    """Algorithmic bytes and flops of one step, split partials excluded.
+
+    bytes = cache rows attended x row bytes + Q + mask cells read + output;
+    flops = 2 * n_head * (576 + 512) per (query row, attended key)."""
+    row_bytes = 1152 if w.kv_type == W.KV_F16 else W.Q8_ROW_BYTES
+    if kept_cells is None:
+        keep = ~np.isneginf(w.mask) if w.mask is not None else None
+        kept_cells = []
+        for b in range(w.n_seq):
+            L = int(w.kv_len[b])
+            if keep is None:
+                kept_cells.append([L] * w.n_q)
+            else:
+                kept_cells.append([int(keep[b, t, :L].sum()) for t in range(w.n_q)])
+    rows_attended = 0  # distinct cache rows read per sequence
+    pairs = 0          # (query token, attended key) pairs
+    mask_bytes = 0
+    for b in range(w.n_seq):
+        rows_attended += max(kept_cells[b])
+        pairs += sum(kept_cells[b])
+        mask_bytes += w.n_q * int(w.kv_len[b]) * 2 if w.mask is not None else 0
+    if w.sparse:
+        mask_bytes = w.n_seq * w.n_kv * 2 + rows_attended * 4 * 2  # mask read + idx write/read
+    q_bytes = w.q.size * 2
+    out_bytes = w.n_seq * w.n_q * w.n_head * 512 * 4
+    kv_bytes = rows_attended * row_bytes
+    flops = 2.0 * w.n_head * (576 + 512) * pairs
+    return {"kv_bytes": kv_bytes, "bytes": kv_bytes + q_bytes + mask_bytes + out_bytes,
+            "flops": flops}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.01):
+        self.index = index
+        self.period = period
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+class Step:
+    """Device-resident inputs and the hot path of one workload."""
+
+    def __init__(self, w, torch, binding):
+        self.w = w
+        self.torch = torch
+        self.b = binding
+        dev = torch.device("cuda")
+        self.q = torch.from_numpy(w.q).to(dev)
+        self.k = torch.from_numpy(w.kcache).to(dev)
+        self.mask = torch.from_numpy(w.mask).to(dev) if w.mask is not None else None
+        self.out = torch.empty(w.q.shape[:3] + (512,), dtype=torch.float32, device=dev)
+        self.kv_len = [int(x) for x in w.kv_len]
+        self.args, self._keep = binding.make_args(self.q, self.k, w.kv_type, self.mask, self.out,
+                                                  w.scale, kv_len=self.kv_len)
+        need = binding.mla_fa_workspace_size(self.args)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.ws_used = need > 0
+
+    def run(self, stream=None):
+        self.b.mla_fa_forward_ex(self.args, self.ws if self.ws_used else None, stream)
+
+
+def gpu_arm(args, rank, world):
+    import torch
+
+    from mla_flash_attention_attn_b200 import binding
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    binding.load()
+    w = W.make(args.workload)
+    acc = algorithmic(w)
+    step = Step(w, torch, binding)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def l2_flush():
+        flush.fill_(1.0)
+
+    for _ in range(args.warmup):
+        l2_flush()
+        step.run()
+    torch.cuda.synchronize()
+    if binding.mla_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        binding.mla_profile_begin()
+        for i in range(args.steps):
+            l2_flush()
+            starts[i].record(stream)
+            step.run()
+            stops[i].record(stream)
+        torch.cuda.synchronize()
+        prof = binding.mla_profile_end()
+    barrier(world)
+    torch.cuda.synchronize()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
+    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(total_ms, world)
+    status = binding.mla_get_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {binding.mla_status_string(status)}")
+
+    # ---- end to end through the same C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_measure(args, w, step, torch, binding, acc, world)
+
+    ms_per_step = total_ms / args.steps
+    kv_gbs = acc["kv_bytes"] * world / (ms_per_step * 1e-3) / 1e9
+    peaks, peak_kind = load_peaks()
+    dom = "mla_fwd_f16"
+    launches, dom_ms = prof.get(dom, (0, 0.0))
+    dom_avg_ms = dom_ms / max(launches, 1)
+    tensor_bound = acc["flops"] / acc["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        achieved = acc["flops"] / (dom_avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        achieved = acc["bytes"] / (dom_avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["traffic"] = args.traffic
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else \
+        "fallback (profiling recipe)"
+    roof["kernel"] = dom
+    roof["kernel_avg_us"] = round(dom_avg_ms * 1e3, 3)
+    roof["algorithmic_bytes_per_launch"] = acc["bytes"]
+    roof["algorithmic_flops_per_launch"] = acc["flops"]
+    result = {
+        "metric": METRIC,
+        "value": round(kv_gbs, 2),
+        "unit": "GB/s",
+        "us_per_call": round(ms_per_step * 1e3, 3),
+        "tokens_per_s": round(w.n_seq * w.n_q * world / (ms_per_step * 1e-3), 1),
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic (seeded PCG64; DeepSeek-V3/V2-Lite cache geometry, random values)",
+        "config": {"workload": args.workload, "n_seq": w.n_seq, "n_q": w.n_q,
+                   "n_head": w.n_head, "n_kv": w.n_kv,
+                   "kv_type": "q8_0" if w.kv_type else "f16",
+                   "kv_len": [int(x) for x in w.kv_len][:16],
+                   "parallelism": f"replicas x{world}",
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)"},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": int(sum(v[0] for v in prof.values())),
+        "kernels": {k: {"launches": v[0], "total_ms": round(v[1], 4)} for k, v in prof.items()},
+        "clocks": clocks.summary(),
+        "impl": "ours",
+    }
+    return result, w
+
+
+def e2e_measure(args, w, step, torch, binding, acc, world):
+    """Same hot path, with the inputs copied from pinned host memory each step and the
+    output copied back, all inside the CUDA-event timed region."""
+    hq = torch.from_numpy(w.q).pin_memory()
+    hk = torch.from_numpy(w.kcache).pin_memory()
+    hm = torch.from_numpy(w.mask).pin_memory() if w.mask is not None else None
+    hout = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
+    stream = torch.cuda.current_stream()
+    n = max(1, min(args.steps, args.e2e_steps))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for i in range(n + 1):
+        s, e = ev[i - 1] if i else (None, None)
+        if s is not None:
+            s.record(stream)
+        step.q.copy_(hq, non_blocking=True)
+        step.k.copy_(hk, non_blocking=True)
+        if hm is not None:
+            step.mask.copy_(hm, non_blocking=True)
+        step.run()
+        hout.copy_(step.out, non_blocking=True)
+        if e is not None:
+            e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), world) / n
+    h2d = hq.numel() * 2 + hk.numel() * hk.element_size() + (hm.numel() * 2 if hm is not None else 0)
+    return {"value": round(acc["kv_bytes"] * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "us_per_call": round(ms * 1e3, 2), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(hout.numel() * 4), "steps": n}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_throughput(w, acc, budget_s):
+    """Time the oracle on a bounded sample of query rows; scale to the metric's unit."""
+    import oracle
+
+    rows_total = w.n_seq * w.n_q * w.n_head
+    # rows per second estimate from one small probe, then a sample sized to the budget
+    t0 = time.perf_counter()
+    _oracle_rows(oracle, w, 1)
+    per_row = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(rows_total, max(oracle.max_threads(), budget_s / per_row * oracle.max_threads())))
+    t0 = time.perf_counter()
+    _oracle_rows(oracle, w, n)
+    dt = time.perf_counter() - t0
+    full_s = dt * rows_total / n
+    return {"value": round(acc["kv_bytes"] / full_s / 1e9, 6), "unit": "GB/s",
+            "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} of {rows_total} query rows, {dt:.1f} s on the host; "
+                      f"time scaled by rows to the full step",
+            "us_per_call_equiv": round(full_s * 1e6, 1)}
+
+
+def _oracle_rows(oracle, w, n):
+    """Compute n query rows spread over the sequences (sparse: over the kept indices)."""
+    per_seq = max(1, n // w.n_seq)
+    done = 0
+    for b in range(w.n_seq):
+        if done >= n:
+            break
+        k = min(per_seq, n - done, w.n_q * w.n_head)
+        rows = np.linspace(0, w.n_q * w.n_head - 1, k).astype(np.int32)
+        mask = w.mask[b] if w.mask is not None else None
+        idx = None
+        if w.sparse:
+            idx = oracle.compact(w.mask[b, 0])
+        oracle.attention(w.q[b], w.kcache[b], w.kv_type, mask, w.scale, rows=rows, idx=idx)
+        done += k
+
+
+def reference_arm(args, rank, world):
+    """The oracle as the reference arm: each step computes a bounded sample of the step's
+    rows on the host cores; the per-step time is scaled by rows to the full step."""
+    if rank != 0:
+        return None
+    import oracle
+
+    w = W.make(args.workload)
+    acc = algorithmic(w)
+    rows_total = w.n_seq * w.n_q * w.n_head
+    per_step_budget = max(0.5, args.ref_budget_s / max(1, args.steps + args.warmup))
+    t0 = time.perf_counter()
+    _oracle_rows(oracle, w, 1)
+    per_row = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(rows_total, max(1, per_step_budget / per_row * oracle.max_threads())))
+    for _ in range(args.warmup):
+        _oracle_rows(oracle, w, max(1, n // 8))
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_rows(oracle, w, n)
+        times.append((time.perf_counter() - t0) * rows_total / n)
+    ms = 1e3 * sum(times) / len(times)
+    value = acc["kv_bytes"] / (ms * 1e-3) / 1e9
+    cpu = {"value": round(value, 6), "unit": "GB/s", "cores": oracle.max_threads(),
+           "kind": "oracle",
+           "sample": f"{n} of {rows_total} query rows per step, time scaled by rows"}
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded PCG64)",
+        "config": {"workload": args.workload, "n_seq": w.n_seq, "n_q": w.n_q,
+                   "n_head": w.n_head, "n_kv": w.n_kv, "parallelism": "host cores"},
+        "impl": "reference", "cpu_baseline": cpu,
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- ranks
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x)], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def init_ranks(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        backend = "nccl" if (torch.cuda.is_available() and args.impl == "ours") else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-budget-s", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel, if captured")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world = init_ranks(args)
+    try:
+        if args.impl == "reference":
+            res = reference_arm(args, rank, world)
+        else:
+            res, w = gpu_arm(args, rank, world)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = oracle_throughput(w, algorithmic(w), args.cpu_budget_s)
+            elif rank == 0:
+                res["cpu_baseline"] = None
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

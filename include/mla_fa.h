@@ -1,0 +1,191 @@
+/*
+ * mla_fa.h -- C ABI of libmla_fa.so: fused flash attention for Multi-head
+ * Latent Attention (MLA) over the compressed KV cache, on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (one query row = one (token t, head h) pair):
+ *
+ *     S[j]   = scale * dot(q[t,h,0:576], k[j,0:576]) + mask[t,j]
+ *     P      = softmax over j of S
+ *     out[t,h,0:512] = sum_j P[j] * k[j,0:512]
+ *
+ * Sources (web pages on MLA flash attention):
+ *  - Cache row = kv_lora_rank (512) latent followed by the n_embd_head_qk_rope
+ *    (64) RoPE key, 576 values, one row per token, shared by all query heads:
+ *    ik_llama.cpp "-mla" guide, section "MLA 是什麼".
+ *  - With flash attention there is only a K cache; V is derived from it. Here
+ *    V = the first 512 columns of the same row: ik_llama.cpp "-mla" guide,
+ *    section "-mla四檔語義". Q arrives already absorbed (576 wide); the
+ *    up/down projections are outside this library.
+ *  - Block-wise online softmax with a running max m and running sum l, so the
+ *    score matrix never reaches device memory: Vulkan FA for DeepSeek MLA
+ *    article, sections 2.1-2.2.
+ *  - f16 additive mask: baguaai flash-attention tag page (PR #23764 item).
+ *  - Quantised q8_0 K cache (-ctk q8_0): ik_llama.cpp "-mla" guide, section
+ *    on recommended command lines; sparse FA over a quantised cache and the
+ *    single-scan mask-index compaction: llama.cpp b11413 release note.
+ *
+ * Conventions for every entry point:
+ *  - All pointers to tensors are DEVICE pointers owned by the caller, except
+ *    where an argument says HOST. The library never frees caller memory.
+ *  - Every call checks its arguments on the host before any launch and
+ *    returns a mla_status; nothing aborts, throws or prints.
+ *  - Launches go to the given CUDA stream (cudaStream_t passed as void*;
+ *    NULL = the legacy default stream). No call synchronises the stream except
+ *    mla_get_device_status.
+ *  - Errors a kernel meets at run time (a bounded wait that ran out) are
+ *    recorded in a per-device status word read by mla_get_device_status.
+ */
+#ifndef MLA_FA_H
+#define MLA_FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_DK 576            /* cache row / query width: 512 latent + 64 rope */
+#define MLA_DV 512            /* value width: the first 512 columns of a row   */
+#define MLA_Q8_0_BLOCK 32     /* q8_0: 32 int8 per block                        */
+#define MLA_Q8_0_ROW_BYTES 612 /* q8_0: 18 blocks x {f16 d; int8 q[32]}         */
+#define MLA_MAX_HEADS 128
+
+typedef enum {
+  MLA_KV_F16 = 0,  /* row = 576 f16 (1152 bytes) */
+  MLA_KV_Q8_0 = 1  /* row = 18 blocks of {f16 d; int8 q[32]} (612 bytes), value = d*q */
+} mla_kv_type;
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_NULL = -1,        /* a required pointer is NULL                      */
+  MLA_ERR_SHAPE = -2,       /* a size or stride is out of range                */
+  MLA_ERR_TYPE = -3,        /* unknown kcache_type                             */
+  MLA_ERR_ALIGN = -4,       /* a pointer or stride breaks 16-byte alignment    */
+  MLA_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required      */
+  MLA_ERR_CUDA = -6,        /* a CUDA runtime call failed                      */
+  MLA_ERR_TIMEOUT = -7,     /* a kernel's bounded wait ran out (device status) */
+  MLA_ERR_UNSUPPORTED = -8, /* valid but unsupported (e.g. no sm_100 device)   */
+  MLA_ERR_INDEX = -9        /* a sparse index outside [0, n_kv) (device status) */
+} mla_status;
+
+/* Full argument set of the batched / sparse forward pass.
+ *
+ * q       f16, element (b, t, h, c) at q[b*q_seq_stride + (t*n_head + h)*576 + c]
+ * kcache  row (b, j) at byte offset (b*k_seq_stride + j) * row_bytes, where
+ *         row_bytes = 1152 (MLA_KV_F16) or 612 (MLA_KV_Q8_0)
+ * mask    f16 or NULL, element (b, t, j) at mask[b*mask_seq_stride + t*mask_row_stride + j];
+ *         0 keeps a cell, -inf drops it, any finite value is added to the score;
+ *         shared by all heads of a token
+ * out     fp32, element (b, t, h, d) at out[b*out_seq_stride + (t*n_head + h)*512 + d]
+ * kv_len  HOST int32[n_seq] or NULL: cells j >= kv_len[b] are not read (treated as
+ *         dropped); NULL means n_kv for every sequence
+ * idx     DEVICE int32 or NULL (sparse): sequence b attends only to cache rows
+ *         idx[b*idx_seq_stride + i] for i < idx_count[b], each in [0, n_kv) and,
+ *         as mla_compact_mask writes them, ascending; the mask (if any) is still
+ *         indexed by the original cell j = idx[...]
+ * idx_count DEVICE int32[n_seq]; required with idx. Read on the device: no host sync.
+ * A stride of 0 means "dense" (the natural value for the given sizes).
+ */
+typedef struct mla_fa_args {
+  const void* q;
+  const void* kcache;
+  int kcache_type;
+  const void* mask;
+  float* out;
+  int n_seq;
+  int n_q;
+  int n_head;
+  int n_kv;
+  float scale;
+  int64_t q_seq_stride;     /* elements; 0 = n_q*n_head*576                    */
+  int64_t k_seq_stride;     /* rows;     0 = n_kv                              */
+  int64_t mask_seq_stride;  /* elements; 0 = n_q*mask_row_stride               */
+  int64_t mask_row_stride;  /* elements; 0 = n_kv                              */
+  int64_t out_seq_stride;   /* elements; 0 = n_q*n_head*512                    */
+  const int32_t* kv_len;    /* HOST, optional                                  */
+  const int32_t* idx;       /* DEVICE, optional (sparse)                       */
+  const int32_t* idx_count; /* DEVICE, required with idx                       */
+  int64_t idx_seq_stride;   /* entries;  0 = n_kv                              */
+} mla_fa_args;
+
+/* Forward pass with the sizes of the single-sequence call:
+ *   q [n_q][n_head][576] f16, kcache [n_kv] rows of kcache_type,
+ *   mask [n_q][n_kv] f16 or NULL, out [n_q][n_head][512] fp32.
+ * Uses the stream set by mla_set_stream (per host thread, default NULL) and a
+ * workspace the library allocates on first use and keeps (grown as needed).
+ * Constraints: 1 <= n_head <= 128, n_q >= 1, n_kv >= 1; q, kcache, out 16-byte aligned.
+ * Returns MLA_OK or the first argument error. */
+int mla_fa_forward(const void* q, const void* kcache, int kcache_type, const void* mask, int n_q,
+                   int n_head, int n_kv, float scale, float* out);
+
+/* Select the stream mla_fa_forward and mla_compact_mask launch on (this thread). */
+int mla_set_stream(void* cuda_stream);
+
+/* Bytes of workspace mla_fa_forward_ex needs for these arguments (0 when the
+ * pass needs no split-KV partials). Returns 0 as well for invalid arguments. */
+size_t mla_fa_workspace_size(const mla_fa_args* a);
+
+/* Batched / sparse forward pass into caller-owned workspace (device memory of
+ * at least mla_fa_workspace_size(a) bytes, 256-byte aligned; may be NULL when
+ * that size is 0). Split-KV partials go to the workspace and are merged by the
+ * log-sum-exp combine before the call's last kernel ends. */
+int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, void* stream);
+
+/* How the pass is divided: units = CTA pairs launched, max_splits = largest
+ * number of KV splits of one (sequence, 128-row group). For tests and tools. */
+int mla_fa_query_plan(const mla_fa_args* a, int* units, int* max_splits);
+
+/* Single-scan mask compaction (llama.cpp b11413 release note, "single-scan
+ * sparse FA index compaction"): writes, in ascending order, the index of every
+ * cell of the f16 mask row whose value is not -inf (bits 0xFC00), and the number
+ * of such cells to *count_out -- both on the device, with no host sync.
+ * mask_row: DEVICE f16[n_kv]; idx_out: DEVICE int32[n_kv]; count_out: DEVICE int32.
+ * Uses a small library-owned workspace (allocated once per device). */
+int mla_compact_mask(const void* mask_row, int n_kv, int32_t* idx_out, int32_t* count_out,
+                     void* stream);
+
+/* Multi-row form with caller workspace: row r of `mask` starts at
+ * mask + r*mask_row_stride (elements); its indices go to idx_out + r*idx_row_stride
+ * and its count to count_out[r]. workspace: DEVICE, >= mla_compact_workspace_size
+ * bytes, 256-byte aligned, zero-filled by the caller before its first use; each
+ * call leaves it ready for the next (calls sharing one workspace must not overlap). */
+size_t mla_compact_workspace_size(int n_rows, int n_kv);
+int mla_compact_mask_ex(const void* mask, int n_rows, int64_t mask_row_stride, int n_kv,
+                        int32_t* idx_out, int64_t idx_row_stride, int32_t* count_out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then return and clear this device's run-time status:
+ * MLA_OK, MLA_ERR_TIMEOUT (a bounded wait in a kernel gave up; that kernel's
+ * results are invalid) or MLA_ERR_INDEX; MLA_ERR_CUDA if the sync failed. */
+int mla_get_device_status(void* stream);
+
+/* Launch a one-CTA kernel that waits on a barrier nothing ever signals, with a
+ * wait limit of timeout_ns; it records MLA_ERR_TIMEOUT and returns. Lets a test
+ * exercise the bounded-wait error path without a fault. */
+int mla_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Per-kernel device timing. Between mla_profile_begin and mla_profile_end the
+ * library records a pair of CUDA events around every kernel it launches (on
+ * that launch's stream) and counts the launches. mla_profile_end synchronises
+ * those events and fills up to max_entries records, one per kernel that ran;
+ * *n_entries gets the number filled. Profiling state is per process. */
+typedef struct mla_profile_entry {
+  char name[48];     /* kernel name, e.g. "mla_fwd_f16" */
+  int launches;      /* launches recorded                */
+  double total_ms;   /* sum of event-timed durations     */
+} mla_profile_entry;
+int mla_profile_begin(void);
+int mla_profile_end(mla_profile_entry* entries, int max_entries, int* n_entries);
+
+/* Human-readable name of a status code (static string). */
+const char* mla_status_string(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_FA_H */

@@ -1,0 +1,261 @@
+"""ctypes binding of libmla_fa.so (include/mla_fa.h), same names as the C ABI.
+
+This module only marshals arguments: torch tensors are turned into device
+pointers and sizes, and every step of the computation runs in the library's
+CUDA kernels. There is no CPU path: if the library is missing or the device is
+not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+LIB_PATH = os.path.join(PKG, "libmla_fa.so")
+HEADER = os.path.join(ROOT, "include", "mla_fa.h")
+
+DK = 576
+DV = 512
+Q8_ROW_BYTES = 612
+KV_F16 = 0
+KV_Q8_0 = 1
+
+MLA_OK = 0
+STATUS_NAMES = {
+    0: "MLA_OK", -1: "MLA_ERR_NULL", -2: "MLA_ERR_SHAPE", -3: "MLA_ERR_TYPE",
+    -4: "MLA_ERR_ALIGN", -5: "MLA_ERR_WORKSPACE", -6: "MLA_ERR_CUDA", -7: "MLA_ERR_TIMEOUT",
+    -8: "MLA_ERR_UNSUPPORTED", -9: "MLA_ERR_INDEX",
+}
+
+
+class MlaError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class mla_fa_args(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p),
+        ("kcache", ctypes.c_void_p),
+        ("kcache_type", ctypes.c_int),
+        ("mask", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("n_seq", ctypes.c_int),
+        ("n_q", ctypes.c_int),
+        ("n_head", ctypes.c_int),
+        ("n_kv", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("q_seq_stride", ctypes.c_int64),
+        ("k_seq_stride", ctypes.c_int64),
+        ("mask_seq_stride", ctypes.c_int64),
+        ("mask_row_stride", ctypes.c_int64),
+        ("out_seq_stride", ctypes.c_int64),
+        ("kv_len", ctypes.c_void_p),
+        ("idx", ctypes.c_void_p),
+        ("idx_count", ctypes.c_void_p),
+        ("idx_seq_stride", ctypes.c_int64),
+    ]
+
+
+class mla_profile_entry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int),
+                ("total_ms", ctypes.c_double)]
+
+
+_lib = None
+
+
+def header_functions():
+    """Names of the functions include/mla_fa.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(mla_\w+)\s*\(", text, flags=re.M)))
+
+
+def load(path: str = LIB_PATH):
+    """Load the library and declare the C signatures. Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(
+            f"{path} is missing: build it with `python -m mla_flash_attention_attn_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, Z, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_uint64
+    lib.mla_fa_forward.argtypes = [P, P, I, P, I, I, I, ctypes.c_float, P]
+    lib.mla_fa_forward.restype = I
+    lib.mla_set_stream.argtypes = [P]
+    lib.mla_set_stream.restype = I
+    lib.mla_fa_workspace_size.argtypes = [ctypes.POINTER(mla_fa_args)]
+    lib.mla_fa_workspace_size.restype = Z
+    lib.mla_fa_forward_ex.argtypes = [ctypes.POINTER(mla_fa_args), P, Z, P]
+    lib.mla_fa_forward_ex.restype = I
+    lib.mla_fa_query_plan.argtypes = [ctypes.POINTER(mla_fa_args), ctypes.POINTER(I),
+                                      ctypes.POINTER(I)]
+    lib.mla_fa_query_plan.restype = I
+    lib.mla_compact_mask.argtypes = [P, I, P, P, P]
+    lib.mla_compact_mask.restype = I
+    lib.mla_compact_workspace_size.argtypes = [I, I]
+    lib.mla_compact_workspace_size.restype = Z
+    lib.mla_compact_mask_ex.argtypes = [P, I, ctypes.c_int64, I, P, ctypes.c_int64, P, P, Z, P]
+    lib.mla_compact_mask_ex.restype = I
+    lib.mla_get_device_status.argtypes = [P]
+    lib.mla_get_device_status.restype = I
+    lib.mla_debug_wait_timeout.argtypes = [U64, P]
+    lib.mla_debug_wait_timeout.restype = I
+    lib.mla_status_string.argtypes = [I]
+    lib.mla_status_string.restype = ctypes.c_char_p
+    lib.mla_version.argtypes = []
+    lib.mla_version.restype = I
+    lib.mla_profile_begin.argtypes = []
+    lib.mla_profile_begin.restype = I
+    lib.mla_profile_end.argtypes = [ctypes.POINTER(mla_profile_entry), I, ctypes.POINTER(I)]
+    lib.mla_profile_end.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(status, what):
+    if status != MLA_OK:
+        raise MlaError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _host_i32(arr):
+    """Keep-alive ctypes int32 array for HOST arguments (kv_len)."""
+    if arr is None:
+        return None
+    vals = [int(v) for v in arr]
+    return (ctypes.c_int32 * len(vals))(*vals)
+
+
+def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None):
+    """Fill mla_fa_args from batched torch tensors.
+
+    q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
+    mask [n_seq][n_q][n_kv] f16 or None; out [n_seq][n_q][n_head][512] f32.
+    Returns (args, keepalive)."""
+    n_seq, n_q, n_head, dk = q.shape
+    if dk != DK:
+        raise ValueError("q must end in 576")
+    a = mla_fa_args()
+    a.q = q.data_ptr()
+    a.kcache = kcache.data_ptr()
+    a.kcache_type = int(kv_type)
+    a.mask = None if mask is None else mask.data_ptr()
+    a.out = out.data_ptr()
+    a.n_seq, a.n_q, a.n_head, a.n_kv = n_seq, n_q, n_head, kcache.shape[1]
+    a.scale = float(scale)
+    a.q_seq_stride = q.stride(0)
+    a.k_seq_stride = kcache.stride(0) // kcache.stride(1)
+    if mask is not None:
+        a.mask_seq_stride = mask.stride(0)
+        a.mask_row_stride = mask.stride(1)
+    a.out_seq_stride = out.stride(0)
+    keep = _host_i32(kv_len)
+    a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
+    if idx is not None:
+        a.idx = idx.data_ptr()
+        a.idx_count = idx_count.data_ptr()
+        a.idx_seq_stride = idx.stride(0)
+    return a, keep
+
+
+def mla_fa_workspace_size(args) -> int:
+    return int(load().mla_fa_workspace_size(ctypes.byref(args)))
+
+
+def mla_fa_query_plan(args):
+    units, splits = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().mla_fa_query_plan(ctypes.byref(args), ctypes.byref(units), ctypes.byref(splits)),
+           "mla_fa_query_plan")
+    return units.value, splits.value
+
+
+def mla_fa_forward_ex(args, workspace=None, stream=None):
+    ws_ptr = None if workspace is None else ctypes.c_void_p(workspace.data_ptr())
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().mla_fa_forward_ex(ctypes.byref(args), ws_ptr, ws_bytes, _stream_ptr(stream)),
+           "mla_fa_forward_ex")
+
+
+def mla_fa_forward(q, kcache, kv_type, mask, scale, out, stream=None):
+    """Single-sequence call: q [n_q][n_head][576], kcache [n_kv][...], mask [n_q][n_kv]."""
+    lib = load()
+    _check(lib.mla_set_stream(_stream_ptr(stream)), "mla_set_stream")
+    n_q, n_head, _ = q.shape
+    _check(lib.mla_fa_forward(_ptr(q), _ptr(kcache), int(kv_type), _ptr(mask), n_q, n_head,
+                              kcache.shape[0], float(scale), _ptr(out)), "mla_fa_forward")
+
+
+def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, idx_count=None,
+            workspace=None, stream=None):
+    """Batched forward through mla_fa_forward_ex; allocates out/workspace with torch if absent."""
+    import torch
+
+    if out is None:
+        out = torch.empty(q.shape[:3] + (DV,), dtype=torch.float32, device=q.device)
+    args, keep = make_args(q, kcache, kv_type, mask, out, scale, kv_len, idx, idx_count)
+    need = mla_fa_workspace_size(args)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    mla_fa_forward_ex(args, workspace if need else None, stream)
+    del keep
+    return out
+
+
+def mla_compact_mask(mask_row, idx_out, count_out, stream=None):
+    _check(load().mla_compact_mask(_ptr(mask_row), mask_row.numel(), _ptr(idx_out), _ptr(count_out),
+                                   _stream_ptr(stream)), "mla_compact_mask")
+
+
+def mla_compact_workspace_size(n_rows, n_kv) -> int:
+    return int(load().mla_compact_workspace_size(int(n_rows), int(n_kv)))
+
+
+def mla_compact_mask_ex(mask, idx_out, count_out, workspace, stream=None):
+    """mask [n_rows][n_kv] f16, idx_out [n_rows][>= n_kv] int32, count_out [n_rows] int32."""
+    n_rows, n_kv = mask.shape
+    _check(load().mla_compact_mask_ex(_ptr(mask), n_rows, mask.stride(0), n_kv, _ptr(idx_out),
+                                      idx_out.stride(0), _ptr(count_out), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream_ptr(stream)), "mla_compact_mask_ex")
+
+
+def mla_get_device_status(stream=None) -> int:
+    return int(load().mla_get_device_status(_stream_ptr(stream)))
+
+
+def mla_debug_wait_timeout(timeout_ns, stream=None):
+    _check(load().mla_debug_wait_timeout(int(timeout_ns), _stream_ptr(stream)),
+           "mla_debug_wait_timeout")
+
+
+def mla_status_string(status) -> str:
+    return load().mla_status_string(int(status)).decode()
+
+
+def mla_profile_begin():
+    _check(load().mla_profile_begin(), "mla_profile_begin")
+
+
+def mla_profile_end():
+    """Stop profiling; returns {kernel name: (launches, total_ms)}."""
+    buf = (mla_profile_entry * 16)()
+    n = ctypes.c_int(0)
+    _check(load().mla_profile_end(buf, 16, ctypes.byref(n)), "mla_profile_end")
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n.value)}

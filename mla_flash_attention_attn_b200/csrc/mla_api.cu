@@ -1,0 +1,544 @@
+// Host side of libmla_fa.so: argument checks, the split-KV launch plan, TMA
+// tensor maps and the kernel launches behind the C ABI in include/mla_fa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/mla_fa.h"
+#include "mla_common.cuh"
+#include "mla_compact.cuh"
+#include "mla_fwd.cuh"
+
+namespace {
+
+using mla::Plan;
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
+constexpr int kMinTilesPerSplit = 2;
+
+thread_local cudaStream_t t_stream = nullptr;
+
+struct DeviceState {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  bool fwd_attr_set = false;
+  void* fwd_ws = nullptr;  // workspace of mla_fa_forward
+  size_t fwd_ws_bytes = 0;
+  void* cmp_ws = nullptr;  // workspace of mla_compact_mask
+  size_t cmp_ws_bytes = 0;
+  uint32_t cmp_epoch = 1;
+};
+
+std::mutex g_mutex;
+std::vector<DeviceState> g_dev;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+PFN_cuCtxGetCurrent_v4000 g_ctx_get_current = nullptr;
+PFN_cuCtxGetDevice_v2000 g_ctx_get_device = nullptr;
+
+void* driver_fn(const char* name) {
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return fn;
+}
+
+// The library links its own copy of the CUDA runtime. The device the caller
+// works on (e.g. the one torch made current on this thread) is taken from the
+// driver's current context, so both runtimes agree on the device.
+int sync_device_with_context(int* dev) {
+  if (g_ctx_get_current == nullptr) {
+    g_ctx_get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(driver_fn("cuCtxGetCurrent"));
+    g_ctx_get_device = reinterpret_cast<PFN_cuCtxGetDevice_v2000>(driver_fn("cuCtxGetDevice"));
+  }
+  CUcontext ctx = nullptr;
+  CUdevice cdev = 0;
+  if (g_ctx_get_current && g_ctx_get_device && g_ctx_get_current(&ctx) == CUDA_SUCCESS &&
+      ctx != nullptr && g_ctx_get_device(&cdev) == CUDA_SUCCESS) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return MLA_ERR_CUDA;
+    if (cur != (int)cdev && cudaSetDevice((int)cdev) != cudaSuccess) return MLA_ERR_CUDA;
+    *dev = (int)cdev;
+    return MLA_OK;
+  }
+  return cudaGetDevice(dev) == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int current_device(DeviceState** st) {
+  int dev = 0;
+  if (sync_device_with_context(&dev) != MLA_OK) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mutex);
+  if ((int)g_dev.size() <= dev) g_dev.resize(dev + 1);
+  DeviceState& s = g_dev[dev];
+  if (!s.probed) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return MLA_ERR_CUDA;
+    s.supported = (prop.major == 10 && prop.minor == 0);
+    s.sm_count = prop.multiProcessorCount;
+    s.probed = true;
+  }
+  if (!s.supported) return MLA_ERR_UNSUPPORTED;
+  if (g_encode == nullptr) {
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_fn("cuTensorMapEncodeTiled"));
+    if (g_encode == nullptr) return MLA_ERR_CUDA;
+  }
+  *st = &s;
+  return MLA_OK;
+}
+
+// ---------------------------------------------------------------- profiling
+enum KernelId { kKernFwdF16 = 0, kKernCombine = 1, kKernCompact = 2, kKernWaitTest = 3, kNumKernels };
+const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_combine", "mla_compact",
+                                               "mla_wait_timeout"};
+struct ProfRecord {
+  cudaEvent_t start, stop;
+  int kernel;
+};
+std::mutex g_prof_mutex;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof_records;
+std::vector<cudaEvent_t> g_prof_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_prof_pool.empty()) {
+    cudaEvent_t e = g_prof_pool.back();
+    g_prof_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets one launch with events when profiling is on.
+struct ProfScope {
+  cudaEvent_t stop = nullptr;
+  int kernel;
+  cudaStream_t stream;
+  ProfScope(int k, cudaStream_t s) : kernel(k), stream(s) {
+    std::lock_guard<std::mutex> lk(g_prof_mutex);
+    if (!g_prof_on) return;
+    cudaEvent_t start = prof_event();
+    stop = prof_event();
+    cudaEventRecord(start, stream);
+    g_prof_records.push_back({start, stop, k});
+  }
+  ~ProfScope() {
+    if (stop) cudaEventRecord(stop, stream);
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+struct Resolved {
+  mla_fa_args a;
+  int rows;
+  int64_t q_ss, k_ss, m_ss, m_rs, o_ss, idx_ss;
+};
+
+int validate(const mla_fa_args* a, Resolved* r) {
+  if (a == nullptr) return MLA_ERR_NULL;
+  if (a->q == nullptr || a->kcache == nullptr || a->out == nullptr) return MLA_ERR_NULL;
+  if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
+  if (a->n_seq < 1 || a->n_q < 1 || a->n_head < 1 || a->n_head > MLA_MAX_HEADS || a->n_kv < 1)
+    return MLA_ERR_SHAPE;
+  if (!std::isfinite(a->scale)) return MLA_ERR_SHAPE;
+  const int64_t rows = (int64_t)a->n_q * a->n_head;
+  if (rows > (1 << 24)) return MLA_ERR_SHAPE;
+  if (a->idx != nullptr && a->idx_count == nullptr) return MLA_ERR_NULL;
+  r->a = *a;
+  r->rows = (int)rows;
+  r->q_ss = a->q_seq_stride ? a->q_seq_stride : rows * MLA_DK;
+  r->k_ss = a->k_seq_stride ? a->k_seq_stride : a->n_kv;
+  r->m_rs = a->mask_row_stride ? a->mask_row_stride : a->n_kv;
+  r->m_ss = a->mask_seq_stride ? a->mask_seq_stride : (int64_t)a->n_q * r->m_rs;
+  r->o_ss = a->out_seq_stride ? a->out_seq_stride : rows * MLA_DV;
+  r->idx_ss = a->idx_seq_stride ? a->idx_seq_stride : a->n_kv;
+  if (r->q_ss < rows * MLA_DK || r->k_ss < a->n_kv || r->m_rs < a->n_kv ||
+      r->m_ss < (int64_t)(a->n_q - 1) * r->m_rs + a->n_kv || r->o_ss < rows * MLA_DV ||
+      r->idx_ss < 0)
+    return MLA_ERR_SHAPE;
+  if (a->q_seq_stride < 0 || a->k_seq_stride < 0 || a->mask_seq_stride < 0 ||
+      a->mask_row_stride < 0 || a->out_seq_stride < 0 || a->idx_seq_stride < 0)
+    return MLA_ERR_SHAPE;
+  if (!aligned16(a->q) || !aligned16(a->kcache) || !aligned16(a->out)) return MLA_ERR_ALIGN;
+  if ((r->q_ss % 8) != 0 || (r->o_ss % 4) != 0) return MLA_ERR_ALIGN;
+  if (a->mask != nullptr && (reinterpret_cast<uintptr_t>(a->mask) & 1)) return MLA_ERR_ALIGN;
+  if (a->kv_len != nullptr)
+    for (int b = 0; b < a->n_seq; ++b)
+      if (a->kv_len[b] < 0 || a->kv_len[b] > a->n_kv) return MLA_ERR_SHAPE;
+  if (a->kcache_type != MLA_KV_F16 || a->idx != nullptr) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+// Split plan for sequences [s0, s0+n). Returns the partial slots it needs.
+int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
+  std::memset(plan, 0, sizeof(Plan));
+  const mla_fa_args& a = r.a;
+  plan->n_seq = n;
+  plan->seq_offset = s0;
+  plan->rows = r.rows;
+  plan->groups = (r.rows + mla::kRowsPerGroup - 1) / mla::kRowsPerGroup;
+  plan->n_head = a.n_head;
+  plan->n_q = a.n_q;
+  plan->n_kv = a.n_kv;
+  const int pairs = std::max(1, sm_count / 2);
+  int64_t sum_tiles = 0;
+  std::vector<int> tiles(n);
+  for (int b = 0; b < n; ++b) {
+    const int len = a.kv_len ? a.kv_len[s0 + b] : a.n_kv;
+    plan->kv_len[b] = len;
+    tiles[b] = (len + mla::kTileKeys - 1) / mla::kTileKeys;
+    sum_tiles += tiles[b];
+  }
+  const int64_t total_groups = (int64_t)n * plan->groups;
+  int units = 0, slots = 0;
+  for (int b = 0; b < n; ++b) {
+    int ns = 1;
+    if (total_groups < pairs && sum_tiles > 0) {
+      const double want = (double)pairs * tiles[b] / ((double)sum_tiles * plan->groups);
+      ns = (int)std::floor(want + 0.5);
+      ns = std::min(ns, std::max(1, tiles[b] / kMinTilesPerSplit));
+      ns = std::max(ns, 1);
+    }
+    plan->n_split[b] = ns;
+    plan->unit_base[b] = units;
+    units += plan->groups * ns;
+    if (ns > 1) {
+      plan->ws_base[b] = slots;
+      slots += plan->groups * ns;
+    } else {
+      plan->ws_base[b] = -1;
+    }
+  }
+  plan->unit_base[n] = units;
+  plan->total_units = units;
+  return slots;
+}
+
+size_t slot_bytes() { return (size_t)mla::kRowsPerGroup * (mla::kDV + 1) * sizeof(float); }
+
+size_t workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_splits) {
+  size_t need = 0;
+  int mu = 0, ms = 0;
+  Plan plan;
+  for (int s0 = 0; s0 < r.a.n_seq; s0 += mla::kPlanMaxSeq) {
+    const int n = std::min(mla::kPlanMaxSeq, r.a.n_seq - s0);
+    const int slots = build_plan(r, s0, n, sm_count, &plan);
+    need = std::max(need, (size_t)slots * slot_bytes());
+    mu = std::max(mu, plan.total_units);
+    for (int b = 0; b < n; ++b) ms = std::max(ms, plan.n_split[b]);
+  }
+  if (max_units) *max_units = mu;
+  if (max_splits) *max_splits = ms;
+  return need;
+}
+
+int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+             uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1) {
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult res = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const mla_fa_args& a = r.a;
+  const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)))
+    return MLA_ERR_WORKSPACE;
+  CUtensorMap tm_q, tm_k, tm_v;
+  const uint64_t row_bytes = MLA_DK * 2;
+  int rc = make_map(&tm_q, a.q, MLA_DK, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
+  if (rc == MLA_OK)
+    rc = make_map(&tm_k, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
+                  64, 64);
+  if (rc == MLA_OK)
+    rc = make_map(&tm_v, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
+                  64, 32);
+  if (rc != MLA_OK) return rc;
+  if (!st->fwd_attr_set) {
+    if (cudaFuncSetAttribute(mla::mla_fwd_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mla::fwd::kSmemAlloc) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    st->fwd_attr_set = true;
+  }
+  mla::MlaFwdParams p;
+  p.mask = static_cast<const uint16_t*>(a.mask);
+  p.out = a.out;
+  p.mask_seq_stride = r.m_ss;
+  p.mask_row_stride = r.m_rs;
+  p.out_seq_stride = r.o_ss;
+  p.scale_log2 = a.scale * mla::kLog2e;
+  p.mask_vec_ok = (a.mask != nullptr && aligned16(a.mask) && (r.m_ss % 8) == 0 && (r.m_rs % 8) == 0);
+  p.timeout_ns = kDefaultTimeoutNs;
+  Plan plan;
+  for (int s0 = 0; s0 < a.n_seq; s0 += mla::kPlanMaxSeq) {
+    const int n = std::min(mla::kPlanMaxSeq, a.n_seq - s0);
+    const int slots = build_plan(r, s0, n, st->sm_count, &plan);
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                                (size_t)slots * mla::kRowsPerGroup * mla::kDV * 4)
+                     : nullptr;
+    dim3 grid(2 * plan.total_units);
+    {
+      ProfScope prof(kKernFwdF16, stream);
+      mla::mla_fwd_f16_kernel<<<grid, mla::fwd::kThreads, mla::fwd::kSmemAlloc, stream>>>(
+          tm_q, tm_k, tm_v, plan, p);
+    }
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (slots > 0) {
+      dim3 cgrid((r.rows + 3) / 4, n);
+      {
+        ProfScope prof(kKernCombine, stream);
+        mla::mla_combine_kernel<<<cgrid, 128, 0, stream>>>(plan, p.ws_o, p.ws_lse, a.out, r.o_ss);
+      }
+      if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
+  }
+  return MLA_OK;
+}
+
+int ensure_ws(void** ptr, size_t* have, size_t need) {
+  if (*have >= need) return MLA_OK;
+  if (*ptr) cudaFree(*ptr);
+  *ptr = nullptr;
+  *have = 0;
+  if (cudaMalloc(ptr, need) != cudaSuccess) return MLA_ERR_CUDA;
+  *have = need;
+  return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_version(void) { return 100; }
+
+const char* mla_status_string(int status) {
+  switch (status) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_NULL: return "MLA_ERR_NULL: a required pointer is NULL";
+    case MLA_ERR_SHAPE: return "MLA_ERR_SHAPE: a size or stride is out of range";
+    case MLA_ERR_TYPE: return "MLA_ERR_TYPE: unknown kcache_type";
+    case MLA_ERR_ALIGN: return "MLA_ERR_ALIGN: a pointer or stride breaks 16-byte alignment";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace missing or too small";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: a CUDA runtime call failed";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: a kernel's bounded wait ran out";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: valid but unsupported here";
+    case MLA_ERR_INDEX: return "MLA_ERR_INDEX: a sparse index is outside [0, n_kv)";
+    default: return "unknown mla status";
+  }
+}
+
+int mla_set_stream(void* cuda_stream) {
+  t_stream = static_cast<cudaStream_t>(cuda_stream);
+  return MLA_OK;
+}
+
+size_t mla_fa_workspace_size(const mla_fa_args* a) {
+  Resolved r;
+  if (validate(a, &r) != MLA_OK) return 0;
+  DeviceState* st = nullptr;
+  if (current_device(&st) != MLA_OK) return 0;
+  return workspace_for(r, st->sm_count, nullptr, nullptr);
+}
+
+int mla_fa_query_plan(const mla_fa_args* a, int* units, int* max_splits) {
+  Resolved r;
+  int rc = validate(a, &r);
+  if (rc != MLA_OK) return rc;
+  DeviceState* st = nullptr;
+  rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  workspace_for(r, st->sm_count, units, max_splits);
+  return MLA_OK;
+}
+
+int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, void* stream) {
+  Resolved r;
+  int rc = validate(a, &r);
+  if (rc != MLA_OK) return rc;
+  DeviceState* st = nullptr;
+  rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  return run_forward(r, st, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int mla_fa_forward(const void* q, const void* kcache, int kcache_type, const void* mask, int n_q,
+                   int n_head, int n_kv, float scale, float* out) {
+  mla_fa_args a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q;
+  a.kcache = kcache;
+  a.kcache_type = kcache_type;
+  a.mask = mask;
+  a.out = out;
+  a.n_seq = 1;
+  a.n_q = n_q;
+  a.n_head = n_head;
+  a.n_kv = n_kv;
+  a.scale = scale;
+  Resolved r;
+  int rc = validate(&a, &r);
+  if (rc != MLA_OK) return rc;
+  DeviceState* st = nullptr;
+  rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    rc = ensure_ws(&st->fwd_ws, &st->fwd_ws_bytes, need);
+  }
+  if (rc != MLA_OK) return rc;
+  return run_forward(r, st, st->fwd_ws, st->fwd_ws_bytes, t_stream);
+}
+
+size_t mla_compact_workspace_size(int n_rows, int n_kv) {
+  if (n_rows < 1 || n_kv < 1) return 0;
+  const int64_t tiles = (n_kv + mla::compact::kTileCells - 1) / mla::compact::kTileCells;
+  const size_t tickets = (((size_t)n_rows * 4) + 255) / 256 * 256;
+  return tickets + (size_t)n_rows * tiles * 8;
+}
+
+int mla_compact_mask_ex(const void* mask, int n_rows, int64_t mask_row_stride, int n_kv,
+                        int32_t* idx_out, int64_t idx_row_stride, int32_t* count_out,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  if (mask == nullptr || idx_out == nullptr || count_out == nullptr) return MLA_ERR_NULL;
+  if (n_rows < 1 || n_kv < 1) return MLA_ERR_SHAPE;
+  if (mask_row_stride == 0) mask_row_stride = n_kv;
+  if (idx_row_stride == 0) idx_row_stride = n_kv;
+  if (mask_row_stride < n_kv || idx_row_stride < n_kv) return MLA_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(mask) & 1) || (reinterpret_cast<uintptr_t>(idx_out) & 3) ||
+      (reinterpret_cast<uintptr_t>(count_out) & 3))
+    return MLA_ERR_ALIGN;
+  const size_t need = mla_compact_workspace_size(n_rows, n_kv);
+  if (workspace == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return MLA_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  int rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  uint32_t epoch;
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    epoch = st->cmp_epoch;
+    st->cmp_epoch = (st->cmp_epoch + 1) & 0x3FFFFFFFu;
+    if (st->cmp_epoch == 0) st->cmp_epoch = 1;
+  }
+  const int tiles = (n_kv + mla::compact::kTileCells - 1) / mla::compact::kTileCells;
+  const size_t tickets_bytes = (((size_t)n_rows * 4) + 255) / 256 * 256;
+  int* tickets = static_cast<int*>(workspace);
+  auto* flags = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) + tickets_bytes);
+  dim3 grid(tiles, n_rows);
+  {
+    ProfScope prof(kKernCompact, static_cast<cudaStream_t>(stream));
+    mla::mla_compact_kernel<<<grid, mla::compact::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint16_t*>(mask), mask_row_stride, n_kv, idx_out, idx_row_stride,
+        count_out, tickets, flags, epoch, kDefaultTimeoutNs);
+  }
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+int mla_compact_mask(const void* mask_row, int n_kv, int32_t* idx_out, int32_t* count_out,
+                     void* stream) {
+  if (mask_row == nullptr || idx_out == nullptr || count_out == nullptr) return MLA_ERR_NULL;
+  if (n_kv < 1) return MLA_ERR_SHAPE;
+  DeviceState* st = nullptr;
+  int rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  const size_t need = mla_compact_workspace_size(1, n_kv);
+  {
+    std::lock_guard<std::mutex> lk(g_mutex);
+    const bool fresh = st->cmp_ws_bytes < need;
+    rc = ensure_ws(&st->cmp_ws, &st->cmp_ws_bytes, need);
+    if (rc == MLA_OK && fresh &&
+        cudaMemset(st->cmp_ws, 0, st->cmp_ws_bytes) != cudaSuccess)
+      rc = MLA_ERR_CUDA;
+  }
+  if (rc != MLA_OK) return rc;
+  return mla_compact_mask_ex(mask_row, 1, n_kv, n_kv, idx_out, n_kv, count_out, st->cmp_ws,
+                             st->cmp_ws_bytes, stream ? stream : t_stream);
+}
+
+int mla_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, mla::g_status, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(mla::g_status, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return v;
+}
+
+int mla_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
+  DeviceState* st = nullptr;
+  int rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  {
+    ProfScope prof(kKernWaitTest, static_cast<cudaStream_t>(stream));
+    mla::mla_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+  }
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int mla_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mutex);
+  for (auto& rec : g_prof_records) {
+    g_prof_pool.push_back(rec.start);
+    g_prof_pool.push_back(rec.stop);
+  }
+  g_prof_records.clear();
+  g_prof_on = true;
+  return MLA_OK;
+}
+
+int mla_profile_end(mla_profile_entry* entries, int max_entries, int* n_entries) {
+  std::lock_guard<std::mutex> lk(g_prof_mutex);
+  g_prof_on = false;
+  int launches[kNumKernels] = {0};
+  double ms[kNumKernels] = {0.0};
+  int rc = MLA_OK;
+  for (auto& rec : g_prof_records) {
+    float t = 0.f;
+    if (cudaEventSynchronize(rec.stop) != cudaSuccess ||
+        cudaEventElapsedTime(&t, rec.start, rec.stop) != cudaSuccess)
+      rc = MLA_ERR_CUDA;
+    launches[rec.kernel] += 1;
+    ms[rec.kernel] += t;
+    g_prof_pool.push_back(rec.start);
+    g_prof_pool.push_back(rec.stop);
+  }
+  g_prof_records.clear();
+  int n = 0;
+  for (int k = 0; k < kNumKernels; ++k) {
+    if (launches[k] == 0) continue;
+    if (entries != nullptr && n < max_entries) {
+      std::memset(&entries[n], 0, sizeof(mla_profile_entry));
+      std::strncpy(entries[n].name, kKernelNames[k], sizeof(entries[n].name) - 1);
+      entries[n].launches = launches[k];
+      entries[n].total_ms = ms[k];
+    }
+    ++n;
+  }
+  if (n_entries) *n_entries = std::min(n, max_entries);
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+// Single-pass compaction of an f16 mask row into the ascending list of kept
+// cell indices (llama.cpp b11413 release note, "single-scan sparse FA index
+// compaction": contiguous segments, a count per segment, one scan over the
+// counts giving each segment its output offset; the list stays ascending).
+//
+// Mapping: a thread's segment is 8 consecutive cells (one 16-byte load); a CTA
+// covers 256 segments = 2048 cells. The scan over segment counts is done in
+// one pass: warp shuffle scan, then a scan of the 8 warp totals, then a
+// decoupled look-back across CTAs. CTAs take their tile in ticket order
+// (atomicAdd), so every tile a CTA waits on belongs to a CTA that is already
+// running; each wait is bounded and reports MLA_ERR_TIMEOUT instead of hanging.
+// Look-back flags carry a per-call epoch, so stale flags from an earlier call
+// read as "not ready" and the flag array needs no clearing between calls.
+#pragma once
+#include <cuda_fp16.h>
+
+#include "mla_common.cuh"
+#include "mla_fwd.cuh"
+
+namespace mla {
+
+namespace compact {
+constexpr int kThreads = 256;
+constexpr int kCellsPerThread = 8;
+constexpr int kTileCells = kThreads * kCellsPerThread;  // 2048
+constexpr uint32_t kStateAggregate = 1;
+constexpr uint32_t kStateInclusive = 2;
+constexpr uint16_t kNegInfBits = 0xFC00;
+}  // namespace compact
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid: (tiles_per_row, n_rows). Workspace per row: one ticket counter (int) and
+// tiles_per_row look-back flags (u64 = tag<<32 | value, tag = epoch*4 + state).
+__global__ void __launch_bounds__(compact::kThreads)
+    mla_compact_kernel(const uint16_t* __restrict__ mask, int64_t mask_row_stride, int n_kv,
+                       int32_t* __restrict__ idx_out, int64_t idx_row_stride,
+                       int32_t* __restrict__ count_out, int* __restrict__ tickets,
+                       unsigned long long* __restrict__ flags, uint32_t epoch,
+                       uint64_t timeout_ns) {
+  using namespace compact;
+  __shared__ int s_tile;
+  __shared__ int s_warp_tot[kThreads / 32];
+  __shared__ int s_excl;
+  const int row = blockIdx.y;
+  const int n_tiles = gridDim.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_tile = atomicAdd(&tickets[row], 1);
+  __syncthreads();
+  const int tile = s_tile;
+  const uint16_t* mrow = mask + (int64_t)row * mask_row_stride;
+  const int64_t cell0 = (int64_t)tile * kTileCells + (int64_t)tid * kCellsPerThread;
+
+  // keep bits of this thread's 8 cells
+  uint32_t keep = 0;
+  if (cell0 + kCellsPerThread <= n_kv && ((reinterpret_cast<uintptr_t>(mrow + cell0) & 15) == 0)) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(mrow + cell0));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      keep |= (uint32_t)((w[h] & 0xFFFFu) != kNegInfBits) << (2 * h);
+      keep |= (uint32_t)((w[h] >> 16) != kNegInfBits) << (2 * h + 1);
+    }
+  } else {
+    for (int k = 0; k < kCellsPerThread; ++k)
+      if (cell0 + k < n_kv && __ldg(mrow + cell0 + k) != kNegInfBits) keep |= 1u << k;
+  }
+  const int cnt = __popc(keep);
+
+  // warp inclusive scan of the segment counts
+  int inc = cnt;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += y;
+  }
+  if (lane == 31) s_warp_tot[warp] = inc;
+  __syncthreads();
+
+  unsigned long long* rflags = flags + (int64_t)row * n_tiles;
+  if (warp == 0) {
+    int wt = lane < kThreads / 32 ? s_warp_tot[lane] : 0;
+    int winc = wt;
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, winc, d);
+      if (lane >= d) winc += y;
+    }
+    if (lane < kThreads / 32) s_warp_tot[lane] = winc - wt;  // exclusive offsets of warps
+    const int agg = __shfl_sync(0xffffffffu, winc, kThreads / 32 - 1);
+    if (lane == 0) {
+      const unsigned long long tag_agg = (unsigned long long)(epoch * 4u + kStateAggregate) << 32;
+      const unsigned long long tag_inc = (unsigned long long)(epoch * 4u + kStateInclusive) << 32;
+      int excl = 0;
+      if (tile == 0) {
+        st_release_u64(&rflags[0], tag_inc | (uint32_t)agg);
+      } else {
+        st_release_u64(&rflags[tile], tag_agg | (uint32_t)agg);
+        bool ok = true;
+        for (int j = tile - 1; j >= 0;) {
+          unsigned long long f = ld_acquire_u64(&rflags[j]);
+          uint32_t tag = (uint32_t)(f >> 32);
+          if (tag == epoch * 4u + kStateInclusive) {
+            excl += (int)(uint32_t)f;
+            break;
+          }
+          if (tag == epoch * 4u + kStateAggregate) {
+            excl += (int)(uint32_t)f;
+            --j;
+            continue;
+          }
+          // not published yet: poll with a wall-time bound
+          uint64_t t0 = globaltimer_ns();
+          while (true) {
+            f = ld_acquire_u64(&rflags[j]);
+            tag = (uint32_t)(f >> 32);
+            if (tag == epoch * 4u + kStateInclusive || tag == epoch * 4u + kStateAggregate) break;
+            if (globaltimer_ns() - t0 > timeout_ns) {
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+        }
+        if (!ok) record_status(kStatusTimeout);
+        st_release_u64(&rflags[tile], tag_inc | (uint32_t)(excl + agg));
+      }
+      s_excl = excl;
+      if (tile == n_tiles - 1) {
+        count_out[row] = excl + agg;
+        tickets[row] = 0;  // every CTA of this row has drawn its ticket
+      }
+    }
+  }
+  __syncthreads();
+
+  // ascending writes: tile offset + warp offset + offset within the warp
+  int pos = s_excl + s_warp_tot[warp] + (inc - cnt);
+  int32_t* orow = idx_out + (int64_t)row * idx_row_stride;
+  for (int k = 0; k < kCellsPerThread; ++k)
+    if (keep & (1u << k)) orow[pos++] = (int32_t)(cell0 + k);
+}
+
+}  // namespace mla

@@ -1,0 +1,105 @@
+"""C ABI checks that need no GPU: the library builds, loads, exports every symbol
+include/mla_fa.h declares, and rejects bad arguments on the host before any
+launch (no kernel runs here)."""
+import ctypes
+
+import pytest
+
+from mla_flash_attention_attn_b200 import binding, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def test_header_declares_the_boundary():
+    names = binding.header_functions()
+    for required in ("mla_fa_forward", "mla_fa_forward_ex", "mla_fa_workspace_size",
+                     "mla_compact_mask", "mla_compact_mask_ex", "mla_get_device_status",
+                     "mla_status_string", "mla_set_stream"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in binding.header_functions() if not hasattr(lib, n)]
+    assert missing == []
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS_NAMES.items():
+        assert binding.mla_status_string(code).startswith(name)
+    assert "unknown" in binding.mla_status_string(12345)
+    assert lib.mla_version() >= 100
+
+
+FAKE = 0x100000  # 16-byte aligned; never dereferenced: validation runs first
+
+
+def base_args(**kw):
+    a = binding.mla_fa_args()
+    a.q = FAKE
+    a.kcache = FAKE
+    a.out = FAKE
+    a.kcache_type = 0
+    a.n_seq, a.n_q, a.n_head, a.n_kv = 1, 1, 16, 256
+    a.scale = 0.07
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def call_ex(lib, a):
+    return lib.mla_fa_forward_ex(ctypes.byref(a), None, 0, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), -1), (dict(kcache=None), -1), (dict(out=None), -1),
+    (dict(kcache_type=7), -3),
+    (dict(n_head=0), -2), (dict(n_head=129), -2), (dict(n_q=0), -2), (dict(n_kv=0), -2),
+    (dict(n_seq=0), -2), (dict(scale=float("inf")), -2), (dict(scale=float("nan")), -2),
+    (dict(q=FAKE + 8), -4), (dict(kcache=FAKE + 4), -4), (dict(out=FAKE + 2), -4),
+    (dict(mask=FAKE + 1), -4), (dict(q_seq_stride=16 * 576 + 4, n_seq=2), -4),
+    (dict(q_seq_stride=100, n_seq=2), -2), (dict(k_seq_stride=10, n_seq=2), -2),
+    (dict(mask=FAKE, mask_row_stride=5), -2), (dict(out_seq_stride=-1), -2),
+    (dict(idx=FAKE), -1),
+])
+def test_argument_errors_are_returned_before_any_launch(lib, kw, expect):
+    assert call_ex(lib, base_args(**kw)) == expect
+    assert lib.mla_fa_workspace_size(ctypes.byref(base_args(**kw))) == 0
+
+
+def test_kv_len_out_of_range_is_rejected(lib):
+    lens = (ctypes.c_int32 * 2)(10, 300)
+    a = base_args(n_seq=2, kv_len=ctypes.cast(lens, ctypes.c_void_p))
+    assert call_ex(lib, a) == -2
+    lens2 = (ctypes.c_int32 * 2)(-1, 3)
+    a2 = base_args(n_seq=2, kv_len=ctypes.cast(lens2, ctypes.c_void_p))
+    assert call_ex(lib, a2) == -2
+
+
+def test_simple_entry_point_validates(lib):
+    assert lib.mla_fa_forward(None, FAKE, 0, None, 1, 16, 256, 0.1, FAKE) == -1
+    assert lib.mla_fa_forward(FAKE, FAKE, 2, None, 1, 16, 256, 0.1, FAKE) == -3
+    assert lib.mla_fa_forward(FAKE, FAKE, 0, None, 1, 200, 256, 0.1, FAKE) == -2
+
+
+def test_compaction_argument_errors(lib):
+    assert lib.mla_compact_mask(None, 10, FAKE, FAKE, None) == -1
+    assert lib.mla_compact_mask(FAKE, 0, FAKE, FAKE, None) == -2
+    assert lib.mla_compact_mask_ex(FAKE + 1, 1, 10, 10, FAKE, 10, FAKE, FAKE, 4096, None) == -4
+    assert lib.mla_compact_mask_ex(FAKE, 1, 10, 10, FAKE, 10, FAKE, None, 0, None) == -5
+    assert lib.mla_compact_mask_ex(FAKE, 1, 5, 10, FAKE, 10, FAKE, FAKE, 4096, None) == -2
+    assert lib.mla_compact_workspace_size(1, 131072) == 256 + 64 * 8
+    assert lib.mla_compact_workspace_size(0, 10) == 0
+
+
+def test_valid_arguments_reach_the_device_check(lib):
+    # With no CUDA device visible a valid call stops at the device check. The fake
+    # pointers must never reach a kernel, so this runs only where no GPU exists.
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers: only meaningful without a GPU")
+    assert call_ex(lib, base_args()) in (-6, -8)

@@ -1,0 +1,272 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Tolerance (f16 paths): max-abs error <= 1e-2 and relative L2 error <= 2e-3 over
+the compared outputs; compaction indices bit-exact. Outputs are pre-filled with
+NaN and followed by a NaN canary region, so an unwritten or overrun cell shows.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from mla_flash_attention_attn_b200 import binding
+from mla_flash_attention_attn_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+REL_L2 = 2e-3
+CANARY = 4096
+
+
+def torch_mod():
+    import torch
+
+    return torch
+
+
+def assert_parity(got, ref, what=""):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, what
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    nref = np.linalg.norm(ref)
+    err = got - ref
+    maxabs = float(np.max(np.abs(err))) if err.size else 0.0
+    if nref == 0.0:
+        assert maxabs == 0.0, f"{what}: expected exact zeros, max |err| {maxabs}"
+        return
+    rel = float(np.linalg.norm(err) / nref)
+    assert maxabs <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {maxabs:.3g} rel-L2 {rel:.3g}"
+
+
+def run_gpu(w, kv_len="auto", mask="auto", k_pad=0):
+    """Run the workload through mla_fa_forward_ex; returns out [n_seq][n_q][n_head][512]."""
+    torch = torch_mod()
+    dev = torch.device("cuda")
+    q = torch.from_numpy(w.q).to(dev)
+    if k_pad:
+        kbuf = torch.zeros((w.n_seq, w.n_kv + k_pad) + w.kcache.shape[2:], dtype=torch.float16,
+                           device=dev)
+        kbuf[:, : w.n_kv] = torch.from_numpy(w.kcache).to(dev)
+        k = kbuf[:, : w.n_kv]
+    else:
+        k = torch.from_numpy(w.kcache).to(dev)
+    m = None
+    if mask == "auto" and w.mask is not None:
+        m = torch.from_numpy(w.mask).to(dev)
+    n_out = w.n_seq * w.n_q * w.n_head * 512
+    big = torch.full((n_out + CANARY,), float("nan"), dtype=torch.float32, device=dev)
+    out = big[:n_out].view(w.n_seq, w.n_q, w.n_head, 512)
+    lens = w.kv_len if kv_len == "auto" else kv_len
+    binding.forward(q, k, w.kv_type, m, w.scale, out=out, kv_len=lens)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    tail = big[n_out:]
+    assert bool(torch.isnan(tail).all()), "write past the end of out"
+    return out.cpu().numpy()
+
+
+def oracle_rows(w, b, rows=None, use_mask=True):
+    return oracle.attention(w.q[b], w.kcache[b], w.kv_type,
+                            w.mask[b] if (use_mask and w.mask is not None) else None,
+                            w.scale, rows=rows)
+
+
+def check_all_rows(w, got, use_mask=True, what=""):
+    for b in range(w.n_seq):
+        ref = oracle_rows(w, b, use_mask=use_mask)
+        assert_parity(got[b].reshape(-1, 512), ref, f"{what} seq {b}")
+
+
+def test_tiny_decode_full_size():
+    w = W.make("tiny_decode")
+    check_all_rows(w, run_gpu(w), what="tiny_decode")
+
+
+def test_v2lite_decode_full_size():
+    w = W.make("v2lite_decode")
+    check_all_rows(w, run_gpu(w), what="v2lite_decode")
+
+
+@pytest.mark.parametrize("with_len", [True, False])
+def test_v3_batched_reduced(with_len):
+    w = W.make("v3_batched_decode", n_kv=2048, len_lo=100, len_hi=2048)
+    got = run_gpu(w, kv_len="auto" if with_len else None)
+    check_all_rows(w, got, what="v3 reduced")
+
+
+def test_prefill_reduced_causal():
+    w = W.make("prefill_chunk", n_q=8, n_head=128, n_kv=640)
+    check_all_rows(w, run_gpu(w), what="prefill reduced")
+
+
+@pytest.mark.parametrize("n_kv", [1, 2, 31, 63, 65, 127, 129, 255, 257, 1000])
+def test_ragged_kv_lengths(n_kv):
+    rng = np.random.default_rng(n_kv)
+    w = W.make("tiny_decode", n_kv=n_kv)
+    keep = rng.random(n_kv) < 0.8
+    keep[rng.integers(0, n_kv)] = True
+    w.mask[0, 0] = np.where(keep, rng.standard_normal(n_kv).astype(np.float16), -np.inf)
+    check_all_rows(w, run_gpu(w), what=f"n_kv={n_kv}")
+
+
+@pytest.mark.parametrize("n_head,n_q", [(1, 1), (7, 3), (16, 9), (64, 2), (100, 3), (128, 2)])
+def test_head_counts_and_row_groups(n_head, n_q):
+    rng = np.random.default_rng(n_head * 10 + n_q)
+    n_kv = 300
+    w = W.make("prefill_chunk", n_q=n_q, n_head=n_head, n_kv=n_kv)
+    w.mask[0] = np.where(rng.random((n_q, n_kv)) < 0.7, np.float16(0), np.float16(-np.inf))
+    w.mask[0, :, 0] = 0
+    check_all_rows(w, run_gpu(w), what=f"H={n_head} n_q={n_q}")
+
+
+def test_fully_masked_rows_give_zero():
+    w = W.make("prefill_chunk", n_q=4, n_head=16, n_kv=200)
+    w.mask[0, 1, :] = -np.inf
+    w.mask[0, 3, :] = -np.inf
+    got = run_gpu(w)
+    assert np.all(got[0, 1] == 0) and np.all(got[0, 3] == 0)
+    check_all_rows(w, got, what="fully masked")
+
+
+def test_no_mask():
+    w = W.make("tiny_decode", n_kv=333)
+    check_all_rows(w, run_gpu(w, mask=None), use_mask=False, what="no mask")
+
+
+def test_large_finite_mask_values_and_shift():
+    w = W.make("tiny_decode", n_kv=400)
+    rng = np.random.default_rng(3)
+    w.mask[0, 0] = (rng.standard_normal(400) * 30).astype(np.float16)
+    check_all_rows(w, run_gpu(w), what="large mask")
+
+
+def test_zero_length_sequence_and_strided_cache():
+    w = W.make("v3_batched_decode", n_seq=3, n_head=16, n_kv=700, len_lo=0, len_hi=700)
+    w.kv_len[:] = [0, 1, 700]
+    keep = np.arange(700)[None, :] < w.kv_len[:, None]
+    w.mask[:, 0, :] = np.where(keep, np.float16(0), np.float16(-np.inf))
+    got = run_gpu(w, k_pad=64)
+    assert np.all(got[0] == 0)
+    check_all_rows(w, got, what="kv_len 0/1/700")
+
+
+def test_deterministic_repeat():
+    w = W.make("v3_batched_decode", n_seq=2, n_kv=1500, len_lo=900, len_hi=1500)
+    a = run_gpu(w)
+    b = run_gpu(w)
+    assert np.array_equal(a, b)
+
+
+def test_split_plan_is_exercised():
+    torch = torch_mod()
+    w = W.make("v3_batched_decode", n_kv=2048, len_lo=1500, len_hi=2048)
+    q = torch.from_numpy(w.q).cuda()
+    k = torch.from_numpy(w.kcache).cuda()
+    out = torch.empty(w.q.shape[:3] + (512,), dtype=torch.float32, device="cuda")
+    args, keep = binding.make_args(q, k, 0, None, out, w.scale, kv_len=w.kv_len)
+    units, splits = binding.mla_fa_query_plan(args)
+    assert splits > 1 and units >= w.n_seq
+    wp = W.make("prefill_chunk", n_q=64, n_head=128, n_kv=256)
+    qp = torch.from_numpy(wp.q).cuda()
+    kp = torch.from_numpy(wp.kcache).cuda()
+    outp = torch.empty(wp.q.shape[:3] + (512,), dtype=torch.float32, device="cuda")
+    args2, keep2 = binding.make_args(qp, kp, 0, None, outp, wp.scale)
+    units2, splits2 = binding.mla_fa_query_plan(args2)
+    assert splits2 == 1 and units2 == 64
+
+
+def test_simple_entry_point_matches_oracle():
+    torch = torch_mod()
+    w = W.make("v2lite_decode", n_kv=1111)
+    q = torch.from_numpy(w.q[0]).cuda()
+    k = torch.from_numpy(w.kcache[0]).cuda()
+    m = torch.from_numpy(w.mask[0]).cuda()
+    out = torch.full((1, 16, 512), float("nan"), dtype=torch.float32, device="cuda")
+    binding.mla_fa_forward(q, k, 0, m, w.scale, out)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    assert_parity(out.cpu().numpy().reshape(-1, 512), oracle_rows(w, 0), "mla_fa_forward")
+
+
+# ------------------------------------------------------------------ full sizes, sampled rows
+def test_v3_batched_full_size_sampled_rows():
+    w = W.make("v3_batched_decode")
+    got = run_gpu(w)
+    rng = np.random.default_rng(0)
+    for b in range(w.n_seq):
+        rows = np.sort(rng.choice(w.n_q * w.n_head, size=3, replace=False)).astype(np.int32)
+        ref = oracle_rows(w, b, rows=rows)
+        assert_parity(got[b].reshape(-1, 512)[rows], ref, f"v3 full seq {b}")
+
+
+def test_prefill_full_size_sampled_rows():
+    w = W.make("prefill_chunk")
+    got = run_gpu(w)
+    H = w.n_head
+    rows = np.array([t * H + h for t in (0, 1, 255, 510, 511) for h in (0, 77, 127)], np.int32)
+    ref = oracle_rows(w, 0, rows=rows)
+    assert_parity(got[0].reshape(-1, 512)[rows], ref, "prefill full")
+
+
+# ------------------------------------------------------------------ run-time error path
+def test_bounded_wait_timeout_is_reported_and_device_stays_usable():
+    w = W.make("tiny_decode", n_kv=64)
+    binding.mla_debug_wait_timeout(1_000_000)  # 1 ms on a barrier nothing signals
+    assert binding.mla_get_device_status() == -7
+    assert binding.mla_get_device_status() == 0  # reading clears it
+    check_all_rows(w, run_gpu(w), what="after timeout")
+
+
+# ------------------------------------------------------------------ compaction
+def compact_gpu(row_np, lib_ws=True):
+    torch = torch_mod()
+    n = row_np.shape[0]
+    m = torch.from_numpy(row_np).cuda()
+    idx = torch.full((n + CANARY,), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    if lib_ws:
+        binding.mla_compact_mask(m, idx, cnt)
+    else:
+        ws = torch.zeros(binding.mla_compact_workspace_size(1, n), dtype=torch.uint8, device="cuda")
+        binding.mla_compact_mask_ex(m.view(1, n), idx[:n].view(1, n), cnt, ws)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    c = int(cnt.item())
+    idx_h = idx.cpu().numpy()
+    assert np.all(idx_h[c:] == -1), "write beyond the kept count"
+    return idx_h[:c]
+
+
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 2047, 2048, 2049, 5000, 65537])
+@pytest.mark.parametrize("p_keep", [0.0, 0.1, 0.5, 1.0])
+def test_compaction_bit_exact(n, p_keep):
+    rng = np.random.default_rng(n + int(p_keep * 100))
+    keep = rng.random(n) < p_keep
+    row = np.where(keep, rng.standard_normal(n), -np.inf).astype(np.float16)
+    row[rng.random(n) < 0.01] = np.float16(-65504.0)  # finite large negatives are kept
+    assert np.array_equal(compact_gpu(row), oracle.compact(row))
+
+
+def test_compaction_full_size_block_pattern_and_repeats():
+    w = W.make("sparse_q8_decode")
+    row = w.mask[0, 0]
+    ref = oracle.compact(row)
+    assert len(ref) == 16384
+    for _ in range(3):  # repeated calls reuse the workspace (epoch-tagged flags)
+        assert np.array_equal(compact_gpu(row), ref)
+    assert np.array_equal(compact_gpu(row, lib_ws=False), ref)
+
+
+def test_compaction_unaligned_row_start():
+    torch = torch_mod()
+    rng = np.random.default_rng(5)
+    n = 3001
+    base = np.where(rng.random(n + 1) < 0.4, np.float16(0), np.float16(-np.inf)).astype(np.float16)
+    m = torch.from_numpy(base).cuda()[1:]  # 2-byte aligned only
+    idx = torch.full((n,), -1, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    binding.mla_compact_mask(m, idx, cnt)
+    torch.cuda.synchronize()
+    c = int(cnt.item())
+    assert np.array_equal(idx.cpu().numpy()[:c], oracle.compact(base[1:]))
