@@ -163,13 +163,23 @@ class Step:
         self.mask = torch.from_numpy(w.mask).to(dev) if w.mask is not None else None
         self.out = torch.empty(w.q.shape[:3] + (512,), dtype=torch.float32, device=dev)
         self.kv_len = [int(x) for x in w.kv_len]
+        self.idx = self.cnt = None
+        if w.sparse:
+            # the step starts from the mask row: compaction, then attention over the kept rows
+            self.idx = torch.empty((w.n_seq, w.n_kv), dtype=torch.int32, device=dev)
+            self.cnt = torch.zeros((w.n_seq,), dtype=torch.int32, device=dev)
+            self.cws = torch.zeros(binding.mla_compact_workspace_size(w.n_seq, w.n_kv),
+                                   dtype=torch.uint8, device=dev)
         self.args, self._keep = binding.make_args(self.q, self.k, w.kv_type, self.mask, self.out,
-                                                  w.scale, kv_len=self.kv_len)
+                                                  w.scale, kv_len=self.kv_len, idx=self.idx,
+                                                  idx_count=self.cnt)
         need = binding.mla_fa_workspace_size(self.args)
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
         self.ws_used = need > 0
 
     def run(self, stream=None):
+        if self.idx is not None:
+            self.b.mla_compact_mask_ex(self.mask[:, 0, :], self.idx, self.cnt, self.cws, stream)
         self.b.mla_fa_forward_ex(self.args, self.ws if self.ws_used else None, stream)
 
 
@@ -226,7 +236,7 @@ def gpu_arm(args, rank, world):
     ms_per_step = total_ms / args.steps
     kv_gbs = acc["kv_bytes"] * world / (ms_per_step * 1e-3) / 1e9
     peaks, peak_kind = load_peaks()
-    dom = "mla_fwd_f16"
+    dom = max((k for k in prof if k.startswith("mla_fwd")), key=lambda k: prof[k][1])
     launches, dom_ms = prof.get(dom, (0, 0.0))
     dom_avg_ms = dom_ms / max(launches, 1)
     tensor_bound = acc["flops"] / acc["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)

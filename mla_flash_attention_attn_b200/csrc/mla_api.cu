@@ -97,9 +97,17 @@ int current_device(DeviceState** st) {
 }
 
 // ---------------------------------------------------------------- profiling
-enum KernelId { kKernFwdF16 = 0, kKernCombine = 1, kKernCompact = 2, kKernWaitTest = 3, kNumKernels };
-const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_combine", "mla_compact",
-                                               "mla_wait_timeout"};
+enum KernelId {
+  kKernFwdF16 = 0,
+  kKernFwdGather = 1,
+  kKernFwdQ8 = 2,
+  kKernCombine = 3,
+  kKernCompact = 4,
+  kKernWaitTest = 5,
+  kNumKernels
+};
+const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_fwd_gather_f16", "mla_fwd_q8_0",
+                                               "mla_combine", "mla_compact", "mla_wait_timeout"};
 struct ProfRecord {
   cudaEvent_t start, stop;
   int kernel;
@@ -177,7 +185,9 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (a->kv_len != nullptr)
     for (int b = 0; b < a->n_seq; ++b)
       if (a->kv_len[b] < 0 || a->kv_len[b] > a->n_kv) return MLA_ERR_SHAPE;
-  if (a->kcache_type != MLA_KV_F16 || a->idx != nullptr) return MLA_ERR_UNSUPPORTED;
+  if (a->idx != nullptr && ((reinterpret_cast<uintptr_t>(a->idx) & 3) ||
+                            (reinterpret_cast<uintptr_t>(a->idx_count) & 3)))
+    return MLA_ERR_ALIGN;
   return MLA_OK;
 }
 
@@ -196,7 +206,9 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
   int64_t sum_tiles = 0;
   std::vector<int> tiles(n);
   for (int b = 0; b < n; ++b) {
-    const int len = a.kv_len ? a.kv_len[s0 + b] : a.n_kv;
+    // sparse: the kept count is only known on the device; plan for the most it can be
+    int len = a.kv_len ? a.kv_len[s0 + b] : a.n_kv;
+    if (a.idx != nullptr) len = (int)std::min<int64_t>(len, r.idx_ss);
     plan->kv_len[b] = len;
     tiles[b] = (len + mla::kTileKeys - 1) / mla::kTileKeys;
     sum_tiles += tiles[b];
@@ -262,18 +274,31 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
   if (need > 0 && (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)))
     return MLA_ERR_WORKSPACE;
+  const int mode = a.kcache_type == MLA_KV_Q8_0 ? mla::kModeQ8
+                   : (a.idx != nullptr ? mla::kModeGatherF16 : mla::kModeTma);
   CUtensorMap tm_q, tm_k, tm_v;
   const uint64_t row_bytes = MLA_DK * 2;
   int rc = make_map(&tm_q, a.q, MLA_DK, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
-  if (rc == MLA_OK)
+  if (rc == MLA_OK && mode == mla::kModeTma) {
     rc = make_map(&tm_k, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
                   64, 64);
-  if (rc == MLA_OK)
-    rc = make_map(&tm_v, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
-                  64, 32);
+    if (rc == MLA_OK)
+      rc = make_map(&tm_v, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes,
+                    (uint64_t)r.k_ss * row_bytes, 64, 32);
+  } else {
+    tm_k = tm_q;  // unused by the gather / dequant modes
+    tm_v = tm_q;
+  }
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
-    if (cudaFuncSetAttribute(mla::mla_fwd_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeTma>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mla::fwd::kSmemAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeGatherF16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mla::fwd::kSmemAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeQ8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                              mla::fwd::kSmemAlloc) != cudaSuccess)
       return MLA_ERR_CUDA;
     st->fwd_attr_set = true;
@@ -287,6 +312,12 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   p.scale_log2 = a.scale * mla::kLog2e;
   p.mask_vec_ok = (a.mask != nullptr && aligned16(a.mask) && (r.m_ss % 8) == 0 && (r.m_rs % 8) == 0);
   p.timeout_ns = kDefaultTimeoutNs;
+  p.kcache = static_cast<const uint8_t*>(a.kcache);
+  p.k_seq_stride = r.k_ss;
+  p.n_kv = a.n_kv;
+  p.idx = a.idx;
+  p.idx_count = a.idx_count;
+  p.idx_seq_stride = r.idx_ss;
   Plan plan;
   for (int s0 = 0; s0 < a.n_seq; s0 += mla::kPlanMaxSeq) {
     const int n = std::min(mla::kPlanMaxSeq, a.n_seq - s0);
@@ -296,10 +327,21 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
                                                 (size_t)slots * mla::kRowsPerGroup * mla::kDV * 4)
                      : nullptr;
     dim3 grid(2 * plan.total_units);
-    {
+    if (mode == mla::kModeTma) {
       ProfScope prof(kKernFwdF16, stream);
-      mla::mla_fwd_f16_kernel<<<grid, mla::fwd::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-          tm_q, tm_k, tm_v, plan, p);
+      mla::mla_fwd_kernel<mla::kModeTma>
+          <<<grid, mla::FwdCfg<mla::kModeTma>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
+              tm_q, tm_k, tm_v, plan, p);
+    } else if (mode == mla::kModeGatherF16) {
+      ProfScope prof(kKernFwdGather, stream);
+      mla::mla_fwd_kernel<mla::kModeGatherF16>
+          <<<grid, mla::FwdCfg<mla::kModeGatherF16>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
+              tm_q, tm_k, tm_v, plan, p);
+    } else {
+      ProfScope prof(kKernFwdQ8, stream);
+      mla::mla_fwd_kernel<mla::kModeQ8>
+          <<<grid, mla::FwdCfg<mla::kModeQ8>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
+              tm_q, tm_k, tm_v, plan, p);
     }
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     if (slots > 0) {

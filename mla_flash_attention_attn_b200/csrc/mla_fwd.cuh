@@ -53,6 +53,21 @@ struct MlaFwdParams {
   float scale_log2;          // scale * log2(e)
   int mask_vec_ok;           // mask rows allow 16-byte loads
   uint64_t timeout_ns;
+  // cache rows read by the gather / dequant producer (modes other than TMA)
+  const uint8_t* kcache;     // row (b, j) at (b*k_seq_stride + j) * row_bytes
+  int64_t k_seq_stride;      // rows
+  int n_kv;
+  // sparse: sequence b attends to rows idx[b*idx_seq_stride + i], i < idx_count[b]
+  const int32_t* idx;
+  const int32_t* idx_count;
+  int64_t idx_seq_stride;
+};
+
+// How K/V tiles reach shared memory.
+enum FwdMode {
+  kModeTma = 0,       // f16 cache, contiguous keys: TMA tensor loads
+  kModeGatherF16 = 1, // f16 cache, rows chosen by an index list: warp-group loads
+  kModeQ8 = 2         // q8_0 cache (dense or indexed): warp-group loads + dequant to f16
 };
 
 namespace fwd {
@@ -104,12 +119,40 @@ __device__ __forceinline__ void decode_unit(const Plan& plan, int unit, int& b, 
   s = local - g * ns;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
-    mla_fwd_f16_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Plan plan,
-                       const __grid_constant__ MlaFwdParams p) {
+template <int kMode>
+struct FwdCfg {
+  static constexpr bool kManual = kMode != kModeTma;
+  static constexpr int kThreads = kManual ? 384 : 256;  // + 4 producer warps when manual
+  static constexpr int kRowBytes = kMode == kModeQ8 ? kQ8RowBytes : 2 * kDK;
+};
+
+// q8_0 block (f16 d, then 32 int8) -> 32 f16 values d*q (one rounding each), as
+// 16 half2 words. An int8 q is biased to u = q + 128 and placed in the low
+// mantissa bits of 1024.0 (0x6400), giving exactly 1024 + u; subtracting 1152
+// leaves q exactly, and one f16 multiply by d rounds d*q once.
+__device__ __forceinline__ void dequant_q8_block(const uint8_t* blk, uint32_t (&h)[16]) {
+  const uint16_t dbits = __ldg(reinterpret_cast<const unsigned short*>(blk));
+  const __half2 d2 = __half2half2(__ushort_as_half(dbits));
+  const __half2 bias = __float2half2_rn(1152.f);
+  const unsigned short* qw = reinterpret_cast<const unsigned short*>(blk + 2);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t u = (uint32_t)__ldg(qw + k) ^ 0x8080u;
+    const uint32_t w = __byte_perm(u, 0x64646464u, 0x4140);
+    __half2 v = *reinterpret_cast<const __half2*>(&w);
+    v = __hmul2(__hsub2(v, bias), d2);
+    h[k] = *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+template <int kMode>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThreads, 1)
+    mla_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Plan plan,
+                   const __grid_constant__ MlaFwdParams p) {
   using namespace fwd;
+  constexpr bool kManual = FwdCfg<kMode>::kManual;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -131,7 +174,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
   decode_unit(plan, blockIdx.x >> 1, b, g, s);
   const int b_abs = plan.seq_offset + b;
   const int n_split = plan.n_split[b];
-  const int len = plan.kv_len[b];
+  const bool sparse = p.idx != nullptr;
+  const int len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
   const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
   const int tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
   const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
@@ -142,7 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
   // ---- setup: barriers, TMEM
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bars.ring_full[i], 1);
+      mbar_init(&bars.ring_full[i], kManual ? 8 : 1);
       mbar_init(&bars.ring_empty[i], 1);
     }
     mbar_init(&bars.q_full, 1);
@@ -155,8 +199,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+    if (!kManual) {
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+    }
   }
   if (warp == 1) tmem_alloc_2sm(tmem_slot, kTmemCols);
   tc_fence_before();
@@ -165,14 +211,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   bool failed = false;
 
+  if constexpr (kManual) {
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;");
+  }
   if (warp == 0) {
-    // ================= producer: TMA loads of Q, then K and V chunks
+    // ================= producer: TMA loads of Q, then (TMA mode) K and V chunks
     if (n_tiles > 0 && elect_one()) {
       const uint32_t q_full_l = mapa_shared(smem_u32(&bars.q_full), 0);
       if (rank == 0) mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
       for (int c = 0; c < 9; ++c)
         tma_load_3d_2sm(sQ + c * kChunkBytes, &tm_q, q_full_l, 64 * c,
                         row0 + kRowsPerCta * (int)rank, b_abs);
+    }
+    if (!kManual && n_tiles > 0 && elect_one()) {
       int stage = 0;
       uint32_t ephase = 0;
       auto acquire = [&]() {
@@ -241,7 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
         tc_fence_after();
         for (int kb = 0; kb < 4; ++kb)
           for (int nb = 0; nb < 2; ++nb) {
-            wait_or_fail(&bars.ring_full[stage], fphase, false);
+            wait_or_fail(&bars.ring_full[stage], fphase, kManual);
             tc_fence_after();
             for (int k2 = 0; k2 < 2; ++k2) {
               const int kk = 2 * kb + k2;
@@ -258,7 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
       for (int i = 0; i < n_tiles; ++i) {
         const uint32_t d_s = tmem + (i & 1) * 64;
         for (int c = 0; c < 9; ++c) {
-          wait_or_fail(&bars.ring_full[stage], fphase, false);
+          wait_or_fail(&bars.ring_full[stage], fphase, kManual);
           tc_fence_after();
           for (int kk = 0; kk < 4; ++kk) {
             uint64_t ad = smem_desc_sw128(q_addr + c * kChunkBytes + kk * 32, 16, 1024);
@@ -274,8 +325,100 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
       pv(n_tiles - 1);
     }
     __syncwarp();
+  } else if (warp >= 8) {
+    // ================= gather / dequant producer (manual modes): 4 warps, 128 threads
+    if constexpr (kManual) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 128;");
+      const int pt = threadIdx.x - 256;
+      const int64_t seq_row0 = (int64_t)b_abs * p.k_seq_stride;
+      const int32_t* idx_row = sparse ? p.idx + (int64_t)b_abs * p.idx_seq_stride : nullptr;
+      // cache row of key position `pos` in this unit's selection, or -1 (zero fill)
+      auto resolve = [&](int pos) -> int {
+        if (pos >= len) return -1;
+        if (!sparse) return pos < p.n_kv ? pos : -1;
+        const int key = __ldg(idx_row + pos);
+        if (key < 0 || key >= p.n_kv) {
+          record_status(kStatusIndex);
+          return -1;
+        }
+        return key;
+      };
+      // 32 consecutive values of a cache row, as f16, into 4 swizzled 16-byte chunks
+      auto fill32 = [&](uint8_t* row_dst, int row_in_atom, int key, int col32, int chunk0) {
+        uint32_t h[16];
+        if (key < 0) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) h[k] = 0u;
+        } else if constexpr (kMode == kModeQ8) {
+          const uint8_t* rowp = p.kcache + (seq_row0 + key) * kQ8RowBytes;
+          dequant_q8_block(rowp + col32 * 34, h);
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.kcache + (seq_row0 + key) * (2 * kDK) + col32 * 64);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 v = __ldg(src + k);
+            h[4 * k] = v.x; h[4 * k + 1] = v.y; h[4 * k + 2] = v.z; h[4 * k + 3] = v.w;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(row_dst + (((chunk0 + k) ^ (row_in_atom & 7)) << 4)) =
+              make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3]);
+      };
+      int stage = 0;
+      uint32_t ephase = 0;
+      auto acquire = [&]() {
+        bool ok = failed ? true : mbar_wait(&bars.ring_empty[stage], ephase ^ 1, to);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && !failed) {
+          failed = true;
+          if (lane == 0) record_status(kStatusTimeout);
+        }
+      };
+      auto publish = [&]() {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars.ring_full[stage]), 0));
+        if (++stage == kStages) { stage = 0; ephase ^= 1; }
+      };
+      // K chunk: 64 keys (this CTA's half of the tile) x 64 columns = 2 blocks of 32
+      auto issue_k = [&](int i) {
+        const int kl = pt >> 1, half = pt & 1;
+        const int key = resolve((tile_begin + i) * kTileKeys + 64 * (int)rank + kl);
+        for (int c = 0; c < 9; ++c) {
+          acquire();
+          fill32(sRing + stage * kChunkBytes + kl * 128, kl, key, 2 * c + half, 4 * half);
+          publish();
+        }
+      };
+      // V chunk: 32 keys x this CTA's 128 value columns (two 64-column boxes)
+      auto issue_v = [&](int j) {
+        const int kl = pt >> 2, q4 = pt & 3;
+        const int box = q4 >> 1, half = q4 & 1;
+        const int kbase = (tile_begin + j) * kTileKeys;
+        for (int kb = 0; kb < 4; ++kb) {
+          const int key = resolve(kbase + 32 * kb + kl);
+          for (int nb = 0; nb < 2; ++nb) {
+            acquire();
+            const int col32 = 8 * nb + 4 * (int)rank + q4;
+            fill32(sRing + stage * kChunkBytes + box * 4096 + kl * 128, kl, key, col32, 4 * half);
+            publish();
+          }
+        }
+      };
+      if (n_tiles > 0) {
+        issue_k(0);
+        for (int i = 1; i < n_tiles; ++i) {
+          issue_k(i);
+          issue_v(i - 1);
+        }
+        issue_v(n_tiles - 1);
+      }
+    }
   } else if (warp >= 4) {
     // ================= softmax / correction / epilogue warpgroup
+    if constexpr (kManual) asm volatile("setmaxnreg.inc.sync.aligned.u32 256;");
     const int L = threadIdx.x - 128;          // TMEM lane
     const int r = L & 63;                     // row within this CTA
     const int kh = L >> 6;                    // which 64 keys of a tile this lane holds
@@ -317,7 +460,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd::kThreads, 1)
       // scores in log2 units; cells beyond the unit's keys are dropped
       float x[64];
       const bool full_range = key0 + 64 <= key_end;
-      if (mrow != nullptr && full_range && p.mask_vec_ok) {
+      if (kManual && sparse) {
+        const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const int pos = key0 + j;
+          float mv = 0.f;
+          bool ok = pos < key_end;
+          if (ok) {
+            const int cell = __ldg(ix + pos);
+            ok = cell >= 0 && cell < p.n_kv;
+            if (ok && mrow != nullptr) mv = __half2float(__ushort_as_half(__ldg(mrow + cell)));
+          }
+          x[j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
+        }
+      } else if (mrow != nullptr && full_range && p.mask_vec_ok) {
         const uint4* mv = reinterpret_cast<const uint4*>(mrow + key0);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {

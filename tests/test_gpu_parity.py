@@ -270,3 +270,125 @@ def test_compaction_unaligned_row_start():
     torch.cuda.synchronize()
     c = int(cnt.item())
     assert np.array_equal(idx.cpu().numpy()[:c], oracle.compact(base[1:]))
+
+
+# ------------------------------------------------------------------ q8_0 cache and sparse indices
+def q8_f16_rounded(rows_u8):
+    """q8_0 rows -> f16 cache with each value d*q rounded once to f16 (the product of an
+    f16 scale and an 8-bit integer is exact in float32, so this is RN_f16(d*q))."""
+    n = rows_u8.shape[0]
+    blk = rows_u8.reshape(n, 18, 34)
+    d = blk[:, :, 0:2].copy().view(np.float16).astype(np.float32)  # [n][18][1]
+    q = blk[:, :, 2:].view(np.int8).astype(np.float32)              # [n][18][32]
+    return (d * q).astype(np.float16).reshape(n, 576)
+
+
+def run_sparse_gpu(w, idx_rows=None, counts=None, use_gpu_compaction=True):
+    """Compaction (GPU) then attention over the kept indices; returns (out, idx, count)."""
+    torch = torch_mod()
+    dev = torch.device("cuda")
+    q = torch.from_numpy(w.q).to(dev)
+    k = torch.from_numpy(w.kcache).to(dev)
+    m = torch.from_numpy(w.mask).to(dev)
+    idx = torch.full((w.n_seq, w.n_kv), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros((w.n_seq,), dtype=torch.int32, device=dev)
+    if use_gpu_compaction:
+        ws = torch.zeros(binding.mla_compact_workspace_size(w.n_seq, w.n_kv), dtype=torch.uint8,
+                         device=dev)
+        binding.mla_compact_mask_ex(m[:, 0, :], idx, cnt, ws)
+    else:
+        for b in range(w.n_seq):
+            idx[b, : len(idx_rows[b])] = torch.from_numpy(idx_rows[b]).to(dev)
+        cnt.copy_(torch.tensor(counts, dtype=torch.int32))
+    n_out = w.n_seq * w.n_q * w.n_head * 512
+    big = torch.full((n_out + CANARY,), float("nan"), dtype=torch.float32, device=dev)
+    out = big[:n_out].view(w.n_seq, w.n_q, w.n_head, 512)
+    binding.forward(q, k, w.kv_type, m, w.scale, out=out, idx=idx, idx_count=cnt)
+    torch.cuda.synchronize()
+    status = binding.mla_get_device_status()
+    assert bool(torch.isnan(big[n_out:]).all())
+    return out.cpu().numpy(), idx.cpu().numpy(), cnt.cpu().numpy(), status
+
+
+def test_q8_0_dense_matches_oracle_on_same_dequantised_values():
+    w = W.make("sparse_q8_decode", n_kv=4096, n_head=128, tail_blocks=4)
+    w.sparse = False
+    got = run_gpu(w)
+    kf16 = q8_f16_rounded(w.kcache[0])
+    ref_same = oracle.attention(w.q[0], kf16, oracle.KV_F16, w.mask[0], w.scale)
+    assert_parity(got[0].reshape(-1, 512), ref_same, "q8_0 vs oracle(f16-rounded d*q)")
+    ref_exact = oracle_rows(w, 0)  # exact d*q in fp64
+    assert_parity(got[0].reshape(-1, 512), ref_exact, "q8_0 vs oracle(exact d*q)")
+
+
+@pytest.mark.parametrize("n_head", [16, 128])
+def test_q8_0_ragged_no_mask(n_head):
+    rng = np.random.default_rng(n_head)
+    w = W.make("sparse_q8_decode", n_kv=1000, n_head=n_head, block=8, tail_blocks=2)
+    w.sparse = False
+    w.mask = None
+    got = run_gpu(w, mask=None)
+    ref = oracle.attention(w.q[0], q8_f16_rounded(w.kcache[0]), oracle.KV_F16, None, w.scale)
+    assert_parity(got[0].reshape(-1, 512), ref, f"q8_0 H={n_head} no mask")
+
+
+def test_sparse_f16_gather_equals_dense_masked():
+    w = W.make("v2lite_decode", n_kv=3000, n_head=128, n_pad=0)
+    rng = np.random.default_rng(9)
+    keep = rng.random(3000) < 0.15
+    keep[-7:] = True
+    w.mask[0, 0] = np.where(keep, np.float16(0), np.float16(-np.inf))
+    w.sparse = True
+    got, idx, cnt, status = run_sparse_gpu(w)
+    assert status == 0
+    assert cnt[0] == keep.sum() and np.array_equal(idx[0, : cnt[0]], np.nonzero(keep)[0])
+    ref = oracle_rows(w, 0)  # dense masked path
+    assert_parity(got[0].reshape(-1, 512), ref, "sparse f16 gather")
+
+
+def test_sparse_q8_reduced_chain():
+    w = W.make("sparse_q8_decode", n_kv=16384, n_head=128, tail_blocks=4)
+    got, idx, cnt, status = run_sparse_gpu(w)
+    assert status == 0
+    ref_idx = oracle.compact(w.mask[0, 0])
+    assert cnt[0] == len(ref_idx) and np.array_equal(idx[0, : cnt[0]], ref_idx)
+    kf16 = q8_f16_rounded(w.kcache[0])
+    ref = oracle.attention(w.q[0], kf16, oracle.KV_F16, w.mask[0], w.scale, idx=ref_idx)
+    assert_parity(got[0].reshape(-1, 512), ref, "sparse q8_0 chain")
+
+
+def test_sparse_q8_full_size_sampled_rows():
+    w = W.make("sparse_q8_decode")
+    got, idx, cnt, status = run_sparse_gpu(w)
+    assert status == 0 and cnt[0] == 16384
+    rows = np.array([0, 1, 31, 64, 100, 127], np.int32)
+    ref_idx = oracle.compact(w.mask[0, 0])
+    ref = oracle.attention(w.q[0], w.kcache[0], oracle.KV_Q8_0, w.mask[0], w.scale, rows=rows,
+                           idx=ref_idx)
+    assert_parity(got[0].reshape(-1, 512)[rows], ref, "sparse q8_0 full")
+
+
+def test_sparse_count_zero_and_partial_lists():
+    w = W.make("v3_batched_decode", n_seq=3, n_head=16, n_kv=900, len_lo=900, len_hi=900)
+    w.mask[:] = 0
+    rng = np.random.default_rng(4)
+    lists = [np.array([], np.int32), np.sort(rng.choice(900, 50, replace=False)).astype(np.int32),
+             np.arange(900, dtype=np.int32)]
+    counts = [0, 50, 900]
+    got, _, _, status = run_sparse_gpu(w, idx_rows=lists, counts=counts, use_gpu_compaction=False)
+    assert status == 0
+    assert np.all(got[0] == 0)
+    for b in (1, 2):
+        ref = oracle.attention(w.q[b], w.kcache[b], 0, w.mask[b], w.scale, idx=lists[b])
+        assert_parity(got[b].reshape(-1, 512), ref, f"sparse list {b}")
+
+
+def test_sparse_out_of_range_index_is_reported_not_read():
+    w = W.make("tiny_decode", n_kv=300)
+    w.mask[:] = 0
+    lst = np.array([3, 10, 299, 300 + 5, 17], np.int32)  # one index beyond n_kv
+    got, _, _, status = run_sparse_gpu(w, idx_rows=[lst], counts=[5], use_gpu_compaction=False)
+    assert status == -9  # MLA_ERR_INDEX recorded; the bad row is treated as dropped
+    ok = np.array([3, 10, 299, 17], np.int32)
+    ref = oracle.attention(w.q[0], w.kcache[0], 0, w.mask[0], w.scale, idx=ok)
+    assert_parity(got[0].reshape(-1, 512), ref, "bad index dropped")
