@@ -132,6 +132,33 @@ size_t mla_fa_workspace_size(const mla_fa_args* a);
  * log-sum-exp combine before the call's last kernel ends. */
 int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, void* stream);
 
+/* Forward pass for callers that cannot allocate device memory. The paper has no
+ * counterpart to this entry point; it exists for users of this library.
+ *
+ * Some callers can't let a library call cudaMalloc: an inference engine that
+ * reserves almost all of the GPU's memory for its KV cache at start-up (so a
+ * later cudaMalloc fails or overcommits), a framework whose own allocator must
+ * account for every byte, or a decode loop that cannot afford the device-wide
+ * synchronisation cudaMalloc and cudaFree may cause. This call takes the same
+ * arguments and gives the same results as mla_fa_forward_ex, but allocates
+ * nothing: its split-KV partials go to a scratch array of
+ * MLA_NOALLOC_SCRATCH_BYTES that the library declares in static device memory.
+ * Every GPU that loads the library holds that array until the process exits.
+ * The caller still passes q, kcache, mask and out.
+ *
+ * - If the pass needs more scratch than MLA_NOALLOC_SCRATCH_BYTES
+ *   (mla_fa_workspace_size(a) > MLA_NOALLOC_SCRATCH_BYTES), it returns
+ *   MLA_ERR_WORKSPACE before launching anything.
+ * - The first call on a device looks up the array's device address once
+ *   (cudaGetSymbolAddress) with that device current; make that first call before
+ *   any stream capture.
+ * - All calls share the one array and it keeps the last call's contents. Nothing
+ *   in it needs to start at zero: each call writes every partial it reads. Calls
+ *   that overlap on the GPU (on different streams, or different host threads
+ *   without ordering) race on it and give wrong results. */
+#define MLA_NOALLOC_SCRATCH_BYTES (24u << 20)
+int mla_fa_forward_noalloc(const mla_fa_args* a, void* stream);
+
 /* How the pass is divided: units = CTA pairs launched, max_splits = largest
  * number of KV splits of one (sequence, 128-row group). For tests and tools. */
 int mla_fa_query_plan(const mla_fa_args* a, int* units, int* max_splits);

@@ -110,6 +110,8 @@ def load(path: str = LIB_PATH):
     lib.mla_status_string.restype = ctypes.c_char_p
     lib.mla_version.argtypes = []
     lib.mla_version.restype = I
+    lib.mla_fa_forward_noalloc.argtypes = [ctypes.POINTER(mla_fa_args), P]
+    lib.mla_fa_forward_noalloc.restype = I
     lib.mla_profile_begin.argtypes = []
     lib.mla_profile_begin.restype = I
     lib.mla_profile_end.argtypes = [ctypes.POINTER(mla_profile_entry), I, ctypes.POINTER(I)]
@@ -259,3 +261,13 @@ def mla_profile_end():
     n = ctypes.c_int(0)
     _check(load().mla_profile_end(buf, 16, ctypes.byref(n)), "mla_profile_end")
     return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n.value)}
+
+
+NOALLOC_SCRATCH_BYTES = 24 << 20
+
+
+def mla_fa_forward_noalloc(args, stream=None):
+    """Forward pass that allocates nothing (split-KV partials in the library's
+    static scratch); raises MlaError(MLA_ERR_WORKSPACE) if the pass needs more."""
+    _check(load().mla_fa_forward_noalloc(ctypes.byref(args), _stream_ptr(stream)),
+           "mla_fa_forward_noalloc")

@@ -366,6 +366,28 @@ int ensure_ws(void** ptr, size_t* have, size_t need) {
   return MLA_OK;
 }
 
+// Scratch of mla_fa_forward_noalloc: split-KV partials (fp32 O rows, then lse)
+// of one call, in static device memory so that the call allocates nothing.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mutex;
+std::vector<void*> g_noalloc_ptr;  // per device: device address of g_noalloc_scratch
+
+// Device address of the scratch array on device `dev` (which must be current).
+// Looked up once per device; host code cannot use the symbol itself as a pointer.
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+  if ((int)g_noalloc_ptr.size() <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return MLA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -420,6 +442,23 @@ int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, vo
   rc = current_device(&st);
   if (rc != MLA_OK) return rc;
   return run_forward(r, st, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int mla_fa_forward_noalloc(const mla_fa_args* a, void* stream) {
+  Resolved r;
+  int rc = validate(a, &r);
+  if (rc != MLA_OK) return rc;
+  DeviceState* st = nullptr;
+  rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  if (workspace_for(r, st->sm_count, nullptr, nullptr) > (size_t)MLA_NOALLOC_SCRATCH_BYTES)
+    return MLA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(dev, &scratch);
+  if (rc != MLA_OK) return rc;
+  return run_forward(r, st, scratch, MLA_NOALLOC_SCRATCH_BYTES, static_cast<cudaStream_t>(stream));
 }
 
 int mla_fa_forward(const void* q, const void* kcache, int kcache_type, const void* mask, int n_q,

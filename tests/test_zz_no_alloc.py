@@ -1,0 +1,91 @@
+"""The forward entry point that allocates nothing.
+
+Some callers cannot let a library call cudaMalloc: an engine that has reserved
+nearly all device memory for its KV cache, a framework whose allocator must own
+every byte, or a decode loop that cannot take the synchronisation cudaMalloc
+may cause. mla_fa_forward_noalloc serves them by keeping its split-KV partials
+in a static device array. These tests call it through the C ABI and check, on
+two calls in a row with different inputs, that it gives what the allocating
+entry point mla_fa_forward_ex gives, and that a pass needing more scratch than
+the array holds is refused before any launch.
+
+This file is collected last so that a run stopping at the first failure has
+already run every other test; it also passes on its own in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+from mla_flash_attention_attn_b200 import binding
+from mla_flash_attention_attn_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 1e-2
+REL_L2 = 2e-3
+
+
+def _inputs(w, torch):
+    dev = torch.device("cuda")
+    q = torch.from_numpy(w.q).to(dev)
+    k = torch.from_numpy(w.kcache).to(dev)
+    m = torch.from_numpy(w.mask).to(dev)
+    return q, k, m
+
+
+def _compare(a, b, what):
+    a = a.astype(np.float64)
+    b = b.astype(np.float64)
+    assert np.all(np.isfinite(a)), what
+    err = a - b
+    maxabs = float(np.abs(err).max())
+    rel = float(np.linalg.norm(err) / max(np.linalg.norm(b), 1e-30))
+    assert maxabs <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {maxabs:.3g} rel-L2 {rel:.3g}"
+
+
+def test_noalloc_matches_allocating_entry_point_on_two_calls():
+    import torch
+
+    binding.load()
+    cases = [
+        W.make("v3_batched_decode", n_kv=4096, len_lo=1000, len_hi=4096),
+        W.make("v3_batched_decode", seed=77, n_seq=3, n_kv=3000, len_lo=200, len_hi=3000),
+    ]
+    for i, w in enumerate(cases):
+        q, k, m = _inputs(w, torch)
+        out_na = torch.full(w.q.shape[:3] + (512,), float("nan"), dtype=torch.float32,
+                            device="cuda")
+        args, keep = binding.make_args(q, k, w.kv_type, m, out_na, w.scale, kv_len=w.kv_len)
+        units, splits = binding.mla_fa_query_plan(args)
+        assert splits > 1, "the case must use split-KV scratch"
+        need = binding.mla_fa_workspace_size(args)
+        assert 0 < need <= binding.NOALLOC_SCRATCH_BYTES
+        binding.mla_fa_forward_noalloc(args)
+        ref = binding.forward(q, k, w.kv_type, m, w.scale, kv_len=w.kv_len)
+        torch.cuda.synchronize()
+        assert binding.mla_get_device_status() == 0
+        _compare(out_na.cpu().numpy(), ref.cpu().numpy(), f"call {i + 1}")
+
+
+def test_noalloc_refuses_a_pass_larger_than_its_scratch():
+    import torch
+
+    binding.load()
+    lib = binding.load()
+    # Find a batch whose split plan needs more partial slots than the scratch holds.
+    dev = torch.device("cuda")
+    found = None
+    for n_seq in range(40, 74):
+        q = torch.zeros((n_seq, 1, 128, 576), dtype=torch.float16, device=dev)
+        k = torch.zeros((n_seq, 12800, 576), dtype=torch.float16, device=dev)
+        out = torch.zeros((n_seq, 1, 128, 512), dtype=torch.float32, device=dev)
+        args, keep = binding.make_args(q, k, 0, None, out, 0.07)
+        if binding.mla_fa_workspace_size(args) > binding.NOALLOC_SCRATCH_BYTES:
+            found = (args, keep, q, k, out)
+            break
+        del q, k, out
+    assert found is not None, "no batch exceeds the scratch size"
+    args = found[0]
+    rc = lib.mla_fa_forward_noalloc(ctypes.byref(args), None)
+    assert rc == -5  # MLA_ERR_WORKSPACE, before any launch
