@@ -6,7 +6,8 @@
 // Mapping: a thread's segment is 8 consecutive cells (one 16-byte load); a CTA
 // covers 256 segments = 2048 cells. The scan over segment counts is done in
 // one pass: warp shuffle scan, then a scan of the 8 warp totals, then a
-// decoupled look-back across CTAs. CTAs take their tile in ticket order
+// decoupled look-back across CTAs (one warp reads 32 predecessor flags per
+// round trip). CTAs take their tile in ticket order
 // (atomicAdd), so every tile a CTA waits on belongs to a CTA that is already
 // running; each wait is bounded and reports MLA_ERR_TIMEOUT instead of hanging.
 // Look-back flags carry a per-call epoch, so stale flags from an earlier call
@@ -95,43 +96,53 @@ __global__ void __launch_bounds__(compact::kThreads)
     }
     if (lane < kThreads / 32) s_warp_tot[lane] = winc - wt;  // exclusive offsets of warps
     const int agg = __shfl_sync(0xffffffffu, winc, kThreads / 32 - 1);
-    if (lane == 0) {
-      const unsigned long long tag_agg = (unsigned long long)(epoch * 4u + kStateAggregate) << 32;
-      const unsigned long long tag_inc = (unsigned long long)(epoch * 4u + kStateInclusive) << 32;
-      int excl = 0;
-      if (tile == 0) {
-        st_release_u64(&rflags[0], tag_inc | (uint32_t)agg);
-      } else {
-        st_release_u64(&rflags[tile], tag_agg | (uint32_t)agg);
-        bool ok = true;
-        for (int j = tile - 1; j >= 0;) {
-          unsigned long long f = ld_acquire_u64(&rflags[j]);
-          uint32_t tag = (uint32_t)(f >> 32);
-          if (tag == epoch * 4u + kStateInclusive) {
-            excl += (int)(uint32_t)f;
+    const uint32_t tag_agg = epoch * 4u + kStateAggregate;
+    const uint32_t tag_inc = epoch * 4u + kStateInclusive;
+    int excl = 0;
+    if (tile == 0) {
+      if (lane == 0) st_release_u64(&rflags[0], ((unsigned long long)tag_inc << 32) | (uint32_t)agg);
+    } else {
+      if (lane == 0) st_release_u64(&rflags[tile], ((unsigned long long)tag_agg << 32) | (uint32_t)agg);
+      // Warp-wide look-back: lane l inspects tile (top - l); a window of 32
+      // predecessors costs one round trip. Sum aggregates down to the nearest
+      // inclusive prefix; tiles before 0 count as an inclusive prefix of 0.
+      int top = tile - 1;
+      bool timed_out = false;
+      uint64_t t0 = 0;
+      while (true) {
+        const int j = top - lane;
+        uint32_t state = kStateInclusive, val = 0;
+        if (j >= 0) {
+          const unsigned long long f = ld_acquire_u64(&rflags[j]);
+          const uint32_t tag = (uint32_t)(f >> 32);
+          state = tag == tag_inc ? kStateInclusive : (tag == tag_agg ? kStateAggregate : 0u);
+          val = (uint32_t)f;
+        }
+        const uint32_t inc_mask = __ballot_sync(0xffffffffu, state == kStateInclusive);
+        const uint32_t wait_mask = __ballot_sync(0xffffffffu, state == 0u);
+        const int first_inc = inc_mask ? __ffs(inc_mask) - 1 : 32;
+        const uint32_t upto = first_inc >= 31 ? 0xffffffffu : ((2u << first_inc) - 1u);
+        if (wait_mask & upto) {  // a needed predecessor has not published yet
+          if (t0 == 0) t0 = globaltimer_ns();
+          if (globaltimer_ns() - t0 > timeout_ns) {
+            timed_out = true;
             break;
           }
-          if (tag == epoch * 4u + kStateAggregate) {
-            excl += (int)(uint32_t)f;
-            --j;
-            continue;
-          }
-          // not published yet: poll with a wall-time bound
-          uint64_t t0 = globaltimer_ns();
-          while (true) {
-            f = ld_acquire_u64(&rflags[j]);
-            tag = (uint32_t)(f >> 32);
-            if (tag == epoch * 4u + kStateInclusive || tag == epoch * 4u + kStateAggregate) break;
-            if (globaltimer_ns() - t0 > timeout_ns) {
-              ok = false;
-              break;
-            }
-          }
-          if (!ok) break;
+          continue;
         }
-        if (!ok) record_status(kStatusTimeout);
-        st_release_u64(&rflags[tile], tag_inc | (uint32_t)(excl + agg));
+        int part = (lane <= first_inc) ? (int)val : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        excl += part;
+        if (first_inc < 32) break;
+        top -= 32;
+        t0 = 0;
       }
+      if (timed_out && lane == 0) record_status(kStatusTimeout);
+      if (lane == 0)
+        st_release_u64(&rflags[tile], ((unsigned long long)tag_inc << 32) | (uint32_t)(excl + agg));
+    }
+    if (lane == 0) {
       s_excl = excl;
       if (tile == n_tiles - 1) {
         count_out[row] = excl + agg;

@@ -72,33 +72,42 @@ enum FwdMode {
 
 namespace fwd {
 
-constexpr int kStages = 12;
+constexpr int kKStages = 8;      // ring of Q.K^T operand chunks (K rows)
+constexpr int kVStages = 6;      // ring of P.V operand chunks (V columns, L2-resident)
+constexpr int kSBufs = 3;        // S buffers in TMEM (64 columns each)
 constexpr int kChunkBytes = 8192;                 // one ring stage
 constexpr int kQBytes = 9 * kChunkBytes;          // 64 rows x 576 f16
 constexpr int kPBufBytes = 2 * kChunkBytes;       // 64 rows x 128 keys f16
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kStages * kChunkBytes;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kKStages * kChunkBytes;
+constexpr int kOffP = kOffV + kVStages * kChunkBytes;
 constexpr int kOffBar = kOffP + 2 * kPBufBytes;
-constexpr int kNumBars = 2 * kStages + 1 + 2 + 2 + 2;
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 1 + kSBufs + 2 + 2;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
 constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
 constexpr int kSmemBytes = kOffXl + 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;                   // 1024-byte alignment slack
-constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 128;                                // O columns start
+constexpr uint32_t kTmemO = kSBufs * 64;                        // O columns start
 constexpr float kRescaleThreshold = 8.0f;                       // log2 units
+
+static_assert(kSmemAlloc <= 232448, "shared memory beyond the 227 KB per-CTA limit");
+static_assert(kTmemO + 256 <= kTmemCols, "S buffers and O exceed the TMEM allocation");
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
+              "128-byte swizzle needs 1 KB alignment");
 
 constexpr uint32_t kIdescQK = idesc_f16_f32(128, 128, 0, 0);    // K-major A and B
 constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);    // B (V) MN-major
 
 struct Bars {
-  uint64_t ring_full[kStages];   // leader: both CTAs' TMA bytes for a stage
-  uint64_t ring_empty[kStages];  // both: the MMAs reading a stage are done
+  uint64_t k_full[kKStages];     // leader: both CTAs' K chunk bytes landed
+  uint64_t k_empty[kKStages];    // both: the Q.K^T MMAs reading a K stage are done
+  uint64_t v_full[kVStages];     // leader: both CTAs' V chunk bytes landed
+  uint64_t v_empty[kVStages];    // both: the P.V MMAs reading a V stage are done
   uint64_t q_full;               // leader: Q of both CTAs loaded
-  uint64_t s_full[2];            // both: S buffer written by Q.K^T
+  uint64_t s_full[kSBufs];       // both: S buffer written by Q.K^T
   uint64_t p_full[2];            // leader: P written (8 warp arrivals, both CTAs)
   uint64_t o_done[2];            // both: P.V of a tile (parity-indexed) complete
 };
@@ -157,7 +166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem + kOffQ;
-  uint8_t* sRing = smem + kOffRing;
+  uint8_t* sK = smem + kOffK;
+  uint8_t* sV = smem + kOffV;
   uint8_t* sP = smem + kOffP;
   Bars& bars = *reinterpret_cast<Bars*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
@@ -185,13 +195,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 
   // ---- setup: barriers, TMEM
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bars.ring_full[i], kManual ? 8 : 1);
-      mbar_init(&bars.ring_empty[i], 1);
+    // manual modes: 2 producer warps per ring in each CTA arrive on the leader
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&bars.k_full[i], kManual ? 4 : 1);
+      mbar_init(&bars.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&bars.v_full[i], kManual ? 4 : 1);
+      mbar_init(&bars.v_empty[i], 1);
     }
     mbar_init(&bars.q_full, 1);
+    for (int i = 0; i < kSBufs; ++i) mbar_init(&bars.s_full[i], 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], 8);
       mbar_init(&bars.o_done[i], 1);
     }
@@ -224,112 +239,146 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                         row0 + kRowsPerCta * (int)rank, b_abs);
     }
     if (!kManual && n_tiles > 0 && elect_one()) {
+      // K ring: this CTA's 64 keys of each tile, 9 chunks of 64 columns, as far
+      // ahead as the ring allows (only Q.K^T consumption frees K stages)
       int stage = 0;
       uint32_t ephase = 0;
-      auto acquire = [&]() {
-        if (!failed && !mbar_wait(&bars.ring_empty[stage], ephase ^ 1, to)) {
-          failed = true;
-          record_status(kStatusTimeout);
-        }
-        if (rank == 0) mbar_arrive_expect_tx(&bars.ring_full[stage], 2 * kChunkBytes);
-      };
-      auto full_l = [&]() { return mapa_shared(smem_u32(&bars.ring_full[stage]), 0); };
-      auto advance = [&]() {
-        if (++stage == kStages) { stage = 0; ephase ^= 1; }
-      };
-      auto issue_k = [&](int i) {
+      for (int i = 0; i < n_tiles; ++i) {
         const int key0 = (tile_begin + i) * kTileKeys + 64 * (int)rank;
         for (int c = 0; c < 9; ++c) {
-          acquire();
-          tma_load_3d_2sm(sRing + stage * kChunkBytes, &tm_k, full_l(), 64 * c, key0, b_abs);
-          advance();
+          if (!failed && !mbar_wait(&bars.k_empty[stage], ephase ^ 1, to)) {
+            failed = true;
+            record_status(kStatusTimeout);
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kChunkBytes);
+          tma_load_3d_2sm(sK + stage * kChunkBytes, &tm_k,
+                          mapa_shared(smem_u32(&bars.k_full[stage]), 0), 64 * c, key0, b_abs);
+          if (++stage == kKStages) { stage = 0; ephase ^= 1; }
         }
-      };
-      auto issue_v = [&](int j) {
+      }
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ================= V producer (TMA mode): value columns of each tile, own ring
+    if (!kManual && n_tiles > 0 && elect_one()) {
+      int stage = 0;
+      uint32_t ephase = 0;
+      for (int j = 0; j < n_tiles; ++j) {
         const int key0 = (tile_begin + j) * kTileKeys;
         for (int kb = 0; kb < 4; ++kb)
           for (int nb = 0; nb < 2; ++nb) {
-            acquire();
+            if (!failed && !mbar_wait(&bars.v_empty[stage], ephase ^ 1, to)) {
+              failed = true;
+              record_status(kStatusTimeout);
+            }
+            if (rank == 0) mbar_arrive_expect_tx(&bars.v_full[stage], 2 * kChunkBytes);
             const int col = 256 * nb + 128 * (int)rank;
-            uint32_t fl = full_l();
-            tma_load_3d_2sm(sRing + stage * kChunkBytes, &tm_v, fl, col, key0 + 32 * kb, b_abs);
-            tma_load_3d_2sm(sRing + stage * kChunkBytes + 4096, &tm_v, fl, col + 64,
-                            key0 + 32 * kb, b_abs);
-            advance();
+            const uint32_t fl = mapa_shared(smem_u32(&bars.v_full[stage]), 0);
+            tma_load_3d_2sm(sV + stage * kChunkBytes, &tm_v, fl, col, key0 + 32 * kb, b_abs);
+            tma_load_3d_2sm(sV + stage * kChunkBytes + 4096, &tm_v, fl, col + 64, key0 + 32 * kb,
+                            b_abs);
+            if (++stage == kVStages) { stage = 0; ephase ^= 1; }
           }
-      };
-      issue_k(0);
-      for (int i = 1; i < n_tiles; ++i) {
-        issue_k(i);
-        issue_v(i - 1);
       }
-      issue_v(n_tiles - 1);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ================= MMA issuer (leader CTA, one thread)
+    // ================= MMA issuer (leader CTA, one thread): a polling scheduler.
+    // Each step issues whatever is ready: the next P.V chunk (needs P of its tile
+    // and the V stage) first, then the next Q.K^T chunk (needs the K stage, and for
+    // a new tile a free S buffer: the softmax of the tile kSBufs earlier has
+    // published its P). Both rings are consumed in their own FIFO order.
     if (rank == 0 && n_tiles > 0 && elect_one()) {
-      auto wait_or_fail = [&](uint64_t* bar, uint32_t parity, bool cluster_scope) {
-        if (failed) return;
-        bool ok = cluster_scope ? mbar_wait_cluster(bar, parity, to) : mbar_wait(bar, parity, to);
-        if (!ok) {
-          failed = true;
-          record_status(kStatusTimeout);
-        }
-      };
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t ring_addr = smem_u32(sRing);
-      const uint32_t p_addr = smem_u32(sP);
-      wait_or_fail(&bars.q_full, 0, false);
-      tc_fence_after();
-      int stage = 0;
-      uint32_t fphase = 0;
-      auto advance = [&]() {
-        if (++stage == kStages) { stage = 0; fphase ^= 1; }
-      };
-      auto pv = [&](int j) {
-        wait_or_fail(&bars.p_full[j & 1], (j >> 1) & 1, true);
-        tc_fence_after();
-        for (int kb = 0; kb < 4; ++kb)
-          for (int nb = 0; nb < 2; ++nb) {
-            wait_or_fail(&bars.ring_full[stage], fphase, kManual);
-            tc_fence_after();
-            for (int k2 = 0; k2 < 2; ++k2) {
-              const int kk = 2 * kb + k2;
-              uint64_t ad = smem_desc_sw128(
-                  p_addr + (j & 1) * kPBufBytes + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024);
-              uint64_t bd = smem_desc_sw128(ring_addr + stage * kChunkBytes + k2 * 2048, 4096, 1024);
-              mma_f16_ss_2sm(tmem + kTmemO + nb * 128, ad, bd, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            mma_commit_2sm_mc(&bars.ring_empty[stage], 0x3);
-            advance();
-          }
-        mma_commit_2sm_mc(&bars.o_done[j & 1], 0x3);
-      };
-      for (int i = 0; i < n_tiles; ++i) {
-        const uint32_t d_s = tmem + (i & 1) * 64;
-        for (int c = 0; c < 9; ++c) {
-          wait_or_fail(&bars.ring_full[stage], fphase, kManual);
-          tc_fence_after();
-          for (int kk = 0; kk < 4; ++kk) {
-            uint64_t ad = smem_desc_sw128(q_addr + c * kChunkBytes + kk * 32, 16, 1024);
-            uint64_t bd = smem_desc_sw128(ring_addr + stage * kChunkBytes + kk * 32, 16, 1024);
-            mma_f16_ss_2sm(d_s, ad, bd, kIdescQK, (c | kk) ? 1u : 0u);
-          }
-          mma_commit_2sm_mc(&bars.ring_empty[stage], 0x3);
-          advance();
-        }
-        mma_commit_2sm_mc(&bars.s_full[i & 1], 0x3);
-        if (i > 0) pv(i - 1);
+      // Descriptor bases; an operand at byte offset `off` within a region is the base
+      // plus off/16 (the start address field is the low 14 bits, no carry possible
+      // below 256 KB). Everything per MMA below is a 64-bit add of a constant.
+      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv = smem_desc_sw128(smem_u32(sV), 4096, 1024);
+      const uint64_t dp = smem_desc_sw128(smem_u32(sP), 16, 1024);
+      constexpr uint32_t kStageUnits = kChunkBytes >> 4;
+      if (!mbar_wait(&bars.q_full, 0, to)) {
+        failed = true;
+        record_status(kStatusTimeout);
       }
-      pv(n_tiles - 1);
+      tc_fence_after();
+      int kst = 0, vst = 0;
+      uint32_t kph = 0, vph = 0;
+      int qk_t = 0, qk_c = 0;  // next Q.K^T tile / 64-column chunk
+      int pv_t = 0, pv_c = 0;  // next P.V tile / (32-key, 256-column) chunk
+      bool p_ok = false;       // P of tile pv_t observed (with cluster-scope acquire)
+      uint64_t idle_since = 0;
+      // Cheap CTA-scope probes; a phase completed by arrivals from the peer CTA is
+      // then acquired once at cluster scope before its data is used.
+      auto ready = [&](uint64_t* bar, uint32_t parity, bool remote) -> bool {
+        if (failed) return true;
+        if (!mbar_test(bar, parity)) return false;
+        if (remote) (void)mbar_test_cluster(bar, parity);
+        return true;
+      };
+      while (pv_t < n_tiles) {
+        bool progressed = false;
+        if (!p_ok) p_ok = ready(&bars.p_full[pv_t & 1], (pv_t >> 1) & 1, true);
+        if (p_ok && ready(&bars.v_full[vst], vph, kManual)) {
+          tc_fence_after();
+          const int kb = pv_c >> 1, nb = pv_c & 1;
+          const uint64_t a0 = dp + (uint32_t)((pv_t & 1) * (kPBufBytes >> 4) + (kb >> 1) * kStageUnits +
+                                              (kb & 1) * 4);
+          const uint64_t b0 = dv + (uint32_t)(vst * kStageUnits);
+          const uint32_t d = tmem + kTmemO + nb * 128;
+          mma_f16_ss_2sm(d, a0, b0, kIdescPV, (pv_t > 0 || kb > 0) ? 1u : 0u);
+          mma_f16_ss_2sm(d, a0 + 2, b0 + 128, kIdescPV, 1u);
+          mma_commit_2sm_mc(&bars.v_empty[vst], 0x3);
+          if (++vst == kVStages) { vst = 0; vph ^= 1; }
+          if (++pv_c == 8) {
+            mma_commit_2sm_mc(&bars.o_done[pv_t & 1], 0x3);
+            pv_c = 0;
+            ++pv_t;
+            p_ok = false;
+          }
+          progressed = true;
+        }
+        const int pv_seen = pv_t + (p_ok ? 1 : 0);
+        if (qk_t < n_tiles && (qk_c > 0 || qk_t < pv_seen + kSBufs) &&
+            ready(&bars.k_full[kst], kph, kManual)) {
+          const uint32_t d_s = tmem + (qk_t % kSBufs) * 64;
+          const uint64_t a0 = dq + (uint32_t)(qk_c * kStageUnits);
+          const uint64_t b0 = dk + (uint32_t)(kst * kStageUnits);
+          const uint32_t acc0 = qk_c ? 1u : 0u;
+          mma_f16_ss_2sm(d_s, a0, b0, kIdescQK, acc0);
+          mma_f16_ss_2sm(d_s, a0 + 2, b0 + 2, kIdescQK, 1u);
+          mma_f16_ss_2sm(d_s, a0 + 4, b0 + 4, kIdescQK, 1u);
+          mma_f16_ss_2sm(d_s, a0 + 6, b0 + 6, kIdescQK, 1u);
+          mma_commit_2sm_mc(&bars.k_empty[kst], 0x3);
+          if (++kst == kKStages) { kst = 0; kph ^= 1; }
+          if (++qk_c == 9) {
+            mma_commit_2sm_mc(&bars.s_full[qk_t % kSBufs], 0x3);
+            qk_c = 0;
+            ++qk_t;
+          }
+          progressed = true;
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else if (!failed) {
+          const uint64_t now = globaltimer_ns();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > to) {
+            failed = true;
+            record_status(kStatusTimeout);
+          }
+        }
+      }
     }
     __syncwarp();
   } else if (warp >= 8) {
-    // ================= gather / dequant producer (manual modes): 4 warps, 128 threads
+    // ================= gather / dequant producers (manual modes): warps 8-9 fill the
+    // K ring, warps 10-11 the V ring; 64 threads per ring, 2 of a stage's 128 items each
     if constexpr (kManual) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 128;");
-      const int pt = threadIdx.x - 256;
+      const bool k_side = warp < 10;
+      const int pt = (threadIdx.x - 256) & 63;
       const int64_t seq_row0 = (int64_t)b_abs * p.k_seq_stride;
       const int32_t* idx_row = sparse ? p.idx + (int64_t)b_abs * p.idx_seq_stride : nullptr;
       // cache row of key position `pos` in this unit's selection, or -1 (zero fill)
@@ -366,10 +415,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           *reinterpret_cast<uint4*>(row_dst + (((chunk0 + k) ^ (row_in_atom & 7)) << 4)) =
               make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3]);
       };
+      const int n_stages = k_side ? kKStages : kVStages;
+      uint64_t* full = k_side ? bars.k_full : bars.v_full;
+      uint64_t* empty = k_side ? bars.k_empty : bars.v_empty;
+      uint8_t* ring = k_side ? sK : sV;
       int stage = 0;
       uint32_t ephase = 0;
       auto acquire = [&]() {
-        bool ok = failed ? true : mbar_wait(&bars.ring_empty[stage], ephase ^ 1, to);
+        bool ok = failed ? true : mbar_wait(&empty[stage], ephase ^ 1, to);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok && !failed) {
           failed = true;
@@ -379,41 +432,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       auto publish = [&]() {
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars.ring_full[stage]), 0));
-        if (++stage == kStages) { stage = 0; ephase ^= 1; }
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[stage]), 0));
+        if (++stage == n_stages) { stage = 0; ephase ^= 1; }
       };
-      // K chunk: 64 keys (this CTA's half of the tile) x 64 columns = 2 blocks of 32
-      auto issue_k = [&](int i) {
-        const int kl = pt >> 1, half = pt & 1;
-        const int key = resolve((tile_begin + i) * kTileKeys + 64 * (int)rank + kl);
-        for (int c = 0; c < 9; ++c) {
-          acquire();
-          fill32(sRing + stage * kChunkBytes + kl * 128, kl, key, 2 * c + half, 4 * half);
-          publish();
-        }
-      };
-      // V chunk: 32 keys x this CTA's 128 value columns (two 64-column boxes)
-      auto issue_v = [&](int j) {
-        const int kl = pt >> 2, q4 = pt & 3;
-        const int box = q4 >> 1, half = q4 & 1;
-        const int kbase = (tile_begin + j) * kTileKeys;
-        for (int kb = 0; kb < 4; ++kb) {
-          const int key = resolve(kbase + 32 * kb + kl);
-          for (int nb = 0; nb < 2; ++nb) {
+      if (k_side) {
+        // K chunk items: 64 keys (this CTA's half of the tile) x 2 blocks of 32 columns
+        for (int i = 0; i < n_tiles; ++i) {
+          const int kbase = (tile_begin + i) * kTileKeys + 64 * (int)rank;
+          const int key_a = resolve(kbase + (pt >> 1));
+          const int key_b = resolve(kbase + 32 + (pt >> 1));
+          const int half = pt & 1;
+          for (int c = 0; c < 9; ++c) {
             acquire();
-            const int col32 = 8 * nb + 4 * (int)rank + q4;
-            fill32(sRing + stage * kChunkBytes + box * 4096 + kl * 128, kl, key, col32, 4 * half);
+            fill32(ring + stage * kChunkBytes + (pt >> 1) * 128, pt >> 1, key_a, 2 * c + half,
+                   4 * half);
+            fill32(ring + stage * kChunkBytes + (32 + (pt >> 1)) * 128, 32 + (pt >> 1), key_b,
+                   2 * c + half, 4 * half);
             publish();
           }
         }
-      };
-      if (n_tiles > 0) {
-        issue_k(0);
-        for (int i = 1; i < n_tiles; ++i) {
-          issue_k(i);
-          issue_v(i - 1);
+      } else {
+        // V chunk items: 32 keys x this CTA's 128 value columns (4 blocks, two boxes)
+        const int q4 = pt & 3, box = q4 >> 1, half = q4 & 1;
+        for (int j = 0; j < n_tiles; ++j) {
+          const int kbase = (tile_begin + j) * kTileKeys;
+          for (int kb = 0; kb < 4; ++kb) {
+            const int kl_a = pt >> 2, kl_b = 16 + (pt >> 2);
+            const int key_a = resolve(kbase + 32 * kb + kl_a);
+            const int key_b = resolve(kbase + 32 * kb + kl_b);
+            for (int nb = 0; nb < 2; ++nb) {
+              acquire();
+              const int col32 = 8 * nb + 4 * (int)rank + q4;
+              uint8_t* st = ring + stage * kChunkBytes + box * 4096;
+              fill32(st + kl_a * 128, kl_a, key_a, col32, 4 * half);
+              fill32(st + kl_b * 128, kl_b, key_b, col32, 4 * half);
+              publish();
+            }
+          }
         }
-        issue_v(n_tiles - 1);
       }
     }
   } else if (warp >= 4) {
@@ -445,21 +501,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     float l_part = 0.f;       // this lane's half of the row sum, relative to m_ref
 
     for (int i = 0; i < n_tiles; ++i) {
-      const int sb = i & 1;
+      const int sb = i & 1;          // P buffer and max-exchange slot
+      const int sbuf = i % kSBufs;   // S buffer in TMEM
       const int key0 = (tile_begin + i) * kTileKeys + 64 * kh;
-      wait_local(&bars.s_full[sb], (i >> 1) & 1);
+      const bool full_range = key0 + 64 <= key_end;
+      // issue this tile's mask loads before waiting for S, to hide their latency
+      const bool vec_mask = !(kManual && sparse) && mrow != nullptr && full_range && p.mask_vec_ok;
+      uint4 mvec[8];
+      if (vec_mask) {
+        const uint4* mv = reinterpret_cast<const uint4*>(mrow + key0);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) mvec[c] = __ldg(mv + c);
+      }
+      wait_local(&bars.s_full[sbuf], (i / kSBufs) & 1);
       tc_fence_after();
       uint32_t sr[64];
       {
         uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
         uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tmem_ld32(tmem + lane_base + sb * 64, a);
-        tmem_ld32(tmem + lane_base + sb * 64 + 32, c);
+        tmem_ld32(tmem + lane_base + sbuf * 64, a);
+        tmem_ld32(tmem + lane_base + sbuf * 64 + 32, c);
         tmem_wait_ld();
       }
       // scores in log2 units; cells beyond the unit's keys are dropped
       float x[64];
-      const bool full_range = key0 + 64 <= key_end;
       if (kManual && sparse) {
         const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
 #pragma unroll
@@ -474,11 +539,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           }
           x[j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
         }
-      } else if (mrow != nullptr && full_range && p.mask_vec_ok) {
-        const uint4* mv = reinterpret_cast<const uint4*>(mrow + key0);
+      } else if (vec_mask) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          uint4 v = __ldg(mv + c);
+          const uint4 v = mvec[c];
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
@@ -609,43 +673,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 //   O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
 // where O_s is split s normalised by its own sum and lse_s = log2 of that sum
 // relative to the split's max; splits with no kept cell have lse_s = -inf.
+// Lane s holds the weight of split s (in chunks of 32 splits); the partial
+// rows are then read with independent, unrolled 16-byte loads.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant__ Plan plan,
                                                           const float* __restrict__ ws_o,
                                                           const float* __restrict__ ws_lse,
                                                           float* __restrict__ out,
                                                           int64_t out_seq_stride) {
   const int b = blockIdx.y;
-  const int ns = plan.n_split[b];
   if (plan.ws_base[b] < 0) return;
+  const int ns = plan.n_split[b];
   const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (row >= plan.rows) return;
   const int lane = threadIdx.x & 31;
   const int g = row / kRowsPerGroup;
   const int rin = row % kRowsPerGroup;
   const int slot0 = plan.ws_base[b] + g * ns;
+  const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
   float mx = -INFINITY;
-  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, ws_lse[(int64_t)(slot0 + s) * kRowsPerGroup + rin]);
+  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)s * kRowsPerGroup));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float4 acc[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
   if (mx != -INFINITY) {
-    float wsum = 0.f;
-    for (int s = 0; s < ns; ++s) {
-      const float lse = ws_lse[(int64_t)(slot0 + s) * kRowsPerGroup + rin];
-      if (lse == -INFINITY) continue;
-      const float w = ex2_approx(lse - mx);
-      wsum += w;
-      const float4* src =
-          reinterpret_cast<const float4*>(ws_o + ((int64_t)(slot0 + s) * kRowsPerGroup + rin) * kDV);
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      const int s = s0 + lane;
+      float wl = 0.f;
+      if (s < ns) {
+        const float lse = __ldg(lse_col + (int64_t)s * kRowsPerGroup);
+        wl = lse == -INFINITY ? 0.f : ex2_approx(lse - mx);
+      }
+      wsum += wl;
+      const int cnt = min(32, ns - s0);
+#pragma unroll 4
+      for (int j = 0; j < cnt; ++j) {
+        const float w = __shfl_sync(0xffffffffu, wl, j);
+        const float4* src = reinterpret_cast<const float4*>(
+            ws_o + ((int64_t)(slot0 + s0 + j) * kRowsPerGroup + rin) * kDV);
+        float4 v[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 v = __ldg(src + lane + 32 * k);
-        acc[k].x = fmaf(w, v.x, acc[k].x);
-        acc[k].y = fmaf(w, v.y, acc[k].y);
-        acc[k].z = fmaf(w, v.z, acc[k].z);
-        acc[k].w = fmaf(w, v.w, acc[k].w);
+        for (int k = 0; k < 4; ++k) v[k] = __ldg(src + lane + 32 * k);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc[k].x = fmaf(w, v[k].x, acc[k].x);
+          acc[k].y = fmaf(w, v[k].y, acc[k].y);
+          acc[k].z = fmaf(w, v[k].z, acc[k].z);
+          acc[k].w = fmaf(w, v[k].w, acc[k].w);
+        }
       }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     const float inv = 1.f / wsum;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
