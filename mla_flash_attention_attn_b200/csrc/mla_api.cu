@@ -269,6 +269,19 @@ int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
   return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// fp32 [d2][d1][512] output view for the kernel's TMA stores: boxes of 32 rows x 32
+// columns, 128-byte swizzle (the layout the kernel stages in shared memory).
+int make_out_map(CUtensorMap* m, void* base, uint64_t d1, uint64_t d2, uint64_t stride2_bytes) {
+  cuuint64_t dims[3] = {(cuuint64_t)MLA_DV, d1, d2};
+  cuuint64_t strides[2] = {(cuuint64_t)MLA_DV * 4, stride2_bytes};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult res = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const mla_fa_args& a = r.a;
   const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
@@ -281,14 +294,27 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   int rc = make_map(&tm_q, a.q, MLA_DK, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
   if (rc == MLA_OK && mode == mla::kModeTma) {
     rc = make_map(&tm_k, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
-                  64, 64);
-    if (rc == MLA_OK)
-      rc = make_map(&tm_v, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes,
-                    (uint64_t)r.k_ss * row_bytes, 64, 32);
+                  64, mla::kTileKeys / 2);
+    if (rc == MLA_OK) {
+      // value view: {64 columns, keys, 8 column blocks, sequences}; a box of
+      // {64, 64, 2, 1} lands as [column block][key][64 columns]
+      cuuint64_t dims[4] = {64, (cuuint64_t)a.n_kv, 8, (cuuint64_t)a.n_seq};
+      cuuint64_t strides[3] = {row_bytes, 128, (cuuint64_t)r.k_ss * row_bytes};
+      cuuint32_t box[4] = {64, 64, 2, 1};
+      cuuint32_t es[4] = {1, 1, 1, 1};
+      CUresult res = g_encode(&tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(a.kcache),
+                              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      rc = res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+    }
   } else {
     tm_k = tm_q;  // unused by the gather / dequant modes
     tm_v = tm_q;
   }
+  CUtensorMap tm_o;
+  if (rc == MLA_OK)
+    rc = make_out_map(&tm_o, a.out, (uint64_t)r.rows, (uint64_t)a.n_seq, (uint64_t)r.o_ss * 4);
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
     if (cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeTma>,
@@ -326,22 +352,28 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                 (size_t)slots * mla::kRowsPerGroup * mla::kDV * 4)
                      : nullptr;
+    CUtensorMap tm_w = tm_o;  // unused when no sequence of this launch is split
+    if (slots > 0) {
+      rc = make_out_map(&tm_w, ws, (uint64_t)slots * mla::kRowsPerGroup, 1,
+                        (uint64_t)slots * mla::kRowsPerGroup * MLA_DV * 4);
+      if (rc != MLA_OK) return rc;
+    }
     dim3 grid(2 * plan.total_units);
     if (mode == mla::kModeTma) {
       ProfScope prof(kKernFwdF16, stream);
       mla::mla_fwd_kernel<mla::kModeTma>
           <<<grid, mla::FwdCfg<mla::kModeTma>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-              tm_q, tm_k, tm_v, plan, p);
+              tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
     } else if (mode == mla::kModeGatherF16) {
       ProfScope prof(kKernFwdGather, stream);
       mla::mla_fwd_kernel<mla::kModeGatherF16>
           <<<grid, mla::FwdCfg<mla::kModeGatherF16>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-              tm_q, tm_k, tm_v, plan, p);
+              tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
     } else {
       ProfScope prof(kKernFwdQ8, stream);
       mla::mla_fwd_kernel<mla::kModeQ8>
           <<<grid, mla::FwdCfg<mla::kModeQ8>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-              tm_q, tm_k, tm_v, plan, p);
+              tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
     }
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     if (slots > 0) {

@@ -9,7 +9,7 @@ constexpr int kDK = 576;             // cache row / query width (512 latent + 64
 constexpr int kDV = 512;             // value width: first 512 columns of the row
 constexpr int kRowsPerGroup = 128;   // M of the 2-SM MMA (64 rows in each CTA)
 constexpr int kRowsPerCta = 64;
-constexpr int kTileKeys = 128;       // N of one Q.K^T MMA: keys per tile
+constexpr int kTileKeys = 256;       // N of one Q.K^T MMA: keys per tile
 constexpr int kPlanMaxSeq = 128;     // sequences per launch (larger batches are chunked)
 constexpr int kQ8RowBytes = 612;     // q8_0: 18 blocks of {f16 d; int8 q[32]}
 constexpr float kLog2e = 1.4426950408889634f;

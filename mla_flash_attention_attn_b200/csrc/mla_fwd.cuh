@@ -12,18 +12,26 @@
 // Hardware mapping (cta_group::2, M = 128 rows, 64 rows in each CTA):
 //  * Each CTA keeps its 64 Q rows in shared memory (9 chunks of 64 columns,
 //    128-byte swizzle) for the whole unit.
-//  * Q.K^T: N = 128 keys; CTA c loads keys [64c, 64c+64) of each tile, so the
-//    pair reads every K byte once. In TMEM, lane r holds keys 0..63 of row r
-//    and lane r+64 keys 64..127 (64 columns per S buffer, two buffers).
-//  * P.V: N = 256 value columns per MMA, two MMAs per 16 keys; CTA c loads
-//    value columns [256j+128c, +128) of the tile's rows. O lives in TMEM
-//    (256 columns per CTA: lane r holds 128 of row r's values per MMA half).
-//  * K and V chunks (8 KB each) stream through one ring of shared-memory
-//    stages filled by TMA; the MMA thread releases a stage with tcgen05.commit.
+//  * Q.K^T: N = 256 keys (a tile); CTA c loads keys [128c, 128c+128) of each
+//    tile, so the pair reads every K byte once. In TMEM, lane r holds keys
+//    0..127 of row r and lane r+64 keys 128..255 (128 columns per S buffer, two
+//    buffers). N = 256 halves the MMAs (and their issue cost) per key.
+//  * P.V: N = 256 value columns per MMA (one value half), K = 16 keys; CTA c
+//    loads value columns [256j+128c, +128) of the tile's rows. O lives in TMEM
+//    (256 columns per CTA: lane r holds 128 of row r's values per value half).
+//  * K stages (16 KB: 128 keys x 64 columns) and V stages (16 KB: 64 keys x 128
+//    value columns) stream through two rings of shared-memory stages; every
+//    stage is 4 MMAs and one tcgen05.commit releases it.
+//  * Two threads issue MMAs: one for Q.K^T, one for P.V. An issuing thread
+//    cannot run ahead of the tensor pipe, so the cycles it spends waiting on a
+//    barrier would idle the pipe; with two issuers one's wait is covered by the
+//    other's MMAs.
 //  * Softmax warpgroup: thread = TMEM lane; the two lanes of a row exchange
 //    their tile maximum through shared memory. The reference max is raised
 //    only when a tile's max exceeds it by more than 2^8, so O is rescaled in
-//    TMEM rarely; P (f16, <= 256) goes to shared memory as the A operand.
+//    TMEM rarely; P (f16, <= 256) goes to one shared-memory buffer as the A
+//    operand, written once P.V of the previous tile has finished.
+//  * Epilogue: O / l is staged in shared memory and written by TMA stores.
 //
 // Every mbarrier wait is bounded (MlaFwdParams::timeout_ns). On a timeout the
 // thread records MLA_ERR_TIMEOUT in the device status word and "fails
@@ -72,17 +80,20 @@ enum FwdMode {
 
 namespace fwd {
 
-constexpr int kKStages = 8;      // ring of Q.K^T operand chunks (K rows)
-constexpr int kVStages = 6;      // ring of P.V operand chunks (V columns, L2-resident)
-constexpr int kSBufs = 3;        // S buffers in TMEM (64 columns each)
-constexpr int kChunkBytes = 8192;                 // one ring stage
+constexpr int kKStages = 3;      // ring of Q.K^T operand stages (K rows)
+constexpr int kVStages = 4;      // ring of P.V operand stages (V columns, L2-resident)
+constexpr int kSBufs = 2;        // S buffers in TMEM (128 columns each)
+constexpr int kSCols = 128;      // TMEM columns of one S buffer
+constexpr int kChunkBytes = 8192;                 // 64 rows x 64 f16 (one swizzle tile)
+constexpr int kKChunkBytes = 2 * kChunkBytes;     // K stage: 128 keys x 64 columns
+constexpr int kVStageBytes = 2 * kChunkBytes;     // V stage: 64 keys x 128 value columns
 constexpr int kQBytes = 9 * kChunkBytes;          // 64 rows x 576 f16
-constexpr int kPBufBytes = 2 * kChunkBytes;       // 64 rows x 128 keys f16
+constexpr int kPBufBytes = 4 * kChunkBytes;       // 64 rows x 256 keys f16
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKStages * kChunkBytes;
-constexpr int kOffP = kOffV + kVStages * kChunkBytes;
-constexpr int kOffBar = kOffP + 2 * kPBufBytes;
+constexpr int kOffV = kOffK + kKStages * kKChunkBytes;
+constexpr int kOffP = kOffV + kVStages * kVStageBytes;
+constexpr int kOffBar = kOffP + kPBufBytes;
 constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 1 + kSBufs + 2 + 2;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
@@ -90,7 +101,7 @@ constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
 constexpr int kSmemBytes = kOffXl + 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;                   // 1024-byte alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = kSBufs * 64;                        // O columns start
+constexpr uint32_t kTmemO = kSBufs * kSCols;                    // O columns start
 constexpr float kRescaleThreshold = 8.0f;                       // log2 units
 
 static_assert(kSmemAlloc <= 232448, "shared memory beyond the 227 KB per-CTA limit");
@@ -98,7 +109,7 @@ static_assert(kTmemO + 256 <= kTmemCols, "S buffers and O exceed the TMEM alloca
 static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
               "128-byte swizzle needs 1 KB alignment");
 
-constexpr uint32_t kIdescQK = idesc_f16_f32(128, 128, 0, 0);    // K-major A and B
+constexpr uint32_t kIdescQK = idesc_f16_f32(128, 256, 0, 0);    // K-major A and B
 constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);    // B (V) MN-major
 
 struct Bars {
@@ -158,7 +169,9 @@ template <int kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThreads, 1)
     mla_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ Plan plan,
+                   const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_o,
+                   const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ Plan plan,
                    const __grid_constant__ MlaFwdParams p) {
   using namespace fwd;
   constexpr bool kManual = FwdCfg<kMode>::kManual;
@@ -244,14 +257,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       int stage = 0;
       uint32_t ephase = 0;
       for (int i = 0; i < n_tiles; ++i) {
-        const int key0 = (tile_begin + i) * kTileKeys + 64 * (int)rank;
+        const int key0 = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
         for (int c = 0; c < 9; ++c) {
           if (!failed && !mbar_wait(&bars.k_empty[stage], ephase ^ 1, to)) {
             failed = true;
             record_status(kStatusTimeout);
           }
-          if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kChunkBytes);
-          tma_load_3d_2sm(sK + stage * kChunkBytes, &tm_k,
+          if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kKChunkBytes);
+          tma_load_3d_2sm(sK + stage * kKChunkBytes, &tm_k,
                           mapa_shared(smem_u32(&bars.k_full[stage]), 0), 64 * c, key0, b_abs);
           if (++stage == kKStages) { stage = 0; ephase ^= 1; }
         }
@@ -265,110 +278,107 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       uint32_t ephase = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int key0 = (tile_begin + j) * kTileKeys;
-        for (int kb = 0; kb < 4; ++kb)
+        for (int kg = 0; kg < kTileKeys / 64; ++kg)
           for (int nb = 0; nb < 2; ++nb) {
             if (!failed && !mbar_wait(&bars.v_empty[stage], ephase ^ 1, to)) {
               failed = true;
               record_status(kStatusTimeout);
             }
-            if (rank == 0) mbar_arrive_expect_tx(&bars.v_full[stage], 2 * kChunkBytes);
-            const int col = 256 * nb + 128 * (int)rank;
+            if (rank == 0) mbar_arrive_expect_tx(&bars.v_full[stage], 2 * kVStageBytes);
+            // one 16 KB box: 64 keys x 2 column blocks of 64 (this CTA's 128 value columns
+            // of value half nb), landing as [column block][key][64 columns]
             const uint32_t fl = mapa_shared(smem_u32(&bars.v_full[stage]), 0);
-            tma_load_3d_2sm(sV + stage * kChunkBytes, &tm_v, fl, col, key0 + 32 * kb, b_abs);
-            tma_load_3d_2sm(sV + stage * kChunkBytes + 4096, &tm_v, fl, col + 64, key0 + 32 * kb,
-                            b_abs);
+            tma_load_4d_2sm(sV + stage * kVStageBytes, &tm_v, fl, 0, key0 + 64 * kg,
+                            4 * nb + 2 * (int)rank, b_abs);
             if (++stage == kVStages) { stage = 0; ephase ^= 1; }
           }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ================= MMA issuer (leader CTA, one thread): a polling scheduler.
-    // Each step issues whatever is ready: the next P.V chunk (needs P of its tile
-    // and the V stage) first, then the next Q.K^T chunk (needs the K stage, and for
-    // a new tile a free S buffer: the softmax of the tile kSBufs earlier has
-    // published its P). Both rings are consumed in their own FIFO order.
+    // ================= Q.K^T issuer (leader CTA, one thread). Two threads issue MMAs:
+    // an issuing thread cannot run ahead of the tensor pipe, so the time it spends
+    // waiting on a barrier would leave the pipe idle; with Q.K^T and P.V on separate
+    // threads one thread's wait is covered by the other's MMAs. A commit tracks the
+    // MMAs of the thread that issues it.
     if (rank == 0 && n_tiles > 0 && elect_one()) {
       // Descriptor bases; an operand at byte offset `off` within a region is the base
       // plus off/16 (the start address field is the low 14 bits, no carry possible
-      // below 256 KB). Everything per MMA below is a 64-bit add of a constant.
+      // below 256 KB).
       const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dk = smem_desc_sw128(smem_u32(sK), 16, 1024);
-      const uint64_t dv = smem_desc_sw128(smem_u32(sV), 4096, 1024);
-      const uint64_t dp = smem_desc_sw128(smem_u32(sP), 16, 1024);
-      constexpr uint32_t kStageUnits = kChunkBytes >> 4;
+      constexpr uint32_t kQUnits = kChunkBytes >> 4;    // Q chunk stride
+      constexpr uint32_t kKUnits = kKChunkBytes >> 4;   // K stage stride
       if (!mbar_wait(&bars.q_full, 0, to)) {
         failed = true;
         record_status(kStatusTimeout);
       }
-      tc_fence_after();
-      int kst = 0, vst = 0;
-      uint32_t kph = 0, vph = 0;
-      int qk_t = 0, qk_c = 0;  // next Q.K^T tile / 64-column chunk
-      int pv_t = 0, pv_c = 0;  // next P.V tile / (32-key, 256-column) chunk
-      bool p_ok = false;       // P of tile pv_t observed (with cluster-scope acquire)
-      uint64_t idle_since = 0;
-      // Cheap CTA-scope probes; a phase completed by arrivals from the peer CTA is
-      // then acquired once at cluster scope before its data is used.
-      auto ready = [&](uint64_t* bar, uint32_t parity, bool remote) -> bool {
-        if (failed) return true;
-        if (!mbar_test(bar, parity)) return false;
-        if (remote) (void)mbar_test_cluster(bar, parity);
-        return true;
-      };
-      while (pv_t < n_tiles) {
-        bool progressed = false;
-        if (!p_ok) p_ok = ready(&bars.p_full[pv_t & 1], (pv_t >> 1) & 1, true);
-        if (p_ok && ready(&bars.v_full[vst], vph, kManual)) {
-          tc_fence_after();
-          const int kb = pv_c >> 1, nb = pv_c & 1;
-          const uint64_t a0 = dp + (uint32_t)((pv_t & 1) * (kPBufBytes >> 4) + (kb >> 1) * kStageUnits +
-                                              (kb & 1) * 4);
-          const uint64_t b0 = dv + (uint32_t)(vst * kStageUnits);
-          const uint32_t d = tmem + kTmemO + nb * 128;
-          mma_f16_ss_2sm(d, a0, b0, kIdescPV, (pv_t > 0 || kb > 0) ? 1u : 0u);
-          mma_f16_ss_2sm(d, a0 + 2, b0 + 128, kIdescPV, 1u);
-          mma_commit_2sm_mc(&bars.v_empty[vst], 0x3);
-          if (++vst == kVStages) { vst = 0; vph ^= 1; }
-          if (++pv_c == 8) {
-            mma_commit_2sm_mc(&bars.o_done[pv_t & 1], 0x3);
-            pv_c = 0;
-            ++pv_t;
-            p_ok = false;
-          }
-          progressed = true;
+      int kst = 0;
+      uint32_t kph = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        // S buffer t % kSBufs is free once the softmax of tile t - kSBufs published its P
+        if (t >= kSBufs && !failed &&
+            !mbar_wait_cluster(&bars.p_full[(t - kSBufs) & 1], ((t - kSBufs) >> 1) & 1, to)) {
+          failed = true;
+          record_status(kStatusTimeout);
         }
-        const int pv_seen = pv_t + (p_ok ? 1 : 0);
-        if (qk_t < n_tiles && (qk_c > 0 || qk_t < pv_seen + kSBufs) &&
-            ready(&bars.k_full[kst], kph, kManual)) {
-          const uint32_t d_s = tmem + (qk_t % kSBufs) * 64;
-          const uint64_t a0 = dq + (uint32_t)(qk_c * kStageUnits);
-          const uint64_t b0 = dk + (uint32_t)(kst * kStageUnits);
-          const uint32_t acc0 = qk_c ? 1u : 0u;
-          mma_f16_ss_2sm(d_s, a0, b0, kIdescQK, acc0);
+        const uint32_t d_s = tmem + (t % kSBufs) * kSCols;
+        for (int c = 0; c < 9; ++c) {
+          const bool ok = kManual ? mbar_wait_cluster(&bars.k_full[kst], kph, to)
+                                  : mbar_wait(&bars.k_full[kst], kph, to);
+          if (!failed && !ok) {
+            failed = true;
+            record_status(kStatusTimeout);
+          }
+          tc_fence_after();
+          const uint64_t a0 = dq + (uint32_t)(c * kQUnits);
+          const uint64_t b0 = dk + (uint32_t)(kst * kKUnits);
+          mma_f16_ss_2sm(d_s, a0, b0, kIdescQK, c ? 1u : 0u);
           mma_f16_ss_2sm(d_s, a0 + 2, b0 + 2, kIdescQK, 1u);
           mma_f16_ss_2sm(d_s, a0 + 4, b0 + 4, kIdescQK, 1u);
           mma_f16_ss_2sm(d_s, a0 + 6, b0 + 6, kIdescQK, 1u);
           mma_commit_2sm_mc(&bars.k_empty[kst], 0x3);
           if (++kst == kKStages) { kst = 0; kph ^= 1; }
-          if (++qk_c == 9) {
-            mma_commit_2sm_mc(&bars.s_full[qk_t % kSBufs], 0x3);
-            qk_c = 0;
-            ++qk_t;
-          }
-          progressed = true;
         }
-        if (progressed) {
-          idle_since = 0;
-        } else if (!failed) {
-          const uint64_t now = globaltimer_ns();
-          if (idle_since == 0) {
-            idle_since = now;
-          } else if (now - idle_since > to) {
-            failed = true;
-            record_status(kStatusTimeout);
-          }
+        mma_commit_2sm_mc(&bars.s_full[t % kSBufs], 0x3);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ================= P.V issuer (leader CTA, one thread): per tile, wait for P, then
+    // consume the V stages (64 keys x one 256-column half each) in the producer's order.
+    if (rank == 0 && n_tiles > 0 && elect_one()) {
+      const uint64_t dv = smem_desc_sw128(smem_u32(sV), 8192, 1024);
+      const uint64_t dp = smem_desc_sw128(smem_u32(sP), 16, 1024);
+      constexpr uint32_t kPUnits = kChunkBytes >> 4;    // P block (64 keys) stride
+      constexpr uint32_t kVUnits = kVStageBytes >> 4;   // V stage stride
+      int vst = 0;
+      uint32_t vph = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        if (!failed && !mbar_wait_cluster(&bars.p_full[t & 1], (t >> 1) & 1, to)) {
+          failed = true;
+          record_status(kStatusTimeout);
         }
+        for (int kg = 0; kg < kTileKeys / 64; ++kg)
+          for (int nb = 0; nb < 2; ++nb) {
+            const bool ok = kManual ? mbar_wait_cluster(&bars.v_full[vst], vph, to)
+                                    : mbar_wait(&bars.v_full[vst], vph, to);
+            if (!failed && !ok) {
+              failed = true;
+              record_status(kStatusTimeout);
+            }
+            tc_fence_after();
+            const uint64_t a0 = dp + (uint32_t)(kg * kPUnits);
+            const uint64_t b0 = dv + (uint32_t)(vst * kVUnits);
+            const uint32_t d = tmem + kTmemO + nb * 128;
+            mma_f16_ss_2sm(d, a0, b0, kIdescPV, (t > 0 || kg > 0) ? 1u : 0u);
+            mma_f16_ss_2sm(d, a0 + 2, b0 + 128, kIdescPV, 1u);
+            mma_f16_ss_2sm(d, a0 + 4, b0 + 256, kIdescPV, 1u);
+            mma_f16_ss_2sm(d, a0 + 6, b0 + 384, kIdescPV, 1u);
+            mma_commit_2sm_mc(&bars.v_empty[vst], 0x3);
+            if (++vst == kVStages) { vst = 0; vph ^= 1; }
+          }
+        mma_commit_2sm_mc(&bars.o_done[t & 1], 0x3);
       }
     }
     __syncwarp();
@@ -436,36 +446,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         if (++stage == n_stages) { stage = 0; ephase ^= 1; }
       };
       if (k_side) {
-        // K chunk items: 64 keys (this CTA's half of the tile) x 2 blocks of 32 columns
+        // K chunk items: 128 keys (this CTA's half of the tile) x 2 blocks of 32 columns;
+        // thread pt takes keys pt/2 + 32q (q = 0..3) and block half pt%2
         for (int i = 0; i < n_tiles; ++i) {
-          const int kbase = (tile_begin + i) * kTileKeys + 64 * (int)rank;
-          const int key_a = resolve(kbase + (pt >> 1));
-          const int key_b = resolve(kbase + 32 + (pt >> 1));
+          const int kbase = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
           const int half = pt & 1;
+          int keys[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) keys[q] = resolve(kbase + 32 * q + (pt >> 1));
           for (int c = 0; c < 9; ++c) {
             acquire();
-            fill32(ring + stage * kChunkBytes + (pt >> 1) * 128, pt >> 1, key_a, 2 * c + half,
-                   4 * half);
-            fill32(ring + stage * kChunkBytes + (32 + (pt >> 1)) * 128, 32 + (pt >> 1), key_b,
-                   2 * c + half, 4 * half);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int kl = 32 * q + (pt >> 1);
+              fill32(ring + stage * kKChunkBytes + kl * 128, kl, keys[q], 2 * c + half, 4 * half);
+            }
             publish();
           }
         }
       } else {
-        // V chunk items: 32 keys x this CTA's 128 value columns (4 blocks, two boxes)
+        // V stage items: 64 keys x this CTA's 128 value columns of one value half (4
+        // blocks of 32 in two 64-column boxes); thread pt takes keys pt/4 + 16q and
+        // 32-column block pt%4
         const int q4 = pt & 3, box = q4 >> 1, half = q4 & 1;
         for (int j = 0; j < n_tiles; ++j) {
           const int kbase = (tile_begin + j) * kTileKeys;
-          for (int kb = 0; kb < 4; ++kb) {
-            const int kl_a = pt >> 2, kl_b = 16 + (pt >> 2);
-            const int key_a = resolve(kbase + 32 * kb + kl_a);
-            const int key_b = resolve(kbase + 32 * kb + kl_b);
+          for (int kg = 0; kg < kTileKeys / 64; ++kg) {
+            int keys[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) keys[q] = resolve(kbase + 64 * kg + (pt >> 2) + 16 * q);
             for (int nb = 0; nb < 2; ++nb) {
               acquire();
               const int col32 = 8 * nb + 4 * (int)rank + q4;
-              uint8_t* st = ring + stage * kChunkBytes + box * 4096;
-              fill32(st + kl_a * 128, kl_a, key_a, col32, 4 * half);
-              fill32(st + kl_b * 128, kl_b, key_b, col32, 4 * half);
+              uint8_t* st = ring + stage * kVStageBytes + box * 8192;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int kl = (pt >> 2) + 16 * q;
+                fill32(st + kl * 128, kl, keys[q], col32, 4 * half);
+              }
               publish();
             }
           }
@@ -501,70 +519,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     float l_part = 0.f;       // this lane's half of the row sum, relative to m_ref
 
     for (int i = 0; i < n_tiles; ++i) {
-      const int sb = i & 1;          // P buffer and max-exchange slot
+      const int sb = i & 1;          // max-exchange slot and p_full barrier
       const int sbuf = i % kSBufs;   // S buffer in TMEM
-      const int key0 = (tile_begin + i) * kTileKeys + 64 * kh;
-      const bool full_range = key0 + 64 <= key_end;
+      constexpr int kHalf = kTileKeys / 2;  // keys of one lane (128)
+      const int key0 = (tile_begin + i) * kTileKeys + kHalf * kh;
+      const bool full_range = key0 + kHalf <= key_end;
       // issue this tile's mask loads before waiting for S, to hide their latency
       const bool vec_mask = !(kManual && sparse) && mrow != nullptr && full_range && p.mask_vec_ok;
-      uint4 mvec[8];
+      uint4 mvec[kHalf / 8];
       if (vec_mask) {
         const uint4* mv = reinterpret_cast<const uint4*>(mrow + key0);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mvec[c] = __ldg(mv + c);
+        for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
       }
       wait_local(&bars.s_full[sbuf], (i / kSBufs) & 1);
       tc_fence_after();
-      uint32_t sr[64];
-      {
-        uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tmem_ld32(tmem + lane_base + sbuf * 64, a);
-        tmem_ld32(tmem + lane_base + sbuf * 64 + 32, c);
+      // scores in log2 units (scale folded in, mask added); cells beyond the unit's keys
+      // are dropped. 128 values per lane, read from TMEM in 4 x 32 columns.
+      float x[kHalf];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(tmem + lane_base + sbuf * kSCols + 32 * q, sr);
         tmem_wait_ld();
-      }
-      // scores in log2 units; cells beyond the unit's keys are dropped
-      float x[64];
-      if (kManual && sparse) {
-        const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
+        if (kManual && sparse) {
+          const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int pos = key0 + j;
-          float mv = 0.f;
-          bool ok = pos < key_end;
-          if (ok) {
-            const int cell = __ldg(ix + pos);
-            ok = cell >= 0 && cell < p.n_kv;
-            if (ok && mrow != nullptr) mv = __half2float(__ushort_as_half(__ldg(mrow + cell)));
+          for (int j = 0; j < 32; ++j) {
+            const int pos = key0 + 32 * q + j;
+            float mv = 0.f;
+            bool ok = pos < key_end;
+            if (ok) {
+              const int cell = __ldg(ix + pos);
+              ok = cell >= 0 && cell < p.n_kv;
+              if (ok && mrow != nullptr) mv = __half2float(__ushort_as_half(__ldg(mrow + cell)));
+            }
+            x[32 * q + j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
           }
-          x[j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
-        }
-      } else if (vec_mask) {
+        } else if (vec_mask) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = mvec[c];
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          for (int c = 0; c < 4; ++c) {
+            const uint4 v = mvec[4 * q + c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
-            x[8 * c + 2 * h] = fmaf(__uint_as_float(sr[8 * c + 2 * h]), p.scale_log2, f.x * kLog2e);
-            x[8 * c + 2 * h + 1] =
-                fmaf(__uint_as_float(sr[8 * c + 2 * h + 1]), p.scale_log2, f.y * kLog2e);
+            for (int h = 0; h < 4; ++h) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
+              const int j = 8 * c + 2 * h;
+              x[32 * q + j] = fmaf(__uint_as_float(sr[j]), p.scale_log2, f.x * kLog2e);
+              x[32 * q + j + 1] = fmaf(__uint_as_float(sr[j + 1]), p.scale_log2, f.y * kLog2e);
+            }
           }
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int key = key0 + j;
-          float mv = 0.f;
-          if (mrow != nullptr && key < key_end)
-            mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
-          x[j] = key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
+          for (int j = 0; j < 32; ++j) {
+            const int key = key0 + 32 * q + j;
+            float mv = 0.f;
+            if (mrow != nullptr && key < key_end)
+              mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
+            x[32 * q + j] =
+                key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
+          }
         }
       }
       float mt = x[0];
 #pragma unroll
-      for (int j = 1; j < 64; ++j) mt = fmaxf(mt, x[j]);
+      for (int j = 1; j < kHalf; ++j) mt = fmaxf(mt, x[j]);
       xmax[sb * 128 + L] = mt;
       named_bar_sync(1, 128);
       mt = fmaxf(mt, xmax[sb * 128 + (L ^ 64)]);
@@ -576,31 +595,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         m_ref = mt;
       }
       const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint32_t pk[32];
+      uint32_t pk[kHalf / 2];
       float lsum = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < kHalf / 2; ++j) {
         __half2 h2 = __floats2half2_rn(ex2_approx(x[2 * j] - mref_use),
                                        ex2_approx(x[2 * j + 1] - mref_use));
         pk[j] = *reinterpret_cast<uint32_t*>(&h2);
-        float2 f2 = __half22float2(h2);
+        const float2 f2 = __half22float2(h2);
         lsum += f2.x + f2.y;
       }
       l_part = l_part * alpha + lsum;
 
-      // P buffer sb is free once P.V of tile i-2 has completed
-      if (i >= 2) wait_local(&bars.o_done[sb], ((i - 2) >> 1) & 1);
+      // The single P buffer (and O, for a rescale) are free once P.V(i-1) has completed.
+      if (i >= 1) wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
       {
-        uint8_t* base = sP + sb * kPBufBytes + kh * kChunkBytes + r * 128;
+        // this lane's 128 keys are P blocks 2*kh and 2*kh+1 (64 keys each) of row r
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          *reinterpret_cast<uint4*>(base + ((c ^ (r & 7)) << 4)) = v;
+        for (int blk = 0; blk < 2; ++blk) {
+          uint8_t* base = sP + (2 * kh + blk) * kChunkBytes + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const int w = 32 * blk + 4 * c;
+            *reinterpret_cast<uint4*>(base + ((c ^ (r & 7)) << 4)) =
+                make_uint4(pk[w], pk[w + 1], pk[w + 2], pk[w + 3]);
+          }
         }
       }
       // rescale O (only when some row of this warp raised its reference max)
       if (__any_sync(0xffffffffu, need && i > 0)) {
-        wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
@@ -628,13 +651,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     const float l_tot = l_part + xl[L ^ 64];
     const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
     const int ws_slot = plan.ws_base[b] >= 0 ? plan.ws_base[b] + g * n_split + s : -1;
-    float* dst = nullptr;
-    if (ws_slot < 0)
-      dst = p.out + (int64_t)b_abs * p.out_seq_stride + (int64_t)row * kDV;
-    else
-      dst = p.ws_o + ((int64_t)ws_slot * kRowsPerGroup + kRowsPerCta * rank + r) * kDV;
-    for (int nb = 0; nb < 2; ++nb)
-      for (int cc = 0; cc < 4; ++cc) {
+    // O / l goes out through shared memory: each warp stages its 32 rows as eight
+    // 32 x 32 fp32 boxes (128-byte rows, 16-byte chunks XOR-swizzled by row, the
+    // layout of a 128-byte-swizzle tensor map) and one lane stores them with TMA.
+    // Every MMA has finished (last o_done), so the operand rings are free; the 4
+    // warps use the first 128 KB. Rows beyond the tensor are clipped by the store.
+    {
+      const int wq = warp - 4;  // row half (wq & 1) of key half kh = wq >> 1
+      uint8_t* wbox = smem + wq * 8 * 4096;
+#pragma unroll 1
+      for (int i = 0; i < 8; ++i) {
+        const int nb = i >> 2, cc = i & 3;
         uint32_t v[32];
         if (n_tiles > 0) {
           tmem_ld32(tmem + lane_base + kTmemO + nb * 128 + cc * 32, v);
@@ -643,16 +670,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = 0u;
         }
-        if (row_valid) {
-          float4* o4 = reinterpret_cast<float4*>(dst + 256 * nb + 128 * kh + 32 * cc);
+        uint8_t* rowp = wbox + i * 4096 + lane * 128;
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            o4[q4] = make_float4(__uint_as_float(v[4 * q4]) * inv_l,
-                                 __uint_as_float(v[4 * q4 + 1]) * inv_l,
-                                 __uint_as_float(v[4 * q4 + 2]) * inv_l,
-                                 __uint_as_float(v[4 * q4 + 3]) * inv_l);
-        }
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+              make_float4(__uint_as_float(v[4 * c]) * inv_l, __uint_as_float(v[4 * c + 1]) * inv_l,
+                          __uint_as_float(v[4 * c + 2]) * inv_l,
+                          __uint_as_float(v[4 * c + 3]) * inv_l);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const CUtensorMap* tm = ws_slot >= 0 ? &tm_w : &tm_o;
+        const int y = (ws_slot >= 0 ? ws_slot * kRowsPerGroup : row0) + kRowsPerCta * (int)rank +
+                      32 * (wq & 1);
+        const int z = ws_slot >= 0 ? 0 : b_abs;
+        for (int i = 0; i < 8; ++i)
+          tma_store_3d(tm, wbox + i * 4096, 256 * (i >> 2) + 128 * kh + 32 * (i & 3), y, z);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+      __syncwarp();
+    }
     if (ws_slot >= 0 && kh == 0 && row_valid)
       p.ws_lse[(int64_t)ws_slot * kRowsPerGroup + kRowsPerCta * rank + r] =
           l_tot > 0.f ? m_ref + __log2f(l_tot) : -INFINITY;
