@@ -335,10 +335,12 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   p.mask_seq_stride = r.m_ss;
   p.mask_row_stride = r.m_rs;
   p.out_seq_stride = r.o_ss;
-  p.scale_log2 = a.scale * mla::kLog2e;
+  p.scale = a.scale;
   p.mask_vec_ok = (a.mask != nullptr && aligned16(a.mask) && (r.m_ss % 8) == 0 && (r.m_rs % 8) == 0);
   p.timeout_ns = kDefaultTimeoutNs;
   p.kcache = static_cast<const uint8_t*>(a.kcache);
+  p.q = static_cast<const uint16_t*>(a.q);
+  p.q_seq_stride = r.q_ss;
   p.k_seq_stride = r.k_ss;
   p.n_kv = a.n_kv;
   p.idx = a.idx;
@@ -377,12 +379,25 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     }
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     if (slots > 0) {
-      dim3 cgrid((r.rows + 3) / 4, n);
+      // one CTA per query row, launched as a programmatic dependent of the forward
+      // kernel so that its launch overlaps the forward's last CTAs
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(r.rows, n);
+      cfg.blockDim = dim3(128);
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      cudaError_t ce;
       {
         ProfScope prof(kKernCombine, stream);
-        mla::mla_combine_kernel<<<cgrid, 128, 0, stream>>>(plan, p.ws_o, p.ws_lse, a.out, r.o_ss);
+        ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const float*)p.ws_o,
+                                (const float*)p.ws_lse, a.out, (int64_t)r.o_ss);
       }
-      if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+      if (ce != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }
   }
   return MLA_OK;

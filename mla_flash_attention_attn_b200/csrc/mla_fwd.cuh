@@ -29,8 +29,8 @@
 //  * Softmax warpgroup: thread = TMEM lane; the two lanes of a row exchange
 //    their tile maximum through shared memory. The reference max is raised
 //    only when a tile's max exceeds it by more than 2^8, so O is rescaled in
-//    TMEM rarely; P (f16, <= 256) goes to one shared-memory buffer as the A
-//    operand, written once P.V of the previous tile has finished.
+//    TMEM rarely; P (f16, <= 256) goes to one of two shared-memory buffers as
+//    the A operand, written once P.V of the tile two earlier has finished.
 //  * Epilogue: O / l is staged in shared memory and written by TMA stores.
 //
 // Every mbarrier wait is bounded (MlaFwdParams::timeout_ns). On a timeout the
@@ -58,13 +58,16 @@ struct MlaFwdParams {
   int64_t mask_seq_stride;   // elements
   int64_t mask_row_stride;   // elements
   int64_t out_seq_stride;    // elements
-  float scale_log2;          // scale * log2(e)
+  float scale;               // softmax scale (natural units)
   int mask_vec_ok;           // mask rows allow 16-byte loads
   uint64_t timeout_ns;
   // cache rows read by the gather / dequant producer (modes other than TMA)
   const uint8_t* kcache;     // row (b, j) at (b*k_seq_stride + j) * row_bytes
   int64_t k_seq_stride;      // rows
   int n_kv;
+  // query rows read by the manual producers: row r of sequence b at q + b*q_seq_stride + r*576
+  const uint16_t* q;
+  int64_t q_seq_stride;      // elements
   // sparse: sequence b attends to rows idx[b*idx_seq_stride + i], i < idx_count[b]
   const int32_t* idx;
   const int32_t* idx_count;
@@ -80,21 +83,24 @@ enum FwdMode {
 
 namespace fwd {
 
-constexpr int kKStages = 3;      // ring of Q.K^T operand stages (K rows)
+constexpr int kKStages = 4;      // ring of Q.K^T operand stages (K chunk + Q chunk)
 constexpr int kVStages = 4;      // ring of P.V operand stages (V columns, L2-resident)
 constexpr int kSBufs = 2;        // S buffers in TMEM (128 columns each)
 constexpr int kSCols = 128;      // TMEM columns of one S buffer
 constexpr int kChunkBytes = 8192;                 // 64 rows x 64 f16 (one swizzle tile)
-constexpr int kKChunkBytes = 2 * kChunkBytes;     // K stage: 128 keys x 64 columns
+constexpr int kKChunkBytes = 2 * kChunkBytes;     // 128 keys x 64 columns
+// A Q.K^T stage holds a K chunk and the matching 64-column chunk of this CTA's 64
+// query rows: Q is re-read from L2 with every tile rather than kept resident, which
+// leaves room for more K stages in flight (the K stream comes from DRAM).
+constexpr int kKStageBytes = kKChunkBytes + kChunkBytes;
 constexpr int kVStageBytes = 2 * kChunkBytes;     // V stage: 64 keys x 128 value columns
-constexpr int kQBytes = 9 * kChunkBytes;          // 64 rows x 576 f16
 constexpr int kPBufBytes = 4 * kChunkBytes;       // 64 rows x 256 keys f16
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKStages * kKChunkBytes;
+constexpr int kPBufs = 2;        // P buffers: tile i uses buffer i % 2
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kKStages * kKStageBytes;
 constexpr int kOffP = kOffV + kVStages * kVStageBytes;
-constexpr int kOffBar = kOffP + kPBufBytes;
-constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 1 + kSBufs + 2 + 2;
+constexpr int kOffBar = kOffP + kPBufs * kPBufBytes;
+constexpr int kNumBars = 2 * kKStages + 2 * kVStages + kSBufs + 2 + 2;
 constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
 constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
 constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
@@ -102,7 +108,7 @@ constexpr int kSmemBytes = kOffXl + 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;                   // 1024-byte alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = kSBufs * kSCols;                    // O columns start
-constexpr float kRescaleThreshold = 8.0f;                       // log2 units
+constexpr float kRescaleThreshold = 5.5451774f;                 // 8 ln 2 (natural units)
 
 static_assert(kSmemAlloc <= 232448, "shared memory beyond the 227 KB per-CTA limit");
 static_assert(kTmemO + 256 <= kTmemCols, "S buffers and O exceed the TMEM allocation");
@@ -113,11 +119,10 @@ constexpr uint32_t kIdescQK = idesc_f16_f32(128, 256, 0, 0);    // K-major A and
 constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);    // B (V) MN-major
 
 struct Bars {
-  uint64_t k_full[kKStages];     // leader: both CTAs' K chunk bytes landed
-  uint64_t k_empty[kKStages];    // both: the Q.K^T MMAs reading a K stage are done
+  uint64_t k_full[kKStages];     // leader: both CTAs' K and Q chunk bytes landed
+  uint64_t k_empty[kKStages];    // both: the Q.K^T MMAs reading a stage are done
   uint64_t v_full[kVStages];     // leader: both CTAs' V chunk bytes landed
   uint64_t v_empty[kVStages];    // both: the P.V MMAs reading a V stage are done
-  uint64_t q_full;               // leader: Q of both CTAs loaded
   uint64_t s_full[kSBufs];       // both: S buffer written by Q.K^T
   uint64_t p_full[2];            // leader: P written (8 warp arrivals, both CTAs)
   uint64_t o_done[2];            // both: P.V of a tile (parity-indexed) complete
@@ -178,7 +183,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem + kOffQ;
   uint8_t* sK = smem + kOffK;
   uint8_t* sV = smem + kOffV;
   uint8_t* sP = smem + kOffP;
@@ -217,7 +221,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       mbar_init(&bars.v_full[i], kManual ? 4 : 1);
       mbar_init(&bars.v_empty[i], 1);
     }
-    mbar_init(&bars.q_full, 1);
     for (int i = 0; i < kSBufs; ++i) mbar_init(&bars.s_full[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.p_full[i], 8);
@@ -240,20 +243,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   bool failed = false;
 
   if constexpr (kManual) {
-    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;");
+    // registers per thread: warps 0-3 (TMA, MMA issuers) 112, producers 128, softmax
+    // 256; 4 warps x 32 x (112 + 128 + 256) = 63488 of the 384 x 168 = 64512 launched
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
   }
   if (warp == 0) {
-    // ================= producer: TMA loads of Q, then (TMA mode) K and V chunks
-    if (n_tiles > 0 && elect_one()) {
-      const uint32_t q_full_l = mapa_shared(smem_u32(&bars.q_full), 0);
-      if (rank == 0) mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
-      for (int c = 0; c < 9; ++c)
-        tma_load_3d_2sm(sQ + c * kChunkBytes, &tm_q, q_full_l, 64 * c,
-                        row0 + kRowsPerCta * (int)rank, b_abs);
-    }
+    // ================= producer (TMA mode): K chunks with their Q chunks
     if (!kManual && n_tiles > 0 && elect_one()) {
-      // K ring: this CTA's 64 keys of each tile, 9 chunks of 64 columns, as far
-      // ahead as the ring allows (only Q.K^T consumption frees K stages)
+      // this CTA's 128 keys of each tile, 9 chunks of 64 columns, as far ahead as the
+      // ring allows (only Q.K^T consumption frees stages); each stage also gets the
+      // same 64 columns of this CTA's 64 query rows
       int stage = 0;
       uint32_t ephase = 0;
       for (int i = 0; i < n_tiles; ++i) {
@@ -263,9 +262,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             failed = true;
             record_status(kStatusTimeout);
           }
-          if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kKChunkBytes);
-          tma_load_3d_2sm(sK + stage * kKChunkBytes, &tm_k,
-                          mapa_shared(smem_u32(&bars.k_full[stage]), 0), 64 * c, key0, b_abs);
+          if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kKStageBytes);
+          const uint32_t fl = mapa_shared(smem_u32(&bars.k_full[stage]), 0);
+          uint8_t* st = sK + stage * kKStageBytes;
+          tma_load_3d_2sm(st, &tm_k, fl, 64 * c, key0, b_abs);
+          tma_load_3d_2sm(st + kKChunkBytes, &tm_q, fl, 64 * c, row0 + kRowsPerCta * (int)rank,
+                          b_abs);
           if (++stage == kKStages) { stage = 0; ephase ^= 1; }
         }
       }
@@ -305,14 +307,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       // Descriptor bases; an operand at byte offset `off` within a region is the base
       // plus off/16 (the start address field is the low 14 bits, no carry possible
       // below 256 KB).
-      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t dk = smem_desc_sw128(smem_u32(sK), 16, 1024);
-      constexpr uint32_t kQUnits = kChunkBytes >> 4;    // Q chunk stride
-      constexpr uint32_t kKUnits = kKChunkBytes >> 4;   // K stage stride
-      if (!mbar_wait(&bars.q_full, 0, to)) {
-        failed = true;
-        record_status(kStatusTimeout);
-      }
+      constexpr uint32_t kStageUnits = kKStageBytes >> 4;  // stage stride
+      constexpr uint32_t kQUnits = kKChunkBytes >> 4;      // Q chunk within a stage
       int kst = 0;
       uint32_t kph = 0;
       for (int t = 0; t < n_tiles; ++t) {
@@ -331,8 +328,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             record_status(kStatusTimeout);
           }
           tc_fence_after();
-          const uint64_t a0 = dq + (uint32_t)(c * kQUnits);
-          const uint64_t b0 = dk + (uint32_t)(kst * kKUnits);
+          const uint64_t b0 = dk + (uint32_t)(kst * kStageUnits);
+          const uint64_t a0 = b0 + kQUnits;
           mma_f16_ss_2sm(d_s, a0, b0, kIdescQK, c ? 1u : 0u);
           mma_f16_ss_2sm(d_s, a0 + 2, b0 + 2, kIdescQK, 1u);
           mma_f16_ss_2sm(d_s, a0 + 4, b0 + 4, kIdescQK, 1u);
@@ -351,6 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       const uint64_t dv = smem_desc_sw128(smem_u32(sV), 8192, 1024);
       const uint64_t dp = smem_desc_sw128(smem_u32(sP), 16, 1024);
       constexpr uint32_t kPUnits = kChunkBytes >> 4;    // P block (64 keys) stride
+      constexpr uint32_t kPBufUnits = kPBufBytes >> 4;  // P buffer stride
       constexpr uint32_t kVUnits = kVStageBytes >> 4;   // V stage stride
       int vst = 0;
       uint32_t vph = 0;
@@ -368,7 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               record_status(kStatusTimeout);
             }
             tc_fence_after();
-            const uint64_t a0 = dp + (uint32_t)(kg * kPUnits);
+            const uint64_t a0 = dp + (uint32_t)((t & 1) * kPBufUnits + kg * kPUnits);
             const uint64_t b0 = dv + (uint32_t)(vst * kVUnits);
             const uint32_t d = tmem + kTmemO + nb * 128;
             mma_f16_ss_2sm(d, a0, b0, kIdescPV, (t > 0 || kg > 0) ? 1u : 0u);
@@ -384,7 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     __syncwarp();
   } else if (warp >= 8) {
     // ================= gather / dequant producers (manual modes): warps 8-9 fill the
-    // K ring, warps 10-11 the V ring; 64 threads per ring, 2 of a stage's 128 items each
+    // K ring, warps 10-11 the V ring (64 threads per ring)
     if constexpr (kManual) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 128;");
       const bool k_side = warp < 10;
@@ -448,6 +446,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       if (k_side) {
         // K chunk items: 128 keys (this CTA's half of the tile) x 2 blocks of 32 columns;
         // thread pt takes keys pt/2 + 32q (q = 0..3) and block half pt%2
+        const int q_row = row0 + kRowsPerCta * (int)rank + pt;
+        const uint16_t* q_src = p.q + (int64_t)b_abs * p.q_seq_stride + (int64_t)q_row * kDK;
         for (int i = 0; i < n_tiles; ++i) {
           const int kbase = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
           const int half = pt & 1;
@@ -456,10 +456,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           for (int q = 0; q < 4; ++q) keys[q] = resolve(kbase + 32 * q + (pt >> 1));
           for (int c = 0; c < 9; ++c) {
             acquire();
+            uint8_t* st = ring + stage * kKStageBytes;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const int kl = 32 * q + (pt >> 1);
-              fill32(ring + stage * kKChunkBytes + kl * 128, kl, keys[q], 2 * c + half, 4 * half);
+              fill32(st + kl * 128, kl, keys[q], 2 * c + half, 4 * half);
+            }
+            // Q chunk c: thread pt copies the 64 columns of query row pt (rows beyond
+            // the sequence's rows are zero)
+            {
+              uint4 v[8];
+              if (q_row < plan.rows) {
+                const uint4* src = reinterpret_cast<const uint4*>(q_src + 64 * c);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = __ldg(src + k);
+              } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) v[k] = make_uint4(0u, 0u, 0u, 0u);
+              }
+              uint8_t* dq = st + kKChunkBytes + pt * 128;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dq + ((k ^ (pt & 7)) << 4)) = v[k];
             }
             publish();
           }
@@ -515,75 +532,91 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       }
     };
 
-    float m_ref = -INFINITY;  // reference max (log2 units) used for exponentiation
+    float m_ref = -INFINITY;  // reference max (natural units) used for exponentiation
     float l_part = 0.f;       // this lane's half of the row sum, relative to m_ref
+
+    constexpr int kHalf = kTileKeys / 2;  // keys of one lane (128)
+    // The mask loads of a tile are issued while the previous tile is still being
+    // processed (right after its scores are formed), so their latency is hidden.
+    uint4 mvec[kHalf / 8];
+    auto mask_vec_ok = [&](int t) {
+      const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
+      return !(kManual && sparse) && mrow != nullptr && k0 + kHalf <= key_end && p.mask_vec_ok;
+    };
+    auto load_mask = [&](int t) {
+      const uint4* mv =
+          reinterpret_cast<const uint4*>(mrow + (tile_begin + t) * kTileKeys + kHalf * kh);
+#pragma unroll
+      for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
+    };
+    bool vec_next = n_tiles > 0 && mask_vec_ok(0);
+    if (vec_next) load_mask(0);
 
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;          // max-exchange slot and p_full barrier
       const int sbuf = i % kSBufs;   // S buffer in TMEM
-      constexpr int kHalf = kTileKeys / 2;  // keys of one lane (128)
       const int key0 = (tile_begin + i) * kTileKeys + kHalf * kh;
-      const bool full_range = key0 + kHalf <= key_end;
-      // issue this tile's mask loads before waiting for S, to hide their latency
-      const bool vec_mask = !(kManual && sparse) && mrow != nullptr && full_range && p.mask_vec_ok;
-      uint4 mvec[kHalf / 8];
-      if (vec_mask) {
-        const uint4* mv = reinterpret_cast<const uint4*>(mrow + key0);
-#pragma unroll
-        for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
-      }
+      const bool vec_mask = vec_next;
       wait_local(&bars.s_full[sbuf], (i / kSBufs) & 1);
       tc_fence_after();
-      // scores in log2 units (scale folded in, mask added); cells beyond the unit's keys
-      // are dropped. 128 values per lane, read from TMEM in 4 x 32 columns.
+      // scores x = scale * s + mask (natural units); cells beyond the unit's keys are
+      // dropped. 128 values per lane, read from TMEM with 4 loads and one wait.
+      uint32_t sr[kHalf];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        tmem_ld32(tmem + lane_base + sbuf * kSCols + 32 * q,
+                  *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * q));
+      tmem_wait_ld();
       float x[kHalf];
+      if (kManual && sparse) {
+        const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t sr[32];
-        tmem_ld32(tmem + lane_base + sbuf * kSCols + 32 * q, sr);
-        tmem_wait_ld();
-        if (kManual && sparse) {
-          const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int pos = key0 + 32 * q + j;
-            float mv = 0.f;
-            bool ok = pos < key_end;
-            if (ok) {
-              const int cell = __ldg(ix + pos);
-              ok = cell >= 0 && cell < p.n_kv;
-              if (ok && mrow != nullptr) mv = __half2float(__ushort_as_half(__ldg(mrow + cell)));
-            }
-            x[32 * q + j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
+        for (int j = 0; j < kHalf; ++j) {
+          const int pos = key0 + j;
+          float mv = 0.f;
+          bool ok = pos < key_end;
+          if (ok) {
+            const int cell = __ldg(ix + pos);
+            ok = cell >= 0 && cell < p.n_kv;
+            if (ok && mrow != nullptr) mv = __half2float(__ushort_as_half(__ldg(mrow + cell)));
           }
-        } else if (vec_mask) {
+          x[j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
+        }
+      } else if (vec_mask) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 v = mvec[4 * q + c];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        for (int c = 0; c < kHalf / 8; ++c) {
+          const uint4 v = mvec[c];
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
-              const int j = 8 * c + 2 * h;
-              x[32 * q + j] = fmaf(__uint_as_float(sr[j]), p.scale_log2, f.x * kLog2e);
-              x[32 * q + j + 1] = fmaf(__uint_as_float(sr[j + 1]), p.scale_log2, f.y * kLog2e);
-            }
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int key = key0 + 32 * q + j;
-            float mv = 0.f;
-            if (mrow != nullptr && key < key_end)
-              mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
-            x[32 * q + j] =
-                key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale_log2, mv * kLog2e) : -INFINITY;
+          for (int h = 0; h < 4; ++h) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
+            const int j = 8 * c + 2 * h;
+            x[j] = fmaf(__uint_as_float(sr[j]), p.scale, f.x);
+            x[j + 1] = fmaf(__uint_as_float(sr[j + 1]), p.scale, f.y);
           }
         }
-      }
-      float mt = x[0];
+      } else {
 #pragma unroll
-      for (int j = 1; j < kHalf; ++j) mt = fmaxf(mt, x[j]);
+        for (int j = 0; j < kHalf; ++j) {
+          const int key = key0 + j;
+          float mv = 0.f;
+          if (mrow != nullptr && key < key_end)
+            mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
+          x[j] = key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
+        }
+      }
+      // next tile's mask: its loads overlap the rest of this tile
+      vec_next = i + 1 < n_tiles && mask_vec_ok(i + 1);
+      if (vec_next) load_mask(i + 1);
+
+      // row max over this lane's 128 keys (8 independent chains), then over the pair
+      float m8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m8[u] = x[u];
+#pragma unroll
+      for (int j = 8; j < kHalf; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+      float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       xmax[sb * 128 + L] = mt;
       named_bar_sync(1, 128);
       mt = fmaxf(mt, xmax[sb * 128 + (L ^ 64)]);
@@ -591,29 +624,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       const bool need = mt > m_ref + kRescaleThreshold;
       float alpha = 1.f;
       if (need) {
-        alpha = ex2_approx(m_ref - mt);  // 0 when m_ref = -inf
+        alpha = ex2_approx((m_ref - mt) * kLog2e);  // 0 when m_ref = -inf
         m_ref = mt;
       }
-      const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // p = 2^(x log2 e - m_ref log2 e), rounded to f16 for the P.V MMA; the row sum
+      // adds the unrounded values (8 independent chains)
+      const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref * kLog2e;
       uint32_t pk[kHalf / 2];
-      float lsum = 0.f;
+      float ls8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ls8[u] = 0.f;
 #pragma unroll
       for (int j = 0; j < kHalf / 2; ++j) {
-        __half2 h2 = __floats2half2_rn(ex2_approx(x[2 * j] - mref_use),
-                                       ex2_approx(x[2 * j + 1] - mref_use));
+        const float e0 = ex2_approx(fmaf(x[2 * j], kLog2e, nb));
+        const float e1 = ex2_approx(fmaf(x[2 * j + 1], kLog2e, nb));
+        __half2 h2 = __floats2half2_rn(e0, e1);
         pk[j] = *reinterpret_cast<uint32_t*>(&h2);
-        const float2 f2 = __half22float2(h2);
-        lsum += f2.x + f2.y;
+        ls8[j & 7] += e0 + e1;
       }
+      const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       l_part = l_part * alpha + lsum;
 
-      // The single P buffer (and O, for a rescale) are free once P.V(i-1) has completed.
-      if (i >= 1) wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
+      // P buffer i % 2 is free once P.V(i-2) has completed
+      if (i >= 2) wait_local(&bars.o_done[i & 1], ((i - 2) >> 1) & 1);
       {
         // this lane's 128 keys are P blocks 2*kh and 2*kh+1 (64 keys each) of row r
+        uint8_t* pbuf = sP + (i & 1) * kPBufBytes;
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
-          uint8_t* base = sP + (2 * kh + blk) * kChunkBytes + r * 128;
+          uint8_t* base = pbuf + (2 * kh + blk) * kChunkBytes + r * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const int w = 32 * blk + 4 * c;
@@ -622,8 +661,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           }
         }
       }
-      // rescale O (only when some row of this warp raised its reference max)
+      // rescale O (only when some row of this warp raised its reference max), once
+      // P.V(i-1) has completed
       if (__any_sync(0xffffffffu, need && i > 0)) {
+        wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
         tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
@@ -645,6 +686,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 
     // ---- epilogue
     if (n_tiles > 0) wait_local(&bars.o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+    // a dependent (combine) launch may start scheduling; it waits for this grid's end
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_after();
     xl[L] = l_part;
     named_bar_sync(1, 128);
@@ -694,7 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     }
     if (ws_slot >= 0 && kh == 0 && row_valid)
       p.ws_lse[(int64_t)ws_slot * kRowsPerGroup + kRowsPerCta * rank + r] =
-          l_tot > 0.f ? m_ref + __log2f(l_tot) : -INFINITY;
+          l_tot > 0.f ? m_ref * kLog2e + __log2f(l_tot) : -INFINITY;
   }
 
   // ---- teardown
@@ -708,22 +751,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   }
 }
 
-// LSE combine of split-KV partials (one warp per query row):
+// LSE combine of split-KV partials (one CTA of 128 threads per query row, thread t
+// owning value columns 4t..4t+3):
 //   O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
 // where O_s is split s normalised by its own sum and lse_s = log2 of that sum
 // relative to the split's max; splits with no kept cell have lse_s = -inf.
-// Lane s holds the weight of split s (in chunks of 32 splits); the partial
-// rows are then read with independent, unrolled 16-byte loads.
+// Every warp derives the weights itself (lane s holds split s, 32 at a time) and
+// broadcasts them with shuffles; the partial rows are read with independent,
+// unrolled 16-byte loads. Launched as a programmatic dependent of the forward
+// kernel: griddepcontrol.wait returns once the forward grid has completed and its
+// partials are visible.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant__ Plan plan,
                                                           const float* __restrict__ ws_o,
                                                           const float* __restrict__ ws_lse,
                                                           float* __restrict__ out,
                                                           int64_t out_seq_stride) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.y;
-  if (plan.ws_base[b] < 0) return;
+  const int row = blockIdx.x;
+  if (plan.ws_base[b] < 0 || row >= plan.rows) return;
   const int ns = plan.n_split[b];
-  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (row >= plan.rows) return;
   const int lane = threadIdx.x & 31;
   const int g = row / kRowsPerGroup;
   const int rin = row % kRowsPerGroup;
@@ -733,11 +780,12 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)s * kRowsPerGroup));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float4 acc[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (mx != -INFINITY) {
+    float wsum = 0.f;
+    constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
+    const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
+                         threadIdx.x;
     for (int s0 = 0; s0 < ns; s0 += 32) {
       const int s = s0 + lane;
       float wl = 0.f;
@@ -747,35 +795,25 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
       }
       wsum += wl;
       const int cnt = min(32, ns - s0);
-#pragma unroll 4
+      const float4* src = src0 + s0 * kSplitStride4;
+#pragma unroll 8
       for (int j = 0; j < cnt; ++j) {
         const float w = __shfl_sync(0xffffffffu, wl, j);
-        const float4* src = reinterpret_cast<const float4*>(
-            ws_o + ((int64_t)(slot0 + s0 + j) * kRowsPerGroup + rin) * kDV);
-        float4 v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = __ldg(src + lane + 32 * k);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          acc[k].x = fmaf(w, v[k].x, acc[k].x);
-          acc[k].y = fmaf(w, v[k].y, acc[k].y);
-          acc[k].z = fmaf(w, v[k].z, acc[k].z);
-          acc[k].w = fmaf(w, v[k].w, acc[k].w);
-        }
+        const float4 v = __ldg(src + j * kSplitStride4);
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     const float inv = 1.f / wsum;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      acc[k].x *= inv; acc[k].y *= inv; acc[k].z *= inv; acc[k].w *= inv;
-    }
+    acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
   }
   float4* dst = reinterpret_cast<float4*>(out + (int64_t)(plan.seq_offset + b) * out_seq_stride +
                                           (int64_t)row * kDV);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) dst[lane + 32 * k] = acc[k];
+  dst[threadIdx.x] = acc;
 }
 
 // Waits on a barrier that nothing ever signals, with a bounded wait, and records
