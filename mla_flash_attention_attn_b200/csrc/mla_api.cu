@@ -21,7 +21,7 @@ namespace {
 using mla::Plan;
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
-constexpr int kMinTilesPerSplit = 2;
+constexpr int kMinTilesPerSplit = 1;
 
 thread_local cudaStream_t t_stream = nullptr;
 

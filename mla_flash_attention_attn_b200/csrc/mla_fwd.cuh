@@ -155,18 +155,63 @@ struct FwdCfg {
 // 16 half2 words. An int8 q is biased to u = q + 128 and placed in the low
 // mantissa bits of 1024.0 (0x6400), giving exactly 1024 + u; subtracting 1152
 // leaves q exactly, and one f16 multiply by d rounds d*q once.
-__device__ __forceinline__ void dequant_q8_block(const uint8_t* blk, uint32_t (&h)[16]) {
-  const uint16_t dbits = __ldg(reinterpret_cast<const unsigned short*>(blk));
-  const __half2 d2 = __half2half2(__ushort_as_half(dbits));
-  const __half2 bias = __float2half2_rn(1152.f);
-  const unsigned short* qw = reinterpret_cast<const unsigned short*>(blk + 2);
+//
+// A block is 34 bytes at 2-byte alignment (rows are 612 bytes): it is read as the
+// 9 aligned 32-bit words that cover it. An even block starts 4-byte aligned and is
+// never the last block of its row; an odd block starts 2 bytes into its first
+// word; either way the 36 bytes read stay inside the row.
+struct RawBlock {
+  uint32_t w[16];  // f16: the 32 values; q8_0: words 0..8 cover the block
+  bool odd;        // q8_0: the block starts 2 bytes into w[0]
+  bool valid;      // false: zero fill
+};
+
+template <int kMode>
+__device__ __forceinline__ void load_block(const uint8_t* kcache, int64_t row, int col32,
+                                           RawBlock& rb) {
+  if constexpr (kMode == kModeQ8) {
+    const uint8_t* blk = kcache + row * kQ8RowBytes + col32 * 34;
+    const uintptr_t a = reinterpret_cast<uintptr_t>(blk);
+    const uint32_t* w4 = reinterpret_cast<const uint32_t*>(a & ~static_cast<uintptr_t>(3));
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const uint32_t u = (uint32_t)__ldg(qw + k) ^ 0x8080u;
-    const uint32_t w = __byte_perm(u, 0x64646464u, 0x4140);
-    __half2 v = *reinterpret_cast<const __half2*>(&w);
-    v = __hmul2(__hsub2(v, bias), d2);
-    h[k] = *reinterpret_cast<uint32_t*>(&v);
+    for (int i = 0; i < 9; ++i) rb.w[i] = __ldg(w4 + i);
+    rb.odd = (a & 2) != 0;
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(kcache + row * (2 * kDK) + col32 * 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 v = __ldg(src + k);
+      rb.w[4 * k] = v.x; rb.w[4 * k + 1] = v.y; rb.w[4 * k + 2] = v.z; rb.w[4 * k + 3] = v.w;
+    }
+  }
+}
+
+template <int kMode>
+__device__ __forceinline__ void block_values(const RawBlock& rb, uint32_t (&h)[16]) {
+  if (!rb.valid) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) h[k] = 0u;
+    return;
+  }
+  if constexpr (kMode == kModeQ8) {
+    // half-word i of the block (0: d, 1..16: int8 pairs)
+    auto hw = [&](int i) -> uint32_t {
+      return rb.odd ? ((i & 1) ? (rb.w[(i + 1) >> 1] & 0xFFFFu) : (rb.w[i >> 1] >> 16))
+                    : ((i & 1) ? (rb.w[i >> 1] >> 16) : (rb.w[i >> 1] & 0xFFFFu));
+    };
+    const __half2 d2 = __half2half2(__ushort_as_half((unsigned short)hw(0)));
+    const __half2 bias = __float2half2_rn(1152.f);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t u = hw(k + 1) ^ 0x8080u;
+      const uint32_t w = __byte_perm(u, 0x64646464u, 0x4140);
+      __half2 v = *reinterpret_cast<const __half2*>(&w);
+      v = __hmul2(__hsub2(v, bias), d2);
+      h[k] = *reinterpret_cast<uint32_t*>(&v);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) h[k] = rb.w[k];
   }
 }
 
@@ -400,24 +445,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         }
         return key;
       };
-      // 32 consecutive values of a cache row, as f16, into 4 swizzled 16-byte chunks
-      auto fill32 = [&](uint8_t* row_dst, int row_in_atom, int key, int col32, int chunk0) {
+      // 32 consecutive values of a cache row: read (all of a stage's blocks first, so
+      // that their loads overlap), then convert to f16 and store as 4 swizzled 16-byte
+      // chunks of the row
+      // blocks loaded before any is stored: 4 for q8_0 (9 words each), 2 for f16 (16)
+      constexpr int kLoadBatch = kMode == kModeQ8 ? 4 : 2;
+      auto load32 = [&](int key, int col32, RawBlock& rb) {
+        rb.valid = key >= 0;
+        rb.odd = false;
+        if (rb.valid) load_block<kMode>(p.kcache, seq_row0 + key, col32, rb);
+      };
+      auto store32 = [&](uint8_t* row_dst, int row_in_atom, int chunk0, const RawBlock& rb) {
         uint32_t h[16];
-        if (key < 0) {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) h[k] = 0u;
-        } else if constexpr (kMode == kModeQ8) {
-          const uint8_t* rowp = p.kcache + (seq_row0 + key) * kQ8RowBytes;
-          dequant_q8_block(rowp + col32 * 34, h);
-        } else {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.kcache + (seq_row0 + key) * (2 * kDK) + col32 * 64);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 v = __ldg(src + k);
-            h[4 * k] = v.x; h[4 * k + 1] = v.y; h[4 * k + 2] = v.z; h[4 * k + 3] = v.w;
-          }
-        }
+        block_values<kMode>(rb, h);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           *reinterpret_cast<uint4*>(row_dst + (((chunk0 + k) ^ (row_in_atom & 7)) << 4)) =
@@ -454,13 +494,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           int keys[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) keys[q] = resolve(kbase + 32 * q + (pt >> 1));
+          // Bring this CTA's rows of the tile into L2 now: the 9 stages below then read
+          // them at L2 latency. The two threads of a key split the row's 128-byte lines
+          // (every prefetched address lies inside the row).
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (keys[q] < 0) continue;
+            const uint8_t* rowp = p.kcache + (seq_row0 + keys[q]) * FwdCfg<kMode>::kRowBytes;
+            for (int off = 128 * half; off < FwdCfg<kMode>::kRowBytes; off += 256) prefetch_l2(rowp + off);
+            if (half == 1) prefetch_l2(rowp + FwdCfg<kMode>::kRowBytes - 1);
+          }
           for (int c = 0; c < 9; ++c) {
             acquire();
             uint8_t* st = ring + stage * kKStageBytes;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int kl = 32 * q + (pt >> 1);
-              fill32(st + kl * 128, kl, keys[q], 2 * c + half, 4 * half);
+            for (int q0 = 0; q0 < 4; q0 += kLoadBatch) {
+              RawBlock rb[kLoadBatch];
+#pragma unroll
+              for (int q = 0; q < kLoadBatch; ++q) load32(keys[q0 + q], 2 * c + half, rb[q]);
+#pragma unroll
+              for (int q = 0; q < kLoadBatch; ++q) {
+                const int kl = 32 * (q0 + q) + (pt >> 1);
+                store32(st + kl * 128, kl, 4 * half, rb[q]);
+              }
             }
             // Q chunk c: thread pt copies the 64 columns of query row pt (rows beyond
             // the sequence's rows are zero)
@@ -497,9 +553,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               const int col32 = 8 * nb + 4 * (int)rank + q4;
               uint8_t* st = ring + stage * kVStageBytes + box * 8192;
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int kl = (pt >> 2) + 16 * q;
-                fill32(st + kl * 128, kl, keys[q], col32, 4 * half);
+              for (int q0 = 0; q0 < 4; q0 += kLoadBatch) {
+                RawBlock rb[kLoadBatch];
+#pragma unroll
+                for (int q = 0; q < kLoadBatch; ++q) load32(keys[q0 + q], col32, rb[q]);
+#pragma unroll
+                for (int q = 0; q < kLoadBatch; ++q) {
+                  const int kl = (pt >> 2) + 16 * (q0 + q);
+                  store32(st + kl * 128, kl, 4 * half, rb[q]);
+                }
               }
               publish();
             }
@@ -539,15 +601,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // The mask loads of a tile are issued while the previous tile is still being
     // processed (right after its scores are formed), so their latency is hidden.
     uint4 mvec[kHalf / 8];
+    // Sparse (index list): every tile takes this path; mvec then holds, as f16 pairs,
+    // the mask value of each position's kept cell (0 without a mask) or -inf for a
+    // position past the list or an invalid cell. The index loads of a group of 64
+    // positions are issued together, then its mask gathers.
     auto mask_vec_ok = [&](int t) {
+      if (kManual && sparse) return true;
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
-      return !(kManual && sparse) && mrow != nullptr && k0 + kHalf <= key_end && p.mask_vec_ok;
+      return mrow != nullptr && k0 + kHalf <= key_end && p.mask_vec_ok;
     };
     auto load_mask = [&](int t) {
-      const uint4* mv =
-          reinterpret_cast<const uint4*>(mrow + (tile_begin + t) * kTileKeys + kHalf * kh);
+      const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
+      if (kManual && sparse) {
+        const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
+        uint32_t* mw = reinterpret_cast<uint32_t*>(mvec);
 #pragma unroll
-      for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
+        for (int g = 0; g < 2; ++g) {
+          int cl[64];
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const int pos = k0 + 64 * g + j;
+            cl[j] = pos < key_end ? __ldg(ix + pos) : -1;
+          }
+          unsigned short hv[64];
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const bool ok = cl[j] >= 0 && cl[j] < p.n_kv;
+            unsigned short h = ok ? (unsigned short)0 : (unsigned short)0xFC00u;  // 0 or -inf
+            if (ok && mrow != nullptr) h = __ldg(mrow + cl[j]);
+            hv[j] = h;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mw[32 * g + j] = (uint32_t)hv[2 * j] | ((uint32_t)hv[2 * j + 1] << 16);
+        }
+      } else {
+        const uint4* mv = reinterpret_cast<const uint4*>(mrow + k0);
+#pragma unroll
+        for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
+      }
     };
     bool vec_next = n_tiles > 0 && mask_vec_ok(0);
     if (vec_next) load_mask(0);
@@ -568,21 +659,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                   *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * q));
       tmem_wait_ld();
       float x[kHalf];
-      if (kManual && sparse) {
-        const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
-#pragma unroll
-        for (int j = 0; j < kHalf; ++j) {
-          const int pos = key0 + j;
-          float mv = 0.f;
-          bool ok = pos < key_end;
-          if (ok) {
-            const int cell = __ldg(ix + pos);
-            ok = cell >= 0 && cell < p.n_kv;
-            if (ok && mrow != nullptr) mv = __half2float(__ushort_as_half(__ldg(mrow + cell)));
-          }
-          x[j] = ok ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
-        }
-      } else if (vec_mask) {
+      if (vec_mask) {
 #pragma unroll
         for (int c = 0; c < kHalf / 8; ++c) {
           const uint4 v = mvec[c];
