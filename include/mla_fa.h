@@ -78,8 +78,11 @@ typedef enum {
  *         0 keeps a cell, -inf drops it, any finite value is added to the score;
  *         shared by all heads of a token
  * out     fp32, element (b, t, h, d) at out[b*out_seq_stride + (t*n_head + h)*512 + d]
- * kv_len  HOST int32[n_seq] or NULL: cells j >= kv_len[b] are not read (treated as
- *         dropped); NULL means n_kv for every sequence
+ * kv_len  HOST int32[n_seq] or NULL: cells j >= kv_len[b] are dropped; NULL means
+ *         n_kv for every sequence. With an f16 cache and no idx, whole 256-key tiles
+ *         are loaded: rows from kv_len[b] up to the next multiple of 256 (and below
+ *         n_kv) are read and weighted by exactly 0, so they must hold finite values
+ *         (a NaN or Inf there would reach the output)
  * idx     DEVICE int32 or NULL (sparse): sequence b attends only to cache rows
  *         idx[b*idx_seq_stride + i] for i < idx_count[b], each in [0, n_kv) and,
  *         as mla_compact_mask writes them, ascending; the mask (if any) is still
