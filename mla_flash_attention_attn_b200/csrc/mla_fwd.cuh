@@ -300,12 +300,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       // same 64 columns of this CTA's 64 query rows
       int stage = 0;
       uint32_t ephase = 0;
-      for (int i = 0; i < n_tiles; ++i) {
+      for (int i = 0; i < n_tiles && !failed; ++i) {
         const int key0 = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
         for (int c = 0; c < 9; ++c) {
-          if (!failed && !mbar_wait(&bars.k_empty[stage], ephase ^ 1, to)) {
+          if (!mbar_wait(&bars.k_empty[stage], ephase ^ 1, to)) {
+            // stop issuing: a stage may still be in use, and the copies already in
+            // flight (at most one ring) land before the teardown
             failed = true;
             record_status(kStatusTimeout);
+            break;
           }
           if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kKStageBytes);
           const uint32_t fl = mapa_shared(smem_u32(&bars.k_full[stage]), 0);
@@ -323,13 +326,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     if (!kManual && n_tiles > 0 && elect_one()) {
       int stage = 0;
       uint32_t ephase = 0;
-      for (int j = 0; j < n_tiles; ++j) {
+      for (int j = 0; j < n_tiles && !failed; ++j) {
         const int key0 = (tile_begin + j) * kTileKeys;
-        for (int kg = 0; kg < kTileKeys / 64; ++kg)
+        for (int kg = 0; kg < kTileKeys / 64 && !failed; ++kg)
           for (int nb = 0; nb < 2; ++nb) {
-            if (!failed && !mbar_wait(&bars.v_empty[stage], ephase ^ 1, to)) {
-              failed = true;
+            if (!mbar_wait(&bars.v_empty[stage], ephase ^ 1, to)) {
+              failed = true;  // stop issuing (see the K producer)
               record_status(kStatusTimeout);
+              break;
             }
             if (rank == 0) mbar_arrive_expect_tx(&bars.v_full[stage], 2 * kVStageBytes);
             // one 16 KB box: 64 keys x 2 column blocks of 64 (this CTA's 128 value columns
@@ -357,20 +361,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       constexpr uint32_t kQUnits = kKChunkBytes >> 4;      // Q chunk within a stage
       int kst = 0;
       uint32_t kph = 0;
-      for (int t = 0; t < n_tiles; ++t) {
+      // On a timeout the issuer stops (no further MMAs or commits); the waits that
+      // depend on its commits then time out in turn and the kernel winds down.
+      for (int t = 0; t < n_tiles && !failed; ++t) {
         // S buffer t % kSBufs is free once the softmax of tile t - kSBufs published its P
-        if (t >= kSBufs && !failed &&
+        if (t >= kSBufs &&
             !mbar_wait_cluster(&bars.p_full[(t - kSBufs) & 1], ((t - kSBufs) >> 1) & 1, to)) {
           failed = true;
           record_status(kStatusTimeout);
+          break;
         }
         const uint32_t d_s = tmem + (t % kSBufs) * kSCols;
         for (int c = 0; c < 9; ++c) {
           const bool ok = kManual ? mbar_wait_cluster(&bars.k_full[kst], kph, to)
                                   : mbar_wait(&bars.k_full[kst], kph, to);
-          if (!failed && !ok) {
+          if (!ok) {
             failed = true;
             record_status(kStatusTimeout);
+            break;
           }
           tc_fence_after();
           const uint64_t b0 = dk + (uint32_t)(kst * kStageUnits);
@@ -382,6 +390,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           mma_commit_2sm_mc(&bars.k_empty[kst], 0x3);
           if (++kst == kKStages) { kst = 0; kph ^= 1; }
         }
+        if (failed) break;
         mma_commit_2sm_mc(&bars.s_full[t % kSBufs], 0x3);
       }
     }
@@ -397,18 +406,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       constexpr uint32_t kVUnits = kVStageBytes >> 4;   // V stage stride
       int vst = 0;
       uint32_t vph = 0;
-      for (int t = 0; t < n_tiles; ++t) {
-        if (!failed && !mbar_wait_cluster(&bars.p_full[t & 1], (t >> 1) & 1, to)) {
+      for (int t = 0; t < n_tiles && !failed; ++t) {  // stops on a timeout, as above
+        if (!mbar_wait_cluster(&bars.p_full[t & 1], (t >> 1) & 1, to)) {
           failed = true;
           record_status(kStatusTimeout);
+          break;
         }
-        for (int kg = 0; kg < kTileKeys / 64; ++kg)
+        for (int kg = 0; kg < kTileKeys / 64 && !failed; ++kg)
           for (int nb = 0; nb < 2; ++nb) {
             const bool ok = kManual ? mbar_wait_cluster(&bars.v_full[vst], vph, to)
                                     : mbar_wait(&bars.v_full[vst], vph, to);
-            if (!failed && !ok) {
+            if (!ok) {
               failed = true;
               record_status(kStatusTimeout);
+              break;
             }
             tc_fence_after();
             const uint64_t a0 = dp + (uint32_t)((t & 1) * kPBufUnits + kg * kPUnits);
@@ -421,6 +432,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             mma_commit_2sm_mc(&bars.v_empty[vst], 0x3);
             if (++vst == kVStages) { vst = 0; vph ^= 1; }
           }
+        if (failed) break;
         mma_commit_2sm_mc(&bars.o_done[t & 1], 0x3);
       }
     }
@@ -818,7 +830,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   }
 
   // ---- teardown
-  if (failed) nanosleep_ns(100000);  // let copies issued before the failure land
+  // A thread that gave up stops issuing at once; the copies and MMAs it issued before
+  // (at most one ring of stages) land well within 100 us, before the cluster barrier
+  // lets either CTA exit or free TMEM.
+  if (failed) sleep_at_least_ns(100000);
   tc_fence_before();
   __syncwarp();
   cluster_sync();

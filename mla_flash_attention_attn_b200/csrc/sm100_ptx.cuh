@@ -376,6 +376,11 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ void nanosleep_ns(uint32_t ns) {
   asm volatile("nanosleep.u32 %0;" ::"r"(ns));
 }
+// Waits at least `ns` of wall time (nanosleep alone may return early).
+__device__ __forceinline__ void sleep_at_least_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) nanosleep_ns(1000);
+}
 
 // Named barrier among `nthreads` threads (multiple of 32).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
