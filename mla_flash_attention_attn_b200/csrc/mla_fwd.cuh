@@ -908,6 +908,105 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   dst[threadIdx.x] = acc;
 }
 
+// The same combine for rows with many splits (one CTA per query row: blockDim.x / 128 groups
+// of 128 threads, at most kCombineGroups; thread t of a group owns value columns
+// 4t..4t+3).
+// Group q takes the splits s with s % groups == q (16 loads in flight per thread), so
+// a row's partials are read with groups x 16 loads in flight; the groups' sums and
+// weight totals meet in shared memory. The host uses it from 32 splits on, with one
+// group per 16 splits. Every warp derives M itself; lane l of a group holds the weight of the
+// group's split l (32 at a time) and broadcasts it with shuffles.
+// Launched as a programmatic dependent of the forward kernel:
+// griddepcontrol.wait returns once the forward grid has completed and its partials
+// are visible.
+constexpr int kCombineGroups = 4;
+
+__global__ void __launch_bounds__(128 * kCombineGroups)
+    mla_combine_grouped_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
+                       const float* __restrict__ ws_lse, float* __restrict__ out,
+                       int64_t out_seq_stride) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // groups 1.. hand their sums to group 0: (groups-1) x 128 float4, then the weight
+  // totals (dynamic shared memory, none with a single group)
+  extern __shared__ float4 s_comb[];
+  const int b = blockIdx.y;
+  const int row = blockIdx.x;
+  if (plan.ws_base[b] < 0 || row >= plan.rows) return;  // the whole CTA leaves
+  const int ns = plan.n_split[b];
+  const int lane = threadIdx.x & 31;
+  const int grp = threadIdx.x >> 7;
+  const int n_grp = blockDim.x >> 7;
+  const int col = threadIdx.x & 127;
+  const int g = row / kRowsPerGroup;
+  const int rin = row % kRowsPerGroup;
+  const int slot0 = plan.ws_base[b] + g * ns;
+  const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
+  float mx = -INFINITY;
+  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)s * kRowsPerGroup));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
+  if (mx != -INFINITY) {  // the same for every warp
+    constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
+    const float4* src0 =
+        reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + col;
+    // this group's splits are s = grp + n_grp * j; lane l holds the weight of j0 + l
+    const int n_mine = ns > grp ? (ns - grp + n_grp - 1) / n_grp : 0;
+    for (int j0 = 0; j0 < n_mine; j0 += 32) {
+      float wl = 0.f;
+      if (j0 + lane < n_mine) {
+        const float lse = __ldg(lse_col + (int64_t)(grp + n_grp * (j0 + lane)) * kRowsPerGroup);
+        wl = lse == -INFINITY ? 0.f : ex2_approx(lse - mx);
+      }
+      wsum += wl;
+      const int cnt = min(32, n_mine - j0);
+      // batches of 16 loads issued before any is used
+      for (int jb = 0; jb < cnt; jb += 16) {
+        float4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (jb + u < cnt) v[u] = __ldg(src0 + (int64_t)(grp + n_grp * (j0 + jb + u)) * kSplitStride4);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float w = __shfl_sync(0xffffffffu, wl, jb + u);  // lanes past cnt hold 0
+          if (jb + u < cnt) {
+            acc.x = fmaf(w, v[u].x, acc.x);
+            acc.y = fmaf(w, v[u].y, acc.y);
+            acc.z = fmaf(w, v[u].z, acc.z);
+            acc.w = fmaf(w, v[u].w, acc.w);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+  }
+  // wsum: this group's weight total (every warp of the group holds it)
+  float* s_wsum = reinterpret_cast<float*>(s_comb + (n_grp - 1) * 128);
+  if (grp > 0) {
+    s_comb[(grp - 1) * 128 + col] = acc;
+    if (col == 0) s_wsum[grp - 1] = wsum;
+  }
+  if (n_grp > 1) __syncthreads();
+  if (grp == 0) {
+#pragma unroll
+    for (int q = 0; q < kCombineGroups - 1; ++q) {
+      if (q + 1 >= n_grp) break;
+      const float4 o = s_comb[q * 128 + col];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
+      wsum += s_wsum[q];
+    }
+    if (mx != -INFINITY) {
+      const float inv = 1.f / wsum;
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    }
+    float4* dst = reinterpret_cast<float4*>(out + (int64_t)(plan.seq_offset + b) * out_seq_stride +
+                                            (int64_t)row * kDV);
+    dst[col] = acc;
+  }
+}
+
 // Waits on a barrier that nothing ever signals, with a bounded wait, and records
 // the timeout: exercises the run-time error path without faulting anything.
 __global__ void mla_wait_timeout_kernel(uint64_t timeout_ns) {
