@@ -194,18 +194,24 @@ __device__ __forceinline__ void block_values(const RawBlock& rb, uint32_t (&h)[1
     return;
   }
   if constexpr (kMode == kModeQ8) {
-    // half-word i of the block (0: d, 1..16: int8 pairs)
-    auto hw = [&](int i) -> uint32_t {
-      return rb.odd ? ((i & 1) ? (rb.w[(i + 1) >> 1] & 0xFFFFu) : (rb.w[i >> 1] >> 16))
-                    : ((i & 1) ? (rb.w[i >> 1] >> 16) : (rb.w[i >> 1] & 0xFFFFu));
-    };
-    const __half2 d2 = __half2half2(__ushort_as_half((unsigned short)hw(0)));
+    // the block's own 32-bit words B[j] = block bytes 4j..4j+3 (j = 0..8): an odd block
+    // starts 2 bytes into rb.w[0], so each is a funnel shift of two loaded words
+    const uint32_t sh = rb.odd ? 16u : 0u;
+    uint32_t x[9];
+#pragma unroll
+    for (int j = 0; j < 9; ++j) {
+      const uint32_t hi = j < 8 ? rb.w[j + 1] : 0u;  // bytes past the block are unused
+      x[j] = __funnelshift_r(rb.w[j], hi, sh) ^ 0x80808080u;  // int8 q -> q + 128
+    }
+    const __half2 d2 = __half2half2(__ushort_as_half((unsigned short)((x[0] ^ 0x80808080u) & 0xFFFFu)));
     const __half2 bias = __float2half2_rn(1152.f);
+    // int8 pair k sits in block bytes 2+2k, 3+2k: the high half of B[k/2] for even k,
+    // the low half of B[k/2+1] for odd k; each byte goes into 0x64 to make 1024 + u
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
-      const uint32_t u = hw(k + 1) ^ 0x8080u;
-      const uint32_t w = __byte_perm(u, 0x64646464u, 0x4140);
-      __half2 v = *reinterpret_cast<const __half2*>(&w);
+      const uint32_t wd = (k & 1) ? __byte_perm(x[(k >> 1) + 1], 0x64646464u, 0x4140)
+                                  : __byte_perm(x[k >> 1], 0x64646464u, 0x4342);
+      __half2 v = *reinterpret_cast<const __half2*>(&wd);
       v = __hmul2(__hsub2(v, bias), d2);
       h[k] = *reinterpret_cast<uint32_t*>(&v);
     }
