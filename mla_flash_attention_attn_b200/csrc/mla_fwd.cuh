@@ -95,7 +95,7 @@ constexpr int kKChunkBytes = 2 * kChunkBytes;     // 128 keys x 64 columns
 constexpr int kKStageBytes = kKChunkBytes + kChunkBytes;
 constexpr int kVStageBytes = 2 * kChunkBytes;     // V stage: 64 keys x 128 value columns
 constexpr int kPBufBytes = 4 * kChunkBytes;       // 64 rows x 256 keys f16
-constexpr int kPBufs = 2;        // P buffers: tile i uses buffer i % 2
+constexpr int kPBufs = 2;        // P buffers (1 or 2): tile i uses buffer i % kPBufs
 constexpr int kOffK = 0;
 constexpr int kOffV = kOffK + kKStages * kKStageBytes;
 constexpr int kOffP = kOffV + kVStages * kVStageBytes;
@@ -428,7 +428,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               break;
             }
             tc_fence_after();
-            const uint64_t a0 = dp + (uint32_t)((t & 1) * kPBufUnits + kg * kPUnits);
+            const uint64_t a0 = dp + (uint32_t)((t % kPBufs) * kPBufUnits + kg * kPUnits);
             const uint64_t b0 = dv + (uint32_t)(vst * kVUnits);
             const uint32_t d = tmem + kTmemO + nb * 128;
             mma_f16_ss_2sm(d, a0, b0, kIdescPV, (t > 0 || kg > 0) ? 1u : 0u);
@@ -740,11 +740,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       l_part = l_part * alpha + lsum;
 
-      // P buffer i % 2 is free once P.V(i-2) has completed
-      if (i >= 2) wait_local(&bars.o_done[i & 1], ((i - 2) >> 1) & 1);
+      // P buffer i % kPBufs is free once P.V(i - kPBufs) has completed
+      if (i >= kPBufs) wait_local(&bars.o_done[(i - kPBufs) & 1], ((i - kPBufs) >> 1) & 1);
       {
         // this lane's 128 keys are P blocks 2*kh and 2*kh+1 (64 keys each) of row r
-        uint8_t* pbuf = sP + (i & 1) * kPBufBytes;
+        uint8_t* pbuf = sP + (i % kPBufs) * kPBufBytes;
 #pragma unroll
         for (int blk = 0; blk < 2; ++blk) {
           uint8_t* base = pbuf + (2 * kh + blk) * kChunkBytes + r * 128;
