@@ -176,6 +176,27 @@ def test_split_plan_is_exercised():
     assert splits2 == 1 and units2 == 64
 
 
+def test_batch_larger_than_one_launch():
+    # 130 sequences: the host splits the batch into launches of at most 128 sequences,
+    # each with its own plan (and split partials + combine where a sequence splits)
+    w = W.make("v3_batched_decode", n_seq=130, n_head=16, n_kv=600, len_lo=1, len_hi=600)
+    check_all_rows(w, run_gpu(w), what="130 sequences")
+
+
+def test_many_splits_of_one_long_sequence():
+    # one 16-head sequence of 20000 keys: 79 tiles over the 74 SM pairs, so its rows are
+    # combined from 74 partials by the multi-group combine
+    w = W.make("v3_batched_decode", n_seq=1, n_head=16, n_kv=20000, len_lo=20000, len_hi=20000)
+    torch = torch_mod()
+    q = torch.from_numpy(w.q).cuda()
+    k = torch.from_numpy(w.kcache).cuda()
+    out = torch.empty(w.q.shape[:3] + (512,), dtype=torch.float32, device="cuda")
+    args, keep = binding.make_args(q, k, 0, None, out, w.scale, kv_len=w.kv_len)
+    units, splits = binding.mla_fa_query_plan(args)
+    assert splits >= 32, "the case must reach the multi-group combine"
+    check_all_rows(w, run_gpu(w), what="one long sequence")
+
+
 def test_simple_entry_point_matches_oracle():
     torch = torch_mod()
     w = W.make("v2lite_decode", n_kv=1111)
