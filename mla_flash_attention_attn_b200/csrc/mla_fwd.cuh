@@ -623,14 +623,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // the mask value of each position's kept cell (0 without a mask) or -inf for a
     // position past the list or an invalid cell. The index loads of a group of 64
     // positions are issued together, then its mask gathers.
+    // A row past the sequence's rows is computed but never stored: it takes the vector
+    // path with a zero mask, so that its lanes follow the same path as their warp's
+    // valid rows.
     auto mask_vec_ok = [&](int t) {
-      if (kManual && sparse) return true;
+      if ((kManual && sparse) || !row_valid) return true;
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
       return mrow != nullptr && k0 + kHalf <= key_end && p.mask_vec_ok;
     };
     auto load_mask = [&](int t) {
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
-      if (kManual && sparse) {
+      if (!row_valid) {
+#pragma unroll
+        for (int c = 0; c < kHalf / 8; ++c) mvec[c] = make_uint4(0u, 0u, 0u, 0u);
+      } else if (kManual && sparse) {
         const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
         uint32_t* mw = reinterpret_cast<uint32_t*>(mvec);
 #pragma unroll
@@ -794,7 +800,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // layout of a 128-byte-swizzle tensor map) and one lane stores them with TMA.
     // Every MMA has finished (last o_done), so the operand rings are free; the 4
     // warps use the first 128 KB. Rows beyond the tensor are clipped by the store.
-    {
+    // A warp whose 32 rows all lie past the sequence's rows has nothing to store.
+    if (__any_sync(0xffffffffu, row_valid)) {
       const int wq = warp - 4;  // row half (wq & 1) of key half kh = wq >> 1
       uint8_t* wbox = smem + wq * 8 * 4096;
 #pragma unroll 1
