@@ -91,7 +91,9 @@ def test_compaction_argument_errors(lib):
     assert lib.mla_compact_mask_ex(FAKE + 1, 1, 10, 10, FAKE, 10, FAKE, FAKE, 4096, None) == -4
     assert lib.mla_compact_mask_ex(FAKE, 1, 10, 10, FAKE, 10, FAKE, None, 0, None) == -5
     assert lib.mla_compact_mask_ex(FAKE, 1, 5, 10, FAKE, 10, FAKE, FAKE, 4096, None) == -2
-    assert lib.mla_compact_workspace_size(1, 131072) == 256 + 64 * 8
+    # 256 bytes of row tickets, then 8 bytes of look-back state per 16384-cell tile
+    assert lib.mla_compact_workspace_size(1, 131072) == 256 + 8 * 8
+    assert lib.mla_compact_workspace_size(3, 16385) == 256 + 3 * 2 * 8
     assert lib.mla_compact_workspace_size(0, 10) == 0
 
 
