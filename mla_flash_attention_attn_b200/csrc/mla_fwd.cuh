@@ -11,14 +11,17 @@
 //
 // Hardware mapping (cta_group::2, M = 128 rows, 64 rows in each CTA):
 //  * Each CTA keeps its 64 Q rows in shared memory (9 chunks of 64 columns,
-//    128-byte swizzle) for the whole unit.
+//    128-byte swizzle) for the whole unit; they arrive with the first tile's K.
 //  * Q.K^T: N = 256 keys (a tile); CTA c loads keys [128c, 128c+128) of each
 //    tile, so the pair reads every K byte once. In TMEM, lane r holds keys
-//    0..127 of row r and lane r+64 keys 128..255 (128 columns per S buffer, two
-//    buffers). N = 256 halves the MMAs (and their issue cost) per key.
+//    0..127 of row r and lane r+64 keys 128..255 (128 columns of S).
 //  * P.V: N = 256 value columns per MMA (one value half), K = 16 keys; CTA c
-//    loads value columns [256j+128c, +128) of the tile's rows. O lives in TMEM
-//    (256 columns per CTA: lane r holds 128 of row r's values per value half).
+//    loads value columns [256j+128c, +128) of the tile's rows. A (P) is read from
+//    TMEM and O accumulates in TMEM (256 columns per CTA: lane r holds 128 of row
+//    r's values per value half).
+//  * TMEM: S (128 columns), P (128 columns: f16 pairs of all 256 keys of the tile
+//    in both lanes of a row), O (256 columns). The softmax frees S as soon as the
+//    scores are in registers, so Q.K^T of the next tile overlaps the softmax.
 //  * K stages (16 KB: 128 keys x 64 columns) and V stages (16 KB: 64 keys x 128
 //    value columns) stream through two rings of shared-memory stages; every
 //    stage is 4 MMAs and one tcgen05.commit releases it.
@@ -27,10 +30,9 @@
 //    barrier would idle the pipe; with two issuers one's wait is covered by the
 //    other's MMAs.
 //  * Softmax warpgroup: thread = TMEM lane; the two lanes of a row exchange
-//    their tile maximum through shared memory. The reference max is raised
-//    only when a tile's max exceeds it by more than 2^8, so O is rescaled in
-//    TMEM rarely; P (f16, <= 256) goes to one of two shared-memory buffers as
-//    the A operand, written once P.V of the tile two earlier has finished.
+//    their tile maximum and their P halves through shared memory. The reference
+//    max is raised only when a tile's max exceeds it by more than 2^8, so O is
+//    rescaled in TMEM rarely.
 //  * Epilogue: O / l is staged in shared memory and written by TMA stores.
 //
 // Every mbarrier wait is bounded (MlaFwdParams::timeout_ns). On a timeout the
@@ -83,50 +85,55 @@ enum FwdMode {
 
 namespace fwd {
 
-constexpr int kKStages = 4;      // ring of Q.K^T operand stages (K chunk + Q chunk)
-constexpr int kVStages = 4;      // ring of P.V operand stages (V columns, L2-resident)
-constexpr int kSBufs = 2;        // S buffers in TMEM (128 columns each)
-constexpr int kSCols = 128;      // TMEM columns of one S buffer
+constexpr int kKStages = 4;      // ring of Q.K^T operand stages (K chunks, from DRAM)
+constexpr int kVStages = 3;      // ring of P.V operand stages (V columns, L2-resident)
 constexpr int kChunkBytes = 8192;                 // 64 rows x 64 f16 (one swizzle tile)
 constexpr int kKChunkBytes = 2 * kChunkBytes;     // 128 keys x 64 columns
-// A Q.K^T stage holds a K chunk and the matching 64-column chunk of this CTA's 64
-// query rows: Q is re-read from L2 with every tile rather than kept resident, which
-// leaves room for more K stages in flight (the K stream comes from DRAM).
-constexpr int kKStageBytes = kKChunkBytes + kChunkBytes;
+constexpr int kQBytes = 9 * kChunkBytes;          // this CTA's 64 query rows x 576, resident
+constexpr int kKStageBytes = kKChunkBytes;
 constexpr int kVStageBytes = 2 * kChunkBytes;     // V stage: 64 keys x 128 value columns
-constexpr int kPBufBytes = 4 * kChunkBytes;       // 64 rows x 256 keys f16
-constexpr int kPBufs = 2;        // P buffers (1 or 2): tile i uses buffer i % kPBufs
-constexpr int kOffK = 0;
+constexpr int kXRounds = 1;                       // P exchange rounds per tile (1 or 2)
+constexpr int kXWords = 64 / kXRounds;            // f16 pairs per lane and round
+constexpr int kXBytes = 128 * kXWords * 4;        // P exchange buffer
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQBytes;
 constexpr int kOffV = kOffK + kKStages * kKStageBytes;
-constexpr int kOffP = kOffV + kVStages * kVStageBytes;
-constexpr int kOffBar = kOffP + kPBufs * kPBufBytes;
-constexpr int kNumBars = 2 * kKStages + 2 * kVStages + kSBufs + 2 + 2;
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+constexpr int kOffX = kOffV + kVStages * kVStageBytes;
+constexpr int kOffBar = kOffX + kXBytes;
+constexpr int kBarBytes = 8 * (2 * kKStages + 2 * kVStages + 1 + 1 + 2 + 2);
+constexpr int kOffTmemSlot = kOffBar + kBarBytes;
 constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
 constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
 constexpr int kSmemBytes = kOffXl + 128 * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;                   // 1024-byte alignment slack
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = kSBufs * kSCols;                    // O columns start
+// TMEM columns: S (fp32 scores of 128 keys per lane), P (f16 pairs of the tile's 256
+// keys per lane), O (256 fp32 columns: 128 values of each value half per lane)
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemP = 128;
+constexpr uint32_t kTmemO = 256;
 constexpr float kRescaleThreshold = 5.5451774f;                 // 8 ln 2 (natural units)
 
 static_assert(kSmemAlloc <= 232448, "shared memory beyond the 227 KB per-CTA limit");
-static_assert(kTmemO + 256 <= kTmemCols, "S buffers and O exceed the TMEM allocation");
-static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0,
+static_assert(kTmemO + 256 <= kTmemCols, "S, P and O exceed the TMEM allocation");
+static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
               "128-byte swizzle needs 1 KB alignment");
+static_assert(kOffBar >= 128 * 1024, "the epilogue stages O in the first 128 KB");
 
 constexpr uint32_t kIdescQK = idesc_f16_f32(128, 256, 0, 0);    // K-major A and B
-constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);    // B (V) MN-major
+constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);    // A (P, TMEM) K-major, B (V) MN-major
 
 struct Bars {
-  uint64_t k_full[kKStages];     // leader: both CTAs' K and Q chunk bytes landed
+  uint64_t k_full[kKStages];     // leader: both CTAs' K chunk bytes landed
   uint64_t k_empty[kKStages];    // both: the Q.K^T MMAs reading a stage are done
   uint64_t v_full[kVStages];     // leader: both CTAs' V chunk bytes landed
   uint64_t v_empty[kVStages];    // both: the P.V MMAs reading a V stage are done
-  uint64_t s_full[kSBufs];       // both: S buffer written by Q.K^T
-  uint64_t p_full[2];            // leader: P written (8 warp arrivals, both CTAs)
+  uint64_t s_full;               // both: S written by Q.K^T
+  uint64_t s_free;               // leader: S read out by the softmax (8 warp arrivals)
+  uint64_t p_full[2];            // leader: P written to TMEM (8 warp arrivals, both CTAs)
   uint64_t o_done[2];            // both: P.V of a tile (parity-indexed) complete
 };
+static_assert(sizeof(Bars) == kBarBytes, "barrier block size");
 
 }  // namespace fwd
 
@@ -234,9 +241,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + kOffQ;
   uint8_t* sK = smem + kOffK;
   uint8_t* sV = smem + kOffV;
-  uint8_t* sP = smem + kOffP;
+  uint4* sX = reinterpret_cast<uint4*>(smem + kOffX);
   Bars& bars = *reinterpret_cast<Bars*>(smem + kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
   float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
@@ -272,7 +280,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       mbar_init(&bars.v_full[i], kManual ? 4 : 1);
       mbar_init(&bars.v_empty[i], 1);
     }
-    for (int i = 0; i < kSBufs; ++i) mbar_init(&bars.s_full[i], 1);
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_free, 8);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.p_full[i], 8);
       mbar_init(&bars.o_done[i], 1);
@@ -299,11 +308,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
   }
   if (warp == 0) {
-    // ================= producer (TMA mode): K chunks with their Q chunks
+    // ================= producer (TMA mode): K chunks; the first tile's stages also
+    // bring the matching chunk of this CTA's 64 query rows, which stay resident
     if (!kManual && n_tiles > 0 && elect_one()) {
       // this CTA's 128 keys of each tile, 9 chunks of 64 columns, as far ahead as the
-      // ring allows (only Q.K^T consumption frees stages); each stage also gets the
-      // same 64 columns of this CTA's 64 query rows
+      // ring allows (only Q.K^T consumption frees stages)
       int stage = 0;
       uint32_t ephase = 0;
       for (int i = 0; i < n_tiles && !failed; ++i) {
@@ -316,12 +325,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             record_status(kStatusTimeout);
             break;
           }
-          if (rank == 0) mbar_arrive_expect_tx(&bars.k_full[stage], 2 * kKStageBytes);
+          if (rank == 0)
+            mbar_arrive_expect_tx(&bars.k_full[stage], 2 * (kKStageBytes + (i == 0 ? kChunkBytes : 0)));
           const uint32_t fl = mapa_shared(smem_u32(&bars.k_full[stage]), 0);
-          uint8_t* st = sK + stage * kKStageBytes;
-          tma_load_3d_2sm(st, &tm_k, fl, 64 * c, key0, b_abs);
-          tma_load_3d_2sm(st + kKChunkBytes, &tm_q, fl, 64 * c, row0 + kRowsPerCta * (int)rank,
-                          b_abs);
+          tma_load_3d_2sm(sK + stage * kKStageBytes, &tm_k, fl, 64 * c, key0, b_abs);
+          if (i == 0)
+            tma_load_3d_2sm(sQ + c * kChunkBytes, &tm_q, fl, 64 * c, row0 + kRowsPerCta * (int)rank,
+                            b_abs);
           if (++stage == kKStages) { stage = 0; ephase ^= 1; }
         }
       }
@@ -363,21 +373,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       // plus off/16 (the start address field is the low 14 bits, no carry possible
       // below 256 KB).
       const uint64_t dk = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
       constexpr uint32_t kStageUnits = kKStageBytes >> 4;  // stage stride
-      constexpr uint32_t kQUnits = kKChunkBytes >> 4;      // Q chunk within a stage
+      constexpr uint32_t kQUnits = kChunkBytes >> 4;       // Q chunk stride
       int kst = 0;
       uint32_t kph = 0;
+      // Q chunk c is resident once the first tile's stage c has landed
       // On a timeout the issuer stops (no further MMAs or commits); the waits that
       // depend on its commits then time out in turn and the kernel winds down.
       for (int t = 0; t < n_tiles && !failed; ++t) {
-        // S buffer t % kSBufs is free once the softmax of tile t - kSBufs published its P
-        if (t >= kSBufs &&
-            !mbar_wait_cluster(&bars.p_full[(t - kSBufs) & 1], ((t - kSBufs) >> 1) & 1, to)) {
+        // S is free once the softmax has read the scores of tile t - 1
+        if (t >= 1 && !mbar_wait_cluster(&bars.s_free, (t - 1) & 1, to)) {
           failed = true;
           record_status(kStatusTimeout);
           break;
         }
-        const uint32_t d_s = tmem + (t % kSBufs) * kSCols;
+        const uint32_t d_s = tmem + kTmemS;
         for (int c = 0; c < 9; ++c) {
           const bool ok = kManual ? mbar_wait_cluster(&bars.k_full[kst], kph, to)
                                   : mbar_wait(&bars.k_full[kst], kph, to);
@@ -388,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           }
           tc_fence_after();
           const uint64_t b0 = dk + (uint32_t)(kst * kStageUnits);
-          const uint64_t a0 = b0 + kQUnits;
+          const uint64_t a0 = dq + (uint32_t)(c * kQUnits);
           mma_f16_ss_2sm(d_s, a0, b0, kIdescQK, c ? 1u : 0u);
           mma_f16_ss_2sm(d_s, a0 + 2, b0 + 2, kIdescQK, 1u);
           mma_f16_ss_2sm(d_s, a0 + 4, b0 + 4, kIdescQK, 1u);
@@ -397,18 +408,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           if (++kst == kKStages) { kst = 0; kph ^= 1; }
         }
         if (failed) break;
-        mma_commit_2sm_mc(&bars.s_full[t % kSBufs], 0x3);
+        mma_commit_2sm_mc(&bars.s_full, 0x3);
       }
     }
     __syncwarp();
   } else if (warp == 3) {
     // ================= P.V issuer (leader CTA, one thread): per tile, wait for P, then
     // consume the V stages (64 keys x one 256-column half each) in the producer's order.
+    // A (P) is read from TMEM: 16 keys per MMA are 8 columns of the P buffer.
     if (rank == 0 && n_tiles > 0 && elect_one()) {
       const uint64_t dv = smem_desc_sw128(smem_u32(sV), 8192, 1024);
-      const uint64_t dp = smem_desc_sw128(smem_u32(sP), 16, 1024);
-      constexpr uint32_t kPUnits = kChunkBytes >> 4;    // P block (64 keys) stride
-      constexpr uint32_t kPBufUnits = kPBufBytes >> 4;  // P buffer stride
       constexpr uint32_t kVUnits = kVStageBytes >> 4;   // V stage stride
       int vst = 0;
       uint32_t vph = 0;
@@ -428,13 +437,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               break;
             }
             tc_fence_after();
-            const uint64_t a0 = dp + (uint32_t)((t % kPBufs) * kPBufUnits + kg * kPUnits);
+            const uint32_t a0 = tmem + kTmemP + (uint32_t)(kg * 32);
             const uint64_t b0 = dv + (uint32_t)(vst * kVUnits);
             const uint32_t d = tmem + kTmemO + nb * 128;
-            mma_f16_ss_2sm(d, a0, b0, kIdescPV, (t > 0 || kg > 0) ? 1u : 0u);
-            mma_f16_ss_2sm(d, a0 + 2, b0 + 128, kIdescPV, 1u);
-            mma_f16_ss_2sm(d, a0 + 4, b0 + 256, kIdescPV, 1u);
-            mma_f16_ss_2sm(d, a0 + 6, b0 + 384, kIdescPV, 1u);
+            mma_f16_ts_2sm(d, a0, b0, kIdescPV, (t > 0 || kg > 0) ? 1u : 0u);
+            mma_f16_ts_2sm(d, a0 + 8, b0 + 128, kIdescPV, 1u);
+            mma_f16_ts_2sm(d, a0 + 16, b0 + 256, kIdescPV, 1u);
+            mma_f16_ts_2sm(d, a0 + 24, b0 + 384, kIdescPV, 1u);
             mma_commit_2sm_mc(&bars.v_empty[vst], 0x3);
             if (++vst == kVStages) { vst = 0; vph ^= 1; }
           }
@@ -504,8 +513,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       if (k_side) {
         // K chunk items: 128 keys (this CTA's half of the tile) x 2 blocks of 32 columns;
         // thread pt takes keys pt/2 + 32q (q = 0..3) and block half pt%2
-        const int q_row = row0 + kRowsPerCta * (int)rank + pt;
-        const uint16_t* q_src = p.q + (int64_t)b_abs * p.q_seq_stride + (int64_t)q_row * kDK;
+        // Q first: thread pt copies the 576 columns of query row pt into the resident Q
+        // chunks (rows beyond the sequence's rows are zero); the first K stage's
+        // publication makes them visible to the MMAs
+        {
+          const int q_row = row0 + kRowsPerCta * (int)rank + pt;
+          const uint4* q_src = reinterpret_cast<const uint4*>(
+              p.q + (int64_t)b_abs * p.q_seq_stride + (int64_t)q_row * kDK);
+          for (int c = 0; c < 9; ++c) {
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = q_row < plan.rows ? __ldg(q_src + 8 * c + k) : make_uint4(0u, 0u, 0u, 0u);
+            uint8_t* dq = sQ + c * kChunkBytes + pt * 128;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dq + ((k ^ (pt & 7)) << 4)) = v[k];
+          }
+        }
         for (int i = 0; i < n_tiles; ++i) {
           const int kbase = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
           const int half = pt & 1;
@@ -535,22 +558,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                 const int kl = 32 * (q0 + q) + (pt >> 1);
                 store32(st + kl * 128, kl, 4 * half, rb[q]);
               }
-            }
-            // Q chunk c: thread pt copies the 64 columns of query row pt (rows beyond
-            // the sequence's rows are zero)
-            {
-              uint4 v[8];
-              if (q_row < plan.rows) {
-                const uint4* src = reinterpret_cast<const uint4*>(q_src + 64 * c);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) v[k] = __ldg(src + k);
-              } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) v[k] = make_uint4(0u, 0u, 0u, 0u);
-              }
-              uint8_t* dq = st + kKChunkBytes + pt * 128;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dq + ((k ^ (pt & 7)) << 4)) = v[k];
             }
             publish();
           }
@@ -601,6 +608,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                                ? p.mask + (int64_t)b_abs * p.mask_seq_stride +
                                      (int64_t)tok * p.mask_row_stride
                                : nullptr;
+    const uint32_t s_free_l = mapa_shared(smem_u32(&bars.s_free), 0);
     const uint32_t p_full_l0 = mapa_shared(smem_u32(&bars.p_full[0]), 0);
     const uint32_t p_full_l1 = mapa_shared(smem_u32(&bars.p_full[1]), 0);
     auto wait_local = [&](uint64_t* bar, uint32_t parity) {
@@ -669,19 +677,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 
     for (int i = 0; i < n_tiles; ++i) {
       const int sb = i & 1;          // max-exchange slot and p_full barrier
-      const int sbuf = i % kSBufs;   // S buffer in TMEM
       const int key0 = (tile_begin + i) * kTileKeys + kHalf * kh;
       const bool vec_mask = vec_next;
-      wait_local(&bars.s_full[sbuf], (i / kSBufs) & 1);
+      wait_local(&bars.s_full, i & 1);
       tc_fence_after();
       // scores x = scale * s + mask (natural units); cells beyond the unit's keys are
       // dropped. 128 values per lane, read from TMEM with 4 loads and one wait.
       uint32_t sr[kHalf];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        tmem_ld32(tmem + lane_base + sbuf * kSCols + 32 * q,
+        tmem_ld32(tmem + lane_base + kTmemS + 32 * q,
                   *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * q));
       tmem_wait_ld();
+      // the scores are in registers: Q.K^T of the next tile may overwrite S (the loads
+      // are complete, so a relaxed arrive suffices)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster_relaxed(s_free_l);
       float x[kHalf];
       if (vec_mask) {
 #pragma unroll
@@ -706,10 +718,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           x[j] = key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
         }
       }
-      // next tile's mask: its loads overlap the rest of this tile
-      vec_next = i + 1 < n_tiles && mask_vec_ok(i + 1);
-      if (vec_next) load_mask(i + 1);
-
       // row max over this lane's 128 keys (8 independent chains), then over the pair
       float m8[8];
 #pragma unroll
@@ -745,28 +753,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       }
       const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       l_part = l_part * alpha + lsum;
+      // next tile's mask: its loads overlap the rest of this tile (the scores are dead)
+      vec_next = i + 1 < n_tiles && mask_vec_ok(i + 1);
+      if (vec_next) load_mask(i + 1);
 
-      // P buffer i % kPBufs is free once P.V(i - kPBufs) has completed
-      if (i >= kPBufs) wait_local(&bars.o_done[(i - kPBufs) & 1], ((i - kPBufs) >> 1) & 1);
+      // P goes to TMEM as the A operand of P.V. That MMA reads A for the value columns
+      // of the first N half from lanes 0-63 and for the second half from lanes 64-127,
+      // so each of a row's two lanes needs all 256 keys: the lanes of a row swap their
+      // 128 keys through shared memory (the previous tile's reads of the exchange
+      // buffer finished before the max exchange barrier above).
       {
-        // this lane's 128 keys are P blocks 2*kh and 2*kh+1 (64 keys each) of row r
-        uint8_t* pbuf = sP + (i % kPBufs) * kPBufBytes;
+        // keys 0..127 of the tile in columns 0..63, keys 128..255 in columns 64..127;
+        // kXRounds rounds of kXWords f16 pairs
+        const uint32_t a = tmem + lane_base + kTmemP;
+        const uint32_t a_own = a + 64 * kh, a_peer = a + 64 * (kh ^ 1);
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          uint8_t* base = pbuf + (2 * kh + blk) * kChunkBytes + r * 128;
+        for (int rd = 0; rd < kXRounds; ++rd) {
+          const int w0 = rd * kXWords;
+          if (rd > 0) named_bar_sync(1, 128);  // the partner has read the previous round
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const int w = 32 * blk + 4 * c;
-            *reinterpret_cast<uint4*>(base + ((c ^ (r & 7)) << 4)) =
-                make_uint4(pk[w], pk[w + 1], pk[w + 2], pk[w + 3]);
+          for (int gq = 0; gq < kXWords / 4; ++gq)
+            sX[gq * 128 + L] = make_uint4(pk[w0 + 4 * gq], pk[w0 + 4 * gq + 1], pk[w0 + 4 * gq + 2],
+                                          pk[w0 + 4 * gq + 3]);
+          named_bar_sync(1, 128);
+          uint32_t pw[kXWords];
+#pragma unroll
+          for (int gq = 0; gq < kXWords / 4; ++gq) {
+            const uint4 v = sX[gq * 128 + (L ^ 64)];
+            pw[4 * gq] = v.x; pw[4 * gq + 1] = v.y; pw[4 * gq + 2] = v.z; pw[4 * gq + 3] = v.w;
           }
+          if (rd == 0) {
+            // the P buffer (and O) are free once P.V of the previous tile has completed
+            if (i > 0) wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int u = 0; u < kXWords / 32; ++u)
+            tmem_st32(a_own + w0 + 32 * u, *reinterpret_cast<uint32_t(*)[32]>(pk + w0 + 32 * u));
+#pragma unroll
+          for (int u = 0; u < kXWords / 32; ++u)
+            tmem_st32(a_peer + w0 + 32 * u, *reinterpret_cast<uint32_t(*)[32]>(pw + 32 * u));
         }
+        tmem_wait_st();
       }
-      // rescale O (only when some row of this warp raised its reference max), once
-      // P.V(i-1) has completed
+      // rescale O (only when some row of this warp raised its reference max); P.V(i-1)
+      // has completed (waited above)
       if (__any_sync(0xffffffffu, need && i > 0)) {
-        wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
-        tc_fence_after();
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t v[32];
@@ -779,10 +811,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         }
         tmem_wait_st();
       }
-      fence_proxy_async_smem();
+      // P is in TMEM and complete (tcgen05.wait::st above): a relaxed arrive hands it over
+      // without waiting for this thread's mask loads of the next tile, which a release
+      // would (that wait cost 1-4 us per tile)
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(sb ? p_full_l1 : p_full_l0);
+      if (lane == 0) mbar_arrive_cluster_relaxed(sb ? p_full_l1 : p_full_l0);
     }
 
     // ---- epilogue
