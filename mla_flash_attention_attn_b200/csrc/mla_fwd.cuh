@@ -625,7 +625,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 
     constexpr int kHalf = kTileKeys / 2;  // keys of one lane (128)
     // The mask loads of a tile are issued while the previous tile is still being
-    // processed (right after its scores are formed), so their latency is hidden.
+    // processed (after its exponentials), so their latency is hidden. Full tiles take
+    // this vector path (zeros without a mask); a ragged last tile goes key by key.
     uint4 mvec[kHalf / 8];
     // Sparse (index list): every tile takes this path; mvec then holds, as f16 pairs,
     // the mask value of each position's kept cell (0 without a mask) or -inf for a
@@ -637,7 +638,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     auto mask_vec_ok = [&](int t) {
       if ((kManual && sparse) || !row_valid) return true;
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
-      return mrow != nullptr && k0 + kHalf <= key_end && p.mask_vec_ok;
+      if (k0 + kHalf > key_end) return false;  // ragged: per-key path
+      return mrow == nullptr || p.mask_vec_ok;  // no mask: zeros
     };
     auto load_mask = [&](int t) {
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
@@ -666,6 +668,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
           for (int j = 0; j < 32; ++j) mw[32 * g + j] = (uint32_t)hv[2 * j] | ((uint32_t)hv[2 * j + 1] << 16);
         }
+      } else if (mrow == nullptr) {
+#pragma unroll
+        for (int c = 0; c < kHalf / 8; ++c) mvec[c] = make_uint4(0u, 0u, 0u, 0u);
       } else {
         const uint4* mv = reinterpret_cast<const uint4*>(mrow + k0);
 #pragma unroll
@@ -838,37 +843,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     if (__any_sync(0xffffffffu, row_valid)) {
       const int wq = warp - 4;  // row half (wq & 1) of key half kh = wq >> 1
       uint8_t* wbox = smem + wq * 8 * 4096;
+      const CUtensorMap* tm = ws_slot >= 0 ? &tm_w : &tm_o;
+      const int y = (ws_slot >= 0 ? ws_slot * kRowsPerGroup : row0) + kRowsPerCta * (int)rank +
+                    32 * (wq & 1);
+      const int z = ws_slot >= 0 ? 0 : b_abs;
+      // groups of kEpi 32-column TMEM loads under one wait (fewer in the manual modes,
+      // whose register budget is smaller); each group's boxes are stored while the next
+      // group is read
+      constexpr int kEpi = kManual ? 2 : 4;
 #pragma unroll 1
-      for (int i = 0; i < 8; ++i) {
-        const int nb = i >> 2, cc = i & 3;
-        uint32_t v[32];
+      for (int g0 = 0; g0 < 8; g0 += kEpi) {
+        uint32_t v[kEpi][32];
         if (n_tiles > 0) {
-          tmem_ld32(tmem + lane_base + kTmemO + nb * 128 + cc * 32, v);
+#pragma unroll
+          for (int u = 0; u < kEpi; ++u) tmem_ld32(tmem + lane_base + kTmemO + 32 * (g0 + u), v[u]);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0u;
-        }
-        uint8_t* rowp = wbox + i * 4096 + lane * 128;
+          for (int u = 0; u < kEpi; ++u)
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) << 4)) =
-              make_float4(__uint_as_float(v[4 * c]) * inv_l, __uint_as_float(v[4 * c + 1]) * inv_l,
-                          __uint_as_float(v[4 * c + 2]) * inv_l,
-                          __uint_as_float(v[4 * c + 3]) * inv_l);
+            for (int j = 0; j < 32; ++j) v[u][j] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kEpi; ++u) {
+          uint8_t* rowp = wbox + (g0 + u) * 4096 + lane * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                make_float4(__uint_as_float(v[u][4 * c]) * inv_l, __uint_as_float(v[u][4 * c + 1]) * inv_l,
+                            __uint_as_float(v[u][4 * c + 2]) * inv_l,
+                            __uint_as_float(v[u][4 * c + 3]) * inv_l);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // box i = TMEM columns 32i..32i+31: value columns 256 (i / 4) + 128 kh + 32 (i % 4)
+          for (int u = 0; u < kEpi; ++u) {
+            const int i = g0 + u;
+            tma_store_3d(tm, wbox + i * 4096, 256 * (i >> 2) + 128 * kh + 32 * (i & 3), y, z);
+          }
+          bulk_commit_group();
+        }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        const CUtensorMap* tm = ws_slot >= 0 ? &tm_w : &tm_o;
-        const int y = (ws_slot >= 0 ? ws_slot * kRowsPerGroup : row0) + kRowsPerCta * (int)rank +
-                      32 * (wq & 1);
-        const int z = ws_slot >= 0 ? 0 : b_abs;
-        for (int i = 0; i < 8; ++i)
-          tma_store_3d(tm, wbox + i * 4096, 256 * (i >> 2) + 128 * kh + 32 * (i & 3), y, z);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-      }
+      if (lane == 0) bulk_wait_group_read0();
       __syncwarp();
     }
     if (ws_slot >= 0 && kh == 0 && row_valid)
@@ -895,11 +912,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 //   O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
 // where O_s is split s normalised by its own sum and lse_s = log2 of that sum
 // relative to the split's max; splits with no kept cell have lse_s = -inf.
-// Every warp derives the weights itself (lane s holds split s, 32 at a time) and
-// broadcasts them with shuffles; the partial rows are read with independent,
-// unrolled 16-byte loads. Launched as a programmatic dependent of the forward
-// kernel: griddepcontrol.wait returns once the forward grid has completed and its
-// partials are visible.
+// Lane s of every warp holds lse_s (the host uses this kernel below 32 splits). The
+// loads of the first 16 partial rows are issued together with the lse loads, before
+// the weights are known, so a row with at most 16 splits costs one round trip to
+// memory. Launched as a programmatic dependent of the forward kernel:
+// griddepcontrol.wait returns once the forward grid has completed and its partials
+// are visible.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant__ Plan plan,
                                                           const float* __restrict__ ws_o,
                                                           const float* __restrict__ ws_lse,
@@ -909,44 +927,45 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   const int b = blockIdx.y;
   const int row = blockIdx.x;
   if (plan.ws_base[b] < 0 || row >= plan.rows) return;
-  const int ns = plan.n_split[b];
+  const int ns = min(plan.n_split[b], 32);
   const int lane = threadIdx.x & 31;
   const int g = row / kRowsPerGroup;
   const int rin = row % kRowsPerGroup;
-  const int slot0 = plan.ws_base[b] + g * ns;
+  const int slot0 = plan.ws_base[b] + g * plan.n_split[b];
   const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
-  float mx = -INFINITY;
-  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)s * kRowsPerGroup));
+  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
+  const float4* src0 =
+      reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + threadIdx.x;
+  const float lse_l = lane < ns ? __ldg(lse_col + (int64_t)lane * kRowsPerGroup) : -INFINITY;
+  constexpr int kFirst = 16;
+  float4 v[kFirst];
+#pragma unroll
+  for (int u = 0; u < kFirst; ++u) v[u] = u < ns ? __ldg(src0 + u * kSplitStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  float mx = lse_l;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (mx != -INFINITY) {
-    float wsum = 0.f;
-    constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
-    const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
-                         threadIdx.x;
-    for (int s0 = 0; s0 < ns; s0 += 32) {
-      const int s = s0 + lane;
-      float wl = 0.f;
-      if (s < ns) {
-        const float lse = __ldg(lse_col + (int64_t)s * kRowsPerGroup);
-        wl = lse == -INFINITY ? 0.f : ex2_approx(lse - mx);
-      }
-      wsum += wl;
-      const int cnt = min(32, ns - s0);
-      const float4* src = src0 + s0 * kSplitStride4;
-#pragma unroll 8
-      for (int j = 0; j < cnt; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wl, j);
-        const float4 v = __ldg(src + j * kSplitStride4);
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
-      }
-    }
+    const float wl = lse_l == -INFINITY ? 0.f : ex2_approx(lse_l - mx);
+    float wsum = wl;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+#pragma unroll
+    for (int u = 0; u < kFirst; ++u) {
+      const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past ns
+      acc.x = fmaf(w, v[u].x, acc.x);
+      acc.y = fmaf(w, v[u].y, acc.y);
+      acc.z = fmaf(w, v[u].z, acc.z);
+      acc.w = fmaf(w, v[u].w, acc.w);
+    }
+    for (int s = kFirst; s < ns; ++s) {
+      const float w = __shfl_sync(0xffffffffu, wl, s);
+      const float4 x = __ldg(src0 + s * kSplitStride4);
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z);
+      acc.w = fmaf(w, x.w, acc.w);
+    }
     const float inv = 1.f / wsum;
     acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
   }
