@@ -100,7 +100,7 @@ constexpr int kOffK = kOffQ + kQBytes;
 constexpr int kOffV = kOffK + kKStages * kKStageBytes;
 constexpr int kOffX = kOffV + kVStages * kVStageBytes;
 constexpr int kOffBar = kOffX + kXBytes;
-constexpr int kBarBytes = 8 * (2 * kKStages + 2 * kVStages + 1 + 1 + 2 + 2);
+constexpr int kBarBytes = 8 * (2 * kKStages + 2 * kVStages + 1 + 1 + 2 + 2 + 1);
 constexpr int kOffTmemSlot = kOffBar + kBarBytes;
 constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
 constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
@@ -132,6 +132,7 @@ struct Bars {
   uint64_t s_free;               // leader: S read out by the softmax (8 warp arrivals)
   uint64_t p_full[2];            // leader: P written to TMEM (8 warp arrivals, both CTAs)
   uint64_t o_done[2];            // both: P.V of a tile (parity-indexed) complete
+  uint64_t q_full;               // leader, gather modes: both CTAs' Q rows landed (TMA)
 };
 static_assert(sizeof(Bars) == kBarBytes, "barrier block size");
 
@@ -167,15 +168,16 @@ struct FwdCfg {
 // 9 aligned 32-bit words that cover it. An even block starts 4-byte aligned and is
 // never the last block of its row; an odd block starts 2 bytes into its first
 // word; either way the 36 bytes read stay inside the row.
+template <int kMode>
 struct RawBlock {
-  uint32_t w[16];  // f16: the 32 values; q8_0: words 0..8 cover the block
+  uint32_t w[kMode == kModeQ8 ? 9 : 16];  // f16: the 32 values; q8_0: 9 words cover the block
   bool odd;        // q8_0: the block starts 2 bytes into w[0]
   bool valid;      // false: zero fill
 };
 
 template <int kMode>
 __device__ __forceinline__ void load_block(const uint8_t* kcache, int64_t row, int col32,
-                                           RawBlock& rb) {
+                                           RawBlock<kMode>& rb) {
   if constexpr (kMode == kModeQ8) {
     const uint8_t* blk = kcache + row * kQ8RowBytes + col32 * 34;
     const uintptr_t a = reinterpret_cast<uintptr_t>(blk);
@@ -194,7 +196,7 @@ __device__ __forceinline__ void load_block(const uint8_t* kcache, int64_t row, i
 }
 
 template <int kMode>
-__device__ __forceinline__ void block_values(const RawBlock& rb, uint32_t (&h)[16]) {
+__device__ __forceinline__ void block_values(const RawBlock<kMode>& rb, uint32_t (&h)[16]) {
   if (!rb.valid) {
 #pragma unroll
     for (int k = 0; k < 16; ++k) h[k] = 0u;
@@ -282,6 +284,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     }
     mbar_init(&bars.s_full, 1);
     mbar_init(&bars.s_free, 8);
+    mbar_init(&bars.q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.p_full[i], 8);
       mbar_init(&bars.o_done[i], 1);
@@ -303,9 +306,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   bool failed = false;
 
   if constexpr (kManual) {
-    // registers per thread: warps 0-3 (TMA, MMA issuers) 112, producers 128, softmax
-    // 256; 4 warps x 32 x (112 + 128 + 256) = 63488 of the 384 x 168 = 64512 launched
-    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 112;");
+    // registers per thread: warps 0-3 (TMA, MMA issuers) 96, producers 152, softmax
+    // 256; 4 warps x 32 x (96 + 152 + 256) = 64512 = the 384 x 168 launched
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
   }
   if (warp == 0) {
     // ================= producer (TMA mode): K chunks; the first tile's stages also
@@ -335,6 +338,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           if (++stage == kKStages) { stage = 0; ephase ^= 1; }
         }
       }
+    }
+    // gather modes: this CTA's Q rows by TMA (the producers gather K and V)
+    if (kManual && n_tiles > 0 && elect_one()) {
+      if (rank == 0) mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
+      const uint32_t fq = mapa_shared(smem_u32(&bars.q_full), 0);
+      for (int c = 0; c < 9; ++c)
+        tma_load_3d_2sm(sQ + c * kChunkBytes, &tm_q, fq, 64 * c, row0 + kRowsPerCta * (int)rank, b_abs);
     }
     __syncwarp();
   } else if (warp == 2) {
@@ -378,7 +388,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       constexpr uint32_t kQUnits = kChunkBytes >> 4;       // Q chunk stride
       int kst = 0;
       uint32_t kph = 0;
-      // Q chunk c is resident once the first tile's stage c has landed
+      // Q chunk c is resident once the first tile's stage c has landed (TMA mode) or
+      // once q_full completes (gather modes)
+      if (kManual && !mbar_wait(&bars.q_full, 0, to)) {
+        failed = true;
+        record_status(kStatusTimeout);
+      }
       // On a timeout the issuer stops (no further MMAs or commits); the waits that
       // depend on its commits then time out in turn and the kernel winds down.
       for (int t = 0; t < n_tiles && !failed; ++t) {
@@ -456,7 +471,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // ================= gather / dequant producers (manual modes): warps 8-9 fill the
     // K ring, warps 10-11 the V ring (64 threads per ring)
     if constexpr (kManual) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 128;");
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 152;");
       const bool k_side = warp < 10;
       const int pt = (threadIdx.x - 256) & 63;
       const int64_t seq_row0 = (int64_t)b_abs * p.k_seq_stride;
@@ -472,17 +487,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         }
         return key;
       };
-      // 32 consecutive values of a cache row: read (all of a stage's blocks first, so
-      // that their loads overlap), then convert to f16 and store as 4 swizzled 16-byte
-      // chunks of the row
-      // blocks loaded before any is stored: 4 for q8_0 (9 words each), 2 for f16 (16)
-      constexpr int kLoadBatch = kMode == kModeQ8 ? 4 : 2;
-      auto load32 = [&](int key, int col32, RawBlock& rb) {
+      // 32 consecutive values of a cache row: read, then convert to f16 and store as 4
+      // swizzled 16-byte chunks of the row.
+      // Blocks per batch: the next batch's loads are in flight while this one is
+      // converted and stored (two batches fit the producers' 152 registers)
+      constexpr int kLoadBatch = 2;
+      auto load32 = [&](int key, int col32, RawBlock<kMode>& rb) {
         rb.valid = key >= 0;
         rb.odd = false;
         if (rb.valid) load_block<kMode>(p.kcache, seq_row0 + key, col32, rb);
       };
-      auto store32 = [&](uint8_t* row_dst, int row_in_atom, int chunk0, const RawBlock& rb) {
+      auto store32 = [&](uint8_t* row_dst, int row_in_atom, int chunk0, const RawBlock<kMode>& rb) {
         uint32_t h[16];
         block_values<kMode>(rb, h);
 #pragma unroll
@@ -512,23 +527,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       };
       if (k_side) {
         // K chunk items: 128 keys (this CTA's half of the tile) x 2 blocks of 32 columns;
-        // thread pt takes keys pt/2 + 32q (q = 0..3) and block half pt%2
-        // Q first: thread pt copies the 576 columns of query row pt into the resident Q
-        // chunks (rows beyond the sequence's rows are zero); the first K stage's
-        // publication makes them visible to the MMAs
-        {
-          const int q_row = row0 + kRowsPerCta * (int)rank + pt;
-          const uint4* q_src = reinterpret_cast<const uint4*>(
-              p.q + (int64_t)b_abs * p.q_seq_stride + (int64_t)q_row * kDK);
-          for (int c = 0; c < 9; ++c) {
-            uint4 v[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = q_row < plan.rows ? __ldg(q_src + 8 * c + k) : make_uint4(0u, 0u, 0u, 0u);
-            uint8_t* dq = sQ + c * kChunkBytes + pt * 128;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(dq + ((k ^ (pt & 7)) << 4)) = v[k];
-          }
-        }
+        // thread pt takes keys pt/2 + 32q (q = 0..3) and block half pt%2. The loads of a
+        // batch of kLoadBatch blocks go out before the previous batch is converted and
+        // stored, so a chunk's load latency overlaps the previous chunk's work.
+        constexpr int kBpc = 4 / kLoadBatch;  // batches per stage
         for (int i = 0; i < n_tiles; ++i) {
           const int kbase = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
           const int half = pt & 1;
@@ -545,19 +547,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             for (int off = 128 * half; off < FwdCfg<kMode>::kRowBytes; off += 256) prefetch_l2(rowp + off);
             if (half == 1) prefetch_l2(rowp + FwdCfg<kMode>::kRowBytes - 1);
           }
+          RawBlock<kMode> cur[kLoadBatch];
+#pragma unroll
+          for (int q = 0; q < kLoadBatch; ++q) load32(keys[q], half, cur[q]);
           for (int c = 0; c < 9; ++c) {
-            acquire();
-            uint8_t* st = ring + stage * kKStageBytes;
+            uint8_t* st = nullptr;
 #pragma unroll
-            for (int q0 = 0; q0 < 4; q0 += kLoadBatch) {
-              RawBlock rb[kLoadBatch];
-#pragma unroll
-              for (int q = 0; q < kLoadBatch; ++q) load32(keys[q0 + q], 2 * c + half, rb[q]);
+            for (int bq = 0; bq < kBpc; ++bq) {
+              const bool last = bq + 1 == kBpc;
+              const int nc = last ? c + 1 : c;          // stage of the next batch
+              const int nq0 = last ? 0 : (bq + 1) * kLoadBatch;
+              RawBlock<kMode> nxt[kLoadBatch];
 #pragma unroll
               for (int q = 0; q < kLoadBatch; ++q) {
-                const int kl = 32 * (q0 + q) + (pt >> 1);
-                store32(st + kl * 128, kl, 4 * half, rb[q]);
+                if (nc < 9) load32(keys[nq0 + q], 2 * nc + half, nxt[q]);
+                else { nxt[q].valid = false; nxt[q].odd = false; }
               }
+              if (bq == 0) {
+                acquire();
+                st = ring + stage * kKStageBytes;
+              }
+#pragma unroll
+              for (int q = 0; q < kLoadBatch; ++q) {
+                const int kl = 32 * (bq * kLoadBatch + q) + (pt >> 1);
+                store32(st + kl * 128, kl, 4 * half, cur[q]);
+              }
+#pragma unroll
+              for (int q = 0; q < kLoadBatch; ++q) cur[q] = nxt[q];
             }
             publish();
           }
@@ -565,31 +581,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       } else {
         // V stage items: 64 keys x this CTA's 128 value columns of one value half (4
         // blocks of 32 in two 64-column boxes); thread pt takes keys pt/4 + 16q and
-        // 32-column block pt%4
+        // 32-column block pt%4. As on the K side, each batch's loads go out before the
+        // previous batch is stored, and the keys of the next 64-key group are resolved
+        // one group ahead.
         const int q4 = pt & 3, box = q4 >> 1, half = q4 & 1;
+        constexpr int kBpc = 4 / kLoadBatch;  // batches per stage
         for (int j = 0; j < n_tiles; ++j) {
           const int kbase = (tile_begin + j) * kTileKeys;
+          int kc[4], kn[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) kc[q] = resolve(kbase + (pt >> 2) + 16 * q);
+          RawBlock<kMode> cur[kLoadBatch];
+#pragma unroll
+          for (int q = 0; q < kLoadBatch; ++q) load32(kc[q], 4 * (int)rank + q4, cur[q]);
           for (int kg = 0; kg < kTileKeys / 64; ++kg) {
-            int keys[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) keys[q] = resolve(kbase + 64 * kg + (pt >> 2) + 16 * q);
+            for (int q = 0; q < 4; ++q)
+              kn[q] = kg + 1 < kTileKeys / 64 ? resolve(kbase + 64 * (kg + 1) + (pt >> 2) + 16 * q) : -1;
+#pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
-              acquire();
-              const int col32 = 8 * nb + 4 * (int)rank + q4;
-              uint8_t* st = ring + stage * kVStageBytes + box * 8192;
+              uint8_t* st = nullptr;
 #pragma unroll
-              for (int q0 = 0; q0 < 4; q0 += kLoadBatch) {
-                RawBlock rb[kLoadBatch];
-#pragma unroll
-                for (int q = 0; q < kLoadBatch; ++q) load32(keys[q0 + q], col32, rb[q]);
+              for (int bq = 0; bq < kBpc; ++bq) {
+                // next batch: the same stage, else the other value half, else the next group
+                const bool last = bq + 1 == kBpc;
+                const bool next_group = last && nb == 1;
+                const int nnb = last ? nb ^ 1 : nb;
+                const int nq0 = last ? 0 : (bq + 1) * kLoadBatch;
+                RawBlock<kMode> nxt[kLoadBatch];
 #pragma unroll
                 for (int q = 0; q < kLoadBatch; ++q) {
-                  const int kl = (pt >> 2) + 16 * (q0 + q);
-                  store32(st + kl * 128, kl, 4 * half, rb[q]);
+                  const int key = next_group ? kn[nq0 + q] : kc[nq0 + q];
+                  if (!next_group || kg + 1 < kTileKeys / 64) load32(key, 8 * nnb + 4 * (int)rank + q4, nxt[q]);
+                  else { nxt[q].valid = false; nxt[q].odd = false; }
                 }
+                if (bq == 0) {
+                  acquire();
+                  st = ring + stage * kVStageBytes + box * 8192;
+                }
+#pragma unroll
+                for (int q = 0; q < kLoadBatch; ++q) {
+                  const int kl = (pt >> 2) + 16 * (bq * kLoadBatch + q);
+                  store32(st + kl * 128, kl, 4 * half, cur[q]);
+                }
+#pragma unroll
+                for (int q = 0; q < kLoadBatch; ++q) cur[q] = nxt[q];
               }
               publish();
             }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) kc[q] = kn[q];
           }
         }
       }
