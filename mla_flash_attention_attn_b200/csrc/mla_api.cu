@@ -379,18 +379,16 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     }
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     if (slots > 0) {
-      // one CTA per query row, launched as a programmatic dependent of the forward
-      // kernel so that its launch overlaps the forward's last CTAs
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(r.rows, n);
+      // launched as a programmatic dependent of the forward kernel so that its launch
+      // overlaps the forward's last CTAs. Up to 16 splits: one 128-thread CTA per row
+      // (one round trip); more: one CTA per (row, quarter of the value columns)
       int ns_max = 1;
       for (int b = 0; b < n; ++b) ns_max = std::max(ns_max, plan.n_split[b]);
-      // up to 31 splits one 128-thread CTA per row walks them; from 32 on, one group of
-      // 128 threads per 16 splits (at most 4) shares the row's splits
-      const bool grouped = ns_max >= 32;
-      const int groups = grouped ? std::min(mla::kCombineGroups, ns_max / 16) : 1;
-      cfg.blockDim = dim3(128 * groups);
-      cfg.dynamicSmemBytes = grouped ? (size_t)(groups - 1) * (128 * 16 + 4) : 0;
+      const bool wide = ns_max > 16;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = wide ? dim3(r.rows, 4, n) : dim3(r.rows, n);
+      cfg.blockDim = dim3(128);
+      cfg.dynamicSmemBytes = 0;
       cfg.stream = stream;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -400,8 +398,8 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       cudaError_t ce;
       {
         ProfScope prof(kKernCombine, stream);
-        if (grouped)
-          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_grouped_kernel, plan, (const float*)p.ws_o,
+        if (wide)
+          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const float*)p.ws_o,
                                   (const float*)p.ws_lse, a.out, (int64_t)r.o_ss);
         else
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const float*)p.ws_o,

@@ -953,7 +953,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 //   O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
 // where O_s is split s normalised by its own sum and lse_s = log2 of that sum
 // relative to the split's max; splits with no kept cell have lse_s = -inf.
-// Lane s of every warp holds lse_s (the host uses this kernel below 32 splits). The
+// Lane s of every warp holds lse_s (the host uses this kernel up to 16 splits). The
 // loads of the first 16 partial rows are issued together with the lse loads, before
 // the weights are known, so a row with at most 16 splits costs one round trip to
 // memory. Launched as a programmatic dependent of the forward kernel:
@@ -1015,102 +1015,103 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   dst[threadIdx.x] = acc;
 }
 
-// The same combine for rows with many splits (one CTA per query row: blockDim.x / 128 groups
-// of 128 threads, at most kCombineGroups; thread t of a group owns value columns
-// 4t..4t+3).
-// Group q takes the splits s with s % groups == q (16 loads in flight per thread), so
-// a row's partials are read with groups x 16 loads in flight; the groups' sums and
-// weight totals meet in shared memory. The host uses it from 32 splits on, with one
-// group per 16 splits. Every warp derives M itself; lane l of a group holds the weight of the
-// group's split l (32 at a time) and broadcasts it with shuffles.
-// Launched as a programmatic dependent of the forward kernel:
-// griddepcontrol.wait returns once the forward grid has completed and its partials
-// are visible.
-constexpr int kCombineGroups = 4;
+// The same combine for rows with many splits: one CTA of 4 warps per (query row,
+// quarter of the value columns), lane l owning columns 128 q + 4l .. +3 of quarter q.
+// Every warp holds the lse of the first 96 splits (lane l: splits l, l+32, l+64) and
+// derives the weights itself; warp w sums the splits s = w (mod 4). The lse loads and
+// the loads of up to kCombPer partial rows per warp are issued together, so a row with
+// at most 96 splits costs one round trip to memory; the warps' sums meet in shared
+// memory. Launched as a programmatic dependent of the forward kernel.
+constexpr int kCombPer = 24;  // partial rows per warp held in registers
 
-__global__ void __launch_bounds__(128 * kCombineGroups)
-    mla_combine_grouped_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
-                       const float* __restrict__ ws_lse, float* __restrict__ out,
-                       int64_t out_seq_stride) {
+__global__ void __launch_bounds__(128)
+    mla_combine_wide_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
+                            const float* __restrict__ ws_lse, float* __restrict__ out,
+                            int64_t out_seq_stride) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // groups 1.. hand their sums to group 0: (groups-1) x 128 float4, then the weight
-  // totals (dynamic shared memory, none with a single group)
-  extern __shared__ float4 s_comb[];
-  const int b = blockIdx.y;
+  __shared__ float4 red[4][32];
+  const int b = blockIdx.z;
   const int row = blockIdx.x;
+  const int qtr = blockIdx.y;
   if (plan.ws_base[b] < 0 || row >= plan.rows) return;  // the whole CTA leaves
   const int ns = plan.n_split[b];
   const int lane = threadIdx.x & 31;
-  const int grp = threadIdx.x >> 7;
-  const int n_grp = blockDim.x >> 7;
-  const int col = threadIdx.x & 127;
+  const int warp = threadIdx.x >> 5;
   const int g = row / kRowsPerGroup;
   const int rin = row % kRowsPerGroup;
   const int slot0 = plan.ws_base[b] + g * ns;
   const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
-  float mx = -INFINITY;
-  for (int s = lane; s < ns; s += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)s * kRowsPerGroup));
+  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
+  const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
+                       qtr * 32 + lane;
+  float lse[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int sp = lane + 32 * k;
+    lse[k] = sp < ns ? __ldg(lse_col + (int64_t)sp * kRowsPerGroup) : -INFINITY;
+  }
+  float4 v[kCombPer];
+#pragma unroll
+  for (int j = 0; j < kCombPer; ++j) {
+    const int sp = warp + 4 * j;
+    v[j] = sp < ns ? __ldg(src0 + sp * kSplitStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float mx = fmaxf(fmaxf(lse[0], lse[1]), lse[2]);
+  for (int sp = lane + 96; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
   if (mx != -INFINITY) {  // the same for every warp
-    constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
-    const float4* src0 =
-        reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + col;
-    // this group's splits are s = grp + n_grp * j; lane l holds the weight of j0 + l
-    const int n_mine = ns > grp ? (ns - grp + n_grp - 1) / n_grp : 0;
-    for (int j0 = 0; j0 < n_mine; j0 += 32) {
-      float wl = 0.f;
-      if (j0 + lane < n_mine) {
-        const float lse = __ldg(lse_col + (int64_t)(grp + n_grp * (j0 + lane)) * kRowsPerGroup);
-        wl = lse == -INFINITY ? 0.f : ex2_approx(lse - mx);
-      }
-      wsum += wl;
-      const int cnt = min(32, n_mine - j0);
-      // batches of 16 loads issued before any is used
-      for (int jb = 0; jb < cnt; jb += 16) {
-        float4 v[16];
+    float w[3];
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          if (jb + u < cnt) v[u] = __ldg(src0 + (int64_t)(grp + n_grp * (j0 + jb + u)) * kSplitStride4);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float w = __shfl_sync(0xffffffffu, wl, jb + u);  // lanes past cnt hold 0
-          if (jb + u < cnt) {
-            acc.x = fmaf(w, v[u].x, acc.x);
-            acc.y = fmaf(w, v[u].y, acc.y);
-            acc.z = fmaf(w, v[u].z, acc.z);
-            acc.w = fmaf(w, v[u].w, acc.w);
-          }
-        }
-      }
+    for (int k = 0; k < 3; ++k) w[k] = lse[k] == -INFINITY ? 0.f : ex2_approx(lse[k] - mx);
+    wsum = (w[0] + w[1]) + w[2];
+    for (int sp = lane + 96; sp < ns; sp += 32) {
+      const float l = __ldg(lse_col + (int64_t)sp * kRowsPerGroup);
+      wsum += l == -INFINITY ? 0.f : ex2_approx(l - mx);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-  }
-  // wsum: this group's weight total (every warp of the group holds it)
-  float* s_wsum = reinterpret_cast<float*>(s_comb + (n_grp - 1) * 128);
-  if (grp > 0) {
-    s_comb[(grp - 1) * 128 + col] = acc;
-    if (col == 0) s_wsum[grp - 1] = wsum;
-  }
-  if (n_grp > 1) __syncthreads();
-  if (grp == 0) {
 #pragma unroll
-    for (int q = 0; q < kCombineGroups - 1; ++q) {
-      if (q + 1 >= n_grp) break;
-      const float4 o = s_comb[q * 128 + col];
-      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
-      wsum += s_wsum[q];
+    for (int j = 0; j < kCombPer; ++j) {
+      const int sp = warp + 4 * j;  // the same in every lane
+      const float wk = sp < 32 ? w[0] : (sp < 64 ? w[1] : w[2]);
+      const float ww = __shfl_sync(0xffffffffu, wk, sp & 31);
+      if (sp < ns && sp < 96) {
+        acc.x = fmaf(ww, v[j].x, acc.x);
+        acc.y = fmaf(ww, v[j].y, acc.y);
+        acc.z = fmaf(ww, v[j].z, acc.z);
+        acc.w = fmaf(ww, v[j].w, acc.w);
+      }
+    }
+    // splits past 96 (this warp's share), one at a time
+    for (int sp = warp + 96; sp < ns; sp += 4) {
+      const float l = __ldg(lse_col + (int64_t)sp * kRowsPerGroup);
+      const float ww = l == -INFINITY ? 0.f : ex2_approx(l - mx);
+      const float4 x = __ldg(src0 + sp * kSplitStride4);
+      acc.x = fmaf(ww, x.x, acc.x);
+      acc.y = fmaf(ww, x.y, acc.y);
+      acc.z = fmaf(ww, x.z, acc.z);
+      acc.w = fmaf(ww, x.w, acc.w);
+    }
+  }
+  red[warp][lane] = acc;
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = red[0][lane];
+#pragma unroll
+    for (int q = 1; q < 4; ++q) {
+      const float4 o = red[q][lane];
+      t.x += o.x; t.y += o.y; t.z += o.z; t.w += o.w;
     }
     if (mx != -INFINITY) {
       const float inv = 1.f / wsum;
-      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+      t.x *= inv; t.y *= inv; t.z *= inv; t.w *= inv;
     }
     float4* dst = reinterpret_cast<float4*>(out + (int64_t)(plan.seq_offset + b) * out_seq_stride +
-                                            (int64_t)row * kDV);
-    dst[col] = acc;
+                                            (int64_t)row * kDV) + qtr * 32 + lane;
+    *dst = t;
   }
 }
 
