@@ -360,23 +360,36 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
                         (uint64_t)slots * mla::kRowsPerGroup * MLA_DV * 4);
       if (rc != MLA_OK) return rc;
     }
-    dim3 grid(2 * plan.total_units);
+    // launched as a programmatic dependent of the stream's previous kernel: its setup
+    // overlaps that kernel's tail, and griddepcontrol.wait in the kernel precedes
+    // every read of its inputs
+    cudaLaunchConfig_t fcfg = {};
+    fcfg.gridDim = dim3(2 * plan.total_units);
+    fcfg.dynamicSmemBytes = mla::fwd::kSmemAlloc;
+    fcfg.stream = stream;
+    cudaLaunchAttribute fattr[1];
+    fattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    fattr[0].val.programmaticStreamSerializationAllowed = 1;
+    fcfg.attrs = fattr;
+    fcfg.numAttrs = 1;
+    cudaError_t fe;
     if (mode == mla::kModeTma) {
       ProfScope prof(kKernFwdF16, stream);
-      mla::mla_fwd_kernel<mla::kModeTma>
-          <<<grid, mla::FwdCfg<mla::kModeTma>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-              tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
+      fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeTma>::kThreads);
+      fe = cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeTma>, tm_q, tm_k, tm_v, tm_o, tm_w,
+                              plan, p);
     } else if (mode == mla::kModeGatherF16) {
       ProfScope prof(kKernFwdGather, stream);
-      mla::mla_fwd_kernel<mla::kModeGatherF16>
-          <<<grid, mla::FwdCfg<mla::kModeGatherF16>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-              tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
+      fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeGatherF16>::kThreads);
+      fe = cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeGatherF16>, tm_q, tm_k, tm_v, tm_o,
+                              tm_w, plan, p);
     } else {
       ProfScope prof(kKernFwdQ8, stream);
-      mla::mla_fwd_kernel<mla::kModeQ8>
-          <<<grid, mla::FwdCfg<mla::kModeQ8>::kThreads, mla::fwd::kSmemAlloc, stream>>>(
-              tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
+      fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeQ8>::kThreads);
+      fe = cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeQ8>, tm_q, tm_k, tm_v, tm_o, tm_w,
+                              plan, p);
     }
+    if (fe != cudaSuccess) return MLA_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     if (slots > 0) {
       // launched as a programmatic dependent of the forward kernel so that its launch

@@ -54,6 +54,9 @@ __global__ void __launch_bounds__(compact::kThreads)
   const int n_tiles = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) s_tile = atomicAdd(&tickets[row], 1);
+  // the attention kernel that follows may start its setup now; it waits for this grid
+  // to complete before it reads the index lists
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __syncthreads();
   const int tile = s_tile;
   const uint16_t* mrow = mask + (int64_t)row * mask_row_stride;

@@ -257,21 +257,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   const uint32_t rank = cluster_ctarank();
   const uint64_t to = p.timeout_ns;
 
-  // ---- work unit
-  int b, g, s;
-  decode_unit(plan, blockIdx.x >> 1, b, g, s);
-  const int b_abs = plan.seq_offset + b;
-  const int n_split = plan.n_split[b];
-  const bool sparse = p.idx != nullptr;
-  const int len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
-  const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
-  const int tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
-  const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
-  const int n_tiles = tile_end - tile_begin;
-  const int key_end = min(len, tile_end * kTileKeys);
-  const int row0 = g * kRowsPerGroup;
-
-  // ---- setup: barriers, TMEM
+  // ---- setup: barriers, TMEM (nothing here reads global memory: the kernel may run
+  // as a programmatic dependent of the kernel that writes its inputs)
   if (threadIdx.x == 0) {
     // manual modes: 2 producer warps per ring in each CTA arrive on the leader
     for (int i = 0; i < kKStages; ++i) {
@@ -303,6 +290,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // inputs written by the previous kernel of the stream (the compaction, say) are
+  // visible from here on; a launch without the programmatic attribute returns at once
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- work unit
+  int b, g, s;
+  decode_unit(plan, blockIdx.x >> 1, b, g, s);
+  const int b_abs = plan.seq_offset + b;
+  const int n_split = plan.n_split[b];
+  const bool sparse = p.idx != nullptr;
+  const int len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
+  const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
+  const int tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
+  const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
+  const int n_tiles = tile_end - tile_begin;
+  const int key_end = min(len, tile_end * kTileKeys);
+  const int row0 = g * kRowsPerGroup;
   bool failed = false;
 
   if constexpr (kManual) {
