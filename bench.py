@@ -86,9 +86,9 @@ def algorithmic(w, kept_cells=None):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "80273b11fa0f634a", "bytes": 182862080},
-    "prefill_chunk": {"source": "80273b11fa0f634a", "bytes": 209875968},
-    "sparse_q8_decode": {"source": "80273b11fa0f634a", "bytes": 10373632},
+    "v3_batched_decode": {"source": "cb8f35c8c8e195e7", "bytes": 171415296},
+    "prefill_chunk": {"source": "cb8f35c8c8e195e7", "bytes": 204832512},
+    "sparse_q8_decode": {"source": "cb8f35c8c8e195e7", "bytes": 10392320},
 }
 
 
