@@ -193,6 +193,14 @@ BUILDERS = {
     "sparse_q8_decode": sparse_q8_decode,
 }
 
+def wv_random(seed=1006, n_head=128, proj_dim=128):
+    """Synthetic value up-projection weights (no trained weights exist here): f16
+    [n_head][512][proj_dim], normal with std 1/sqrt(512) so that a projected row has
+    the scale of an attention row."""
+    rng = np.random.default_rng(seed)
+    return _normal_f16(rng, (n_head, 512, proj_dim), std=1.0 / np.sqrt(512.0))
+
+
 # Full sizes, in the order the five workloads are listed in the benchmark definition.
 WORKLOAD_ORDER = ["tiny_decode", "v2lite_decode", "v3_batched_decode", "prefill_chunk",
                   "sparse_q8_decode"]

@@ -12,7 +12,7 @@ top of ``mla_oracle.c``.
 
 Parity pins (checked by ``tests/test_oracle_pins.py`` against closed forms,
 brute force and invariants, never against the oracle itself):
-  attention / attention_online / attention_split / compact / dequant_q8_0.
+  attention / attention_online / attention_split / compact / dequant_q8_0 / project.
 """
 from __future__ import annotations
 
@@ -78,6 +78,8 @@ def _load():
         lib.oracle_compact.restype = L
         lib.oracle_dequant_q8_0.argtypes = [P, L, P]
         lib.oracle_dequant_q8_0.restype = None
+        lib.oracle_project.argtypes = [P, P, L, P, I, I, P]
+        lib.oracle_project.restype = I
         lib.oracle_init()
         _lib = lib
         return lib
@@ -214,3 +216,23 @@ def attention_batched(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None
         outs.append(attention(q[b], kcache[b], kv_type, None if mask is None else mask[b],
                               scale, None if rows is None else rows[b], ib))
     return outs
+
+
+def project(o, heads, wv):
+    """Value up-projection of attention rows: p[r][n] = sum_d o[r][d] * wv[heads[r]][d][n].
+
+    o: float64 [n_rows][512] attention rows; heads: int [n_rows], the head of each row;
+    wv: f16 [n_head][512][proj_dim]. Returns float64 [n_rows][proj_dim] (fp64 sums of
+    exact products of the f16 weights)."""
+    o = np.ascontiguousarray(o, dtype=np.float64)
+    hd = np.ascontiguousarray(heads, dtype=np.int32)
+    w = _bits16(wv)
+    if o.ndim != 2 or o.shape[1] != DV or w.ndim != 3 or w.shape[1] != DV or len(hd) != o.shape[0]:
+        raise ValueError("project: o [n][512], heads [n], wv [n_head][512][proj_dim]")
+    n_head, _, proj_dim = w.shape
+    out = np.zeros((o.shape[0], proj_dim), dtype=np.float64)
+    rc = _load().oracle_project(_ptr(o), _ptr(hd), o.shape[0], _ptr(np.ascontiguousarray(w)),
+                                n_head, proj_dim, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_project rejected its arguments")
+    return out

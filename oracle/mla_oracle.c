@@ -26,6 +26,9 @@
  *  - f16 additive mask: baguaai flash-attention tag page, item on PR #23764.
  *  - Ascending index compaction of the kept mask cells: llama.cpp b11413
  *    release note, item "single-scan sparse FA index compaction".
+ *  - Value up-projection of each head (oracle_project): wkv_b split per head into
+ *    wk_b and wv_b, "128 x 512 x 128": ik_llama.cpp -mla guide, section on tensor
+ *    derivation; p[n] = sum_d o[d] * wv[h][d][n].
  *
  * Readings where the pages are silent:
  *  - The mask is added after scaling and is not scaled itself.
@@ -324,4 +327,31 @@ long oracle_compact(const uint16_t* mask_row, long n_kv, int32_t* idx_out) {
   for (long j = 0; j < n_kv; ++j)
     if (mask_row[j] != 0xFC00u) idx_out[n++] = (int32_t)j;
   return n;
+}
+
+/* Value up-projection W_UV of each head (ik_llama.cpp -mla guide, section on tensor
+ * derivation: wkv_b is split per head into wk_b and wv_b, "128 x 512 x 128"), applied
+ * to attention rows:
+ *   p[r][n] = sum_{d<512} o[r][d] * wv[h(r)][d][n],   n < proj_dim
+ * o      : double [n_rows][512] (attention rows, e.g. from oracle_attention)
+ * heads  : int32 [n_rows], the head h(r) of each row, in [0, n_head)
+ * wv     : f16 bits [n_head][512][proj_dim]
+ * out    : double [n_rows][proj_dim]
+ * Returns 0, or -1 on a bad argument. */
+int oracle_project(const double* o, const int32_t* heads, long n_rows, const uint16_t* wv,
+                   int n_head, int proj_dim, double* out) {
+  if (!o || !heads || !wv || !out || n_rows < 0 || n_head < 1 || proj_dim < 1) return -1;
+  for (long r = 0; r < n_rows; ++r)
+    if (heads[r] < 0 || heads[r] >= n_head) return -1;
+  oracle_init();
+#pragma omp parallel for schedule(static)
+  for (long r = 0; r < n_rows; ++r) {
+    const uint16_t* w = wv + (long)heads[r] * ORC_DV * proj_dim;
+    for (int n = 0; n < proj_dim; ++n) {
+      double acc = 0.0;
+      for (int d = 0; d < ORC_DV; ++d) acc += o[r * ORC_DV + d] * g_half[w[(long)d * proj_dim + n]];
+      out[r * proj_dim + n] = acc;
+    }
+  }
+  return 0;
 }

@@ -344,3 +344,66 @@ def test_planted_mistakes_are_caught():
     no_rope = route(q_norope, k, k[:, :DV], m64)
     for bad in (wrong_v, scaled_mask, no_rope):
         assert np.max(np.abs(bad - ref)) > 1e-3
+
+
+# ---- value up-projection W_UV (oracle.project), pinned to other computations --------
+
+def _proj_inputs(seed, n_rows=12, n_head=4, proj_dim=128):
+    rng = np.random.default_rng(seed)
+    o = rng.standard_normal((n_rows, oracle.DV))
+    heads = rng.integers(0, n_head, n_rows).astype(np.int32)
+    wv = (rng.standard_normal((n_head, oracle.DV, proj_dim)) * 0.05).astype(np.float16)
+    return o, heads, wv
+
+
+def test_project_one_hot_weights_select_columns_exactly():
+    # wv[h][d][n] = 1 where d = sel[h][n]: each output is one input column, exactly
+    rng = np.random.default_rng(51)
+    n_head, proj_dim, n_rows = 3, 128, 10
+    o = rng.standard_normal((n_rows, oracle.DV))
+    heads = rng.integers(0, n_head, n_rows).astype(np.int32)
+    sel = np.stack([rng.permutation(oracle.DV)[:proj_dim] for _ in range(n_head)])
+    wv = np.zeros((n_head, oracle.DV, proj_dim), dtype=np.float16)
+    for h in range(n_head):
+        wv[h, sel[h], np.arange(proj_dim)] = 1.0
+    got = oracle.project(o, heads, wv)
+    want = np.stack([o[r, sel[heads[r]]] for r in range(n_rows)])
+    assert np.array_equal(got, want)
+
+
+def test_project_weights_of_each_head_are_its_own():
+    # head h scales its selector by 2^h: a row projected with another head's matrix
+    # would come out with the wrong power of two
+    rng = np.random.default_rng(52)
+    n_head, n_rows = 4, 16
+    o = rng.standard_normal((n_rows, oracle.DV))
+    heads = (np.arange(n_rows) % n_head).astype(np.int32)
+    wv = np.zeros((n_head, oracle.DV, 128), dtype=np.float16)
+    for h in range(n_head):
+        wv[h, np.arange(128), np.arange(128)] = 2.0 ** h
+    got = oracle.project(o, heads, wv)
+    want = np.stack([o[r, :128] * 2.0 ** heads[r] for r in range(n_rows)])
+    assert np.array_equal(got, want)
+
+
+def test_project_scales_exactly_with_a_power_of_two():
+    o, heads, wv = _proj_inputs(53)
+    a = oracle.project(o, heads, wv)
+    b = oracle.project(o, heads, (wv.astype(np.float32) * 4).astype(np.float16))
+    assert np.array_equal(b, 4 * a)
+
+
+def test_project_matches_an_independent_contraction():
+    # numpy's fp64 contraction over the exactly converted f16 weights; only the
+    # summation order differs
+    o, heads, wv = _proj_inputs(54)
+    want = np.einsum("rd,rdn->rn", o, wv.astype(np.float64)[heads])
+    got = oracle.project(o, heads, wv)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+def test_project_rejects_bad_heads():
+    o, heads, wv = _proj_inputs(55)
+    heads[3] = 4  # n_head is 4
+    with pytest.raises(ValueError):
+        oracle.project(o, heads, wv)
