@@ -50,6 +50,7 @@ extern "C" {
 #define MLA_Q8_0_BLOCK 32     /* q8_0: 32 int8 per block                        */
 #define MLA_Q8_0_ROW_BYTES 612 /* q8_0: 18 blocks x {f16 d; int8 q[32]}         */
 #define MLA_MAX_HEADS 128
+#define MLA_PROJ_DIM 128      /* output width of the fused value up-projection   */
 
 typedef enum {
   MLA_KV_F16 = 0,  /* row = 576 f16 (1152 bytes) */
@@ -88,6 +89,15 @@ typedef enum {
  *         as mla_compact_mask writes them, ascending; the mask (if any) is still
  *         indexed by the original cell j = idx[...]
  * idx_count DEVICE int32[n_seq]; required with idx. Read on the device: no host sync.
+ * wv      DEVICE f16 or NULL: the value up-projection W_UV of each head, element
+ *         (h, d, n) at wv[(h*512 + d)*proj_dim + n] (wv_b of the ik_llama.cpp -mla guide,
+ *         section on tensor derivation: per head 512 latent columns -> 128). When set,
+ *         the call writes out_proj instead of out (out may then be NULL):
+ *           out_proj(b, t, h, n) = sum_{d<512} O(b, t, h, d) * wv(h, d, n)
+ *         with O the attention row that out would hold; 16-byte aligned
+ * proj_dim output width of the projection; must be MLA_PROJ_DIM (128) when wv is set
+ * out_proj DEVICE fp32, element (b, t, h, n) at
+ *         out_proj[b*out_proj_seq_stride + (t*n_head + h)*proj_dim + n]; 16-byte aligned
  * A stride of 0 means "dense" (the natural value for the given sizes).
  */
 typedef struct mla_fa_args {
@@ -110,6 +120,10 @@ typedef struct mla_fa_args {
   const int32_t* idx;       /* DEVICE, optional (sparse)                       */
   const int32_t* idx_count; /* DEVICE, required with idx                       */
   int64_t idx_seq_stride;   /* entries;  0 = n_kv                              */
+  const void* wv;           /* DEVICE, optional: fused value up-projection     */
+  int proj_dim;             /* MLA_PROJ_DIM when wv is set                     */
+  float* out_proj;          /* DEVICE, required with wv                        */
+  int64_t out_proj_seq_stride; /* elements; 0 = n_q*n_head*proj_dim            */
 } mla_fa_args;
 
 /* Forward pass with the sizes of the single-sequence call:
@@ -132,7 +146,11 @@ size_t mla_fa_workspace_size(const mla_fa_args* a);
 /* Batched / sparse forward pass into caller-owned workspace (device memory of
  * at least mla_fa_workspace_size(a) bytes, 256-byte aligned; may be NULL when
  * that size is 0). Split-KV partials go to the workspace and are merged by the
- * log-sum-exp combine before the call's last kernel ends. */
+ * log-sum-exp combine before the call's last kernel ends. With wv set, every
+ * sequence writes partials (so the workspace is never 0 bytes) and the combine
+ * applies the projection. Errors: wv without out_proj MLA_ERR_NULL, proj_dim other
+ * than MLA_PROJ_DIM MLA_ERR_UNSUPPORTED, misaligned wv / out_proj / stride
+ * MLA_ERR_ALIGN. */
 int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, void* stream);
 
 /* Forward pass for callers that cannot allocate device memory. The paper has no

@@ -57,6 +57,10 @@ class mla_fa_args(ctypes.Structure):
         ("idx", ctypes.c_void_p),
         ("idx_count", ctypes.c_void_p),
         ("idx_seq_stride", ctypes.c_int64),
+        ("wv", ctypes.c_void_p),
+        ("proj_dim", ctypes.c_int),
+        ("out_proj", ctypes.c_void_p),
+        ("out_proj_seq_stride", ctypes.c_int64),
     ]
 
 
@@ -145,12 +149,14 @@ def _host_i32(arr):
     return (ctypes.c_int32 * len(vals))(*vals)
 
 
-def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None):
+def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None,
+              wv=None, out_proj=None):
     """Fill mla_fa_args from batched torch tensors.
 
     q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
-    mask [n_seq][n_q][n_kv] f16 or None; out [n_seq][n_q][n_head][512] f32.
-    Returns (args, keepalive)."""
+    mask [n_seq][n_q][n_kv] f16 or None; out [n_seq][n_q][n_head][512] f32 (or None with
+    wv); wv [n_head][512][128] f16 and out_proj [n_seq][n_q][n_head][128] f32 for the
+    fused value up-projection. Returns (args, keepalive)."""
     n_seq, n_q, n_head, dk = q.shape
     if dk != DK:
         raise ValueError("q must end in 576")
@@ -159,7 +165,7 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     a.kcache = kcache.data_ptr()
     a.kcache_type = int(kv_type)
     a.mask = None if mask is None else mask.data_ptr()
-    a.out = out.data_ptr()
+    a.out = None if out is None else out.data_ptr()
     a.n_seq, a.n_q, a.n_head, a.n_kv = n_seq, n_q, n_head, kcache.shape[1]
     a.scale = float(scale)
     a.q_seq_stride = q.stride(0)
@@ -167,7 +173,12 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     if mask is not None:
         a.mask_seq_stride = mask.stride(0)
         a.mask_row_stride = mask.stride(1)
-    a.out_seq_stride = out.stride(0)
+    a.out_seq_stride = 0 if out is None else out.stride(0)
+    if wv is not None:
+        a.wv = wv.data_ptr()
+        a.proj_dim = int(wv.shape[2])
+        a.out_proj = None if out_proj is None else out_proj.data_ptr()
+        a.out_proj_seq_stride = 0 if out_proj is None else out_proj.stride(0)
     keep = _host_i32(kv_len)
     a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
     if idx is not None:
@@ -218,6 +229,24 @@ def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, id
     mla_fa_forward_ex(args, workspace if need else None, stream)
     del keep
     return out
+
+
+def forward_proj(q, kcache, kv_type, mask, scale, wv, out_proj=None, kv_len=None, idx=None,
+                 idx_count=None, workspace=None, stream=None):
+    """Forward with the fused value up-projection (wv [n_head][512][128] f16); returns
+    out_proj [n_seq][n_q][n_head][128] f32. The 512-wide attention rows are not written."""
+    import torch
+
+    if out_proj is None:
+        out_proj = torch.empty(q.shape[:3] + (int(wv.shape[2]),), dtype=torch.float32, device=q.device)
+    args, keep = make_args(q, kcache, kv_type, mask, None, scale, kv_len, idx, idx_count, wv=wv,
+                           out_proj=out_proj)
+    need = mla_fa_workspace_size(args)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    mla_fa_forward_ex(args, workspace if need else None, stream)
+    del keep
+    return out_proj
 
 
 def mla_compact_mask(mask_row, idx_out, count_out, stream=None):

@@ -151,12 +151,16 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 struct Resolved {
   mla_fa_args a;
   int rows;
-  int64_t q_ss, k_ss, m_ss, m_rs, o_ss, idx_ss;
+  int64_t q_ss, k_ss, m_ss, m_rs, o_ss, idx_ss, op_ss;
+  bool proj;  // fused value up-projection: every sequence writes split partials
 };
 
 int validate(const mla_fa_args* a, Resolved* r) {
   if (a == nullptr) return MLA_ERR_NULL;
-  if (a->q == nullptr || a->kcache == nullptr || a->out == nullptr) return MLA_ERR_NULL;
+  const bool proj = a->wv != nullptr;
+  if (a->q == nullptr || a->kcache == nullptr || (a->out == nullptr && !proj)) return MLA_ERR_NULL;
+  if (proj && a->out_proj == nullptr) return MLA_ERR_NULL;
+  if (proj && a->proj_dim != MLA_PROJ_DIM) return MLA_ERR_UNSUPPORTED;
   if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
   if (a->n_seq < 1 || a->n_q < 1 || a->n_head < 1 || a->n_head > MLA_MAX_HEADS || a->n_kv < 1)
     return MLA_ERR_SHAPE;
@@ -172,6 +176,11 @@ int validate(const mla_fa_args* a, Resolved* r) {
   r->m_ss = a->mask_seq_stride ? a->mask_seq_stride : (int64_t)a->n_q * r->m_rs;
   r->o_ss = a->out_seq_stride ? a->out_seq_stride : rows * MLA_DV;
   r->idx_ss = a->idx_seq_stride ? a->idx_seq_stride : a->n_kv;
+  r->proj = proj;
+  r->op_ss = proj ? (a->out_proj_seq_stride ? a->out_proj_seq_stride : rows * MLA_PROJ_DIM) : 0;
+  if (proj && (a->out_proj_seq_stride < 0 || r->op_ss < rows * MLA_PROJ_DIM)) return MLA_ERR_SHAPE;
+  if (proj && (!aligned16(a->wv) || !aligned16(a->out_proj) || (r->op_ss % 4) != 0))
+    return MLA_ERR_ALIGN;
   if (r->q_ss < rows * MLA_DK || r->k_ss < a->n_kv || r->m_rs < a->n_kv ||
       r->m_ss < (int64_t)(a->n_q - 1) * r->m_rs + a->n_kv || r->o_ss < rows * MLA_DV ||
       r->idx_ss < 0)
@@ -179,7 +188,8 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (a->q_seq_stride < 0 || a->k_seq_stride < 0 || a->mask_seq_stride < 0 ||
       a->mask_row_stride < 0 || a->out_seq_stride < 0 || a->idx_seq_stride < 0)
     return MLA_ERR_SHAPE;
-  if (!aligned16(a->q) || !aligned16(a->kcache) || !aligned16(a->out)) return MLA_ERR_ALIGN;
+  if (!aligned16(a->q) || !aligned16(a->kcache) || (a->out != nullptr && !aligned16(a->out)))
+    return MLA_ERR_ALIGN;
   if ((r->q_ss % 8) != 0 || (r->o_ss % 4) != 0) return MLA_ERR_ALIGN;
   if (a->mask != nullptr && (reinterpret_cast<uintptr_t>(a->mask) & 1)) return MLA_ERR_ALIGN;
   if (a->kv_len != nullptr)
@@ -226,7 +236,7 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
     plan->n_split[b] = ns;
     plan->unit_base[b] = units;
     units += plan->groups * ns;
-    if (ns > 1) {
+    if (ns > 1 || r.proj) {
       plan->ws_base[b] = slots;
       slots += plan->groups * ns;
     } else {
@@ -313,8 +323,15 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     tm_v = tm_q;
   }
   CUtensorMap tm_o;
-  if (rc == MLA_OK)
-    rc = make_out_map(&tm_o, a.out, (uint64_t)r.rows, (uint64_t)a.n_seq, (uint64_t)r.o_ss * 4);
+  // with the projection every sequence writes partials and the kernel never stores
+  // to out (which may be NULL): the output map then views the workspace
+  if (rc == MLA_OK) {
+    if (r.proj)
+      rc = make_out_map(&tm_o, ws, (uint64_t)mla::kRowsPerGroup, 1,
+                        (uint64_t)mla::kRowsPerGroup * MLA_DV * 4);
+    else
+      rc = make_out_map(&tm_o, a.out, (uint64_t)r.rows, (uint64_t)a.n_seq, (uint64_t)r.o_ss * 4);
+  }
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
     if (cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeTma>,
@@ -401,6 +418,12 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = wide ? dim3(r.rows, 4, n) : dim3(r.rows, n);
       cfg.blockDim = dim3(128);
+      if (r.proj) {
+        // fused projection: one CTA per (head, batch of 8 (sequence, token) rows)
+        const int nrows = n * a.n_q;
+        cfg.gridDim = dim3(a.n_head, (nrows + mla::kProjRows - 1) / mla::kProjRows);
+        cfg.blockDim = dim3(256);
+      }
       cfg.dynamicSmemBytes = 0;
       cfg.stream = stream;
       cudaLaunchAttribute attr[1];
@@ -411,7 +434,11 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       cudaError_t ce;
       {
         ProfScope prof(kKernCombine, stream);
-        if (wide)
+        if (r.proj)
+          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_proj_kernel, plan, (const float*)p.ws_o,
+                                  (const float*)p.ws_lse, static_cast<const uint16_t*>(a.wv),
+                                  a.out_proj, (int64_t)r.op_ss);
+        else if (wide)
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const float*)p.ws_o,
                                   (const float*)p.ws_lse, a.out, (int64_t)r.o_ss);
         else

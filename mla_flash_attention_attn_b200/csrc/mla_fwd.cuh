@@ -1119,6 +1119,139 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// LSE combine fused with the value up-projection W_UV of each head (ik_llama.cpp -mla
+// guide, section on tensor derivation: wkv_b is split per head into wk_b and wv_b,
+// "128 x 512 x 128"; Vulkan FA article, section 6.1: fold the projection matrices into
+// the attention kernel):
+//   out_proj[b][t][h][n] = sum_{d<512} O[b][t][h][d] * wv[h][d][n],   n < 128,
+// where O is the combined, normalised attention row (as mla_combine_kernel computes it).
+// One CTA of 8 warps per (head h, batch of kProjRows (b, t) rows of this launch): warp w
+// combines row w of the batch into shared memory; then thread (warp w, lane l) takes
+// latent columns [64w, 64w+64), output columns 8 (l % 16) .. +7 and rows 4 (l / 16) ..
+// +3, reading W_h as 16-byte vectors (W_h, 128 KB, is read once per CTA); the 8 warps'
+// partial sums meet in shared memory. Launched as a programmatic dependent of the
+// forward kernel.
+constexpr int kProjRows = 8;
+constexpr int kProjDim = 128;
+
+__global__ void __launch_bounds__(256)
+    mla_combine_proj_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
+                            const float* __restrict__ ws_lse, const uint16_t* __restrict__ wv,
+                            float* __restrict__ out_proj, int64_t op_seq_stride) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // o_s: the batch's combined rows; afterwards reused for the warps' partial sums
+  __shared__ __align__(16) float smem_f[8 * kProjRows * kProjDim];  // 32 KB
+  float (*o_s)[kDV] = reinterpret_cast<float (*)[kDV]>(smem_f);
+  const int h = blockIdx.x;
+  const int j0 = blockIdx.y * kProjRows;
+  const int nrows = plan.n_seq * plan.n_q;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;
+  {
+    // ---- combine row j0 + warp (lane l owns value columns 4 (l + 32u) .. +3, u < 4)
+    const int j = j0 + warp;
+    float4 acc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < nrows) {
+      const int b = j / plan.n_q, t = j - (j / plan.n_q) * plan.n_q;
+      const int row = t * plan.n_head + h;
+      const int ns = plan.n_split[b];
+      const int slot0 = plan.ws_base[b] + (row / kRowsPerGroup) * ns;
+      const int rin = row % kRowsPerGroup;
+      const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
+      const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + lane;
+      float mx = -INFINITY;
+      for (int sp = lane; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (mx != -INFINITY) {
+        float wsum = 0.f;
+        for (int s0 = 0; s0 < ns; s0 += 32) {
+          float wl = 0.f;
+          if (s0 + lane < ns) {
+            const float l = __ldg(lse_col + (int64_t)(s0 + lane) * kRowsPerGroup);
+            wl = l == -INFINITY ? 0.f : ex2_approx(l - mx);
+          }
+          wsum += wl;
+          const int cnt = min(32, ns - s0);
+#pragma unroll 4
+          for (int jj = 0; jj < cnt; ++jj) {
+            const float w = __shfl_sync(0xffffffffu, wl, jj);
+            const float4* src = src0 + (int64_t)(s0 + jj) * kSplitStride4;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float4 v = __ldg(src + 32 * u);
+              acc[u].x = fmaf(w, v.x, acc[u].x);
+              acc[u].y = fmaf(w, v.y, acc[u].y);
+              acc[u].z = fmaf(w, v.z, acc[u].z);
+              acc[u].w = fmaf(w, v.w, acc[u].w);
+            }
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+        const float inv = 1.f / wsum;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc[u].x *= inv; acc[u].y *= inv; acc[u].z *= inv; acc[u].w *= inv;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) reinterpret_cast<float4*>(o_s[warp])[lane + 32 * u] = acc[u];
+  }
+  __syncthreads();
+  // ---- project: latent columns [64 warp, +64), output columns 8 ng .. +7, rows 4 rg .. +3
+  const int ng = lane & 15, rg = lane >> 4;
+  float a[4][8];
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) a[r][c] = 0.f;
+  const uint4* wrow = reinterpret_cast<const uint4*>(wv + ((int64_t)h * kDV + 64 * warp) * kProjDim) + ng;
+#pragma unroll 16
+  for (int d = 0; d < 64; ++d) {
+    const uint4 w4 = __ldg(wrow + d * (kProjDim / 8));
+    const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+    float wf[8];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[c]));
+      wf[2 * c] = f.x;
+      wf[2 * c + 1] = f.y;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float o = o_s[4 * rg + r][64 * warp + d];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) a[r][c] = fmaf(o, wf[c], a[r][c]);
+    }
+  }
+  __syncthreads();  // every thread has read o_s; the buffer now takes the partial sums
+  float* red = smem_f;  // [warp][row][n]
+#pragma unroll
+  for (int r = 0; r < 4; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      red[(warp * kProjRows + 4 * rg + r) * kProjDim + 8 * ng + c] = a[r][c];
+  __syncthreads();
+  // ---- sum the 8 warps' partials: thread i writes outputs i, i + 256, i + 512, i + 768
+#pragma unroll
+  for (int k = 0; k < kProjRows * kProjDim / 256; ++k) {
+    const int e = threadIdx.x + 256 * k;
+    const int r = e / kProjDim, n = e % kProjDim;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += red[(w * kProjRows + r) * kProjDim + n];
+    const int j = j0 + r;
+    if (j < nrows) {
+      const int b = j / plan.n_q, t = j - (j / plan.n_q) * plan.n_q;
+      out_proj[(int64_t)(plan.seq_offset + b) * op_seq_stride + (int64_t)(t * plan.n_head + h) * kProjDim + n] = sum;
+    }
+  }
+}
+
 // Waits on a barrier that nothing ever signals, with a bounded wait, and records
 // the timeout: exercises the run-time error path without faulting anything.
 __global__ void mla_wait_timeout_kernel(uint64_t timeout_ns) {

@@ -64,10 +64,29 @@ def call_ex(lib, a):
     (dict(q_seq_stride=100, n_seq=2), -2), (dict(k_seq_stride=10, n_seq=2), -2),
     (dict(mask=FAKE, mask_row_stride=5), -2), (dict(out_seq_stride=-1), -2),
     (dict(idx=FAKE), -1),
+    # fused value up-projection
+    (dict(wv=FAKE, proj_dim=128), -1),                                  # no out_proj
+    (dict(wv=FAKE, proj_dim=64, out_proj=FAKE), -8),                    # width not 128
+    (dict(wv=FAKE + 2, proj_dim=128, out_proj=FAKE), -4),
+    (dict(wv=FAKE, proj_dim=128, out_proj=FAKE + 4), -4),
+    (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, out_proj_seq_stride=100, n_seq=2), -2),
+    (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, out_proj_seq_stride=16 * 128 + 2, n_seq=2), -4),
 ])
 def test_argument_errors_are_returned_before_any_launch(lib, kw, expect):
     assert call_ex(lib, base_args(**kw)) == expect
     assert lib.mla_fa_workspace_size(ctypes.byref(base_args(**kw))) == 0
+
+
+def test_projection_lets_out_be_null(lib):
+    # out may be NULL when the projection is requested: without a GPU the valid call
+    # stops at the device check, never at argument validation. The fake pointers must
+    # never reach a kernel, so this runs only where no GPU exists.
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers: only meaningful without a GPU")
+    a = base_args(out=None, wv=FAKE, proj_dim=128, out_proj=FAKE)
+    assert call_ex(lib, a) in (-6, -8)
 
 
 def test_kv_len_out_of_range_is_rejected(lib):

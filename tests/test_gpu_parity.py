@@ -414,3 +414,59 @@ def test_sparse_out_of_range_index_is_reported_not_read():
     ok = np.array([3, 10, 299, 17], np.int32)
     ref = oracle.attention(w.q[0], w.kcache[0], 0, w.mask[0], w.scale, idx=ok)
     assert_parity(got[0].reshape(-1, 512), ref, "bad index dropped")
+
+
+# ---- fused value up-projection (out_proj = O . W_UV per head) ---------------------
+
+def run_gpu_proj(w, wv):
+    """mla_fa_forward_ex with wv set; returns out_proj [n_seq][n_q][n_head][128]."""
+    torch = torch_mod()
+    dev = torch.device("cuda")
+    q = torch.from_numpy(w.q).to(dev)
+    k = torch.from_numpy(w.kcache).to(dev)
+    m = torch.from_numpy(w.mask).to(dev) if w.mask is not None else None
+    n_out = w.n_seq * w.n_q * w.n_head * 128
+    big = torch.full((n_out + CANARY,), float("nan"), dtype=torch.float32, device=dev)
+    out_proj = big[:n_out].view(w.n_seq, w.n_q, w.n_head, 128)
+    binding.forward_proj(q, k, w.kv_type, m, w.scale, torch.from_numpy(wv).to(dev),
+                         out_proj=out_proj, kv_len=w.kv_len)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    assert bool(torch.isnan(big[n_out:]).all()), "write past the end of out_proj"
+    return out_proj.cpu().numpy()
+
+
+def check_proj(w, wv, got, what):
+    rows = w.n_q * w.n_head
+    heads = np.arange(rows) % w.n_head
+    for b in range(w.n_seq):
+        ref = oracle.project(oracle_rows(w, b), heads, wv)
+        assert_parity(got[b].reshape(rows, 128), ref, f"{what} seq {b}")
+
+
+@pytest.mark.parametrize("case", ["v3_split", "tiny_unsplit", "prefill_rows", "ragged_heads"])
+def test_fused_projection_matches_oracle(case):
+    if case == "v3_split":      # 8 sequences, split-KV partials
+        w = W.make("v3_batched_decode", n_kv=2048, len_lo=100, len_hi=2048)
+    elif case == "tiny_unsplit":  # one unit: the partial slot is forced
+        w = W.make("tiny_decode", n_kv=300)
+    elif case == "prefill_rows":  # 8 tokens x 128 heads: row batches span tokens
+        w = W.make("prefill_chunk", n_q=8, n_head=128, n_kv=640)
+    else:                          # 3 tokens x 5 heads: the last row batch is partial
+        w = W.make("prefill_chunk", n_q=3, n_head=5, n_kv=300)
+    wv = W.wv_random(n_head=w.n_head)
+    got = run_gpu_proj(w, wv)
+    check_proj(w, wv, got, case)
+
+
+def test_fused_projection_with_an_empty_sequence():
+    # a zero-length sequence projects a zero row (its lengths also set in the mask,
+    # which the oracle follows)
+    w = W.make("v3_batched_decode", n_seq=3, n_head=16, n_kv=700, len_lo=0, len_hi=700)
+    w.kv_len[:] = [300, 0, 700]
+    keep = np.arange(700)[None, :] < w.kv_len[:, None]
+    w.mask[:, 0, :] = np.where(keep, np.float16(0), np.float16(-np.inf))
+    wv = W.wv_random(n_head=16)
+    got = run_gpu_proj(w, wv)
+    assert np.all(got[1] == 0.0)
+    check_proj(w, wv, got, "kv_len 300/0/700")
