@@ -64,7 +64,9 @@ typedef enum {
   MLA_ERR_TYPE = -3,        /* unknown kcache_type                             */
   MLA_ERR_ALIGN = -4,       /* a pointer or stride breaks 16-byte alignment    */
   MLA_ERR_WORKSPACE = -5,   /* workspace missing or smaller than required      */
-  MLA_ERR_CUDA = -6,        /* a CUDA runtime call failed                      */
+  MLA_ERR_CUDA = -6,        /* a CUDA runtime call failed; as a device status:
+                               a kernel launched with less dynamic shared memory
+                               than it needs (it returned without working)      */
   MLA_ERR_TIMEOUT = -7,     /* a kernel's bounded wait ran out (device status) */
   MLA_ERR_UNSUPPORTED = -8, /* valid but unsupported (e.g. no sm_100 device)   */
   MLA_ERR_INDEX = -9        /* a sparse index outside [0, n_kv) (device status) */

@@ -342,7 +342,10 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
                              mla::fwd::kSmemAlloc) != cudaSuccess ||
         cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeQ8>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             mla::fwd::kSmemAlloc) != cudaSuccess)
+                             mla::fwd::kSmemAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(mla::mla_combine_proj_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mla::kProjSmem) != cudaSuccess)
       return MLA_ERR_CUDA;
     st->fwd_attr_set = true;
   }
@@ -418,13 +421,15 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = wide ? dim3(r.rows, 4, n) : dim3(r.rows, n);
       cfg.blockDim = dim3(128);
-      if (r.proj) {
-        // fused projection: one CTA per (head, batch of 8 (sequence, token) rows)
-        const int nrows = n * a.n_q;
-        cfg.gridDim = dim3(a.n_head, (nrows + mla::kProjRows - 1) / mla::kProjRows);
-        cfg.blockDim = dim3(256);
-      }
       cfg.dynamicSmemBytes = 0;
+      if (r.proj) {
+        // fused projection: a cluster of 4 CTAs (the quarters of the latent columns) per
+        // (head, batch of 8 (sequence, token) rows)
+        const int nrows = n * a.n_q;
+        cfg.gridDim = dim3(a.n_head, 4 * ((nrows + mla::kProjRows - 1) / mla::kProjRows));
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = mla::kProjSmem;
+      }
       cfg.stream = stream;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -15,6 +15,7 @@ constexpr int kQ8RowBytes = 612;     // q8_0: 18 blocks of {f16 d; int8 q[32]}
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Status codes written by kernels (same values as mla_status in mla_fa.h).
+constexpr int kStatusLaunch = -6;   // launched with less dynamic shared memory than it needs
 constexpr int kStatusTimeout = -7;
 constexpr int kStatusIndex = -9;
 

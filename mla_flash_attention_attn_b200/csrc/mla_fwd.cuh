@@ -241,6 +241,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   using namespace fwd;
   constexpr bool kManual = FwdCfg<kMode>::kManual;
   extern __shared__ uint8_t smem_raw[];
+  // a launch with too little dynamic shared memory reports and returns (every CTA takes
+  // this branch, so no cluster barrier is left waiting)
+  if (dynamic_smem_bytes() < (uint32_t)fwd::kSmemAlloc) {
+    if (threadIdx.x == 0) record_status(kStatusLaunch);
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem + kOffQ;
@@ -1125,34 +1131,61 @@ __global__ void __launch_bounds__(128)
 // the attention kernel):
 //   out_proj[b][t][h][n] = sum_{d<512} O[b][t][h][d] * wv[h][d][n],   n < 128,
 // where O is the combined, normalised attention row (as mla_combine_kernel computes it).
-// One CTA of 8 warps per (head h, batch of kProjRows (b, t) rows of this launch): warp w
-// combines row w of the batch into shared memory; then thread (warp w, lane l) takes
-// latent columns [64w, 64w+64), output columns 8 (l % 16) .. +7 and rows 4 (l / 16) ..
-// +3, reading W_h as 16-byte vectors (W_h, 128 KB, is read once per CTA); the 8 warps'
-// partial sums meet in shared memory. Launched as a programmatic dependent of the
-// forward kernel.
+// A cluster of 4 CTAs per (head h, batch of kProjRows (b, t) rows of this launch); CTA q
+// of the cluster takes latent columns [128q, 128q+128). Its 32 KB slice of W_h is one
+// contiguous bulk copy into shared memory, issued first. The combine is separable by
+// column, so CTA q reads only its quarter of the partial rows: warp w combines row w of
+// the batch (lane l: columns 4l..4l+3 of the quarter), with the lse of up to 96 splits
+// and the first 16 partial rows loaded together. Then thread (warp w, lane l) multiplies
+// latent columns 16w..16w+15 of the quarter into output columns 8 (l % 16) .. +7 of rows
+// 4 (l / 16) .. +3; the 8 warps' sums meet in shared memory, and the 4 CTAs' sums over
+// distributed shared memory (CTA q adds up rows 2q, 2q+1). Launched as a programmatic
+// dependent of the forward kernel.
 constexpr int kProjRows = 8;
 constexpr int kProjDim = 128;
+constexpr int kProjWBytes = 128 * kProjDim * 2;                       // W slice: 32 KB
+constexpr int kProjORow = 132;                                        // padded o_s row
+constexpr int kProjSmem = kProjWBytes + kProjRows * kProjORow * 4 +   // W, o_s
+                          8 * kProjRows * kProjDim * 4 +              // warps' sums
+                          kProjRows * kProjDim * 4 + 16;              // CTA sum, barrier
 
-__global__ void __launch_bounds__(256)
+__global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
     mla_combine_proj_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, const uint16_t* __restrict__ wv,
                             float* __restrict__ out_proj, int64_t op_seq_stride) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // o_s: the batch's combined rows; afterwards reused for the warps' partial sums
-  __shared__ __align__(16) float smem_f[8 * kProjRows * kProjDim];  // 32 KB
-  float (*o_s)[kDV] = reinterpret_cast<float (*)[kDV]>(smem_f);
+  extern __shared__ __align__(128) uint8_t proj_smem[];
+  // a launch with too little dynamic shared memory reports and returns (every CTA takes
+  // this branch, so no cluster barrier is left waiting)
+  if (dynamic_smem_bytes() < (uint32_t)kProjSmem) {
+    if (threadIdx.x == 0) record_status(kStatusLaunch);
+    return;
+  }
+  const uint16_t* w_s = reinterpret_cast<const uint16_t*>(proj_smem);               // [128 d][128 n]
+  float (*o_s)[kProjORow] = reinterpret_cast<float (*)[kProjORow]>(proj_smem + kProjWBytes);
+  float (*red)[kProjRows][kProjDim] =
+      reinterpret_cast<float (*)[kProjRows][kProjDim]>(proj_smem + kProjWBytes + kProjRows * kProjORow * 4);
+  float (*part)[kProjDim] = reinterpret_cast<float (*)[kProjDim]>(
+      proj_smem + kProjWBytes + kProjRows * kProjORow * 4 + 8 * kProjRows * kProjDim * 4);
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(
+      proj_smem + kProjWBytes + kProjRows * kProjORow * 4 + 8 * kProjRows * kProjDim * 4 + kProjRows * kProjDim * 4);
   const int h = blockIdx.x;
-  const int j0 = blockIdx.y * kProjRows;
+  const uint32_t qtr = cluster_ctarank();
+  const int j0 = (int)(blockIdx.y >> 2) * kProjRows;
   const int nrows = plan.n_seq * plan.n_q;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;
+  // this CTA's slice of W_h first (it does not depend on the combine)
+  if (threadIdx.x == 0) {
+    mbar_init(wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(wbar, kProjWBytes);
+    bulk_load(proj_smem, wv + ((int64_t)h * kDV + 128 * qtr) * kProjDim, kProjWBytes, wbar);
+  }
   {
-    // ---- combine row j0 + warp (lane l owns value columns 4 (l + 32u) .. +3, u < 4)
+    // ---- combine columns 128 qtr + 4 lane .. +3 of row j0 + warp
     const int j = j0 + warp;
-    float4 acc[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (j < nrows) {
       const int b = j / plan.n_q, t = j - (j / plan.n_q) * plan.n_q;
       const int row = t * plan.n_head + h;
@@ -1160,59 +1193,76 @@ __global__ void __launch_bounds__(256)
       const int slot0 = plan.ws_base[b] + (row / kRowsPerGroup) * ns;
       const int rin = row % kRowsPerGroup;
       const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
-      const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + lane;
-      float mx = -INFINITY;
-      for (int sp = lane; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
+      const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
+                           32 * qtr + lane;
+      float lse[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const int sp = lane + 32 * k;
+        lse[k] = sp < ns ? __ldg(lse_col + (int64_t)sp * kRowsPerGroup) : -INFINITY;
+      }
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        v[u] = u < ns ? __ldg(src0 + (int64_t)u * kSplitStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      float mx = fmaxf(fmaxf(lse[0], lse[1]), lse[2]);
+      for (int sp = lane + 96; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (mx != -INFINITY) {
-        float wsum = 0.f;
-        for (int s0 = 0; s0 < ns; s0 += 32) {
-          float wl = 0.f;
-          if (s0 + lane < ns) {
-            const float l = __ldg(lse_col + (int64_t)(s0 + lane) * kRowsPerGroup);
-            wl = l == -INFINITY ? 0.f : ex2_approx(l - mx);
-          }
-          wsum += wl;
-          const int cnt = min(32, ns - s0);
-#pragma unroll 4
-          for (int jj = 0; jj < cnt; ++jj) {
-            const float w = __shfl_sync(0xffffffffu, wl, jj);
-            const float4* src = src0 + (int64_t)(s0 + jj) * kSplitStride4;
+        float wk[3];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float4 v = __ldg(src + 32 * u);
-              acc[u].x = fmaf(w, v.x, acc[u].x);
-              acc[u].y = fmaf(w, v.y, acc[u].y);
-              acc[u].z = fmaf(w, v.z, acc[u].z);
-              acc[u].w = fmaf(w, v.w, acc[u].w);
-            }
-          }
+        for (int k = 0; k < 3; ++k) wk[k] = lse[k] == -INFINITY ? 0.f : ex2_approx(lse[k] - mx);
+        float wsum = (wk[0] + wk[1]) + wk[2];
+        for (int sp = lane + 96; sp < ns; sp += 32) {
+          const float l = __ldg(lse_col + (int64_t)sp * kRowsPerGroup);
+          wsum += l == -INFINITY ? 0.f : ex2_approx(l - mx);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-        const float inv = 1.f / wsum;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          acc[u].x *= inv; acc[u].y *= inv; acc[u].z *= inv; acc[u].w *= inv;
+        for (int u = 0; u < 16; ++u) {
+          const float w = __shfl_sync(0xffffffffu, wk[0], u);  // 0 past ns
+          acc.x = fmaf(w, v[u].x, acc.x);
+          acc.y = fmaf(w, v[u].y, acc.y);
+          acc.z = fmaf(w, v[u].z, acc.z);
+          acc.w = fmaf(w, v[u].w, acc.w);
         }
+        for (int sp = 16; sp < ns; ++sp) {
+          float w;  // split sp's weight, the same in every lane
+          if (sp < 96) {
+            const float x = sp < 32 ? wk[0] : (sp < 64 ? wk[1] : wk[2]);
+            w = __shfl_sync(0xffffffffu, x, sp & 31);
+          } else {
+            const float l = __ldg(lse_col + (int64_t)sp * kRowsPerGroup);
+            w = l == -INFINITY ? 0.f : ex2_approx(l - mx);
+          }
+          const float4 x = __ldg(src0 + (int64_t)sp * kSplitStride4);
+          acc.x = fmaf(w, x.x, acc.x);
+          acc.y = fmaf(w, x.y, acc.y);
+          acc.z = fmaf(w, x.z, acc.z);
+          acc.w = fmaf(w, x.w, acc.w);
+        }
+        const float inv = 1.f / wsum;
+        acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
       }
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) reinterpret_cast<float4*>(o_s[warp])[lane + 32 * u] = acc[u];
+    *reinterpret_cast<float4*>(&o_s[warp][4 * lane]) = acc;
   }
-  __syncthreads();
-  // ---- project: latent columns [64 warp, +64), output columns 8 ng .. +7, rows 4 rg .. +3
+  __syncthreads();  // o_s complete; the barrier init is visible to every thread
+  if (!mbar_wait(wbar, 0, 2000000000ull)) record_status(kStatusTimeout);
+  // ---- project this quarter: latent columns 16 warp .. +15, output columns 8 ng .. +7,
+  //      rows 4 rg .. +3
   const int ng = lane & 15, rg = lane >> 4;
   float a[4][8];
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
     for (int c = 0; c < 8; ++c) a[r][c] = 0.f;
-  const uint4* wrow = reinterpret_cast<const uint4*>(wv + ((int64_t)h * kDV + 64 * warp) * kProjDim) + ng;
-#pragma unroll 16
-  for (int d = 0; d < 64; ++d) {
-    const uint4 w4 = __ldg(wrow + d * (kProjDim / 8));
+#pragma unroll 4
+  for (int d = 0; d < 16; ++d) {
+    const int dl = 16 * warp + d;  // latent column within the quarter
+    const uint4 w4 = *reinterpret_cast<const uint4*>(w_s + dl * kProjDim + 8 * ng);
     const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
     float wf[8];
 #pragma unroll
@@ -1223,33 +1273,42 @@ __global__ void __launch_bounds__(256)
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float o = o_s[4 * rg + r][64 * warp + d];
+      const float o = o_s[4 * rg + r][dl];
 #pragma unroll
       for (int c = 0; c < 8; ++c) a[r][c] = fmaf(o, wf[c], a[r][c]);
     }
   }
-  __syncthreads();  // every thread has read o_s; the buffer now takes the partial sums
-  float* red = smem_f;  // [warp][row][n]
 #pragma unroll
   for (int r = 0; r < 4; ++r)
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      red[(warp * kProjRows + 4 * rg + r) * kProjDim + 8 * ng + c] = a[r][c];
+    for (int c = 0; c < 8; ++c) red[warp][4 * rg + r][8 * ng + c] = a[r][c];
   __syncthreads();
-  // ---- sum the 8 warps' partials: thread i writes outputs i, i + 256, i + 512, i + 768
 #pragma unroll
   for (int k = 0; k < kProjRows * kProjDim / 256; ++k) {
     const int e = threadIdx.x + 256 * k;
     const int r = e / kProjDim, n = e % kProjDim;
     float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) sum += red[(w * kProjRows + r) * kProjDim + n];
+    for (int w = 0; w < 8; ++w) sum += red[w][r][n];
+    part[r][n] = sum;
+  }
+  // ---- the cluster's 4 quarters: CTA qtr adds up rows 2 qtr, 2 qtr + 1
+  cluster_sync();
+  {
+    const int r = 2 * (int)qtr + (threadIdx.x >> 7), n = threadIdx.x & 127;
+    const uint32_t local = smem_u32(&part[r][n]);
+    float sum = 0.f;
+#pragma unroll
+    for (uint32_t c = 0; c < 4; ++c) sum += ld_shared_cluster_f32(mapa_shared(local, c));
     const int j = j0 + r;
     if (j < nrows) {
       const int b = j / plan.n_q, t = j - (j / plan.n_q) * plan.n_q;
       out_proj[(int64_t)(plan.seq_offset + b) * op_seq_stride + (int64_t)(t * plan.n_head + h) * kProjDim + n] = sum;
     }
   }
+  // the peers have read this CTA's sums before it exits (their loads have returned by
+  // the time they arrive: an execution barrier suffices)
+  cluster_sync_relaxed();
 }
 
 // Waits on a barrier that nothing ever signals, with a bounded wait, and records
