@@ -12,7 +12,8 @@ top of ``mla_oracle.c``.
 
 Parity pins (checked by ``tests/test_oracle_pins.py`` against closed forms,
 brute force and invariants, never against the oracle itself):
-  attention / attention_online / attention_split / compact / dequant_q8_0 / project.
+  attention / attention_online / attention_split / compact / dequant_q8_0 / project /
+  attention_variants.
 """
 from __future__ import annotations
 
@@ -80,6 +81,9 @@ def _load():
         lib.oracle_dequant_q8_0.restype = None
         lib.oracle_project.argtypes = [P, P, L, P, I, I, P]
         lib.oracle_project.restype = I
+        D_ = ctypes.c_double
+        lib.oracle_attention_variants.argtypes = [P, P, I, P, P, L, I, I, L, D_, D_, P, L, P, P]
+        lib.oracle_attention_variants.restype = I
         lib.oracle_init()
         _lib = lib
         return lib
@@ -235,4 +239,23 @@ def project(o, heads, wv):
                                 n_head, proj_dim, _ptr(out))
     if rc != 0:
         raise ValueError("oracle_project rejected its arguments")
+    return out
+
+
+def attention_variants(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, idx=None, softcap=0.0,
+                       slopes=None, pos0=0, sinks=None):
+    """Attention with the optional variants: logit softcap (softcap > 0), ALiBi (slopes
+    [n_head], bias slopes[h] * (j - (pos0 + t))) and attention sinks (sinks [n_head],
+    one extra logit per head in the denominator). Returns float64 [n_q*n_head][512]."""
+    q, kc, m, ix, _, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, None)
+    sl = None if slopes is None else np.ascontiguousarray(slopes, dtype=np.float64)
+    sk = None if sinks is None else np.ascontiguousarray(sinks, dtype=np.float64)
+    if (sl is not None and sl.shape != (n_head,)) or (sk is not None and sk.shape != (n_head,)):
+        raise ValueError("slopes and sinks are per head")
+    rc = _load().oracle_attention_variants(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
+                                           0 if ix is None else len(ix), n_q, n_head, n_kv,
+                                           float(scale), float(softcap), _ptr(sl), int(pos0),
+                                           _ptr(sk), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_attention_variants rejected its arguments")
     return out

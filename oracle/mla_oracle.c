@@ -26,6 +26,9 @@
  *  - f16 additive mask: baguaai flash-attention tag page, item on PR #23764.
  *  - Ascending index compaction of the kept mask cells: llama.cpp b11413
  *    release note, item "single-scan sparse FA index compaction".
+ *  - Attention sinks, ALiBi and logit softcap (oracle_attention_variants), named for
+ *    the Metal FA kernel in the llama.cpp tag page (PR #29570); their formulas are
+ *    this file's readings, written next to the function.
  *  - Value up-projection of each head (oracle_project): wkv_b split per head into
  *    wk_b and wv_b, "128 x 512 x 128": ik_llama.cpp -mla guide, section on tensor
  *    derivation; p[n] = sum_d o[d] * wv[h][d][n].
@@ -352,6 +355,71 @@ int oracle_project(const double* o, const int32_t* heads, long n_rows, const uin
       for (int d = 0; d < ORC_DV; ++d) acc += o[r * ORC_DV + d] * g_half[w[(long)d * proj_dim + n]];
       out[r * proj_dim + n] = acc;
     }
+  }
+  return 0;
+}
+
+/* Variants on the same attention (Metal FA kernel of the llama.cpp tag page, PR
+ * #29570: attention sinks, ALiBi, logit softcap), written out as definitions.
+ * For query row (t, h) and selected cache position j:
+ *   s_j = scale * sum_c q[t,h,c] k[j,c]
+ *   s_j = softcap * tanh(s_j / softcap)                 if softcap > 0
+ *   s_j = s_j + mask[t, j] + slopes[h] * (j - (pos0 + t))  (slopes optional)
+ *   M   = max(max_j s_j, sinks[h])                       (sinks optional)
+ *   L   = sum_j exp(s_j - M) + exp(sinks[h] - M)
+ *   o   = sum_j exp(s_j - M) k[j, :512] / L,  0 when M = -inf
+ * q: f16 bits [n_q][n_head][576]; slopes, sinks: double [n_head] or NULL;
+ * out: double [n_q*n_head][512]. Returns 0, or -1 on a bad argument. */
+int oracle_attention_variants(const uint16_t* q, const void* kcache, int kv_type,
+                              const uint16_t* mask, const int32_t* idx, long n_idx, int n_q,
+                              int n_head, long n_kv, double scale, double softcap,
+                              const double* slopes, long pos0, const double* sinks, double* out) {
+  if (!q || !kcache || !out || n_q < 1 || n_head < 1 || n_kv < 1) return -1;
+  if (kv_type != ORC_KV_F16 && kv_type != ORC_KV_Q8_0) return -1;
+  if (softcap < 0.0) return -1;
+  if (idx) {
+    for (long i = 0; i < n_idx; ++i)
+      if (idx[i] < 0 || idx[i] >= n_kv) return -1;
+  }
+  oracle_init();
+  const long n_sel = idx ? n_idx : n_kv;
+  const long total = (long)n_q * n_head;
+#pragma omp parallel
+  {
+    double* s = (double*)malloc(sizeof(double) * (size_t)(n_sel > 0 ? n_sel : 1));
+    double qd[ORC_DK];
+#pragma omp for schedule(dynamic, 1)
+    for (long row = 0; row < total; ++row) {
+      const long t = row / n_head, h = row % n_head;
+      const uint16_t* qrow = q + row * ORC_DK;
+      for (int c = 0; c < ORC_DK; ++c) qd[c] = g_half[qrow[c]];
+      const uint16_t* mrow = mask ? mask + t * n_kv : NULL;
+      double* o = out + row * ORC_DV;
+      double M = sinks ? sinks[h] : -INFINITY;
+      for (long i = 0; i < n_sel; ++i) {
+        const long key = key_at(idx, i);
+        double dot = 0.0;
+        for (int c = 0; c < ORC_DK; ++c) dot += qd[c] * kval(kcache, kv_type, key, c);
+        double v = scale * dot;
+        if (softcap > 0.0) v = softcap * tanh(v / softcap);
+        if (mrow) v += g_half[mrow[key]];
+        if (slopes) v += slopes[h] * (double)(key - (pos0 + t));
+        s[i] = v;
+        if (v > M) M = v;
+      }
+      for (int d = 0; d < ORC_DV; ++d) o[d] = 0.0;
+      if (M == -INFINITY) continue;
+      double L = sinks ? exp(sinks[h] - M) : 0.0;
+      for (long i = 0; i < n_sel; ++i) {
+        const double p = exp(s[i] - M);
+        L += p;
+        if (p == 0.0) continue;
+        const long key = key_at(idx, i);
+        for (int d = 0; d < ORC_DV; ++d) o[d] += p * kval(kcache, kv_type, key, d);
+      }
+      for (int d = 0; d < ORC_DV; ++d) o[d] /= L;
+    }
+    free(s);
   }
   return 0;
 }

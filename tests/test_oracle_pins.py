@@ -407,3 +407,115 @@ def test_project_rejects_bad_heads():
     heads[3] = 4  # n_head is 4
     with pytest.raises(ValueError):
         oracle.project(o, heads, wv)
+
+
+# ---- attention variants: softcap, ALiBi, sinks (oracle.attention_variants) -----------
+
+def brute_force_variants(q, k, mask, scale, softcap=0.0, slopes=None, pos0=0, sinks=None):
+    """The variants' definitions with explicit float64 numpy matrices (no oracle code)."""
+    qd = q.astype(np.float64)
+    kd = k.astype(np.float64)
+    n_q, H, _ = q.shape
+    n = k.shape[0]
+    out = np.zeros((n_q, H, DV))
+    for t in range(n_q):
+        S = scale * (qd[t] @ kd.T)  # [H][n]
+        if softcap > 0:
+            S = softcap * np.tanh(S / softcap)
+        if mask is not None:
+            S = S + mask[t].astype(np.float64)[None, :]
+        if slopes is not None:
+            S = S + np.asarray(slopes, np.float64)[:, None] * (np.arange(n)[None, :] - (pos0 + t))
+        M = S.max(axis=1)
+        if sinks is not None:
+            M = np.maximum(M, np.asarray(sinks, np.float64))
+        for h in range(H):
+            if np.isneginf(M[h]):
+                continue
+            p = np.where(np.isneginf(S[h]), 0.0, np.exp(S[h] - M[h]))
+            den = p.sum() + (np.exp(sinks[h] - M[h]) if sinks is not None else 0.0)
+            out[t, h] = (p @ kd[:, :DV]) / den
+    return out.reshape(n_q * H, DV)
+
+
+def _variant_inputs(seed, n_q=2, H=4, n=37, masked=True):
+    rng = np.random.default_rng(seed)
+    q = rand_f16(rng, (n_q, H, DK))
+    k = rand_f16(rng, (n, DK))
+    mask = None
+    if masked:
+        mask = rand_f16(rng, (n_q, n), std=0.5)
+        mask[:, rng.choice(n, 5, replace=False)] = NEG
+    return q, k, mask
+
+
+def test_softcap_matches_brute_force():
+    q, k, mask = _variant_inputs(61)
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, softcap=2.5)
+    want = brute_force_variants(q, k, mask, 0.125, softcap=2.5)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_softcap_with_a_huge_cap_is_plain_attention():
+    q, k, mask = _variant_inputs(62)
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, softcap=1e7)
+    want = brute_force(q, k, mask, 0.125).reshape(-1, DV)
+    assert np.allclose(got, want, rtol=1e-9, atol=1e-12)
+
+
+def test_alibi_matches_brute_force_and_is_shift_invariant():
+    q, k, mask = _variant_inputs(63)
+    slopes = np.array([0.5, 0.25, 0.125, 0.0625])
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, slopes=slopes, pos0=36)
+    want = brute_force_variants(q, k, mask, 0.125, slopes=slopes, pos0=36)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
+    # a per-row constant in the bias does not change a softmax
+    shifted = oracle.attention_variants(q, k, mask=mask, scale=0.125, slopes=slopes, pos0=-1000)
+    assert np.allclose(shifted, got, rtol=1e-11, atol=1e-13)
+
+
+def test_alibi_with_zero_slopes_is_plain_attention_exactly():
+    q, k, mask = _variant_inputs(64)
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, slopes=np.zeros(4))
+    assert np.array_equal(got, oracle.attention(q, k, mask=mask, scale=0.125))
+
+
+def test_sinks_match_brute_force():
+    q, k, mask = _variant_inputs(65)
+    sinks = np.array([-1.0, 0.0, 2.0, 7.5])
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, sinks=sinks)
+    want = brute_force_variants(q, k, mask, 0.125, sinks=sinks)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_a_minus_inf_sink_is_plain_attention_exactly():
+    q, k, mask = _variant_inputs(66)
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, sinks=np.full(4, -np.inf))
+    assert np.array_equal(got, oracle.attention(q, k, mask=mask, scale=0.125))
+
+
+def test_sink_with_one_key_is_a_sigmoid():
+    # one key of score s and a sink sigma: o = v * e^s / (e^s + e^sigma) = v * sigmoid(s - sigma)
+    q, k, _ = _variant_inputs(67, n_q=1, H=3, n=1, masked=False)
+    sinks = np.array([-0.5, 0.3, 4.0])
+    got = oracle.attention_variants(q, k, scale=0.2, sinks=sinks)
+    s = 0.2 * (q[0].astype(np.float64) @ k[0].astype(np.float64))
+    want = k[0, :DV].astype(np.float64)[None, :] / (1.0 + np.exp(sinks - s))[:, None]
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-14)
+
+
+def test_sink_on_a_fully_masked_row_gives_zero():
+    q, k, mask = _variant_inputs(68, n_q=1)
+    mask[:] = NEG
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.125, sinks=np.array([0.0, 1.0, 2.0, 3.0]))
+    assert np.array_equal(got, np.zeros_like(got))
+
+
+def test_all_variants_together_match_brute_force():
+    q, k, mask = _variant_inputs(69, n_q=3, H=5, n=50)
+    slopes = np.array([0.5, 0.25, 0.125, 0.0625, 0.03125])
+    sinks = np.array([0.0, -2.0, 1.0, 3.0, -0.5])
+    got = oracle.attention_variants(q, k, mask=mask, scale=0.1, softcap=3.0, slopes=slopes, pos0=47,
+                                    sinks=sinks)
+    want = brute_force_variants(q, k, mask, 0.1, softcap=3.0, slopes=slopes, pos0=47, sinks=sinks)
+    assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
