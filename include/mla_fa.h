@@ -100,6 +100,17 @@ typedef enum {
  * proj_dim output width of the projection; must be MLA_PROJ_DIM (128) when wv is set
  * out_proj DEVICE fp32, element (b, t, h, n) at
  *         out_proj[b*out_proj_seq_stride + (t*n_head + h)*proj_dim + n]; 16-byte aligned
+ * sinks   DEVICE fp32 [n_head] or NULL: attention sinks, one extra logit per head in
+ *         the softmax denominator with no value:
+ *           o = sum_j e^{s_j} v_j / (e^{sinks[h]} + sum_j e^{s_j})
+ * alibi_slopes DEVICE fp32 [n_head] or NULL: ALiBi, s_j += alibi_slopes[h] * (j - p_t)
+ *         with j the key's cache position and p_t = kv_len[b] - n_q + t the query's
+ *         position (the n_q query tokens are the last positions of the sequence).
+ *         Not supported with idx (MLA_ERR_UNSUPPORTED)
+ * softcap > 0: logit softcap, the scaled score becomes softcap * tanh(score / softcap)
+ *         before the mask is added; 0 = off
+ * (the variants are named for the Metal FA kernel of the llama.cpp tag page, PR
+ * #29570; these formulas are this library's reading of them)
  * A stride of 0 means "dense" (the natural value for the given sizes).
  */
 typedef struct mla_fa_args {
@@ -126,6 +137,9 @@ typedef struct mla_fa_args {
   int proj_dim;             /* MLA_PROJ_DIM when wv is set                     */
   float* out_proj;          /* DEVICE, required with wv                        */
   int64_t out_proj_seq_stride; /* elements; 0 = n_q*n_head*proj_dim            */
+  const float* sinks;       /* DEVICE fp32 [n_head], optional                  */
+  const float* alibi_slopes; /* DEVICE fp32 [n_head], optional                 */
+  float softcap;            /* > 0 enables the logit softcap                   */
 } mla_fa_args;
 
 /* Forward pass with the sizes of the single-sequence call:

@@ -61,6 +61,9 @@ class mla_fa_args(ctypes.Structure):
         ("proj_dim", ctypes.c_int),
         ("out_proj", ctypes.c_void_p),
         ("out_proj_seq_stride", ctypes.c_int64),
+        ("sinks", ctypes.c_void_p),
+        ("alibi_slopes", ctypes.c_void_p),
+        ("softcap", ctypes.c_float),
     ]
 
 
@@ -150,13 +153,14 @@ def _host_i32(arr):
 
 
 def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None,
-              wv=None, out_proj=None):
+              wv=None, out_proj=None, sinks=None, alibi_slopes=None, softcap=0.0):
     """Fill mla_fa_args from batched torch tensors.
 
     q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
     mask [n_seq][n_q][n_kv] f16 or None; out [n_seq][n_q][n_head][512] f32 (or None with
     wv); wv [n_head][512][128] f16 and out_proj [n_seq][n_q][n_head][128] f32 for the
-    fused value up-projection. Returns (args, keepalive)."""
+    fused value up-projection; sinks / alibi_slopes fp32 [n_head] and softcap > 0 for
+    the attention variants. Returns (args, keepalive)."""
     n_seq, n_q, n_head, dk = q.shape
     if dk != DK:
         raise ValueError("q must end in 576")
@@ -179,6 +183,9 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
         a.proj_dim = int(wv.shape[2])
         a.out_proj = None if out_proj is None else out_proj.data_ptr()
         a.out_proj_seq_stride = 0 if out_proj is None else out_proj.stride(0)
+    a.sinks = None if sinks is None else sinks.data_ptr()
+    a.alibi_slopes = None if alibi_slopes is None else alibi_slopes.data_ptr()
+    a.softcap = float(softcap)
     keep = _host_i32(kv_len)
     a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
     if idx is not None:
@@ -216,13 +223,14 @@ def mla_fa_forward(q, kcache, kv_type, mask, scale, out, stream=None):
 
 
 def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, idx_count=None,
-            workspace=None, stream=None):
+            workspace=None, stream=None, sinks=None, alibi_slopes=None, softcap=0.0):
     """Batched forward through mla_fa_forward_ex; allocates out/workspace with torch if absent."""
     import torch
 
     if out is None:
         out = torch.empty(q.shape[:3] + (DV,), dtype=torch.float32, device=q.device)
-    args, keep = make_args(q, kcache, kv_type, mask, out, scale, kv_len, idx, idx_count)
+    args, keep = make_args(q, kcache, kv_type, mask, out, scale, kv_len, idx, idx_count,
+                           sinks=sinks, alibi_slopes=alibi_slopes, softcap=softcap)
     need = mla_fa_workspace_size(args)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

@@ -153,6 +153,7 @@ struct Resolved {
   int rows;
   int64_t q_ss, k_ss, m_ss, m_rs, o_ss, idx_ss, op_ss;
   bool proj;  // fused value up-projection: every sequence writes split partials
+  bool sinks; // attention sinks: every sequence writes split partials (the combine adds them)
 };
 
 int validate(const mla_fa_args* a, Resolved* r) {
@@ -161,6 +162,10 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (a->q == nullptr || a->kcache == nullptr || (a->out == nullptr && !proj)) return MLA_ERR_NULL;
   if (proj && a->out_proj == nullptr) return MLA_ERR_NULL;
   if (proj && a->proj_dim != MLA_PROJ_DIM) return MLA_ERR_UNSUPPORTED;
+  if (!(a->softcap >= 0.f) || std::isinf(a->softcap)) return MLA_ERR_SHAPE;  // NaN, <0, inf
+  if (a->alibi_slopes != nullptr && a->idx != nullptr) return MLA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(a->sinks) & 3) || (reinterpret_cast<uintptr_t>(a->alibi_slopes) & 3))
+    return MLA_ERR_ALIGN;
   if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
   if (a->n_seq < 1 || a->n_q < 1 || a->n_head < 1 || a->n_head > MLA_MAX_HEADS || a->n_kv < 1)
     return MLA_ERR_SHAPE;
@@ -177,6 +182,7 @@ int validate(const mla_fa_args* a, Resolved* r) {
   r->o_ss = a->out_seq_stride ? a->out_seq_stride : rows * MLA_DV;
   r->idx_ss = a->idx_seq_stride ? a->idx_seq_stride : a->n_kv;
   r->proj = proj;
+  r->sinks = a->sinks != nullptr;
   r->op_ss = proj ? (a->out_proj_seq_stride ? a->out_proj_seq_stride : rows * MLA_PROJ_DIM) : 0;
   if (proj && (a->out_proj_seq_stride < 0 || r->op_ss < rows * MLA_PROJ_DIM)) return MLA_ERR_SHAPE;
   if (proj && (!aligned16(a->wv) || !aligned16(a->out_proj) || (r->op_ss % 4) != 0))
@@ -236,7 +242,7 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
     plan->n_split[b] = ns;
     plan->unit_base[b] = units;
     units += plan->groups * ns;
-    if (ns > 1 || r.proj) {
+    if (ns > 1 || r.proj || r.sinks) {
       plan->ws_base[b] = slots;
       slots += plan->groups * ns;
     } else {
@@ -334,15 +340,18 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   }
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
-    if (cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeTma>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             mla::fwd::kSmemAlloc) != cudaSuccess ||
-        cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeGatherF16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             mla::fwd::kSmemAlloc) != cudaSuccess ||
-        cudaFuncSetAttribute(mla::mla_fwd_kernel<mla::kModeQ8>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             mla::fwd::kSmemAlloc) != cudaSuccess ||
+    const void* fwd_kernels[] = {
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, true>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true>};
+    bool ok = true;
+    for (const void* k : fwd_kernels)
+      ok = ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      mla::fwd::kSmemAlloc) == cudaSuccess;
+    if (!ok ||
         cudaFuncSetAttribute(mla::mla_combine_proj_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              mla::kProjSmem) != cudaSuccess)
@@ -366,6 +375,8 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   p.idx = a.idx;
   p.idx_count = a.idx_count;
   p.idx_seq_stride = r.idx_ss;
+  p.softcap = a.softcap;
+  p.slopes = a.alibi_slopes;
   Plan plan;
   for (int s0 = 0; s0 < a.n_seq; s0 += mla::kPlanMaxSeq) {
     const int n = std::min(mla::kPlanMaxSeq, a.n_seq - s0);
@@ -393,21 +404,29 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     fcfg.attrs = fattr;
     fcfg.numAttrs = 1;
     cudaError_t fe;
+    // the softcap / ALiBi instance only when the call asks for one of them
+    const bool variant = a.softcap > 0.f || a.alibi_slopes != nullptr;
     if (mode == mla::kModeTma) {
       ProfScope prof(kKernFwdF16, stream);
       fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeTma>::kThreads);
-      fe = cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeTma>, tm_q, tm_k, tm_v, tm_o, tm_w,
-                              plan, p);
+      fe = variant ? cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeTma, true>, tm_q, tm_k,
+                                        tm_v, tm_o, tm_w, plan, p)
+                   : cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeTma, false>, tm_q, tm_k,
+                                        tm_v, tm_o, tm_w, plan, p);
     } else if (mode == mla::kModeGatherF16) {
       ProfScope prof(kKernFwdGather, stream);
       fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeGatherF16>::kThreads);
-      fe = cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeGatherF16>, tm_q, tm_k, tm_v, tm_o,
-                              tm_w, plan, p);
+      fe = variant ? cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeGatherF16, true>, tm_q,
+                                        tm_k, tm_v, tm_o, tm_w, plan, p)
+                   : cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeGatherF16, false>, tm_q,
+                                        tm_k, tm_v, tm_o, tm_w, plan, p);
     } else {
       ProfScope prof(kKernFwdQ8, stream);
       fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeQ8>::kThreads);
-      fe = cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeQ8>, tm_q, tm_k, tm_v, tm_o, tm_w,
-                              plan, p);
+      fe = variant ? cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeQ8, true>, tm_q, tm_k,
+                                        tm_v, tm_o, tm_w, plan, p)
+                   : cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeQ8, false>, tm_q, tm_k,
+                                        tm_v, tm_o, tm_w, plan, p);
     }
     if (fe != cudaSuccess) return MLA_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
@@ -442,13 +461,13 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
         if (r.proj)
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_proj_kernel, plan, (const float*)p.ws_o,
                                   (const float*)p.ws_lse, static_cast<const uint16_t*>(a.wv),
-                                  a.out_proj, (int64_t)r.op_ss);
+                                  a.out_proj, (int64_t)r.op_ss, a.sinks);
         else if (wide)
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const float*)p.ws_o,
-                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss);
+                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks);
         else
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const float*)p.ws_o,
-                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss);
+                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks);
       }
       if (ce != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }

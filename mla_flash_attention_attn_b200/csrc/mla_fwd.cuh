@@ -74,6 +74,9 @@ struct MlaFwdParams {
   const int32_t* idx;
   const int32_t* idx_count;
   int64_t idx_seq_stride;
+  // variants (0 / nullptr = off): logit softcap, ALiBi slopes per head
+  float softcap;
+  const float* slopes;
 };
 
 // How K/V tiles reach shared memory.
@@ -230,7 +233,9 @@ __device__ __forceinline__ void block_values(const RawBlock<kMode>& rb, uint32_t
   }
 }
 
-template <int kMode>
+// kVariant: the instance that applies the logit softcap and ALiBi (the host launches it
+// only when a call asks for one of them, so the common path carries none of that code)
+template <int kMode, bool kVariant>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThreads, 1)
     mla_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -660,6 +665,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                                      (int64_t)tok * p.mask_row_stride
                                : nullptr;
     const uint32_t s_free_l = mapa_shared(smem_u32(&bars.s_free), 0);
+    // variants: the ALiBi bias is slope * (key - position of the query), the query
+    // tokens being the last n_q positions of the sequence (with sinks the softmax is no
+    // longer shift invariant, so this position is the defined one)
+    const float slope =
+        (kVariant && p.slopes != nullptr && row_valid) ? __ldg(p.slopes + row % plan.n_head) : 0.f;
+    const int alibi_ref = len - plan.n_q + tok;
     const uint32_t p_full_l0 = mapa_shared(smem_u32(&bars.p_full[0]), 0);
     const uint32_t p_full_l1 = mapa_shared(smem_u32(&bars.p_full[1]), 0);
     auto wait_local = [&](uint64_t* bar, uint32_t parity) {
@@ -751,27 +762,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster_relaxed(s_free_l);
       float x[kHalf];
-      if (vec_mask) {
-#pragma unroll
-        for (int c = 0; c < kHalf / 8; ++c) {
-          const uint4 v = mvec[c];
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
-            const int j = 8 * c + 2 * h;
-            x[j] = fmaf(__uint_as_float(sr[j]), p.scale, f.x);
-            x[j + 1] = fmaf(__uint_as_float(sr[j + 1]), p.scale, f.y);
-          }
-        }
-      } else {
+      if constexpr (kVariant) {
+        // softcapped (or plainly scaled) score, then the mask, then the ALiBi bias
+        const float cap = p.softcap;
+        const float sc = cap > 0.f ? p.scale / cap : 0.f;
+        const uint32_t* mw = reinterpret_cast<const uint32_t*>(mvec);
 #pragma unroll
         for (int j = 0; j < kHalf; ++j) {
           const int key = key0 + j;
-          float mv = 0.f;
-          if (mrow != nullptr && key < key_end)
-            mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
-          x[j] = key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
+          float sv = __uint_as_float(sr[j]);
+          sv = cap > 0.f ? cap * tanhf(sv * sc) : sv * p.scale;
+          float mv;
+          if (vec_mask) {
+            const uint32_t w = mw[j >> 1];
+            mv = __half2float(__ushort_as_half((unsigned short)((j & 1) ? (w >> 16) : (w & 0xFFFFu))));
+          } else {
+            mv = (mrow != nullptr && key < key_end) ? __half2float(__ushort_as_half(__ldg(mrow + key))) : 0.f;
+          }
+          const float xv = fmaf(slope, (float)(key - alibi_ref), sv + mv);
+          x[j] = (vec_mask || key < key_end) ? xv : -INFINITY;
+        }
+      } else {
+        if (vec_mask) {
+#pragma unroll
+          for (int c = 0; c < kHalf / 8; ++c) {
+            const uint4 v = mvec[c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[h]));
+              const int j = 8 * c + 2 * h;
+              x[j] = fmaf(__uint_as_float(sr[j]), p.scale, f.x);
+              x[j + 1] = fmaf(__uint_as_float(sr[j + 1]), p.scale, f.y);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kHalf; ++j) {
+            const int key = key0 + j;
+            float mv = 0.f;
+            if (mrow != nullptr && key < key_end)
+              mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
+            x[j] = key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
+          }
         }
       }
       // row max over this lane's 128 keys (8 independent chains), then over the pair
@@ -973,7 +1006,8 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
                                                           const float* __restrict__ ws_o,
                                                           const float* __restrict__ ws_lse,
                                                           float* __restrict__ out,
-                                                          int64_t out_seq_stride) {
+                                                          int64_t out_seq_stride,
+                                                          const float* __restrict__ sinks) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.y;
   const int row = blockIdx.x;
@@ -995,12 +1029,16 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   float mx = lse_l;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  // an attention sink is one more split with lse = sink (log2 units) and no value
+  const float snk = sinks != nullptr ? __ldg(sinks + row % plan.n_head) * kLog2e : -INFINITY;
+  mx = fmaxf(mx, snk);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (mx != -INFINITY) {
     const float wl = lse_l == -INFINITY ? 0.f : ex2_approx(lse_l - mx);
     float wsum = wl;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    if (snk != -INFINITY) wsum += ex2_approx(snk - mx);
 #pragma unroll
     for (int u = 0; u < kFirst; ++u) {
       const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past ns
@@ -1037,7 +1075,7 @@ constexpr int kCombPer = 24;  // partial rows per warp held in registers
 __global__ void __launch_bounds__(128)
     mla_combine_wide_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, float* __restrict__ out,
-                            int64_t out_seq_stride) {
+                            int64_t out_seq_stride, const float* __restrict__ sinks) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 red[4][32];
   const int b = blockIdx.z;
@@ -1070,6 +1108,9 @@ __global__ void __launch_bounds__(128)
   for (int sp = lane + 96; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  // an attention sink is one more split with lse = sink (log2 units) and no value
+  const float snk = sinks != nullptr ? __ldg(sinks + row % plan.n_head) * kLog2e : -INFINITY;
+  mx = fmaxf(mx, snk);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float wsum = 0.f;
   if (mx != -INFINITY) {  // the same for every warp
@@ -1083,6 +1124,7 @@ __global__ void __launch_bounds__(128)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    if (snk != -INFINITY) wsum += ex2_approx(snk - mx);
 #pragma unroll
     for (int j = 0; j < kCombPer; ++j) {
       const int sp = warp + 4 * j;  // the same in every lane
@@ -1152,7 +1194,8 @@ constexpr int kProjSmem = kProjWBytes + kProjRows * kProjORow * 4 +   // W, o_s
 __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
     mla_combine_proj_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, const uint16_t* __restrict__ wv,
-                            float* __restrict__ out_proj, int64_t op_seq_stride) {
+                            float* __restrict__ out_proj, int64_t op_seq_stride,
+                            const float* __restrict__ sinks) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(128) uint8_t proj_smem[];
   // a launch with too little dynamic shared memory reports and returns (every CTA takes
@@ -1209,6 +1252,9 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
       for (int sp = lane + 96; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      // an attention sink is one more split with lse = sink (log2 units) and no value
+      const float snk = sinks != nullptr ? __ldg(sinks + h) * kLog2e : -INFINITY;
+      mx = fmaxf(mx, snk);
       if (mx != -INFINITY) {
         float wk[3];
 #pragma unroll
@@ -1220,6 +1266,7 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+        if (snk != -INFINITY) wsum += ex2_approx(snk - mx);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const float w = __shfl_sync(0xffffffffu, wk[0], u);  // 0 past ns

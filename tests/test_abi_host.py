@@ -71,6 +71,10 @@ def call_ex(lib, a):
     (dict(wv=FAKE, proj_dim=128, out_proj=FAKE + 4), -4),
     (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, out_proj_seq_stride=100, n_seq=2), -2),
     (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, out_proj_seq_stride=16 * 128 + 2, n_seq=2), -4),
+    # attention variants
+    (dict(softcap=-1.0), -2), (dict(softcap=float("nan")), -2), (dict(softcap=float("inf")), -2),
+    (dict(alibi_slopes=FAKE, idx=FAKE, idx_count=FAKE), -8),
+    (dict(sinks=FAKE + 2), -4), (dict(alibi_slopes=FAKE + 1), -4),
 ])
 def test_argument_errors_are_returned_before_any_launch(lib, kw, expect):
     assert call_ex(lib, base_args(**kw)) == expect

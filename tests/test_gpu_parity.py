@@ -39,7 +39,7 @@ def assert_parity(got, ref, what=""):
     assert maxabs <= MAX_ABS and rel <= REL_L2, f"{what}: max-abs {maxabs:.3g} rel-L2 {rel:.3g}"
 
 
-def run_gpu(w, kv_len="auto", mask="auto", k_pad=0):
+def run_gpu(w, kv_len="auto", mask="auto", k_pad=0, **variants):
     """Run the workload through mla_fa_forward_ex; returns out [n_seq][n_q][n_head][512]."""
     torch = torch_mod()
     dev = torch.device("cuda")
@@ -58,7 +58,12 @@ def run_gpu(w, kv_len="auto", mask="auto", k_pad=0):
     big = torch.full((n_out + CANARY,), float("nan"), dtype=torch.float32, device=dev)
     out = big[:n_out].view(w.n_seq, w.n_q, w.n_head, 512)
     lens = w.kv_len if kv_len == "auto" else kv_len
-    binding.forward(q, k, w.kv_type, m, w.scale, out=out, kv_len=lens)
+    vt = {}
+    for name in ("sinks", "alibi_slopes"):
+        if variants.get(name) is not None:
+            vt[name] = torch.from_numpy(np.asarray(variants[name], np.float32)).to(dev)
+    binding.forward(q, k, w.kv_type, m, w.scale, out=out, kv_len=lens,
+                    softcap=variants.get("softcap", 0.0), **vt)
     torch.cuda.synchronize()
     assert binding.mla_get_device_status() == 0
     tail = big[n_out:]
@@ -470,3 +475,73 @@ def test_fused_projection_with_an_empty_sequence():
     got = run_gpu_proj(w, wv)
     assert np.all(got[1] == 0.0)
     check_proj(w, wv, got, "kv_len 300/0/700")
+
+
+# ---- attention variants: logit softcap, ALiBi, sinks -----------------------------
+
+def alibi_slopes(n_head):
+    return np.array([2.0 ** (-8.0 * (h + 1) / n_head) for h in range(n_head)])
+
+
+def check_variants(w, got, what, softcap=0.0, slopes=None, sinks=None, kcache=None, kv_type=None):
+    for b in range(w.n_seq):
+        ref = oracle.attention_variants(
+            w.q[b], w.kcache[b] if kcache is None else kcache, w.kv_type if kv_type is None else kv_type,
+            w.mask[b] if w.mask is not None else None, w.scale, softcap=softcap, slopes=slopes,
+            pos0=int(w.kv_len[b]) - w.n_q, sinks=sinks)
+        assert_parity(got[b].reshape(-1, 512), ref, f"{what} seq {b}")
+
+
+def test_softcap_matches_oracle():
+    w = W.make("tiny_decode", n_kv=300)
+    got = run_gpu(w, softcap=5.0)
+    check_variants(w, got, "softcap", softcap=5.0)
+
+
+def test_alibi_matches_oracle_prefill_rows():
+    w = W.make("prefill_chunk", n_q=8, n_head=128, n_kv=640)
+    sl = alibi_slopes(128)
+    got = run_gpu(w, alibi_slopes=sl)
+    check_variants(w, got, "alibi", slopes=sl)
+
+
+def test_alibi_long_sequence_precision():
+    # biases up to 0.5 x 4095 relative to the last key
+    w = W.make("v2lite_decode", n_kv=4096, n_head=16, n_pad=0)
+    sl = alibi_slopes(16)
+    got = run_gpu(w, alibi_slopes=sl)
+    check_variants(w, got, "alibi long", slopes=sl)
+
+
+def test_sinks_with_split_plan():
+    w = W.make("v3_batched_decode", n_kv=2048, len_lo=100, len_hi=2048)
+    sinks = np.random.default_rng(7).normal(0.0, 2.0, 128)
+    got = run_gpu(w, sinks=sinks)
+    check_variants(w, got, "sinks", sinks=sinks)
+
+
+def test_sinks_unsplit_and_empty_sequence():
+    w = W.make("v3_batched_decode", n_seq=3, n_head=16, n_kv=700, len_lo=0, len_hi=700)
+    w.kv_len[:] = [300, 0, 700]
+    keep = np.arange(700)[None, :] < w.kv_len[:, None]
+    w.mask[:, 0, :] = np.where(keep, np.float16(0), np.float16(-np.inf))
+    sinks = np.linspace(-3.0, 3.0, 16)
+    got = run_gpu(w, sinks=sinks)
+    assert np.all(got[1] == 0.0)
+    check_variants(w, got, "sinks kv_len 300/0/700", sinks=sinks)
+
+
+def test_all_variants_together():
+    w = W.make("prefill_chunk", n_q=3, n_head=5, n_kv=300)
+    sl = alibi_slopes(5)
+    sinks = np.array([0.5, -1.0, 2.0, 0.0, 3.0])
+    got = run_gpu(w, softcap=4.0, alibi_slopes=sl, sinks=sinks)
+    check_variants(w, got, "all variants", softcap=4.0, slopes=sl, sinks=sinks)
+
+
+def test_softcap_q8_0_dense():
+    w = W.make("sparse_q8_decode", n_kv=2048, n_head=128, tail_blocks=4)
+    w.sparse = False
+    got = run_gpu(w, softcap=6.0)
+    check_variants(w, got, "softcap q8_0", softcap=6.0, kcache=q8_f16_rounded(w.kcache[0]),
+                   kv_type=oracle.KV_F16)
