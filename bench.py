@@ -49,11 +49,15 @@ DEFAULT_WORKLOAD = "v3_batched_decode"
 
 
 # ----------------------------------------------------------------------------- accounting
-def algorithmic(w, kept_cells=None):
+def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
     """Algorithmic bytes and flops of one step, split partials excluded.
 
     bytes = cache rows attended x row bytes + Q + mask cells read + output;
-    flops = 2 * n_head * (576 + 512) per (query row, attended key)."""
+    flops = 2 * n_head * (576 + 512) per (query row, attended key). With the fused
+    value up-projection (wuv) the output is 128 wide and the step also reads the
+    weights (n_head x 512 x 128 f16) and does 2 x 512 x 128 flops per query row.
+    A sparse step reads its mask row and writes then reads the index list; with the
+    mask gather there is no list: the mask rows are read once."""
     row_bytes = 1152 if w.kv_type == W.KV_F16 else W.Q8_ROW_BYTES
     if kept_cells is None:
         keep = ~np.isneginf(w.mask) if w.mask is not None else None
@@ -71,12 +75,15 @@ def algorithmic(w, kept_cells=None):
         rows_attended += max(kept_cells[b])
         pairs += sum(kept_cells[b])
         mask_bytes += w.n_q * int(w.kv_len[b]) * 2 if w.mask is not None else 0
-    if w.sparse:
+    if w.sparse and not mask_gather:
         mask_bytes = w.n_seq * w.n_kv * 2 + rows_attended * 4 * 2  # mask read + idx write/read
     q_bytes = w.q.size * 2
-    out_bytes = w.n_seq * w.n_q * w.n_head * 512 * 4
+    out_bytes = w.n_seq * w.n_q * w.n_head * (128 if wuv else 512) * 4
     kv_bytes = rows_attended * row_bytes
     flops = 2.0 * w.n_head * (576 + 512) * pairs
+    if wuv:
+        out_bytes += w.n_head * 512 * 128 * 2
+        flops += 2.0 * 512 * 128 * w.n_seq * w.n_q * w.n_head
     return {"kv_bytes": kv_bytes, "bytes": kv_bytes + q_bytes + mask_bytes + out_bytes,
             "flops": flops}
 
@@ -102,6 +109,12 @@ def kernel_source_hash():
             with open(os.path.join(src, f), "rb") as fh:
                 h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def workload_name(args):
+    """The workload as the step runs it: the cache geometry plus the fused options."""
+    return (args.workload + ("+wuv" if args.wuv else "")
+            + ("+mask_gather" if args.mask_gather else ""))
 
 
 def measured_traffic(workload):
@@ -186,7 +199,7 @@ class ClockSampler:
 class Step:
     """Device-resident inputs and the hot path of one workload."""
 
-    def __init__(self, w, torch, binding):
+    def __init__(self, w, torch, binding, wuv=False, mask_gather=False):
         self.w = w
         self.torch = torch
         self.b = binding
@@ -194,18 +207,22 @@ class Step:
         self.q = torch.from_numpy(w.q).to(dev)
         self.k = torch.from_numpy(w.kcache).to(dev)
         self.mask = torch.from_numpy(w.mask).to(dev) if w.mask is not None else None
-        self.out = torch.empty(w.q.shape[:3] + (512,), dtype=torch.float32, device=dev)
+        # with the fused value up-projection the step's result is the 128-wide projection
+        self.wv = torch.from_numpy(W.wv_random(n_head=w.n_head)).to(dev) if wuv else None
+        self.out = torch.empty(w.q.shape[:3] + ((128 if wuv else 512),), dtype=torch.float32,
+                               device=dev)
         self.kv_len = [int(x) for x in w.kv_len]
         self.idx = self.cnt = None
-        if w.sparse:
+        if w.sparse and not mask_gather:
             # the step starts from the mask row: compaction, then attention over the kept rows
             self.idx = torch.empty((w.n_seq, w.n_kv), dtype=torch.int32, device=dev)
             self.cnt = torch.zeros((w.n_seq,), dtype=torch.int32, device=dev)
             self.cws = torch.zeros(binding.mla_compact_workspace_size(w.n_seq, w.n_kv),
                                    dtype=torch.uint8, device=dev)
-        self.args, self._keep = binding.make_args(self.q, self.k, w.kv_type, self.mask, self.out,
-                                                  w.scale, kv_len=self.kv_len, idx=self.idx,
-                                                  idx_count=self.cnt)
+        self.args, self._keep = binding.make_args(
+            self.q, self.k, w.kv_type, self.mask, None if wuv else self.out, w.scale,
+            kv_len=self.kv_len, idx=self.idx, idx_count=self.cnt, wv=self.wv,
+            out_proj=self.out if wuv else None, mask_gather=mask_gather)
         need = binding.mla_fa_workspace_size(self.args)
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
         self.ws_used = need > 0
@@ -224,8 +241,8 @@ def gpu_arm(args, rank, world):
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     binding.load()
     w = W.make(args.workload)
-    acc = algorithmic(w)
-    step = Step(w, torch, binding)
+    acc = algorithmic(w, wuv=args.wuv, mask_gather=args.mask_gather)
+    step = Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather)
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -297,7 +314,8 @@ def gpu_arm(args, rank, world):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
-    roof["traffic"] = args.traffic if args.traffic is not None else measured_traffic(args.workload)
+    roof["traffic"] = (args.traffic if args.traffic is not None
+                       else measured_traffic(workload_name(args)))
     roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else \
         "fallback (profiling recipe)"
     roof["kernel"] = dom
@@ -319,7 +337,8 @@ def gpu_arm(args, rank, world):
         "vs_baseline": None,
         "dtype": "f16",
         "data": "synthetic (seeded PCG64; DeepSeek-V3/V2-Lite cache geometry, random values)",
-        "config": {"workload": args.workload, "n_seq": w.n_seq, "n_q": w.n_q,
+        "config": {"workload": workload_name(args),
+                   "n_seq": w.n_seq, "n_q": w.n_q,
                    "n_head": w.n_head, "n_kv": w.n_kv,
                    "kv_type": "q8_0" if w.kv_type else "f16",
                    "kv_len": [int(x) for x in w.kv_len][:16],
@@ -439,7 +458,8 @@ def reference_arm(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded PCG64)",
-        "config": {"workload": args.workload, "n_seq": w.n_seq, "n_q": w.n_q,
+        "config": {"workload": args.workload,
+                   "n_seq": w.n_seq, "n_q": w.n_q,
                    "n_head": w.n_head, "n_kv": w.n_kv, "parallelism": "host cores"},
         "impl": "reference", "cpu_baseline": cpu,
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -491,6 +511,12 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.WORKLOAD_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--wuv", action="store_true",
+                    help="fuse the value up-projection W_UV (synthetic f16 weights) into the "
+                         "step; the result is the 128-wide projection")
+    ap.add_argument("--mask-gather", action="store_true",
+                    help="masked workloads: sparse attention straight from the mask (the "
+                         "compaction fused into the attention kernel, no index list)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0)
@@ -500,6 +526,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.wuv and args.impl == "reference":
+        ap.error("--wuv applies to --impl ours (the oracle arm times the attention only)")
+    if args.mask_gather and args.impl == "reference":
+        ap.error("--mask-gather applies to --impl ours (the oracle arm runs the unfused chain)")
+    if args.wuv:
+        args.no_cpu_baseline = True  # the oracle baseline times the attention only
     rank, world = init_ranks(args)
     try:
         if args.impl == "reference":

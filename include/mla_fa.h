@@ -111,6 +111,13 @@ typedef enum {
  *         before the mask is added; 0 = off
  * (the variants are named for the Metal FA kernel of the llama.cpp tag page, PR
  * #29570; these formulas are this library's reading of them)
+ * mask_gather 1: sparse attention straight from the mask, without an index list
+ *         (the compaction fused into the attention, for any n_q): the cells, in
+ *         chunks of 8, are dealt round-robin to a sequence's KV splits; every work
+ *         unit compacts its chunks and gathers only the cache rows that some query
+ *         row of its 128-row group keeps (mask != -inf); each row still applies its
+ *         own mask. Requires mask, excludes idx and alibi_slopes. The workspace then
+ *         also holds the units' cell lists
  * A stride of 0 means "dense" (the natural value for the given sizes).
  */
 typedef struct mla_fa_args {
@@ -140,6 +147,7 @@ typedef struct mla_fa_args {
   const float* sinks;       /* DEVICE fp32 [n_head], optional                  */
   const float* alibi_slopes; /* DEVICE fp32 [n_head], optional                 */
   float softcap;            /* > 0 enables the logit softcap                   */
+  int mask_gather;          /* 1: gather the mask's kept cells (no idx)        */
 } mla_fa_args;
 
 /* Forward pass with the sizes of the single-sequence call:

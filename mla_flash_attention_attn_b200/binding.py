@@ -64,6 +64,7 @@ class mla_fa_args(ctypes.Structure):
         ("sinks", ctypes.c_void_p),
         ("alibi_slopes", ctypes.c_void_p),
         ("softcap", ctypes.c_float),
+        ("mask_gather", ctypes.c_int),
     ]
 
 
@@ -153,14 +154,16 @@ def _host_i32(arr):
 
 
 def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None,
-              wv=None, out_proj=None, sinks=None, alibi_slopes=None, softcap=0.0):
+              wv=None, out_proj=None, sinks=None, alibi_slopes=None, softcap=0.0,
+              mask_gather=False):
     """Fill mla_fa_args from batched torch tensors.
 
     q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
     mask [n_seq][n_q][n_kv] f16 or None; out [n_seq][n_q][n_head][512] f32 (or None with
     wv); wv [n_head][512][128] f16 and out_proj [n_seq][n_q][n_head][128] f32 for the
     fused value up-projection; sinks / alibi_slopes fp32 [n_head] and softcap > 0 for
-    the attention variants. Returns (args, keepalive)."""
+    the attention variants; mask_gather=True for sparse attention straight from the mask
+    (the kernel compacts it, no index list). Returns (args, keepalive)."""
     n_seq, n_q, n_head, dk = q.shape
     if dk != DK:
         raise ValueError("q must end in 576")
@@ -186,6 +189,7 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     a.sinks = None if sinks is None else sinks.data_ptr()
     a.alibi_slopes = None if alibi_slopes is None else alibi_slopes.data_ptr()
     a.softcap = float(softcap)
+    a.mask_gather = 1 if mask_gather else 0
     keep = _host_i32(kv_len)
     a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
     if idx is not None:
@@ -223,14 +227,16 @@ def mla_fa_forward(q, kcache, kv_type, mask, scale, out, stream=None):
 
 
 def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, idx_count=None,
-            workspace=None, stream=None, sinks=None, alibi_slopes=None, softcap=0.0):
+            workspace=None, stream=None, sinks=None, alibi_slopes=None, softcap=0.0,
+            mask_gather=False):
     """Batched forward through mla_fa_forward_ex; allocates out/workspace with torch if absent."""
     import torch
 
     if out is None:
         out = torch.empty(q.shape[:3] + (DV,), dtype=torch.float32, device=q.device)
     args, keep = make_args(q, kcache, kv_type, mask, out, scale, kv_len, idx, idx_count,
-                           sinks=sinks, alibi_slopes=alibi_slopes, softcap=softcap)
+                           sinks=sinks, alibi_slopes=alibi_slopes, softcap=softcap,
+                           mask_gather=mask_gather)
     need = mla_fa_workspace_size(args)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -240,7 +246,7 @@ def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, id
 
 
 def forward_proj(q, kcache, kv_type, mask, scale, wv, out_proj=None, kv_len=None, idx=None,
-                 idx_count=None, workspace=None, stream=None):
+                 idx_count=None, workspace=None, stream=None, mask_gather=False):
     """Forward with the fused value up-projection (wv [n_head][512][128] f16); returns
     out_proj [n_seq][n_q][n_head][128] f32. The 512-wide attention rows are not written."""
     import torch
@@ -248,7 +254,7 @@ def forward_proj(q, kcache, kv_type, mask, scale, wv, out_proj=None, kv_len=None
     if out_proj is None:
         out_proj = torch.empty(q.shape[:3] + (int(wv.shape[2]),), dtype=torch.float32, device=q.device)
     args, keep = make_args(q, kcache, kv_type, mask, None, scale, kv_len, idx, idx_count, wv=wv,
-                           out_proj=out_proj)
+                           out_proj=out_proj, mask_gather=mask_gather)
     need = mla_fa_workspace_size(args)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

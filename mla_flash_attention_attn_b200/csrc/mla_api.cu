@@ -164,6 +164,9 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (proj && a->proj_dim != MLA_PROJ_DIM) return MLA_ERR_UNSUPPORTED;
   if (!(a->softcap >= 0.f) || std::isinf(a->softcap)) return MLA_ERR_SHAPE;  // NaN, <0, inf
   if (a->alibi_slopes != nullptr && a->idx != nullptr) return MLA_ERR_UNSUPPORTED;
+  if (a->mask_gather != 0 && a->mask_gather != 1) return MLA_ERR_SHAPE;
+  if (a->mask_gather && a->mask == nullptr) return MLA_ERR_NULL;
+  if (a->mask_gather && (a->idx != nullptr || a->alibi_slopes != nullptr)) return MLA_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(a->sinks) & 3) || (reinterpret_cast<uintptr_t>(a->alibi_slopes) & 3))
     return MLA_ERR_ALIGN;
   if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
@@ -256,6 +259,23 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
 
 size_t slot_bytes() { return (size_t)mla::kRowsPerGroup * (mla::kDV + 1) * sizeof(float); }
 
+// Mask gather: entries of one CTA's cell list (8 per chunk of the most chunks a
+// split is dealt, rounded up to 64) and the bytes of all lists of a launch.
+int64_t gather_stride(const Plan& plan) {
+  int64_t m = 0;
+  for (int b = 0; b < plan.n_seq; ++b) {
+    const int64_t chunks = ((int64_t)plan.kv_len[b] + 7) / 8;
+    m = std::max<int64_t>(m, 8 * ((chunks + plan.n_split[b] - 1) / plan.n_split[b]));
+  }
+  return std::max<int64_t>(64, (m + 63) / 64 * 64);
+}
+size_t gather_bytes(const Resolved& r, const Plan& plan, int slots) {
+  if (!r.a.mask_gather) return 0;
+  const size_t head = (size_t)slots * slot_bytes();
+  const size_t start = (head + 255) / 256 * 256;
+  return start - head + (size_t)2 * plan.total_units * gather_stride(plan) * sizeof(int32_t);
+}
+
 size_t workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_splits) {
   size_t need = 0;
   int mu = 0, ms = 0;
@@ -263,7 +283,7 @@ size_t workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_s
   for (int s0 = 0; s0 < r.a.n_seq; s0 += mla::kPlanMaxSeq) {
     const int n = std::min(mla::kPlanMaxSeq, r.a.n_seq - s0);
     const int slots = build_plan(r, s0, n, sm_count, &plan);
-    need = std::max(need, (size_t)slots * slot_bytes());
+    need = std::max(need, (size_t)slots * slot_bytes() + gather_bytes(r, plan, slots));
     mu = std::max(mu, plan.total_units);
     for (int b = 0; b < n; ++b) ms = std::max(ms, plan.n_split[b]);
   }
@@ -298,13 +318,23 @@ int make_out_map(CUtensorMap* m, void* base, uint64_t d1, uint64_t d2, uint64_t 
   return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// One instance of the attention kernel, with its block size (cfg has the rest).
+template <int kMode, bool kVariant, bool kGather>
+cudaError_t launch_fwd(cudaLaunchConfig_t cfg, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                       const CUtensorMap& tm_v, const CUtensorMap& tm_o, const CUtensorMap& tm_w,
+                       const mla::Plan& plan, const mla::MlaFwdParams& p) {
+  cfg.blockDim = dim3(mla::FwdCfg<kMode>::kThreads);
+  return cudaLaunchKernelEx(&cfg, mla::mla_fwd_kernel<kMode, kVariant, kGather>, tm_q, tm_k, tm_v,
+                            tm_o, tm_w, plan, p);
+}
+
 int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const mla_fa_args& a = r.a;
   const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
   if (need > 0 && (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)))
     return MLA_ERR_WORKSPACE;
   const int mode = a.kcache_type == MLA_KV_Q8_0 ? mla::kModeQ8
-                   : (a.idx != nullptr ? mla::kModeGatherF16 : mla::kModeTma);
+                   : (a.idx != nullptr || a.mask_gather ? mla::kModeGatherF16 : mla::kModeTma);
   CUtensorMap tm_q, tm_k, tm_v;
   const uint64_t row_bytes = MLA_DK * 2;
   int rc = make_map(&tm_q, a.q, MLA_DK, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
@@ -341,12 +371,16 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
     const void* fwd_kernels[] = {
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, true>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true>};
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, true, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, true>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, true>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, false>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, true>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, true>};
     bool ok = true;
     for (const void* k : fwd_kernels)
       ok = ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -385,6 +419,14 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                 (size_t)slots * mla::kRowsPerGroup * mla::kDV * 4)
                      : nullptr;
+    p.mask_gather = a.mask_gather;
+    p.gather_list = nullptr;
+    p.gather_stride = 0;
+    if (a.mask_gather) {
+      const size_t head = (size_t)slots * slot_bytes();
+      p.gather_list = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + (head + 255) / 256 * 256);
+      p.gather_stride = gather_stride(plan);
+    }
     CUtensorMap tm_w = tm_o;  // unused when no sequence of this launch is split
     if (slots > 0) {
       rc = make_out_map(&tm_w, ws, (uint64_t)slots * mla::kRowsPerGroup, 1,
@@ -403,30 +445,27 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     fattr[0].val.programmaticStreamSerializationAllowed = 1;
     fcfg.attrs = fattr;
     fcfg.numAttrs = 1;
-    cudaError_t fe;
-    // the softcap / ALiBi instance only when the call asks for one of them
+    // the softcap / ALiBi instance and the mask-gather instance only when the call
+    // asks for them
     const bool variant = a.softcap > 0.f || a.alibi_slopes != nullptr;
-    if (mode == mla::kModeTma) {
-      ProfScope prof(kKernFwdF16, stream);
-      fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeTma>::kThreads);
-      fe = variant ? cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeTma, true>, tm_q, tm_k,
-                                        tm_v, tm_o, tm_w, plan, p)
-                   : cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeTma, false>, tm_q, tm_k,
-                                        tm_v, tm_o, tm_w, plan, p);
-    } else if (mode == mla::kModeGatherF16) {
-      ProfScope prof(kKernFwdGather, stream);
-      fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeGatherF16>::kThreads);
-      fe = variant ? cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeGatherF16, true>, tm_q,
-                                        tm_k, tm_v, tm_o, tm_w, plan, p)
-                   : cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeGatherF16, false>, tm_q,
-                                        tm_k, tm_v, tm_o, tm_w, plan, p);
-    } else {
-      ProfScope prof(kKernFwdQ8, stream);
-      fcfg.blockDim = dim3(mla::FwdCfg<mla::kModeQ8>::kThreads);
-      fe = variant ? cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeQ8, true>, tm_q, tm_k,
-                                        tm_v, tm_o, tm_w, plan, p)
-                   : cudaLaunchKernelEx(&fcfg, mla::mla_fwd_kernel<mla::kModeQ8, false>, tm_q, tm_k,
-                                        tm_v, tm_o, tm_w, plan, p);
+    const bool gather = a.mask_gather != 0;
+    cudaError_t fe;
+    {
+      ProfScope prof(mode == mla::kModeTma ? kKernFwdF16
+                     : mode == mla::kModeGatherF16 ? kKernFwdGather : kKernFwdQ8, stream);
+      if (mode == mla::kModeTma)
+        fe = variant ? launch_fwd<mla::kModeTma, true, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                     : launch_fwd<mla::kModeTma, false, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
+      else if (mode == mla::kModeGatherF16)
+        fe = gather ? (variant ? launch_fwd<mla::kModeGatherF16, true, true>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                               : launch_fwd<mla::kModeGatherF16, false, true>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p))
+                    : (variant ? launch_fwd<mla::kModeGatherF16, true, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                               : launch_fwd<mla::kModeGatherF16, false, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p));
+      else
+        fe = gather ? (variant ? launch_fwd<mla::kModeQ8, true, true>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                               : launch_fwd<mla::kModeQ8, false, true>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p))
+                    : (variant ? launch_fwd<mla::kModeQ8, true, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                               : launch_fwd<mla::kModeQ8, false, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p));
     }
     if (fe != cudaSuccess) return MLA_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;

@@ -77,6 +77,11 @@ struct MlaFwdParams {
   // variants (0 / nullptr = off): logit softcap, ALiBi slopes per head
   float softcap;
   const float* slopes;
+  // mask gather (no index list): unit u, CTA rank r lists its kept cells at
+  // gather_list + (2u + r) * gather_stride
+  int mask_gather;
+  int32_t* gather_list;
+  int64_t gather_stride;
 };
 
 // How K/V tiles reach shared memory.
@@ -233,9 +238,10 @@ __device__ __forceinline__ void block_values(const RawBlock<kMode>& rb, uint32_t
   }
 }
 
-// kVariant: the instance that applies the logit softcap and ALiBi (the host launches it
-// only when a call asks for one of them, so the common path carries none of that code)
-template <int kMode, bool kVariant>
+// kVariant: the instance that applies the logit softcap and ALiBi; kGather: the instance
+// that compacts the mask itself (gather modes only). The host launches them only when a
+// call asks for them, so the common path carries none of that code.
+template <int kMode, bool kVariant, bool kGather>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThreads, 1)
     mla_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -310,14 +316,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   decode_unit(plan, blockIdx.x >> 1, b, g, s);
   const int b_abs = plan.seq_offset + b;
   const int n_split = plan.n_split[b];
-  const bool sparse = p.idx != nullptr;
-  const int len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
-  const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
-  const int tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
-  const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
-  const int n_tiles = tile_end - tile_begin;
-  const int key_end = min(len, tile_end * kTileKeys);
   const int row0 = g * kRowsPerGroup;
+  constexpr bool gather = kManual && kGather;
+  const bool sparse = p.idx != nullptr || gather;
+  // positions of the unit: an index list (its tiles of the sequence's list), or, with
+  // the mask gather, every kept cell of the chunks dealt to its split (below)
+  int len, tile_begin, n_tiles, key_end;
+  // the unit's index list, recomputed where it is read (cheaper than a live register)
+  auto list_ptr = [&]() -> const int32_t* {
+    return gather ? p.gather_list + (int64_t)(2 * (blockIdx.x >> 1) + rank) * p.gather_stride
+                  : p.idx + (int64_t)b_abs * p.idx_seq_stride;
+  };
+  if (gather) {
+    // The sequence's first kv_len cells, in chunks of 8, are dealt round-robin to its
+    // splits (chunk j to split j mod n_split), so that a run of kept cells (a recent
+    // window, say) is shared out instead of landing on one split. Each split compacts
+    // its chunks here into an ascending list of the cells that some row of this group
+    // keeps (mask != -inf): a thread takes one chunk, a block scan gives its offset.
+    // Both CTAs of the pair build the same list.
+    const int cells = plan.kv_len[b];
+    const int n_chunks = (cells + 7) >> 3;
+    const int t_lo = row0 / plan.n_head;
+    const int t_hi = min(plan.rows - 1, row0 + kRowsPerGroup - 1) / plan.n_head;
+    int32_t* out_list = p.gather_list + (int64_t)(2 * (blockIdx.x >> 1) + rank) * p.gather_stride;
+    int* scan = reinterpret_cast<int*>(xmax);  // warp totals of one pass
+    const uint16_t* mseq = p.mask + (int64_t)b_abs * p.mask_seq_stride;
+    constexpr int kT = FwdCfg<kMode>::kThreads;
+    int base = 0;
+    for (int i0 = 0; (int64_t)s + (int64_t)n_split * i0 < n_chunks; i0 += kT) {
+      const int64_t j = (int64_t)s + (int64_t)n_split * (i0 + (int)threadIdx.x);
+      const int cell0 = (int)(8 * j);
+      uint32_t keep = 0;
+      if (j < n_chunks) {
+        const int n_in = min(8, cells - cell0);
+        for (int t = t_lo; t <= t_hi; ++t) {
+          const uint16_t* mr = mseq + (int64_t)t * p.mask_row_stride + cell0;
+          if (p.mask_vec_ok && n_in == 8) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(mr));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if ((w[k] & 0xFFFFu) != 0xFC00u) keep |= 1u << (2 * k);
+              if ((w[k] >> 16) != 0xFC00u) keep |= 2u << (2 * k);
+            }
+          } else {
+            for (int k = 0; k < n_in; ++k)
+              if (__ldg(mr + k) != 0xFC00u) keep |= 1u << k;
+          }
+        }
+      }
+      const int cnt = __popc(keep);
+      int inc = cnt;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += y;
+      }
+      if (lane == 31) scan[warp] = inc;
+      __syncthreads();
+      int woff = 0, total = 0;
+      for (int w = 0; w < kT / 32; ++w) {
+        const int tw = scan[w];
+        if (w < warp) woff += tw;
+        total += tw;
+      }
+      int pos = base + woff + inc - cnt;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (keep & (1u << k)) out_list[pos++] = cell0 + k;
+      base += total;
+      __syncthreads();  // the warp totals are read before the next pass overwrites them
+    }
+    __syncthreads();  // the list is complete and visible to every thread of this CTA
+    len = base;
+    tile_begin = 0;
+    n_tiles = (len + kTileKeys - 1) / kTileKeys;
+    key_end = len;
+  } else {
+    len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
+    const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
+    tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
+    const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
+    n_tiles = tile_end - tile_begin;
+    key_end = min(len, tile_end * kTileKeys);
+  }
   bool failed = false;
 
   if constexpr (kManual) {
@@ -490,12 +572,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       const bool k_side = warp < 10;
       const int pt = (threadIdx.x - 256) & 63;
       const int64_t seq_row0 = (int64_t)b_abs * p.k_seq_stride;
-      const int32_t* idx_row = sparse ? p.idx + (int64_t)b_abs * p.idx_seq_stride : nullptr;
+      const int32_t* idx_row = sparse ? list_ptr() : nullptr;
       // cache row of key position `pos` in this unit's selection, or -1 (zero fill)
       auto resolve = [&](int pos) -> int {
         if (pos >= len) return -1;
         if (!sparse) return pos < p.n_kv ? pos : -1;
-        const int key = __ldg(idx_row + pos);
+        const int key = idx_row[pos];  // plain load: the gather list is written in this kernel
         if (key < 0 || key >= p.n_kv) {
           record_status(kStatusIndex);
           return -1;
@@ -709,7 +791,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
         for (int c = 0; c < kHalf / 8; ++c) mvec[c] = make_uint4(0u, 0u, 0u, 0u);
       } else if (kManual && sparse) {
-        const int32_t* ix = p.idx + (int64_t)b_abs * p.idx_seq_stride;
+        const int32_t* ix = list_ptr();
         uint32_t* mw = reinterpret_cast<uint32_t*>(mvec);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -717,7 +799,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
           for (int j = 0; j < 64; ++j) {
             const int pos = k0 + 64 * g + j;
-            cl[j] = pos < key_end ? __ldg(ix + pos) : -1;
+            cl[j] = pos < key_end ? ix[pos] : -1;
           }
           unsigned short hv[64];
 #pragma unroll

@@ -2,6 +2,9 @@
 include/mla_fa.h declares, and rejects bad arguments on the host before any
 launch (no kernel runs here)."""
 import ctypes
+import os
+import shutil
+import subprocess
 
 import pytest
 
@@ -25,6 +28,25 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(lib):
     missing = [n for n in binding.header_functions() if not hasattr(lib, n)]
     assert missing == []
+
+
+def test_argument_struct_matches_the_header(tmp_path):
+    # the ctypes mirror of mla_fa_args must agree with the C compiler on every field's
+    # offset and on the size, or every field after a mismatch is read wrongly
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    fields = [f[0] for f in binding.mla_fa_args._fields_]
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include \"mla_fa.h\"\nint main(void) {\n"
+                   + "".join(f'  printf("%zu\\n", offsetof(mla_fa_args, {f}));\n' for f in fields)
+                   + '  printf("%zu\\n", sizeof(mla_fa_args));\n  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True,
+                                          text=True).stdout.split()]
+    want = [getattr(binding.mla_fa_args, f).offset for f in fields] + [ctypes.sizeof(binding.mla_fa_args)]
+    assert got == want
 
 
 def test_status_strings(lib):
@@ -75,6 +97,10 @@ def call_ex(lib, a):
     (dict(softcap=-1.0), -2), (dict(softcap=float("nan")), -2), (dict(softcap=float("inf")), -2),
     (dict(alibi_slopes=FAKE, idx=FAKE, idx_count=FAKE), -8),
     (dict(sinks=FAKE + 2), -4), (dict(alibi_slopes=FAKE + 1), -4),
+    # mask gather: needs the mask, excludes an index list and ALiBi
+    (dict(mask_gather=2, mask=FAKE), -2), (dict(mask_gather=1), -1),
+    (dict(mask_gather=1, mask=FAKE, idx=FAKE, idx_count=FAKE), -8),
+    (dict(mask_gather=1, mask=FAKE, alibi_slopes=FAKE), -8),
 ])
 def test_argument_errors_are_returned_before_any_launch(lib, kw, expect):
     assert call_ex(lib, base_args(**kw)) == expect

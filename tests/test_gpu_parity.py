@@ -63,7 +63,8 @@ def run_gpu(w, kv_len="auto", mask="auto", k_pad=0, **variants):
         if variants.get(name) is not None:
             vt[name] = torch.from_numpy(np.asarray(variants[name], np.float32)).to(dev)
     binding.forward(q, k, w.kv_type, m, w.scale, out=out, kv_len=lens,
-                    softcap=variants.get("softcap", 0.0), **vt)
+                    softcap=variants.get("softcap", 0.0),
+                    mask_gather=variants.get("mask_gather", False), **vt)
     torch.cuda.synchronize()
     assert binding.mla_get_device_status() == 0
     tail = big[n_out:]
@@ -423,7 +424,103 @@ def test_sparse_out_of_range_index_is_reported_not_read():
 
 # ---- fused value up-projection (out_proj = O . W_UV per head) ---------------------
 
-def run_gpu_proj(w, wv):
+# ---- mask gather: sparse attention straight from the mask (the compaction fused in) ----
+# Dropping the cells whose mask is -inf leaves every row's softmax unchanged, so the
+# reference is the oracle's dense masked attention.
+def sparse_rows_mask(rng, n_q, n_kv, p_keep, shared_frac=0.0):
+    """Per-token keep patterns: a shared random part plus each token's own cells."""
+    shared = rng.random(n_kv) < p_keep * shared_frac
+    own = rng.random((n_q, n_kv)) < p_keep * (1.0 - shared_frac)
+    keep = own | shared[None]
+    vals = rng.standard_normal((n_q, n_kv)).astype(np.float16)
+    return np.where(keep, vals, np.float16(-np.inf)).astype(np.float16)
+
+
+def test_mask_gather_f16_single_query():
+    w = W.make("v2lite_decode", n_kv=3000, n_head=128, n_pad=0)
+    rng = np.random.default_rng(21)
+    keep = rng.random(3000) < 0.15
+    keep[-7:] = True
+    w.mask[0, 0] = np.where(keep, np.float16(0), np.float16(-np.inf))
+    check_all_rows(w, run_gpu(w, mask_gather=True), what="mask gather f16")
+
+
+@pytest.mark.parametrize("n_head,n_q", [(16, 8), (16, 19), (100, 3), (128, 3), (7, 5)])
+def test_mask_gather_multi_query(n_head, n_q):
+    # 128-row groups that span several tokens take the union of their masks; each row
+    # still applies its own
+    rng = np.random.default_rng(n_head * 100 + n_q)
+    n_kv = 2500
+    w = W.make("prefill_chunk", n_q=n_q, n_head=n_head, n_kv=n_kv)
+    w.mask[0] = sparse_rows_mask(rng, n_q, n_kv, 0.2, shared_frac=0.5)
+    w.mask[0, :, rng.integers(0, n_kv)] = 0
+    check_all_rows(w, run_gpu(w, mask_gather=True), what=f"mask gather H={n_head} n_q={n_q}")
+
+
+def test_mask_gather_ragged_batch_with_splits_and_empty_rows():
+    w = W.make("v3_batched_decode", n_seq=5, n_head=16, n_kv=9000, len_lo=1, len_hi=9000)
+    rng = np.random.default_rng(33)
+    w.q = rng.standard_normal((5, 2, 16, 576)).astype(np.float16)
+    w.kv_len = np.array([9000, 1, 0, 4097, 257], np.int32)
+    w.mask = np.stack([sparse_rows_mask(rng, 2, 9000, 0.1) for _ in range(5)])
+    w.mask[3] = np.float16(-np.inf)           # no kept cell in the whole sequence
+    w.mask[4, 1] = np.float16(-np.inf)        # one token with no kept cell
+    w.mask[1, :, 0] = 0
+    got = run_gpu(w, mask_gather=True)
+    assert np.all(got[2] == 0) and np.all(got[3] == 0) and np.all(got[4, 1] == 0)
+    for b in range(w.n_seq):
+        n = int(w.kv_len[b])
+        ref = oracle.attention(w.q[b], w.kcache[b][:n], w.kv_type, w.mask[b][:, :n], w.scale) if n \
+            else np.zeros((w.n_q * w.n_head, 512))
+        assert_parity(got[b].reshape(-1, 512), ref, f"mask gather ragged seq {b}")
+
+
+def test_mask_gather_every_cell_kept_equals_dense():
+    w = W.make("v3_batched_decode", n_seq=2, n_head=128, n_kv=3000, len_lo=3000, len_hi=3000)
+    dense = run_gpu(w)
+    gath = run_gpu(w, mask_gather=True)
+    assert_parity(gath.reshape(-1, 512), dense.reshape(-1, 512), "all kept vs dense")
+    check_all_rows(w, gath, what="mask gather all kept")
+
+
+def test_mask_gather_q8_0_reduced():
+    w = W.make("sparse_q8_decode", n_kv=16384, n_head=128, tail_blocks=4)
+    got = run_gpu(w, mask_gather=True)
+    ref = oracle.attention(w.q[0], q8_f16_rounded(w.kcache[0]), oracle.KV_F16, w.mask[0], w.scale)
+    assert_parity(got[0].reshape(-1, 512), ref, "mask gather q8_0")
+
+
+def test_mask_gather_q8_0_full_size_sampled_rows():
+    w = W.make("sparse_q8_decode")
+    got = run_gpu(w, mask_gather=True)
+    rows = np.array([0, 1, 31, 64, 100, 127], np.int32)
+    ref = oracle.attention(w.q[0], w.kcache[0], oracle.KV_Q8_0, w.mask[0], w.scale, rows=rows)
+    assert_parity(got[0].reshape(-1, 512)[rows], ref, "mask gather q8_0 full")
+
+
+def test_mask_gather_q8_0_multi_query_ragged():
+    rng = np.random.default_rng(44)
+    w = W.make("sparse_q8_decode", n_kv=5000, n_head=16, block=8, tail_blocks=2)
+    q = rng.standard_normal((1, 6, 16, 576)).astype(np.float16)
+    w.q = q
+    w.mask = sparse_rows_mask(rng, 6, 5000, 0.12, shared_frac=0.3)[None]
+    got = run_gpu(w, mask_gather=True)
+    ref = oracle.attention(w.q[0], q8_f16_rounded(w.kcache[0]), oracle.KV_F16, w.mask[0], w.scale)
+    assert_parity(got[0].reshape(-1, 512), ref, "mask gather q8_0 multi-query")
+
+
+def test_mask_gather_with_variants():
+    w = W.make("prefill_chunk", n_q=4, n_head=16, n_kv=3000)
+    rng = np.random.default_rng(55)
+    w.mask[0] = sparse_rows_mask(rng, 4, 3000, 0.25)
+    sinks = rng.standard_normal(16).astype(np.float32)
+    got = run_gpu(w, mask_gather=True, sinks=sinks, softcap=30.0)
+    ref = oracle.attention_variants(w.q[0], w.kcache[0], w.kv_type, w.mask[0], w.scale,
+                                    softcap=30.0, sinks=sinks)
+    assert_parity(got[0].reshape(-1, 512), ref, "mask gather + sinks + softcap")
+
+
+def run_gpu_proj(w, wv, mask_gather=False):
     """mla_fa_forward_ex with wv set; returns out_proj [n_seq][n_q][n_head][128]."""
     torch = torch_mod()
     dev = torch.device("cuda")
@@ -434,7 +531,7 @@ def run_gpu_proj(w, wv):
     big = torch.full((n_out + CANARY,), float("nan"), dtype=torch.float32, device=dev)
     out_proj = big[:n_out].view(w.n_seq, w.n_q, w.n_head, 128)
     binding.forward_proj(q, k, w.kv_type, m, w.scale, torch.from_numpy(wv).to(dev),
-                         out_proj=out_proj, kv_len=w.kv_len)
+                         out_proj=out_proj, kv_len=w.kv_len, mask_gather=mask_gather)
     torch.cuda.synchronize()
     assert binding.mla_get_device_status() == 0
     assert bool(torch.isnan(big[n_out:]).all()), "write past the end of out_proj"
@@ -462,6 +559,14 @@ def test_fused_projection_matches_oracle(case):
     wv = W.wv_random(n_head=w.n_head)
     got = run_gpu_proj(w, wv)
     check_proj(w, wv, got, case)
+
+
+def test_fused_projection_with_mask_gather():
+    w = W.make("prefill_chunk", n_q=3, n_head=128, n_kv=4000)
+    rng = np.random.default_rng(66)
+    w.mask[0] = sparse_rows_mask(rng, 3, 4000, 0.1)
+    wv = W.wv_random(n_head=128)
+    check_proj(w, wv, run_gpu_proj(w, wv, mask_gather=True), "projection + mask gather")
 
 
 def test_fused_projection_with_an_empty_sequence():
