@@ -257,7 +257,8 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
   return slots;
 }
 
-size_t slot_bytes() { return (size_t)mla::kRowsPerGroup * (mla::kDV + 1) * sizeof(float); }
+// One split partial: 128 rows of O_s / l_s in f16, and their 128 fp32 log-sum-exps.
+size_t slot_bytes() { return (size_t)mla::kRowsPerGroup * (mla::kDV * 2 + sizeof(float)); }
 
 // Mask gather: entries of one CTA's cell list (8 per chunk of the most chunks a
 // split is dealt, rounded up to 64) and the bytes of all lists of a launch.
@@ -318,6 +319,19 @@ int make_out_map(CUtensorMap* m, void* base, uint64_t d1, uint64_t d2, uint64_t 
   return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
+// f16 [rows][512] view of the split partials for the kernel's TMA stores: boxes of 32
+// rows x 64 columns (128-byte rows), 128-byte swizzle.
+int make_part_map(CUtensorMap* m, void* base, uint64_t rows) {
+  cuuint64_t dims[3] = {(cuuint64_t)MLA_DV, rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)MLA_DV * 2, (cuuint64_t)rows * MLA_DV * 2};
+  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult res = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, base, dims, strides, box, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // One instance of the attention kernel, with its block size (cfg has the rest).
 template <int kMode, bool kVariant, bool kGather>
 cudaError_t launch_fwd(cudaLaunchConfig_t cfg, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
@@ -360,11 +374,12 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   }
   CUtensorMap tm_o;
   // with the projection every sequence writes partials and the kernel never stores
-  // to out (which may be NULL): the output map then views the workspace
+  // to out (which may be NULL): the output map then views the workspace (the first
+  // 64 fp32 rows, inside the first slot)
   if (rc == MLA_OK) {
     if (r.proj)
-      rc = make_out_map(&tm_o, ws, (uint64_t)mla::kRowsPerGroup, 1,
-                        (uint64_t)mla::kRowsPerGroup * MLA_DV * 4);
+      rc = make_out_map(&tm_o, ws, (uint64_t)mla::kRowsPerGroup / 2, 1,
+                        (uint64_t)mla::kRowsPerGroup / 2 * MLA_DV * 4);
     else
       rc = make_out_map(&tm_o, a.out, (uint64_t)r.rows, (uint64_t)a.n_seq, (uint64_t)r.o_ss * 4);
   }
@@ -415,9 +430,9 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   for (int s0 = 0; s0 < a.n_seq; s0 += mla::kPlanMaxSeq) {
     const int n = std::min(mla::kPlanMaxSeq, a.n_seq - s0);
     const int slots = build_plan(r, s0, n, st->sm_count, &plan);
-    p.ws_o = static_cast<float*>(ws);
+    p.ws_o = static_cast<uint16_t*>(ws);
     p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                                (size_t)slots * mla::kRowsPerGroup * mla::kDV * 4)
+                                                (size_t)slots * mla::kRowsPerGroup * mla::kDV * 2)
                      : nullptr;
     p.mask_gather = a.mask_gather;
     p.gather_list = nullptr;
@@ -429,8 +444,7 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     }
     CUtensorMap tm_w = tm_o;  // unused when no sequence of this launch is split
     if (slots > 0) {
-      rc = make_out_map(&tm_w, ws, (uint64_t)slots * mla::kRowsPerGroup, 1,
-                        (uint64_t)slots * mla::kRowsPerGroup * MLA_DV * 4);
+      rc = make_part_map(&tm_w, ws, (uint64_t)slots * mla::kRowsPerGroup);
       if (rc != MLA_OK) return rc;
     }
     // launched as a programmatic dependent of the stream's previous kernel: its setup
@@ -498,14 +512,14 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       {
         ProfScope prof(kKernCombine, stream);
         if (r.proj)
-          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_proj_kernel, plan, (const float*)p.ws_o,
+          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_proj_kernel, plan, (const uint16_t*)p.ws_o,
                                   (const float*)p.ws_lse, static_cast<const uint16_t*>(a.wv),
                                   a.out_proj, (int64_t)r.op_ss, a.sinks);
         else if (wide)
-          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const float*)p.ws_o,
+          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const uint16_t*)p.ws_o,
                                   (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks);
         else
-          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const float*)p.ws_o,
+          ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const uint16_t*)p.ws_o,
                                   (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks);
       }
       if (ce != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;

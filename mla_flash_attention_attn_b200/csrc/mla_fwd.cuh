@@ -55,7 +55,7 @@ __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0
 struct MlaFwdParams {
   const uint16_t* mask;      // f16 bits, or nullptr
   float* out;                // fp32 [seq][rows][512]
-  float* ws_o;               // fp32 [slot][128][512] split partials
+  uint16_t* ws_o;            // f16 [slot][128][512] split partials (O_s / l_s)
   float* ws_lse;             // fp32 [slot][128] log2-sum-exp of each partial
   int64_t mask_seq_stride;   // elements
   int64_t mask_row_stride;   // elements
@@ -1001,15 +1001,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
     const int ws_slot = plan.ws_base[b] >= 0 ? plan.ws_base[b] + g * n_split + s : -1;
     // O / l goes out through shared memory: each warp stages its 32 rows as eight
-    // 32 x 32 fp32 boxes (128-byte rows, 16-byte chunks XOR-swizzled by row, the
-    // layout of a 128-byte-swizzle tensor map) and one lane stores them with TMA.
+    // 32 x 32 fp32 boxes, or for a split partial four 32 x 64 f16 boxes (128-byte rows,
+    // 16-byte chunks XOR-swizzled by row, the layout of a 128-byte-swizzle tensor map),
+    // and one lane stores them with TMA.
     // Every MMA has finished (last o_done), so the operand rings are free; the 4
     // warps use the first 128 KB. Rows beyond the tensor are clipped by the store.
     // A warp whose 32 rows all lie past the sequence's rows has nothing to store.
     if (__any_sync(0xffffffffu, row_valid)) {
       const int wq = warp - 4;  // row half (wq & 1) of key half kh = wq >> 1
       uint8_t* wbox = smem + wq * 8 * 4096;
-      const CUtensorMap* tm = ws_slot >= 0 ? &tm_w : &tm_o;
+      const bool part = ws_slot >= 0;  // f16 partial (tm_w) or the fp32 output (tm_o)
+      const CUtensorMap* tm = part ? &tm_w : &tm_o;
       const int y = (ws_slot >= 0 ? ws_slot * kRowsPerGroup : row0) + kRowsPerCta * (int)rank +
                     32 * (wq & 1);
       const int z = ws_slot >= 0 ? 0 : b_abs;
@@ -1030,23 +1032,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[u][j] = 0u;
         }
+        if (part) {
+          // TMEM groups i, i+1 (i even) are 64 adjacent value columns: one f16 box
 #pragma unroll
-        for (int u = 0; u < kEpi; ++u) {
-          uint8_t* rowp = wbox + (g0 + u) * 4096 + lane * 128;
+          for (int u = 0; u < kEpi; u += 2) {
+            uint8_t* rowp = wbox + ((g0 + u) >> 1) * 4096 + lane * 128;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) << 4)) =
-                make_float4(__uint_as_float(v[u][4 * c]) * inv_l, __uint_as_float(v[u][4 * c + 1]) * inv_l,
-                            __uint_as_float(v[u][4 * c + 2]) * inv_l,
-                            __uint_as_float(v[u][4 * c + 3]) * inv_l);
+            for (int c = 0; c < 8; ++c) {
+              const uint32_t* x = &v[u + (c >> 2)][8 * (c & 3)];
+              uint32_t h[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const __half2 hh = __floats2half2_rn(__uint_as_float(x[2 * k]) * inv_l,
+                                                     __uint_as_float(x[2 * k + 1]) * inv_l);
+                h[k] = *reinterpret_cast<const uint32_t*>(&hh);
+              }
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < kEpi; ++u) {
+            uint8_t* rowp = wbox + (g0 + u) * 4096 + lane * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<float4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+                  make_float4(__uint_as_float(v[u][4 * c]) * inv_l, __uint_as_float(v[u][4 * c + 1]) * inv_l,
+                              __uint_as_float(v[u][4 * c + 2]) * inv_l,
+                              __uint_as_float(v[u][4 * c + 3]) * inv_l);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          // box i = TMEM columns 32i..32i+31: value columns 256 (i / 4) + 128 kh + 32 (i % 4)
-          for (int u = 0; u < kEpi; ++u) {
-            const int i = g0 + u;
-            tma_store_3d(tm, wbox + i * 4096, 256 * (i >> 2) + 128 * kh + 32 * (i & 3), y, z);
+          // TMEM columns 32i..32i+31 are value columns 256 (i / 4) + 128 kh + 32 (i % 4)
+          if (part) {
+            for (int u = 0; u < kEpi; u += 2) {
+              const int i = g0 + u;
+              tma_store_3d(tm, wbox + (i >> 1) * 4096, 256 * (i >> 2) + 128 * kh + 32 * (i & 3), y, z);
+            }
+          } else {
+            for (int u = 0; u < kEpi; ++u) {
+              const int i = g0 + u;
+              tma_store_3d(tm, wbox + i * 4096, 256 * (i >> 2) + 128 * kh + 32 * (i & 3), y, z);
+            }
           }
           bulk_commit_group();
         }
@@ -1073,6 +1102,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   }
 }
 
+// Four consecutive f16 partial values (one 8-byte load) as floats.
+__device__ __forceinline__ float4 part4(uint2 r) {
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 // LSE combine of split-KV partials (one CTA of 128 threads per query row, thread t
 // owning value columns 4t..4t+3):
 //   O = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),  M = max_s lse_s,
@@ -1085,7 +1121,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 // griddepcontrol.wait returns once the forward grid has completed and its partials
 // are visible.
 __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant__ Plan plan,
-                                                          const float* __restrict__ ws_o,
+                                                          const uint16_t* __restrict__ ws_o,
                                                           const float* __restrict__ ws_lse,
                                                           float* __restrict__ out,
                                                           int64_t out_seq_stride,
@@ -1100,14 +1136,14 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   const int rin = row % kRowsPerGroup;
   const int slot0 = plan.ws_base[b] + g * plan.n_split[b];
   const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
-  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
-  const float4* src0 =
-      reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + threadIdx.x;
+  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // 4-value groups per slot
+  const uint2* src0 =
+      reinterpret_cast<const uint2*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) + threadIdx.x;
   const float lse_l = lane < ns ? __ldg(lse_col + (int64_t)lane * kRowsPerGroup) : -INFINITY;
   constexpr int kFirst = 16;
-  float4 v[kFirst];
+  uint2 v[kFirst];
 #pragma unroll
-  for (int u = 0; u < kFirst; ++u) v[u] = u < ns ? __ldg(src0 + u * kSplitStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int u = 0; u < kFirst; ++u) v[u] = u < ns ? __ldg(src0 + u * kSplitStride4) : make_uint2(0u, 0u);
   float mx = lse_l;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -1124,14 +1160,15 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
 #pragma unroll
     for (int u = 0; u < kFirst; ++u) {
       const float w = __shfl_sync(0xffffffffu, wl, u);  // 0 past ns
-      acc.x = fmaf(w, v[u].x, acc.x);
-      acc.y = fmaf(w, v[u].y, acc.y);
-      acc.z = fmaf(w, v[u].z, acc.z);
-      acc.w = fmaf(w, v[u].w, acc.w);
+      const float4 x = part4(v[u]);
+      acc.x = fmaf(w, x.x, acc.x);
+      acc.y = fmaf(w, x.y, acc.y);
+      acc.z = fmaf(w, x.z, acc.z);
+      acc.w = fmaf(w, x.w, acc.w);
     }
     for (int s = kFirst; s < ns; ++s) {
       const float w = __shfl_sync(0xffffffffu, wl, s);
-      const float4 x = __ldg(src0 + s * kSplitStride4);
+      const float4 x = part4(__ldg(src0 + s * kSplitStride4));
       acc.x = fmaf(w, x.x, acc.x);
       acc.y = fmaf(w, x.y, acc.y);
       acc.z = fmaf(w, x.z, acc.z);
@@ -1155,7 +1192,7 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
 constexpr int kCombPer = 24;  // partial rows per warp held in registers
 
 __global__ void __launch_bounds__(128)
-    mla_combine_wide_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
+    mla_combine_wide_kernel(const __grid_constant__ Plan plan, const uint16_t* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, float* __restrict__ out,
                             int64_t out_seq_stride, const float* __restrict__ sinks) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -1171,20 +1208,20 @@ __global__ void __launch_bounds__(128)
   const int rin = row % kRowsPerGroup;
   const int slot0 = plan.ws_base[b] + g * ns;
   const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
-  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // float4 per slot
-  const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
-                       qtr * 32 + lane;
+  constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // 4-value groups per slot
+  const uint2* src0 = reinterpret_cast<const uint2*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
+                      qtr * 32 + lane;
   float lse[3];
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     const int sp = lane + 32 * k;
     lse[k] = sp < ns ? __ldg(lse_col + (int64_t)sp * kRowsPerGroup) : -INFINITY;
   }
-  float4 v[kCombPer];
+  uint2 v[kCombPer];
 #pragma unroll
   for (int j = 0; j < kCombPer; ++j) {
     const int sp = warp + 4 * j;
-    v[j] = sp < ns ? __ldg(src0 + sp * kSplitStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[j] = sp < ns ? __ldg(src0 + sp * kSplitStride4) : make_uint2(0u, 0u);
   }
   float mx = fmaxf(fmaxf(lse[0], lse[1]), lse[2]);
   for (int sp = lane + 96; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
@@ -1213,17 +1250,18 @@ __global__ void __launch_bounds__(128)
       const float wk = sp < 32 ? w[0] : (sp < 64 ? w[1] : w[2]);
       const float ww = __shfl_sync(0xffffffffu, wk, sp & 31);
       if (sp < ns && sp < 96) {
-        acc.x = fmaf(ww, v[j].x, acc.x);
-        acc.y = fmaf(ww, v[j].y, acc.y);
-        acc.z = fmaf(ww, v[j].z, acc.z);
-        acc.w = fmaf(ww, v[j].w, acc.w);
+        const float4 x = part4(v[j]);
+        acc.x = fmaf(ww, x.x, acc.x);
+        acc.y = fmaf(ww, x.y, acc.y);
+        acc.z = fmaf(ww, x.z, acc.z);
+        acc.w = fmaf(ww, x.w, acc.w);
       }
     }
     // splits past 96 (this warp's share), one at a time
     for (int sp = warp + 96; sp < ns; sp += 4) {
       const float l = __ldg(lse_col + (int64_t)sp * kRowsPerGroup);
       const float ww = l == -INFINITY ? 0.f : ex2_approx(l - mx);
-      const float4 x = __ldg(src0 + sp * kSplitStride4);
+      const float4 x = part4(__ldg(src0 + sp * kSplitStride4));
       acc.x = fmaf(ww, x.x, acc.x);
       acc.y = fmaf(ww, x.y, acc.y);
       acc.z = fmaf(ww, x.z, acc.z);
@@ -1274,7 +1312,7 @@ constexpr int kProjSmem = kProjWBytes + kProjRows * kProjORow * 4 +   // W, o_s
                           kProjRows * kProjDim * 4 + 16;              // CTA sum, barrier
 
 __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
-    mla_combine_proj_kernel(const __grid_constant__ Plan plan, const float* __restrict__ ws_o,
+    mla_combine_proj_kernel(const __grid_constant__ Plan plan, const uint16_t* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, const uint16_t* __restrict__ wv,
                             float* __restrict__ out_proj, int64_t op_seq_stride,
                             const float* __restrict__ sinks) {
@@ -1318,18 +1356,18 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
       const int slot0 = plan.ws_base[b] + (row / kRowsPerGroup) * ns;
       const int rin = row % kRowsPerGroup;
       const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
-      const float4* src0 = reinterpret_cast<const float4*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
-                           32 * qtr + lane;
+      const uint2* src0 = reinterpret_cast<const uint2*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +
+                          32 * qtr + lane;
       float lse[3];
 #pragma unroll
       for (int k = 0; k < 3; ++k) {
         const int sp = lane + 32 * k;
         lse[k] = sp < ns ? __ldg(lse_col + (int64_t)sp * kRowsPerGroup) : -INFINITY;
       }
-      float4 v[16];
+      uint2 v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u)
-        v[u] = u < ns ? __ldg(src0 + (int64_t)u * kSplitStride4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[u] = u < ns ? __ldg(src0 + (int64_t)u * kSplitStride4) : make_uint2(0u, 0u);
       float mx = fmaxf(fmaxf(lse[0], lse[1]), lse[2]);
       for (int sp = lane + 96; sp < ns; sp += 32) mx = fmaxf(mx, __ldg(lse_col + (int64_t)sp * kRowsPerGroup));
 #pragma unroll
@@ -1352,10 +1390,11 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const float w = __shfl_sync(0xffffffffu, wk[0], u);  // 0 past ns
-          acc.x = fmaf(w, v[u].x, acc.x);
-          acc.y = fmaf(w, v[u].y, acc.y);
-          acc.z = fmaf(w, v[u].z, acc.z);
-          acc.w = fmaf(w, v[u].w, acc.w);
+          const float4 x = part4(v[u]);
+          acc.x = fmaf(w, x.x, acc.x);
+          acc.y = fmaf(w, x.y, acc.y);
+          acc.z = fmaf(w, x.z, acc.z);
+          acc.w = fmaf(w, x.w, acc.w);
         }
         for (int sp = 16; sp < ns; ++sp) {
           float w;  // split sp's weight, the same in every lane
@@ -1366,7 +1405,7 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
             const float l = __ldg(lse_col + (int64_t)sp * kRowsPerGroup);
             w = l == -INFINITY ? 0.f : ex2_approx(l - mx);
           }
-          const float4 x = __ldg(src0 + (int64_t)sp * kSplitStride4);
+          const float4 x = part4(__ldg(src0 + (int64_t)sp * kSplitStride4));
           acc.x = fmaf(w, x.x, acc.x);
           acc.y = fmaf(w, x.y, acc.y);
           acc.z = fmaf(w, x.z, acc.z);

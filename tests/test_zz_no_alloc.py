@@ -73,16 +73,19 @@ def test_noalloc_refuses_a_pass_larger_than_its_scratch():
 
     binding.load()
     lib = binding.load()
-    # Find a batch whose split plan needs more partial slots than the scratch holds.
+    # Find a batch that needs more partial slots than the scratch holds: with attention
+    # sinks every sequence's 128-row groups write partials (a plain pass uses about one
+    # slot per CTA pair, which always fits).
     dev = torch.device("cuda")
     found = None
-    for n_seq in range(40, 74):
-        q = torch.zeros((n_seq, 1, 128, 576), dtype=torch.float16, device=dev)
-        k = torch.zeros((n_seq, 12800, 576), dtype=torch.float16, device=dev)
-        out = torch.zeros((n_seq, 1, 128, 512), dtype=torch.float32, device=dev)
-        args, keep = binding.make_args(q, k, 0, None, out, 0.07)
+    sinks = torch.zeros((128,), dtype=torch.float32, device=dev)
+    for n_seq in (32, 64, 96, 128):
+        q = torch.zeros((n_seq, 2, 128, 576), dtype=torch.float16, device=dev)
+        k = torch.zeros((n_seq, 256, 576), dtype=torch.float16, device=dev)
+        out = torch.zeros((n_seq, 2, 128, 512), dtype=torch.float32, device=dev)
+        args, keep = binding.make_args(q, k, 0, None, out, 0.07, sinks=sinks)
         if binding.mla_fa_workspace_size(args) > binding.NOALLOC_SCRATCH_BYTES:
-            found = (args, keep, q, k, out)
+            found = (args, keep, q, k, out, sinks)
             break
         del q, k, out
     assert found is not None, "no batch exceeds the scratch size"
