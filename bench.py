@@ -93,9 +93,9 @@ def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "cb8f35c8c8e195e7", "bytes": 171415296},
-    "prefill_chunk": {"source": "cb8f35c8c8e195e7", "bytes": 204832512},
-    "sparse_q8_decode": {"source": "cb8f35c8c8e195e7", "bytes": 10392320},
+    "v3_batched_decode": {"source": "ccab4893bcd64589", "bytes": 170689536},
+    "prefill_chunk": {"source": "ccab4893bcd64589", "bytes": 204933376},
+    "sparse_q8_decode": {"source": "ccab4893bcd64589", "bytes": 10393600},
 }
 
 
