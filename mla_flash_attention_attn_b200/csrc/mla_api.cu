@@ -175,6 +175,12 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (!std::isfinite(a->scale)) return MLA_ERR_SHAPE;
   const int64_t rows = (int64_t)a->n_q * a->n_head;
   if (rows > (1 << 24)) return MLA_ERR_SHAPE;
+  // the projection's grid has 4 CTAs per 8 (sequence, token) rows of a launch in its y
+  // dimension (at most 65535)
+  if (proj && (int64_t)4 *
+                  (((int64_t)std::min(a->n_seq, mla::kPlanMaxSeq) * a->n_q + mla::kProjRows - 1) /
+                   mla::kProjRows) > 65535)
+    return MLA_ERR_SHAPE;
   if (a->idx != nullptr && a->idx_count == nullptr) return MLA_ERR_NULL;
   r->a = *a;
   r->rows = (int)rows;

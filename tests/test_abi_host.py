@@ -93,6 +93,8 @@ def call_ex(lib, a):
     (dict(wv=FAKE, proj_dim=128, out_proj=FAKE + 4), -4),
     (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, out_proj_seq_stride=100, n_seq=2), -2),
     (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, out_proj_seq_stride=16 * 128 + 2, n_seq=2), -4),
+    # the projection grid's y dimension: 4 CTAs per 8 (sequence, token) rows <= 65535
+    (dict(wv=FAKE, proj_dim=128, out_proj=FAKE, n_seq=128, n_q=1050, n_head=1), -2),
     # attention variants
     (dict(softcap=-1.0), -2), (dict(softcap=float("nan")), -2), (dict(softcap=float("inf")), -2),
     (dict(alibi_slopes=FAKE, idx=FAKE, idx_count=FAKE), -8),
