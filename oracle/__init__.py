@@ -71,6 +71,8 @@ def _load():
         common = [P, P, I, P, P, L, I, I, L, D, P, L]
         lib.oracle_attention.argtypes = common + [P]
         lib.oracle_attention.restype = I
+        lib.oracle_attention_lse.argtypes = common + [P, P]
+        lib.oracle_attention_lse.restype = I
         lib.oracle_attention_online.argtypes = common + [L, P]
         lib.oracle_attention_online.restype = I
         lib.oracle_attention_split.argtypes = common + [P, I, P]
@@ -157,6 +159,47 @@ def attention(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None, idx=No
     if rc != 0:
         raise ValueError("oracle_attention rejected its arguments")
     return out
+
+
+def attention_lse(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None, idx=None):
+    """attention() and, per row, the natural log-sum-exp of the scores,
+    lse = log sum_j exp(scale*q.k_j + mask_j) (-inf for a row with nothing kept).
+    Returns (float64 [rows][512], float64 [rows])."""
+    q, kc, m, ix, rw, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, rows)
+    lse = np.zeros(out.shape[0], dtype=np.float64)
+    rc = _load().oracle_attention_lse(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
+                                      0 if ix is None else len(ix), n_q, n_head, n_kv, float(scale),
+                                      _ptr(rw), 0 if rw is None else len(rw), _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle_attention_lse rejected its arguments")
+    return out, lse
+
+
+def combine(o_parts, lse_parts):
+    """Merge partial attention results of the same rows over disjoint key sets
+    (split-KV across devices): with M = max_p lse_p and w_p = exp(lse_p - M),
+    out = sum_p w_p o_p / sum_p w_p and lse = M + log(sum_p w_p). A row whose parts
+    are all -inf gets out = 0 and lse = -inf. The merge follows from the softmax
+    definition: o_p = sum_{j in part p} e^{s_j} v_j / e^{lse_p}. The pages give the
+    running-max rescaling inside one pass (Vulkan FA for DeepSeek MLA article, section
+    2.2); the merge across parts is the same rule applied to whole parts.
+    o_parts float [P][rows][512], lse_parts float [P][rows]; returns float64
+    ([rows][512], [rows])."""
+    o = np.asarray(o_parts, dtype=np.float64)
+    lse = np.asarray(lse_parts, dtype=np.float64)
+    if o.ndim != 3 or lse.shape != o.shape[:2]:
+        raise ValueError("o_parts [P][rows][512] and lse_parts [P][rows]")
+    n_rows = o.shape[1]
+    out = np.zeros((n_rows, o.shape[2]), dtype=np.float64)
+    out_lse = np.full(n_rows, -np.inf)
+    for r in range(n_rows):
+        M = np.max(lse[:, r])
+        if M == -np.inf:
+            continue
+        w = np.exp(lse[:, r] - M)
+        out[r] = (w[:, None] * o[:, r, :]).sum(axis=0) / w.sum()
+        out_lse[r] = M + np.log(w.sum())
+    return out, out_lse
 
 
 def attention_online(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, tile=64, rows=None,

@@ -12,6 +12,7 @@
  *   p_j  = exp(s_j - M)
  *   L    = sum_j p_j
  *   o[d] = sum_j p_j * k[j,d] / L              for d < 512
+ *   lse  = M + log(L)                          (oracle_attention_lse)
  *
  * Sources (web pages on MLA flash attention):
  *  - Cache row = 512-wide latent followed by the 64-wide RoPE key, 576 in
@@ -140,16 +141,19 @@ static inline double score(const double* q, const void* kc, int kv_type, long ke
 /* Selected keys: all of 0..n_kv-1 when idx == NULL, else idx[0..n_sel). */
 static inline long key_at(const int32_t* idx, long i) { return idx ? (long)idx[i] : i; }
 
-/* Two-pass softmax-weighted sum for one query row. */
+/* Two-pass softmax-weighted sum for one query row; with lse != NULL also the
+ * row's natural log-sum-exp of the scores, M + log(L) (-inf when every cell is
+ * masked). */
 static void attend_two_pass(const double* q, const void* kc, int kv_type, const uint16_t* mrow,
                             const int32_t* idx, long n_sel, double scale, double* s,
-                            double* out) {
+                            double* out, double* lse) {
   double M = -INFINITY;
   for (long i = 0; i < n_sel; ++i) {
     s[i] = score(q, kc, kv_type, key_at(idx, i), mrow, scale);
     if (s[i] > M) M = s[i];
   }
   for (int d = 0; d < ORC_DV; ++d) out[d] = 0.0;
+  if (lse) *lse = -INFINITY;
   if (M == -INFINITY) return; /* every cell masked: o = 0 */
   double L = 0.0;
   for (long i = 0; i < n_sel; ++i) {
@@ -160,6 +164,7 @@ static void attend_two_pass(const double* q, const void* kc, int kv_type, const 
     for (int d = 0; d < ORC_DV; ++d) out[d] += p * kval(kc, kv_type, key, d);
   }
   for (int d = 0; d < ORC_DV; ++d) out[d] /= L;
+  if (lse) *lse = M + log(L);
 }
 
 /* One-pass tiled online softmax for one query row: running max m and running
@@ -252,11 +257,12 @@ enum { MODE_TWO_PASS = 0, MODE_ONLINE = 1, MODE_SPLIT = 2 };
  * idx    : NULL for all keys, else n_idx ascending cache rows (sparse)
  * rows   : NULL for every (t, h) in order, else n_rows row ids t*n_head + h
  * out    : double [n_rows or n_q*n_head][512]
+ * lse    : NULL, or double [n_rows or n_q*n_head] (two-pass mode only)
  * Returns 0, or -1 on a bad argument. */
 static int run(int mode, const uint16_t* q, const void* kcache, int kv_type, const uint16_t* mask,
                const int32_t* idx, long n_idx, int n_q, int n_head, long n_kv, double scale,
                const int32_t* rows, long n_rows, long tile, const int32_t* bounds, int n_split,
-               double* out) {
+               double* out, double* lse) {
   if (!q || !kcache || !out || n_q < 1 || n_head < 1 || n_kv < 1) return -1;
   if (kv_type != ORC_KV_F16 && kv_type != ORC_KV_Q8_0) return -1;
   if (idx) {
@@ -284,7 +290,7 @@ static int run(int mode, const uint16_t* q, const void* kcache, int kv_type, con
       const uint16_t* mrow = mask ? mask + t * n_kv : NULL;
       double* o = out + r * ORC_DV;
       if (mode == MODE_TWO_PASS)
-        attend_two_pass(qd, kcache, kv_type, mrow, idx, n_sel, scale, s, o);
+        attend_two_pass(qd, kcache, kv_type, mrow, idx, n_sel, scale, s, o, lse ? lse + r : NULL);
       else if (mode == MODE_ONLINE)
         attend_online(qd, kcache, kv_type, mrow, idx, n_sel, scale, tile, s, o);
       else
@@ -299,7 +305,17 @@ int oracle_attention(const uint16_t* q, const void* kcache, int kv_type, const u
                      const int32_t* idx, long n_idx, int n_q, int n_head, long n_kv, double scale,
                      const int32_t* rows, long n_rows, double* out) {
   return run(MODE_TWO_PASS, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, 0, NULL, 0, out);
+             n_rows, 0, NULL, 0, out, NULL);
+}
+
+/* oracle_attention plus each row's natural log-sum-exp of its scores. */
+int oracle_attention_lse(const uint16_t* q, const void* kcache, int kv_type, const uint16_t* mask,
+                         const int32_t* idx, long n_idx, int n_q, int n_head, long n_kv,
+                         double scale, const int32_t* rows, long n_rows, double* out,
+                         double* lse) {
+  if (!lse) return -1;
+  return run(MODE_TWO_PASS, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
+             n_rows, 0, NULL, 0, out, lse);
 }
 
 int oracle_attention_online(const uint16_t* q, const void* kcache, int kv_type,
@@ -308,7 +324,7 @@ int oracle_attention_online(const uint16_t* q, const void* kcache, int kv_type,
                             long tile, double* out) {
   if (tile < 1) return -1;
   return run(MODE_ONLINE, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, tile, NULL, 0, out);
+             n_rows, tile, NULL, 0, out, NULL);
 }
 
 int oracle_attention_split(const uint16_t* q, const void* kcache, int kv_type,
@@ -320,7 +336,7 @@ int oracle_attention_split(const uint16_t* q, const void* kcache, int kv_type,
   for (int i = 0; i < n_split; ++i)
     if (bounds[i + 1] < bounds[i]) return -1;
   return run(MODE_SPLIT, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, 0, bounds, n_split, out);
+             n_rows, 0, bounds, n_split, out, NULL);
 }
 
 /* Keep rule: a cell is kept iff its f16 bits are not -inf (0xFC00).

@@ -519,3 +519,86 @@ def test_all_variants_together_match_brute_force():
                                     sinks=sinks)
     want = brute_force_variants(q, k, mask, 0.1, softcap=3.0, slopes=slopes, pos0=47, sinks=sinks)
     assert np.allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+# ---- log-sum-exp of a row and the merge of partial results (split-KV across devices) --
+
+def test_lse_of_equal_scores_is_log_count():
+    # Q = 0 and a zero mask: every score is 0, so lse = log(n) exactly
+    rng = np.random.default_rng(40)
+    for n in (1, 2, 7, 300):
+        q = np.zeros((1, 3, DK), np.float16)
+        k = rand_f16(rng, (n, DK))
+        _, lse = oracle.attention_lse(q, k, mask=np.zeros((1, n), np.float16), scale=0.3)
+        np.testing.assert_allclose(lse, np.full(3, math.log(n)), rtol=0, atol=1e-13)
+
+
+def test_lse_with_a_one_hot_query_is_a_library_logsumexp():
+    # q = e_c: the score of key j is scale * k[j, c] + mask[j], so the row's lse is
+    # scipy's logsumexp of those numbers
+    from scipy.special import logsumexp
+
+    rng = np.random.default_rng(41)
+    n, c, scale = 200, 517, 0.37
+    k = rand_f16(rng, (n, DK), std=3.0)
+    mask = rand_f16(rng, (1, n))
+    mask[0, rng.random(n) < 0.3] = NEG
+    q = np.zeros((1, 1, DK), np.float16)
+    q[0, 0, c] = 1.0
+    _, lse = oracle.attention_lse(q, k, mask=mask, scale=scale)
+    s = scale * k[:, c].astype(np.float64) + mask[0].astype(np.float64)
+    np.testing.assert_allclose(lse[0], logsumexp(s), rtol=0, atol=1e-12)
+
+
+def test_lse_of_a_fully_masked_row_is_minus_inf_and_shifts_with_the_mask():
+    rng = np.random.default_rng(42)
+    q = rand_f16(rng, (2, 2, DK))
+    k = rand_f16(rng, (50, DK))
+    mask = np.zeros((2, 50), np.float16)
+    mask[1, :] = NEG
+    mask[0, 40:] = NEG
+    _, lse = oracle.attention_lse(q, k, mask=mask, scale=0.07)
+    assert np.all(np.isneginf(lse[2:])) and np.all(np.isfinite(lse[:2]))
+    shifted = np.where(np.isneginf(mask), mask, mask + np.float16(6.0)).astype(np.float16)
+    _, lse2 = oracle.attention_lse(q, k, mask=shifted, scale=0.07)
+    np.testing.assert_allclose(lse2[:2], lse[:2] + 6.0, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("cuts", [(0, 300), (0, 100, 300), (0, 1, 150, 151, 300), (0, 60, 120, 300)])
+def test_combine_of_key_range_parts_equals_the_whole(cuts):
+    # attention over disjoint key ranges, merged by the log-sum-exp rule, is the
+    # attention over all keys: pins the merge against the softmax definition. The
+    # (0, 60, 120, 300) cut has a part whose keys are all masked (lse -inf).
+    rng = np.random.default_rng(43)
+    n = 300
+    q = rand_f16(rng, (3, 4, DK))
+    k = rand_f16(rng, (n, DK))
+    mask = rand_f16(rng, (3, n))
+    mask[:, 60:120] = NEG
+    o_all, lse_all = oracle.attention_lse(q, k, mask=mask, scale=0.06)
+    parts = [oracle.attention_lse(q, k[a:b], mask=mask[:, a:b], scale=0.06)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    o, lse = oracle.combine(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    np.testing.assert_allclose(o, o_all, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_all, rtol=0, atol=1e-12)
+
+
+def test_combine_closed_forms():
+    rng = np.random.default_rng(44)
+    o = rng.standard_normal((2, 5, DV))
+    lse0 = rng.standard_normal(5)
+    # one part: the identity
+    oo, ll = oracle.combine(o[:1], lse0[None])
+    np.testing.assert_array_equal(oo, o[0])
+    np.testing.assert_array_equal(ll, lse0)
+    # weights 1 : 3
+    lse = np.stack([lse0, lse0 + math.log(3.0)])
+    oo, ll = oracle.combine(o, lse)
+    np.testing.assert_allclose(oo, (o[0] + 3.0 * o[1]) / 4.0, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(ll, lse0 + math.log(4.0), rtol=0, atol=1e-13)
+    # a -inf part is ignored; all parts -inf give 0 and -inf
+    lse = np.stack([lse0, np.full(5, -np.inf)])
+    oo, ll = oracle.combine(o, lse)
+    np.testing.assert_array_equal(oo, o[0])
+    oo, ll = oracle.combine(o, np.full((2, 5), -np.inf))
+    assert np.all(oo == 0) and np.all(np.isneginf(ll))
