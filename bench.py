@@ -93,9 +93,9 @@ def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "d2f9cebac91a0ba1", "bytes": 170689536},
-    "prefill_chunk": {"source": "d2f9cebac91a0ba1", "bytes": 204933376},
-    "sparse_q8_decode": {"source": "d2f9cebac91a0ba1", "bytes": 10393600},
+    "v3_batched_decode": {"source": "c4969cb3127192b8", "bytes": 170689536},
+    "prefill_chunk": {"source": "c4969cb3127192b8", "bytes": 204933376},
+    "sparse_q8_decode": {"source": "c4969cb3127192b8", "bytes": 10393600},
 }
 
 

@@ -118,6 +118,12 @@ typedef enum {
  *         row of its 128-row group keeps (mask != -inf); each row still applies its
  *         own mask. Requires mask, excludes idx and alibi_slopes. The workspace then
  *         also holds the units' cell lists
+ * out_lse DEVICE fp32 [n_seq][n_q][n_head] or NULL: each row's natural log-sum-exp of
+ *         its scores, lse = log sum_j exp(scale q.k_j + mask_j) (-inf for a row with
+ *         nothing kept), next to out. With it, partial results of the same rows over
+ *         disjoint key ranges (a cache split across devices, say) merge exactly with
+ *         mla_fa_combine. Every sequence then writes partials. Excludes sinks and wv
+ *         (MLA_ERR_UNSUPPORTED); 4-byte aligned
  * A stride of 0 means "dense" (the natural value for the given sizes).
  */
 typedef struct mla_fa_args {
@@ -148,6 +154,7 @@ typedef struct mla_fa_args {
   const float* alibi_slopes; /* DEVICE fp32 [n_head], optional                 */
   float softcap;            /* > 0 enables the logit softcap                   */
   int mask_gather;          /* 1: gather the mask's kept cells (no idx)        */
+  float* out_lse;           /* DEVICE, optional: natural log-sum-exp per row   */
 } mla_fa_args;
 
 /* Forward pass with the sizes of the single-sequence call:
@@ -203,6 +210,22 @@ int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, vo
  *   without ordering) race on it and give wrong results. */
 #define MLA_NOALLOC_SCRATCH_BYTES (24u << 20)
 int mla_fa_forward_noalloc(const mla_fa_args* a, void* stream);
+
+/* Merge of partial results of the same query rows over disjoint key sets (the
+ * log-sum-exp rule of the split-KV combine, applied across calls, e.g. a cache
+ * split across devices whose per-device results were gathered):
+ *   M = max_p lse_p[r],  w_p = exp(lse_p[r] - M),
+ *   out[r] = sum_p w_p o_p[r] / sum_p w_p,   out_lse[r] = M + log(sum_p w_p).
+ * A row whose parts are all -inf gets out = 0 and out_lse = -inf.
+ * o_parts DEVICE fp32 [n_parts][rows][512], part p at o_parts + p*rows*512;
+ * lse_parts DEVICE fp32 [n_parts][rows] (natural log, as out_lse of
+ * mla_fa_forward_ex writes it); out DEVICE fp32 [rows][512]; out_lse DEVICE fp32
+ * [rows] or NULL. 1 <= n_parts <= MLA_COMBINE_MAX_PARTS, rows >= 1; o_parts and
+ * out 16-byte aligned, the lse arrays 4-byte aligned. out may not overlap the
+ * inputs. Runs on `stream` (NULL: the legacy default stream); no host sync. */
+#define MLA_COMBINE_MAX_PARTS 1024
+int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows,
+                   float* out, float* out_lse, void* stream);
 
 /* How the pass is divided: units = CTA pairs launched, max_splits = largest
  * number of KV splits of one (sequence, 128-row group). For tests and tools. */

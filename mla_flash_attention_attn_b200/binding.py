@@ -65,6 +65,7 @@ class mla_fa_args(ctypes.Structure):
         ("alibi_slopes", ctypes.c_void_p),
         ("softcap", ctypes.c_float),
         ("mask_gather", ctypes.c_int),
+        ("out_lse", ctypes.c_void_p),
     ]
 
 
@@ -124,6 +125,8 @@ def load(path: str = LIB_PATH):
     lib.mla_profile_begin.restype = I
     lib.mla_profile_end.argtypes = [ctypes.POINTER(mla_profile_entry), I, ctypes.POINTER(I)]
     lib.mla_profile_end.restype = I
+    lib.mla_fa_combine.argtypes = [P, P, I, ctypes.c_int64, P, P, P]
+    lib.mla_fa_combine.restype = I
     _lib = lib
     return lib
 
@@ -155,7 +158,7 @@ def _host_i32(arr):
 
 def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None,
               wv=None, out_proj=None, sinks=None, alibi_slopes=None, softcap=0.0,
-              mask_gather=False):
+              mask_gather=False, out_lse=None):
     """Fill mla_fa_args from batched torch tensors.
 
     q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
@@ -163,7 +166,8 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     wv); wv [n_head][512][128] f16 and out_proj [n_seq][n_q][n_head][128] f32 for the
     fused value up-projection; sinks / alibi_slopes fp32 [n_head] and softcap > 0 for
     the attention variants; mask_gather=True for sparse attention straight from the mask
-    (the kernel compacts it, no index list). Returns (args, keepalive)."""
+    (the kernel compacts it, no index list); out_lse fp32 [n_seq][n_q][n_head] for each
+    row's natural log-sum-exp. Returns (args, keepalive)."""
     n_seq, n_q, n_head, dk = q.shape
     if dk != DK:
         raise ValueError("q must end in 576")
@@ -190,6 +194,7 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     a.alibi_slopes = None if alibi_slopes is None else alibi_slopes.data_ptr()
     a.softcap = float(softcap)
     a.mask_gather = 1 if mask_gather else 0
+    a.out_lse = None if out_lse is None else out_lse.data_ptr()
     keep = _host_i32(kv_len)
     a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
     if idx is not None:
@@ -228,7 +233,7 @@ def mla_fa_forward(q, kcache, kv_type, mask, scale, out, stream=None):
 
 def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, idx_count=None,
             workspace=None, stream=None, sinks=None, alibi_slopes=None, softcap=0.0,
-            mask_gather=False):
+            mask_gather=False, out_lse=None):
     """Batched forward through mla_fa_forward_ex; allocates out/workspace with torch if absent."""
     import torch
 
@@ -236,7 +241,7 @@ def forward(q, kcache, kv_type, mask, scale, out=None, kv_len=None, idx=None, id
         out = torch.empty(q.shape[:3] + (DV,), dtype=torch.float32, device=q.device)
     args, keep = make_args(q, kcache, kv_type, mask, out, scale, kv_len, idx, idx_count,
                            sinks=sinks, alibi_slopes=alibi_slopes, softcap=softcap,
-                           mask_gather=mask_gather)
+                           mask_gather=mask_gather, out_lse=out_lse)
     need = mla_fa_workspace_size(args)
     if need and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -261,6 +266,29 @@ def forward_proj(q, kcache, kv_type, mask, scale, wv, out_proj=None, kv_len=None
     mla_fa_forward_ex(args, workspace if need else None, stream)
     del keep
     return out_proj
+
+
+COMBINE_MAX_PARTS = 1024  # MLA_COMBINE_MAX_PARTS
+
+
+def combine(o_parts, lse_parts, out=None, out_lse=None, stream=None):
+    """mla_fa_combine: merge partial results of the same rows over disjoint key sets.
+    o_parts fp32 [n_parts][rows][512] (or [n_parts][..][512], rows = the product of the
+    middle sizes), lse_parts fp32 [n_parts][rows] (natural log); returns out fp32
+    [rows][512] (allocated if absent); out_lse fp32 [rows] is written if given."""
+    import torch
+
+    n_parts = o_parts.shape[0]
+    o = o_parts.reshape(n_parts, -1, DV)
+    rows = o.shape[1]
+    lse = lse_parts.reshape(n_parts, rows)
+    if not (o.is_contiguous() and lse.is_contiguous()):
+        raise ValueError("o_parts and lse_parts must be contiguous")
+    if out is None:
+        out = torch.empty((rows, DV), dtype=torch.float32, device=o_parts.device)
+    _check(load().mla_fa_combine(_ptr(o), _ptr(lse), n_parts, rows, _ptr(out), _ptr(out_lse),
+                                 _stream_ptr(stream)), "mla_fa_combine")
+    return out
 
 
 def mla_compact_mask(mask_row, idx_out, count_out, stream=None):

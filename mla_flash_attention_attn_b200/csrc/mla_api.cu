@@ -104,10 +104,12 @@ enum KernelId {
   kKernCombine = 3,
   kKernCompact = 4,
   kKernWaitTest = 5,
+  kKernMerge = 6,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_fwd_gather_f16", "mla_fwd_q8_0",
-                                               "mla_combine", "mla_compact", "mla_wait_timeout"};
+                                               "mla_combine", "mla_compact", "mla_wait_timeout",
+                                               "mla_merge"};
 struct ProfRecord {
   cudaEvent_t start, stop;
   int kernel;
@@ -154,6 +156,7 @@ struct Resolved {
   int64_t q_ss, k_ss, m_ss, m_rs, o_ss, idx_ss, op_ss;
   bool proj;  // fused value up-projection: every sequence writes split partials
   bool sinks; // attention sinks: every sequence writes split partials (the combine adds them)
+  bool lse;   // per-row log-sum-exp output: every sequence writes partials (the combine writes it)
 };
 
 int validate(const mla_fa_args* a, Resolved* r) {
@@ -167,7 +170,9 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (a->mask_gather != 0 && a->mask_gather != 1) return MLA_ERR_SHAPE;
   if (a->mask_gather && a->mask == nullptr) return MLA_ERR_NULL;
   if (a->mask_gather && (a->idx != nullptr || a->alibi_slopes != nullptr)) return MLA_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(a->sinks) & 3) || (reinterpret_cast<uintptr_t>(a->alibi_slopes) & 3))
+  if (a->out_lse != nullptr && (a->sinks != nullptr || proj)) return MLA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(a->sinks) & 3) || (reinterpret_cast<uintptr_t>(a->alibi_slopes) & 3) ||
+      (reinterpret_cast<uintptr_t>(a->out_lse) & 3))
     return MLA_ERR_ALIGN;
   if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
   if (a->n_seq < 1 || a->n_q < 1 || a->n_head < 1 || a->n_head > MLA_MAX_HEADS || a->n_kv < 1)
@@ -192,6 +197,7 @@ int validate(const mla_fa_args* a, Resolved* r) {
   r->idx_ss = a->idx_seq_stride ? a->idx_seq_stride : a->n_kv;
   r->proj = proj;
   r->sinks = a->sinks != nullptr;
+  r->lse = a->out_lse != nullptr;
   r->op_ss = proj ? (a->out_proj_seq_stride ? a->out_proj_seq_stride : rows * MLA_PROJ_DIM) : 0;
   if (proj && (a->out_proj_seq_stride < 0 || r->op_ss < rows * MLA_PROJ_DIM)) return MLA_ERR_SHAPE;
   if (proj && (!aligned16(a->wv) || !aligned16(a->out_proj) || (r->op_ss % 4) != 0))
@@ -251,7 +257,7 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
     plan->n_split[b] = ns;
     plan->unit_base[b] = units;
     units += plan->groups * ns;
-    if (ns > 1 || r.proj || r.sinks) {
+    if (ns > 1 || r.proj || r.sinks || r.lse) {
       plan->ws_base[b] = slots;
       slots += plan->groups * ns;
     } else {
@@ -523,10 +529,10 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
                                   a.out_proj, (int64_t)r.op_ss, a.sinks);
         else if (wide)
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const uint16_t*)p.ws_o,
-                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks);
+                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks, a.out_lse);
         else
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const uint16_t*)p.ws_o,
-                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks);
+                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks, a.out_lse);
       }
       if (ce != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }
@@ -709,6 +715,26 @@ int mla_compact_mask_ex(const void* mask, int n_rows, int64_t mask_row_stride, i
     mla::mla_compact_kernel<<<grid, mla::compact::kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint16_t*>(mask), mask_row_stride, n_kv, idx_out, idx_row_stride,
         count_out, tickets, flags, epoch, kDefaultTimeoutNs);
+  }
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows,
+                   float* out, float* out_lse, void* stream) {
+  if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return MLA_ERR_NULL;
+  if (n_parts < 1 || n_parts > MLA_COMBINE_MAX_PARTS || rows < 1) return MLA_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(o_parts) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
+      (reinterpret_cast<uintptr_t>(lse_parts) & 3) || (reinterpret_cast<uintptr_t>(out_lse) & 3))
+    return MLA_ERR_ALIGN;
+  DeviceState* st = nullptr;
+  int rc = current_device(&st);
+  if (rc != MLA_OK) return rc;
+  const unsigned grid = (unsigned)std::min<int64_t>(rows, (int64_t)1 << 30);
+  {
+    ProfScope prof(kKernMerge, static_cast<cudaStream_t>(stream));
+    mla::mla_merge_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(o_parts, lse_parts, n_parts,
+                                                                               rows, out, out_lse);
   }
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;

@@ -13,6 +13,7 @@ constexpr int kTileKeys = 256;       // N of one Q.K^T MMA: keys per tile
 constexpr int kPlanMaxSeq = 128;     // sequences per launch (larger batches are chunked)
 constexpr int kQ8RowBytes = 612;     // q8_0: 18 blocks of {f16 d; int8 q[32]}
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // Status codes written by kernels (same values as mla_status in mla_fa.h).
 constexpr int kStatusLaunch = -6;   // launched with less dynamic shared memory than it needs

@@ -1125,7 +1125,8 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
                                                           const float* __restrict__ ws_lse,
                                                           float* __restrict__ out,
                                                           int64_t out_seq_stride,
-                                                          const float* __restrict__ sinks) {
+                                                          const float* __restrict__ sinks,
+                                                          float* __restrict__ out_lse) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.y;
   const int row = blockIdx.x;
@@ -1151,9 +1152,10 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   const float snk = sinks != nullptr ? __ldg(sinks + row % plan.n_head) * kLog2e : -INFINITY;
   mx = fmaxf(mx, snk);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float wsum = 0.f;
   if (mx != -INFINITY) {
     const float wl = lse_l == -INFINITY ? 0.f : ex2_approx(lse_l - mx);
-    float wsum = wl;
+    wsum = wl;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     if (snk != -INFINITY) wsum += ex2_approx(snk - mx);
@@ -1180,6 +1182,10 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
   float4* dst = reinterpret_cast<float4*>(out + (int64_t)(plan.seq_offset + b) * out_seq_stride +
                                           (int64_t)row * kDV);
   dst[threadIdx.x] = acc;
+  // the row's natural log-sum-exp (mx and wsum are in log2 units)
+  if (out_lse != nullptr && threadIdx.x == 0)
+    out_lse[(int64_t)(plan.seq_offset + b) * plan.rows + row] =
+        mx == -INFINITY ? -INFINITY : (mx + log2f(wsum)) * kLn2;
 }
 
 // The same combine for rows with many splits: one CTA of 4 warps per (query row,
@@ -1194,7 +1200,8 @@ constexpr int kCombPer = 24;  // partial rows per warp held in registers
 __global__ void __launch_bounds__(128)
     mla_combine_wide_kernel(const __grid_constant__ Plan plan, const uint16_t* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, float* __restrict__ out,
-                            int64_t out_seq_stride, const float* __restrict__ sinks) {
+                            int64_t out_seq_stride, const float* __restrict__ sinks,
+                            float* __restrict__ out_lse) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 red[4][32];
   const int b = blockIdx.z;
@@ -1284,6 +1291,45 @@ __global__ void __launch_bounds__(128)
     float4* dst = reinterpret_cast<float4*>(out + (int64_t)(plan.seq_offset + b) * out_seq_stride +
                                             (int64_t)row * kDV) + qtr * 32 + lane;
     *dst = t;
+    // the row's natural log-sum-exp (mx and wsum are in log2 units)
+    if (out_lse != nullptr && qtr == 0 && lane == 0)
+      out_lse[(int64_t)(plan.seq_offset + b) * plan.rows + row] =
+          mx == -INFINITY ? -INFINITY : (mx + log2f(wsum)) * kLn2;
+  }
+}
+
+// Merge of n_parts partial results of the same rows over disjoint key sets
+// (mla_fa_combine): the log-sum-exp combine across calls, with natural-log lse.
+// One CTA of 128 threads per row (grid-stride over the rows), thread i owning value
+// columns 4i..4i+3; every thread reads the parts' lse (the same addresses across the
+// CTA), then sums the weighted parts.
+__global__ void __launch_bounds__(128)
+    mla_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts,
+                     int n_parts, int64_t rows, float* __restrict__ out, float* __restrict__ out_lse) {
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    float mx = -INFINITY;
+    for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, __ldg(lse_parts + (int64_t)p * rows + r));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll 4
+      for (int p = 0; p < n_parts; ++p) {
+        const float l = __ldg(lse_parts + (int64_t)p * rows + r);
+        const float w = l == -INFINITY ? 0.f : ex2_approx((l - mx) * kLog2e);
+        if (w == 0.f) continue;  // the same in every thread of the CTA
+        const float4 x =
+            __ldg(reinterpret_cast<const float4*>(o_parts + ((int64_t)p * rows + r) * kDV) + threadIdx.x);
+        acc.x = fmaf(w, x.x, acc.x);
+        acc.y = fmaf(w, x.y, acc.y);
+        acc.z = fmaf(w, x.z, acc.z);
+        acc.w = fmaf(w, x.w, acc.w);
+        wsum += w;
+      }
+      const float inv = 1.f / wsum;
+      acc.x *= inv; acc.y *= inv; acc.z *= inv; acc.w *= inv;
+    }
+    reinterpret_cast<float4*>(out + r * kDV)[threadIdx.x] = acc;
+    if (out_lse != nullptr && threadIdx.x == 0) out_lse[r] = mx == -INFINITY ? -INFINITY : mx + logf(wsum);
   }
 }
 

@@ -99,6 +99,10 @@ def call_ex(lib, a):
     (dict(softcap=-1.0), -2), (dict(softcap=float("nan")), -2), (dict(softcap=float("inf")), -2),
     (dict(alibi_slopes=FAKE, idx=FAKE, idx_count=FAKE), -8),
     (dict(sinks=FAKE + 2), -4), (dict(alibi_slopes=FAKE + 1), -4),
+    # per-row lse: excludes sinks and the projection; 4-byte aligned
+    (dict(out_lse=FAKE, sinks=FAKE), -8),
+    (dict(out_lse=FAKE, wv=FAKE, proj_dim=128, out_proj=FAKE), -8),
+    (dict(out_lse=FAKE + 2), -4),
     # mask gather: needs the mask, excludes an index list and ALiBi
     (dict(mask_gather=2, mask=FAKE), -2), (dict(mask_gather=1), -1),
     (dict(mask_gather=1, mask=FAKE, idx=FAKE, idx_count=FAKE), -8),
@@ -146,6 +150,20 @@ def test_compaction_argument_errors(lib):
     assert lib.mla_compact_workspace_size(1, 131072) == 256 + 8 * 8
     assert lib.mla_compact_workspace_size(3, 16385) == 256 + 3 * 2 * 8
     assert lib.mla_compact_workspace_size(0, 10) == 0
+
+
+def test_combine_argument_errors(lib):
+    f = lib.mla_fa_combine
+    assert f(None, FAKE, 2, 10, FAKE, None, None) == -1
+    assert f(FAKE, None, 2, 10, FAKE, None, None) == -1
+    assert f(FAKE, FAKE, 2, 10, None, None, None) == -1
+    assert f(FAKE, FAKE, 0, 10, FAKE, None, None) == -2
+    assert f(FAKE, FAKE, binding.COMBINE_MAX_PARTS + 1, 10, FAKE, None, None) == -2
+    assert f(FAKE, FAKE, 2, 0, FAKE, None, None) == -2
+    assert f(FAKE + 4, FAKE, 2, 10, FAKE, None, None) == -4
+    assert f(FAKE, FAKE, 2, 10, FAKE + 8, None, None) == -4
+    assert f(FAKE, FAKE + 2, 2, 10, FAKE, None, None) == -4
+    assert f(FAKE, FAKE, 2, 10, FAKE, FAKE + 1, None) == -4
 
 
 def test_valid_arguments_reach_the_device_check(lib):

@@ -650,3 +650,134 @@ def test_softcap_q8_0_dense():
     got = run_gpu(w, softcap=6.0)
     check_variants(w, got, "softcap q8_0", softcap=6.0, kcache=q8_f16_rounded(w.kcache[0]),
                    kv_type=oracle.KV_F16)
+
+
+# ---- per-row log-sum-exp and the merge across calls (split-KV across devices) ----------
+# Tolerance of the lse: 2e-3 absolute. A merge weighs a part by e^{lse}, so an lse error
+# d changes that part's relative weight by about d; 2e-3 keeps merged rows inside the
+# rel-L2 2e-3 budget of the attention output.
+LSE_ATOL = 2e-3
+
+
+def run_gpu_lse(w, idx=None, idx_count=None, mask_gather=False):
+    torch = torch_mod()
+    dev = torch.device("cuda")
+    q = torch.from_numpy(w.q).to(dev)
+    k = torch.from_numpy(w.kcache).to(dev)
+    m = torch.from_numpy(w.mask).to(dev) if w.mask is not None else None
+    rows = w.n_seq * w.n_q * w.n_head
+    out = torch.full((w.n_seq, w.n_q, w.n_head, 512), float("nan"), device=dev)
+    big = torch.full((rows + CANARY,), float("nan"), device=dev)
+    lse = big[:rows].view(w.n_seq, w.n_q, w.n_head)
+    binding.forward(q, k, w.kv_type, m, w.scale, out=out, kv_len=w.kv_len, idx=idx,
+                    idx_count=idx_count, out_lse=lse, mask_gather=mask_gather)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    assert bool(torch.isnan(big[rows:]).all()), "write past the end of out_lse"
+    return out.cpu().numpy(), lse.cpu().numpy()
+
+
+def assert_lse(got, ref, what):
+    got = np.asarray(got, np.float64).ravel()
+    ref = np.asarray(ref, np.float64).ravel()
+    assert np.array_equal(np.isneginf(got), np.isneginf(ref)), f"{what}: -inf rows differ"
+    fin = np.isfinite(ref)
+    assert np.all(np.isfinite(got[fin])), f"{what}: non-finite lse"
+    err = float(np.max(np.abs(got[fin] - ref[fin]))) if fin.any() else 0.0
+    assert err <= LSE_ATOL, f"{what}: lse max-abs {err:.3g}"
+
+
+@pytest.mark.parametrize("case", ["v3_split", "tiny_unsplit", "prefill_rows", "empty_and_masked"])
+def test_out_lse_matches_oracle(case):
+    if case == "v3_split":
+        w = W.make("v3_batched_decode", n_kv=2048, len_lo=100, len_hi=2048)
+    elif case == "tiny_unsplit":
+        w = W.make("tiny_decode", n_kv=300)
+    elif case == "prefill_rows":
+        w = W.make("prefill_chunk", n_q=3, n_head=100, n_kv=700)
+    else:
+        w = W.make("v3_batched_decode", n_seq=3, n_head=16, n_kv=600, len_lo=600, len_hi=600)
+        w.kv_len[:] = [600, 0, 350]
+        w.mask[2] = np.float16(-np.inf)
+    got, lse = run_gpu_lse(w)
+    for b in range(w.n_seq):
+        n = int(w.kv_len[b])
+        if n == 0:
+            assert np.all(got[b] == 0) and np.all(np.isneginf(lse[b]))
+            continue
+        o_ref, l_ref = oracle.attention_lse(w.q[b], w.kcache[b][:n], w.kv_type,
+                                            None if w.mask is None else w.mask[b][:, :n], w.scale)
+        assert_parity(got[b].reshape(-1, 512), o_ref, f"{case} out seq {b}")
+        assert_lse(lse[b], l_ref, f"{case} lse seq {b}")
+
+
+def test_out_lse_sparse_q8_and_mask_gather():
+    torch = torch_mod()
+    w = W.make("sparse_q8_decode", n_kv=16384, n_head=128, tail_blocks=4)
+    ref_idx = oracle.compact(w.mask[0, 0])
+    kf16 = q8_f16_rounded(w.kcache[0])
+    o_ref, l_ref = oracle.attention_lse(w.q[0], kf16, oracle.KV_F16, w.mask[0], w.scale)
+    idx = torch.full((1, w.n_kv), -1, dtype=torch.int32, device="cuda")
+    idx[0, : len(ref_idx)] = torch.from_numpy(ref_idx).cuda()
+    cnt = torch.tensor([len(ref_idx)], dtype=torch.int32, device="cuda")
+    for what, kw in (("index list", dict(idx=idx, idx_count=cnt)), ("mask gather", dict(mask_gather=True))):
+        got, lse = run_gpu_lse(w, **kw)
+        assert_parity(got[0].reshape(-1, 512), o_ref, f"q8_0 {what} out")
+        assert_lse(lse[0], l_ref, f"q8_0 {what} lse")
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_split_kv_decode_emulated_on_one_gpu(world):
+    # the ranks' calls of a split-KV decode, made one after another on one GPU: each
+    # attends over its range of the cache with the lse, mla_fa_combine merges them
+    torch = torch_mod()
+    from mla_flash_attention_attn_b200 import split_kv
+
+    w = W.make("v3_batched_decode", n_kv=4096, len_lo=100, len_hi=4096)
+    dev = torch.device("cuda")
+    q = torch.from_numpy(w.q).to(dev)
+    rows = w.n_seq * w.n_q * w.n_head
+    o_all = torch.empty((world, rows, 512), device=dev)
+    lse_all = torch.empty((world, rows), device=dev)
+    for r, (lo, hi) in enumerate(split_kv.shard_bounds(w.n_kv, world)):
+        k = torch.from_numpy(w.kcache[:, lo:hi].copy()).to(dev)
+        m = torch.from_numpy(w.mask[:, :, lo:hi].copy()).to(dev)
+        binding.forward(q, k, w.kv_type, m, w.scale, out=o_all[r].view(w.n_seq, 1, w.n_head, 512),
+                        kv_len=split_kv.shard_lengths(w.kv_len, lo, hi),
+                        out_lse=lse_all[r].view(w.n_seq, 1, w.n_head))
+    lse_out = torch.empty((rows,), device=dev)
+    out = binding.combine(o_all, lse_all, out_lse=lse_out)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    got = out.cpu().numpy().reshape(w.n_seq, -1, 512)
+    lse = lse_out.cpu().numpy().reshape(w.n_seq, -1)
+    for b in range(w.n_seq):
+        n = int(w.kv_len[b])
+        o_ref, l_ref = oracle.attention_lse(w.q[b], w.kcache[b][:n], w.kv_type, w.mask[b][:, :n], w.scale)
+        assert_parity(got[b], o_ref, f"split-KV x{world} seq {b}")
+        assert_lse(lse[b], l_ref, f"split-KV x{world} lse seq {b}")
+
+
+@pytest.mark.parametrize("n_parts,rows", [(1, 5), (2, 1), (5, 1000), (33, 77)])
+def test_combine_entry_point_matches_oracle(n_parts, rows):
+    torch = torch_mod()
+    rng = np.random.default_rng(n_parts * 1000 + rows)
+    o = rng.standard_normal((n_parts, rows, 512)).astype(np.float32)
+    lse = (rng.standard_normal((n_parts, rows)) * 20).astype(np.float32)
+    lse[rng.random((n_parts, rows)) < 0.2] = -np.inf
+    lse[:, 0] = -np.inf  # a row with no kept key in any part
+    o_ref, l_ref = oracle.combine(o, lse)
+    big = torch.full((rows * 512 + CANARY,), float("nan"), device="cuda")
+    out = big[: rows * 512].view(rows, 512)
+    lse_out = torch.empty((rows,), device="cuda")
+    binding.combine(torch.from_numpy(o).cuda(), torch.from_numpy(lse).cuda(), out=out, out_lse=lse_out)
+    torch.cuda.synchronize()
+    assert bool(torch.isnan(big[rows * 512:]).all())
+    got = out.cpu().numpy()
+    assert np.all(got[0] == 0)
+    # fp32 arithmetic on fp32 inputs: a few ulp of the largest term
+    np.testing.assert_allclose(got, o_ref, rtol=1e-5, atol=2e-5)
+    lg = lse_out.cpu().numpy()
+    assert np.array_equal(np.isneginf(lg), np.isneginf(l_ref))
+    fin = np.isfinite(l_ref)
+    np.testing.assert_allclose(lg[fin], l_ref[fin], rtol=0, atol=1e-4)
