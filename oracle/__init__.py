@@ -73,6 +73,8 @@ def _load():
         lib.oracle_attention.restype = I
         lib.oracle_attention_lse.argtypes = common + [P, P]
         lib.oracle_attention_lse.restype = I
+        lib.oracle_attention_dk.argtypes = [P, P, P, P, L, I, I, L, I, D, P, L, P, P]
+        lib.oracle_attention_dk.restype = I
         lib.oracle_attention_online.argtypes = common + [L, P]
         lib.oracle_attention_online.restype = I
         lib.oracle_attention_split.argtypes = common + [P, I, P]
@@ -119,13 +121,15 @@ def half_to_double(bits: int) -> float:
 
 def _prep(q, kcache, kv_type, mask, idx, rows):
     q = _bits16(q)
-    if q.ndim != 3 or q.shape[2] != DK:
-        raise ValueError("q must be [n_q][n_head][576]")
-    n_q, n_head, _ = q.shape
+    if q.ndim != 3 or q.shape[2] not in (DK, DV):
+        raise ValueError("q must be [n_q][n_head][576] (or [..][512], f16 cache)")
+    n_q, n_head, dk = q.shape
+    if dk != DK and kv_type != KV_F16:
+        raise ValueError("the 512-wide head shape takes an f16 cache")
     if kv_type == KV_F16:
         kc = _bits16(kcache)
-        if kc.ndim != 2 or kc.shape[1] != DK:
-            raise ValueError("f16 kcache must be [n_kv][576]")
+        if kc.ndim != 2 or kc.shape[1] != dk:
+            raise ValueError("f16 kcache must be [n_kv][dk], dk as q's")
     elif kv_type == KV_Q8_0:
         kc = np.ascontiguousarray(kcache, dtype=np.uint8)
         if kc.ndim != 2 or kc.shape[1] != Q8_ROW_BYTES:
@@ -148,11 +152,20 @@ def _prep(q, kcache, kv_type, mask, idx, rows):
 def attention(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None, idx=None):
     """Two-pass fp64 softmax(scale*Q.K^T + mask).V with V = K[:, :512].
 
-    q: f16 [n_q][n_head][576]; kcache: f16 [n_kv][576] or q8_0 bytes [n_kv][612];
+    q: f16 [n_q][n_head][576]; kcache: f16 [n_kv][576] or q8_0 bytes [n_kv][612]
+    (or q [..][512] with an f16 kcache [n_kv][512]: the DK = DV = 512 head shape);
     mask: f16 [n_q][n_kv] or None; idx: optional int32 kept rows (sparse);
     rows: optional row ids t*n_head+h to compute. Returns float64 [rows][512].
     """
     q, kc, m, ix, rw, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, rows)
+    if q.shape[2] != DK:  # the DK = DV = 512 head shape
+        rc = _load().oracle_attention_dk(_ptr(q), _ptr(kc), _ptr(m), _ptr(ix),
+                                         0 if ix is None else len(ix), n_q, n_head, n_kv,
+                                         q.shape[2], float(scale), _ptr(rw),
+                                         0 if rw is None else len(rw), _ptr(out), None)
+        if rc != 0:
+            raise ValueError("oracle_attention_dk rejected its arguments")
+        return out
     rc = _load().oracle_attention(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
                                   0 if ix is None else len(ix), n_q, n_head, n_kv, float(scale),
                                   _ptr(rw), 0 if rw is None else len(rw), _ptr(out))
@@ -167,6 +180,14 @@ def attention_lse(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, rows=None, id
     Returns (float64 [rows][512], float64 [rows])."""
     q, kc, m, ix, rw, n_q, n_head, n_kv, out = _prep(q, kcache, kv_type, mask, idx, rows)
     lse = np.zeros(out.shape[0], dtype=np.float64)
+    if q.shape[2] != DK:  # the DK = DV = 512 head shape
+        rc = _load().oracle_attention_dk(_ptr(q), _ptr(kc), _ptr(m), _ptr(ix),
+                                         0 if ix is None else len(ix), n_q, n_head, n_kv,
+                                         q.shape[2], float(scale), _ptr(rw),
+                                         0 if rw is None else len(rw), _ptr(out), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle_attention_dk rejected its arguments")
+        return out, lse
     rc = _load().oracle_attention_lse(_ptr(q), _ptr(kc), kv_type, _ptr(m), _ptr(ix),
                                       0 if ix is None else len(ix), n_q, n_head, n_kv, float(scale),
                                       _ptr(rw), 0 if rw is None else len(rw), _ptr(out), _ptr(lse))

@@ -41,6 +41,11 @@
  *  - q8_0 row = 18 blocks of {f16 d; int8 q[32]} (34 bytes), 612 bytes per
  *    row; value = d * q, exact in double.
  *
+ * Head width: the cache row and the query are dk wide, 576 above; the
+ * DK = DV = 512 shape (one of the head shapes the llama.cpp tag page lists for the
+ * Metal FA kernel, PR #29570) takes dk = 512 with the same V = first 512 columns,
+ * i.e. the whole row (oracle_attention_dk, f16 cache only).
+ *
  * Everything is fp64: each f16 input is converted exactly to double
  * (-inf stays -inf, exp(-inf) = 0); results are returned as double and
  * rounded to fp32 once by the caller.
@@ -107,11 +112,11 @@ double oracle_half_to_double(uint16_t h) {
   return g_half[h];
 }
 
-/* Value of column c of cache row `key`. */
-static inline double kval(const void* kc, int kv_type, long key, int c) {
+/* Value of column c of cache row `key` (f16 rows are dk wide). */
+static inline double kval_w(const void* kc, int kv_type, long key, int c, int dk) {
   if (kv_type == ORC_KV_F16) {
     const uint16_t* k = (const uint16_t*)kc;
-    return g_half[k[key * ORC_DK + c]];
+    return g_half[k[key * dk + c]];
   } else {
     const uint8_t* row = (const uint8_t*)kc + key * ORC_Q8_ROW_BYTES;
     const uint8_t* blk = row + (c / ORC_Q8_BLOCK) * ORC_Q8_BLOCK_BYTES;
@@ -121,6 +126,9 @@ static inline double kval(const void* kc, int kv_type, long key, int c) {
     return g_half[dbits] * (double)qv;
   }
 }
+static inline double kval(const void* kc, int kv_type, long key, int c) {
+  return kval_w(kc, kv_type, key, c, ORC_DK);
+}
 
 void oracle_dequant_q8_0(const uint8_t* rows, long n_rows, double* out) {
   oracle_init();
@@ -129,13 +137,17 @@ void oracle_dequant_q8_0(const uint8_t* rows, long n_rows, double* out) {
 }
 
 /* Score of key `key` for query row q (576 doubles). */
-static inline double score(const double* q, const void* kc, int kv_type, long key,
-                           const uint16_t* mrow, double scale) {
+static inline double score_w(const double* q, const void* kc, int kv_type, long key,
+                             const uint16_t* mrow, double scale, int dk) {
   double dot = 0.0;
-  for (int c = 0; c < ORC_DK; ++c) dot += q[c] * kval(kc, kv_type, key, c);
+  for (int c = 0; c < dk; ++c) dot += q[c] * kval_w(kc, kv_type, key, c, dk);
   double s = scale * dot;
   if (mrow) s += g_half[mrow[key]];
   return s;
+}
+static inline double score(const double* q, const void* kc, int kv_type, long key,
+                           const uint16_t* mrow, double scale) {
+  return score_w(q, kc, kv_type, key, mrow, scale, ORC_DK);
 }
 
 /* Selected keys: all of 0..n_kv-1 when idx == NULL, else idx[0..n_sel). */
@@ -146,10 +158,10 @@ static inline long key_at(const int32_t* idx, long i) { return idx ? (long)idx[i
  * masked). */
 static void attend_two_pass(const double* q, const void* kc, int kv_type, const uint16_t* mrow,
                             const int32_t* idx, long n_sel, double scale, double* s,
-                            double* out, double* lse) {
+                            double* out, double* lse, int dk) {
   double M = -INFINITY;
   for (long i = 0; i < n_sel; ++i) {
-    s[i] = score(q, kc, kv_type, key_at(idx, i), mrow, scale);
+    s[i] = score_w(q, kc, kv_type, key_at(idx, i), mrow, scale, dk);
     if (s[i] > M) M = s[i];
   }
   for (int d = 0; d < ORC_DV; ++d) out[d] = 0.0;
@@ -161,7 +173,7 @@ static void attend_two_pass(const double* q, const void* kc, int kv_type, const 
     L += p;
     if (p == 0.0) continue;
     long key = key_at(idx, i);
-    for (int d = 0; d < ORC_DV; ++d) out[d] += p * kval(kc, kv_type, key, d);
+    for (int d = 0; d < ORC_DV; ++d) out[d] += p * kval_w(kc, kv_type, key, d, dk);
   }
   for (int d = 0; d < ORC_DV; ++d) out[d] /= L;
   if (lse) *lse = M + log(L);
@@ -262,9 +274,10 @@ enum { MODE_TWO_PASS = 0, MODE_ONLINE = 1, MODE_SPLIT = 2 };
 static int run(int mode, const uint16_t* q, const void* kcache, int kv_type, const uint16_t* mask,
                const int32_t* idx, long n_idx, int n_q, int n_head, long n_kv, double scale,
                const int32_t* rows, long n_rows, long tile, const int32_t* bounds, int n_split,
-               double* out, double* lse) {
+               double* out, double* lse, int dk) {
   if (!q || !kcache || !out || n_q < 1 || n_head < 1 || n_kv < 1) return -1;
   if (kv_type != ORC_KV_F16 && kv_type != ORC_KV_Q8_0) return -1;
+  if (dk != ORC_DK && (dk != ORC_DV || kv_type != ORC_KV_F16 || mode != MODE_TWO_PASS)) return -1;
   if (idx) {
     for (long i = 0; i < n_idx; ++i)
       if (idx[i] < 0 || idx[i] >= n_kv) return -1;
@@ -285,12 +298,12 @@ static int run(int mode, const uint16_t* q, const void* kcache, int kv_type, con
         continue;
       }
       long t = row / n_head;
-      const uint16_t* qrow = q + row * ORC_DK;
-      for (int c = 0; c < ORC_DK; ++c) qd[c] = g_half[qrow[c]];
+      const uint16_t* qrow = q + row * dk;
+      for (int c = 0; c < dk; ++c) qd[c] = g_half[qrow[c]];
       const uint16_t* mrow = mask ? mask + t * n_kv : NULL;
       double* o = out + r * ORC_DV;
       if (mode == MODE_TWO_PASS)
-        attend_two_pass(qd, kcache, kv_type, mrow, idx, n_sel, scale, s, o, lse ? lse + r : NULL);
+        attend_two_pass(qd, kcache, kv_type, mrow, idx, n_sel, scale, s, o, lse ? lse + r : NULL, dk);
       else if (mode == MODE_ONLINE)
         attend_online(qd, kcache, kv_type, mrow, idx, n_sel, scale, tile, s, o);
       else
@@ -305,7 +318,17 @@ int oracle_attention(const uint16_t* q, const void* kcache, int kv_type, const u
                      const int32_t* idx, long n_idx, int n_q, int n_head, long n_kv, double scale,
                      const int32_t* rows, long n_rows, double* out) {
   return run(MODE_TWO_PASS, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, 0, NULL, 0, out, NULL);
+             n_rows, 0, NULL, 0, out, NULL, ORC_DK);
+}
+
+/* Two-pass attention with the head width dk (576, or 512 for the DK = DV = 512
+ * shape, f16 cache only): q [n_q][n_head][dk], kcache [n_kv][dk], V = the first 512
+ * columns. lse may be NULL. */
+int oracle_attention_dk(const uint16_t* q, const void* kcache, const uint16_t* mask,
+                        const int32_t* idx, long n_idx, int n_q, int n_head, long n_kv, int dk,
+                        double scale, const int32_t* rows, long n_rows, double* out, double* lse) {
+  return run(MODE_TWO_PASS, q, kcache, ORC_KV_F16, mask, idx, n_idx, n_q, n_head, n_kv, scale,
+             rows, n_rows, 0, NULL, 0, out, lse, dk);
 }
 
 /* oracle_attention plus each row's natural log-sum-exp of its scores. */
@@ -315,7 +338,7 @@ int oracle_attention_lse(const uint16_t* q, const void* kcache, int kv_type, con
                          double* lse) {
   if (!lse) return -1;
   return run(MODE_TWO_PASS, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, 0, NULL, 0, out, lse);
+             n_rows, 0, NULL, 0, out, lse, ORC_DK);
 }
 
 int oracle_attention_online(const uint16_t* q, const void* kcache, int kv_type,
@@ -324,7 +347,7 @@ int oracle_attention_online(const uint16_t* q, const void* kcache, int kv_type,
                             long tile, double* out) {
   if (tile < 1) return -1;
   return run(MODE_ONLINE, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, tile, NULL, 0, out, NULL);
+             n_rows, tile, NULL, 0, out, NULL, ORC_DK);
 }
 
 int oracle_attention_split(const uint16_t* q, const void* kcache, int kv_type,
@@ -336,7 +359,7 @@ int oracle_attention_split(const uint16_t* q, const void* kcache, int kv_type,
   for (int i = 0; i < n_split; ++i)
     if (bounds[i + 1] < bounds[i]) return -1;
   return run(MODE_SPLIT, q, kcache, kv_type, mask, idx, n_idx, n_q, n_head, n_kv, scale, rows,
-             n_rows, 0, bounds, n_split, out, NULL);
+             n_rows, 0, bounds, n_split, out, NULL, ORC_DK);
 }
 
 /* Keep rule: a cell is kept iff its f16 bits are not -inf (0xFC00).

@@ -602,3 +602,38 @@ def test_combine_closed_forms():
     np.testing.assert_array_equal(oo, o[0])
     oo, ll = oracle.combine(o, np.full((2, 5), -np.inf))
     assert np.all(oo == 0) and np.all(np.isneginf(ll))
+
+
+# ---- the DK = DV = 512 head shape (V = the whole 512-wide row) ---------------------------
+
+def test_dk512_matches_brute_force():
+    rng = np.random.default_rng(50)
+    q = rand_f16(rng, (3, 2, 512))
+    k = rand_f16(rng, (37, 512))
+    mask = rand_f16(rng, (3, 37))
+    mask[1, ::3] = NEG
+    got = oracle.attention(q, k, mask=mask, scale=0.05)
+    np.testing.assert_allclose(got, brute_force(q, k, mask, 0.05), rtol=1e-12, atol=1e-13)
+
+
+def test_dk512_single_key_gives_the_row():
+    rng = np.random.default_rng(51)
+    q = rand_f16(rng, (1, 4, 512))
+    k = rand_f16(rng, (1, 512))
+    got = oracle.attention(q, k, scale=0.3)
+    np.testing.assert_array_equal(got, np.repeat(k.astype(np.float64), 4, axis=0))
+
+
+def test_dk512_equals_dk576_with_zero_rope_columns_exactly():
+    # 64 zero columns appended to q and to every cache row add exact zeros to each
+    # score and leave V (the first 512 columns) as it is
+    rng = np.random.default_rng(52)
+    q = rand_f16(rng, (2, 3, 512))
+    k = rand_f16(rng, (90, 512))
+    mask = rand_f16(rng, (2, 90))
+    mask[0, 40:] = NEG
+    pad = lambda x: np.concatenate([x, np.zeros(x.shape[:-1] + (64,), np.float16)], axis=-1)
+    o512, l512 = oracle.attention_lse(q, k, mask=mask, scale=0.07)
+    o576, l576 = oracle.attention_lse(pad(q), pad(k), mask=mask, scale=0.07)
+    np.testing.assert_array_equal(o512, o576)
+    np.testing.assert_array_equal(l512, l576)
