@@ -74,9 +74,10 @@ typedef enum {
 
 /* Full argument set of the batched / sparse forward pass.
  *
- * q       f16, element (b, t, h, c) at q[b*q_seq_stride + (t*n_head + h)*576 + c]
+ * q       f16, element (b, t, h, c) at q[b*q_seq_stride + (t*n_head + h)*dk + c], dk the
+ *         head width (576, or 512 with head_dim = 512)
  * kcache  row (b, j) at byte offset (b*k_seq_stride + j) * row_bytes, where
- *         row_bytes = 1152 (MLA_KV_F16) or 612 (MLA_KV_Q8_0)
+ *         row_bytes = 2*dk (MLA_KV_F16: 1152, or 1024) or 612 (MLA_KV_Q8_0)
  * mask    f16 or NULL, element (b, t, j) at mask[b*mask_seq_stride + t*mask_row_stride + j];
  *         0 keeps a cell, -inf drops it, any finite value is added to the score;
  *         shared by all heads of a token
@@ -124,6 +125,12 @@ typedef enum {
  *         disjoint key ranges (a cache split across devices, say) merge exactly with
  *         mla_fa_combine. Every sequence then writes partials. Excludes sinks and wv
  *         (MLA_ERR_UNSUPPORTED); 4-byte aligned
+ * head_dim 0 or MLA_DK (576): the latent + RoPE row above. MLA_DV (512): the DK = DV =
+ *         512 head shape (one of the head shapes the llama.cpp tag page lists for the
+ *         Metal FA kernel, PR #29570): q and the cache rows are 512 wide and V is the
+ *         whole row. f16 cache only (else MLA_ERR_UNSUPPORTED); dense or index-list
+ *         attention, with sinks, out_lse and wv as above; softcap, ALiBi and mask_gather
+ *         MLA_ERR_UNSUPPORTED. Other values MLA_ERR_SHAPE
  * A stride of 0 means "dense" (the natural value for the given sizes).
  */
 typedef struct mla_fa_args {
@@ -137,7 +144,7 @@ typedef struct mla_fa_args {
   int n_head;
   int n_kv;
   float scale;
-  int64_t q_seq_stride;     /* elements; 0 = n_q*n_head*576                    */
+  int64_t q_seq_stride;     /* elements; 0 = n_q*n_head*dk                     */
   int64_t k_seq_stride;     /* rows;     0 = n_kv                              */
   int64_t mask_seq_stride;  /* elements; 0 = n_q*mask_row_stride               */
   int64_t mask_row_stride;  /* elements; 0 = n_kv                              */
@@ -155,6 +162,7 @@ typedef struct mla_fa_args {
   float softcap;            /* > 0 enables the logit softcap                   */
   int mask_gather;          /* 1: gather the mask's kept cells (no idx)        */
   float* out_lse;           /* DEVICE, optional: natural log-sum-exp per row   */
+  int head_dim;             /* 0 / MLA_DK: 576-wide heads; MLA_DV: 512         */
 } mla_fa_args;
 
 /* Forward pass with the sizes of the single-sequence call:

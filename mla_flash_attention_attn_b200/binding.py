@@ -66,6 +66,7 @@ class mla_fa_args(ctypes.Structure):
         ("softcap", ctypes.c_float),
         ("mask_gather", ctypes.c_int),
         ("out_lse", ctypes.c_void_p),
+        ("head_dim", ctypes.c_int),
     ]
 
 
@@ -162,6 +163,7 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     """Fill mla_fa_args from batched torch tensors.
 
     q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
+    q [..][512] with kcache [..][512] f16 selects the DK = DV = 512 head shape;
     mask [n_seq][n_q][n_kv] f16 or None; out [n_seq][n_q][n_head][512] f32 (or None with
     wv); wv [n_head][512][128] f16 and out_proj [n_seq][n_q][n_head][128] f32 for the
     fused value up-projection; sinks / alibi_slopes fp32 [n_head] and softcap > 0 for
@@ -169,8 +171,8 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     (the kernel compacts it, no index list); out_lse fp32 [n_seq][n_q][n_head] for each
     row's natural log-sum-exp. Returns (args, keepalive)."""
     n_seq, n_q, n_head, dk = q.shape
-    if dk != DK:
-        raise ValueError("q must end in 576")
+    if dk not in (DK, DV):
+        raise ValueError("q must end in 576 (or 512: the DK = DV = 512 head shape)")
     a = mla_fa_args()
     a.q = q.data_ptr()
     a.kcache = kcache.data_ptr()
@@ -195,6 +197,7 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     a.softcap = float(softcap)
     a.mask_gather = 1 if mask_gather else 0
     a.out_lse = None if out_lse is None else out_lse.data_ptr()
+    a.head_dim = dk
     keep = _host_i32(kv_len)
     a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
     if idx is not None:

@@ -157,6 +157,7 @@ struct Resolved {
   bool proj;  // fused value up-projection: every sequence writes split partials
   bool sinks; // attention sinks: every sequence writes split partials (the combine adds them)
   bool lse;   // per-row log-sum-exp output: every sequence writes partials (the combine writes it)
+  int dk;     // head width: MLA_DK, or MLA_DV for the DK = DV = 512 shape
 };
 
 int validate(const mla_fa_args* a, Resolved* r) {
@@ -175,6 +176,13 @@ int validate(const mla_fa_args* a, Resolved* r) {
       (reinterpret_cast<uintptr_t>(a->out_lse) & 3))
     return MLA_ERR_ALIGN;
   if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
+  // head width: 576, or 512 (f16 cache; dense or index-list attention, no softcap,
+  // ALiBi or mask gather)
+  const int dk = a->head_dim == 0 ? MLA_DK : a->head_dim;
+  if (dk != MLA_DK && dk != MLA_DV) return MLA_ERR_SHAPE;
+  if (dk == MLA_DV && (a->kcache_type != MLA_KV_F16 || a->softcap > 0.f || a->alibi_slopes != nullptr ||
+                       a->mask_gather != 0))
+    return MLA_ERR_UNSUPPORTED;
   if (a->n_seq < 1 || a->n_q < 1 || a->n_head < 1 || a->n_head > MLA_MAX_HEADS || a->n_kv < 1)
     return MLA_ERR_SHAPE;
   if (!std::isfinite(a->scale)) return MLA_ERR_SHAPE;
@@ -189,7 +197,8 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (a->idx != nullptr && a->idx_count == nullptr) return MLA_ERR_NULL;
   r->a = *a;
   r->rows = (int)rows;
-  r->q_ss = a->q_seq_stride ? a->q_seq_stride : rows * MLA_DK;
+  r->dk = dk;
+  r->q_ss = a->q_seq_stride ? a->q_seq_stride : rows * dk;
   r->k_ss = a->k_seq_stride ? a->k_seq_stride : a->n_kv;
   r->m_rs = a->mask_row_stride ? a->mask_row_stride : a->n_kv;
   r->m_ss = a->mask_seq_stride ? a->mask_seq_stride : (int64_t)a->n_q * r->m_rs;
@@ -202,7 +211,7 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (proj && (a->out_proj_seq_stride < 0 || r->op_ss < rows * MLA_PROJ_DIM)) return MLA_ERR_SHAPE;
   if (proj && (!aligned16(a->wv) || !aligned16(a->out_proj) || (r->op_ss % 4) != 0))
     return MLA_ERR_ALIGN;
-  if (r->q_ss < rows * MLA_DK || r->k_ss < a->n_kv || r->m_rs < a->n_kv ||
+  if (r->q_ss < rows * dk || r->k_ss < a->n_kv || r->m_rs < a->n_kv ||
       r->m_ss < (int64_t)(a->n_q - 1) * r->m_rs + a->n_kv || r->o_ss < rows * MLA_DV ||
       r->idx_ss < 0)
     return MLA_ERR_SHAPE;
@@ -345,12 +354,12 @@ int make_part_map(CUtensorMap* m, void* base, uint64_t rows) {
 }
 
 // One instance of the attention kernel, with its block size (cfg has the rest).
-template <int kMode, bool kVariant, bool kGather>
+template <int kMode, bool kVariant, bool kGather, int kNC = 9>
 cudaError_t launch_fwd(cudaLaunchConfig_t cfg, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                        const CUtensorMap& tm_v, const CUtensorMap& tm_o, const CUtensorMap& tm_w,
                        const mla::Plan& plan, const mla::MlaFwdParams& p) {
   cfg.blockDim = dim3(mla::FwdCfg<kMode>::kThreads);
-  return cudaLaunchKernelEx(&cfg, mla::mla_fwd_kernel<kMode, kVariant, kGather>, tm_q, tm_k, tm_v,
+  return cudaLaunchKernelEx(&cfg, mla::mla_fwd_kernel<kMode, kVariant, kGather, kNC>, tm_q, tm_k, tm_v,
                             tm_o, tm_w, plan, p);
 }
 
@@ -362,10 +371,10 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   const int mode = a.kcache_type == MLA_KV_Q8_0 ? mla::kModeQ8
                    : (a.idx != nullptr || a.mask_gather ? mla::kModeGatherF16 : mla::kModeTma);
   CUtensorMap tm_q, tm_k, tm_v;
-  const uint64_t row_bytes = MLA_DK * 2;
-  int rc = make_map(&tm_q, a.q, MLA_DK, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
+  const uint64_t row_bytes = (uint64_t)r.dk * 2;
+  int rc = make_map(&tm_q, a.q, r.dk, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
   if (rc == MLA_OK && mode == mla::kModeTma) {
-    rc = make_map(&tm_k, a.kcache, MLA_DK, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
+    rc = make_map(&tm_k, a.kcache, r.dk, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
                   64, mla::kTileKeys / 2);
     if (rc == MLA_OK) {
       // value view: {64 columns, keys, 8 column blocks, sequences}; a box of
@@ -398,16 +407,18 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
     const void* fwd_kernels[] = {
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, true, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, true>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, true>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, false>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, true>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, true>};
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, true, false, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, false, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, true, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, true, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, false, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, false, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, true, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, true, 9>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 8>,
+        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false, 8>};
     bool ok = true;
     for (const void* k : fwd_kernels)
       ok = ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -479,7 +490,11 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     {
       ProfScope prof(mode == mla::kModeTma ? kKernFwdF16
                      : mode == mla::kModeGatherF16 ? kKernFwdGather : kKernFwdQ8, stream);
-      if (mode == mla::kModeTma)
+      if (r.dk != MLA_DK)  // the DK = DV = 512 shape: dense or index-list, f16 cache
+        fe = mode == mla::kModeTma
+                 ? launch_fwd<mla::kModeTma, false, false, 8>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                 : launch_fwd<mla::kModeGatherF16, false, false, 8>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
+      else if (mode == mla::kModeTma)
         fe = variant ? launch_fwd<mla::kModeTma, true, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
                      : launch_fwd<mla::kModeTma, false, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
       else if (mode == mla::kModeGatherF16)

@@ -164,7 +164,6 @@ template <int kMode>
 struct FwdCfg {
   static constexpr bool kManual = kMode != kModeTma;
   static constexpr int kThreads = kManual ? 384 : 256;  // + 4 producer warps when manual
-  static constexpr int kRowBytes = kMode == kModeQ8 ? kQ8RowBytes : 2 * kDK;
 };
 
 // q8_0 block (f16 d, then 32 int8) -> 32 f16 values d*q (one rounding each), as
@@ -183,7 +182,8 @@ struct RawBlock {
   bool valid;      // false: zero fill
 };
 
-template <int kMode>
+// kRowBytes: bytes of an f16 cache row (2 x its head width)
+template <int kMode, int kRowBytes>
 __device__ __forceinline__ void load_block(const uint8_t* kcache, int64_t row, int col32,
                                            RawBlock<kMode>& rb) {
   if constexpr (kMode == kModeQ8) {
@@ -194,7 +194,7 @@ __device__ __forceinline__ void load_block(const uint8_t* kcache, int64_t row, i
     for (int i = 0; i < 9; ++i) rb.w[i] = __ldg(w4 + i);
     rb.odd = (a & 2) != 0;
   } else {
-    const uint4* src = reinterpret_cast<const uint4*>(kcache + row * (2 * kDK) + col32 * 64);
+    const uint4* src = reinterpret_cast<const uint4*>(kcache + row * kRowBytes + col32 * 64);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint4 v = __ldg(src + k);
@@ -240,8 +240,10 @@ __device__ __forceinline__ void block_values(const RawBlock<kMode>& rb, uint32_t
 
 // kVariant: the instance that applies the logit softcap and ALiBi; kGather: the instance
 // that compacts the mask itself (gather modes only). The host launches them only when a
-// call asks for them, so the common path carries none of that code.
-template <int kMode, bool kVariant, bool kGather>
+// call asks for them, so the common path carries none of that code. kNC: 64-column
+// chunks of the head width, 9 (576: 512 latent + 64 RoPE) or 8 (the DK = DV = 512
+// shape, f16 cache, V the whole row).
+template <int kMode, bool kVariant, bool kGather, int kNC>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThreads, 1)
     mla_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -251,6 +253,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                    const __grid_constant__ MlaFwdParams p) {
   using namespace fwd;
   constexpr bool kManual = FwdCfg<kMode>::kManual;
+  static_assert(kNC == 9 || (kNC == 8 && kMode != kModeQ8), "head width 576, or 512 with an f16 cache");
+  // bytes of a cache row: q8_0 rows are 612 bytes; f16 rows 2 x the head width
+  constexpr int kRowBytes = kMode == kModeQ8 ? kQ8RowBytes : 128 * kNC;
   extern __shared__ uint8_t smem_raw[];
   // a launch with too little dynamic shared memory reports and returns (every CTA takes
   // this branch, so no cluster barrier is left waiting)
@@ -417,7 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       uint32_t ephase = 0;
       for (int i = 0; i < n_tiles && !failed; ++i) {
         const int key0 = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
-        for (int c = 0; c < 9; ++c) {
+        for (int c = 0; c < kNC; ++c) {
           if (!mbar_wait(&bars.k_empty[stage], ephase ^ 1, to)) {
             // stop issuing: a stage may still be in use, and the copies already in
             // flight (at most one ring) land before the teardown
@@ -438,9 +443,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     }
     // gather modes: this CTA's Q rows by TMA (the producers gather K and V)
     if (kManual && n_tiles > 0 && elect_one()) {
-      if (rank == 0) mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
+      if (rank == 0) mbar_arrive_expect_tx(&bars.q_full, 2 * kNC * kChunkBytes);
       const uint32_t fq = mapa_shared(smem_u32(&bars.q_full), 0);
-      for (int c = 0; c < 9; ++c)
+      for (int c = 0; c < kNC; ++c)
         tma_load_3d_2sm(sQ + c * kChunkBytes, &tm_q, fq, 64 * c, row0 + kRowsPerCta * (int)rank, b_abs);
     }
     __syncwarp();
@@ -501,7 +506,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           break;
         }
         const uint32_t d_s = tmem + kTmemS;
-        for (int c = 0; c < 9; ++c) {
+        for (int c = 0; c < kNC; ++c) {
           const bool ok = kManual ? mbar_wait_cluster(&bars.k_full[kst], kph, to)
                                   : mbar_wait(&bars.k_full[kst], kph, to);
           if (!ok) {
@@ -592,7 +597,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       auto load32 = [&](int key, int col32, RawBlock<kMode>& rb) {
         rb.valid = key >= 0;
         rb.odd = false;
-        if (rb.valid) load_block<kMode>(p.kcache, seq_row0 + key, col32, rb);
+        if (rb.valid) load_block<kMode, kRowBytes>(p.kcache, seq_row0 + key, col32, rb);
       };
       auto store32 = [&](uint8_t* row_dst, int row_in_atom, int chunk0, const RawBlock<kMode>& rb) {
         uint32_t h[16];
@@ -640,14 +645,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             if (keys[q] < 0) continue;
-            const uint8_t* rowp = p.kcache + (seq_row0 + keys[q]) * FwdCfg<kMode>::kRowBytes;
-            for (int off = 128 * half; off < FwdCfg<kMode>::kRowBytes; off += 256) prefetch_l2(rowp + off);
-            if (half == 1) prefetch_l2(rowp + FwdCfg<kMode>::kRowBytes - 1);
+            const uint8_t* rowp = p.kcache + (seq_row0 + keys[q]) * kRowBytes;
+            for (int off = 128 * half; off < kRowBytes; off += 256) prefetch_l2(rowp + off);
+            if (half == 1) prefetch_l2(rowp + kRowBytes - 1);
           }
           RawBlock<kMode> cur[kLoadBatch];
 #pragma unroll
           for (int q = 0; q < kLoadBatch; ++q) load32(keys[q], half, cur[q]);
-          for (int c = 0; c < 9; ++c) {
+          for (int c = 0; c < kNC; ++c) {
             uint8_t* st = nullptr;
 #pragma unroll
             for (int bq = 0; bq < kBpc; ++bq) {
@@ -657,7 +662,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               RawBlock<kMode> nxt[kLoadBatch];
 #pragma unroll
               for (int q = 0; q < kLoadBatch; ++q) {
-                if (nc < 9) load32(keys[nq0 + q], 2 * nc + half, nxt[q]);
+                if (nc < kNC) load32(keys[nq0 + q], 2 * nc + half, nxt[q]);
                 else { nxt[q].valid = false; nxt[q].odd = false; }
               }
               if (bq == 0) {

@@ -103,6 +103,11 @@ def call_ex(lib, a):
     (dict(out_lse=FAKE, sinks=FAKE), -8),
     (dict(out_lse=FAKE, wv=FAKE, proj_dim=128, out_proj=FAKE), -8),
     (dict(out_lse=FAKE + 2), -4),
+    # head width: 576 or 512; 512 takes an f16 cache, no softcap, ALiBi or mask gather
+    (dict(head_dim=256), -2), (dict(head_dim=513), -2),
+    (dict(head_dim=512, kcache_type=1), -8), (dict(head_dim=512, softcap=5.0), -8),
+    (dict(head_dim=512, alibi_slopes=FAKE), -8), (dict(head_dim=512, mask=FAKE, mask_gather=1), -8),
+    (dict(head_dim=512, q_seq_stride=16 * 512 - 8, n_seq=2), -2),
     # mask gather: needs the mask, excludes an index list and ALiBi
     (dict(mask_gather=2, mask=FAKE), -2), (dict(mask_gather=1), -1),
     (dict(mask_gather=1, mask=FAKE, idx=FAKE, idx_count=FAKE), -8),

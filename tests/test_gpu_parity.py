@@ -781,3 +781,77 @@ def test_combine_entry_point_matches_oracle(n_parts, rows):
     assert np.array_equal(np.isneginf(lg), np.isneginf(l_ref))
     fin = np.isfinite(l_ref)
     np.testing.assert_allclose(lg[fin], l_ref[fin], rtol=0, atol=1e-4)
+
+
+# ---- the DK = DV = 512 head shape (f16 cache, V = the whole row) -------------------------
+
+def run_dk512(q, k, mask, scale, kv_len=None, idx=None, idx_count=None, **kw):
+    torch = torch_mod()
+    dev = torch.device("cuda")
+    n_seq, n_q, n_head, _ = q.shape
+    n_out = n_seq * n_q * n_head * 512
+    big = torch.full((n_out + CANARY,), float("nan"), device=dev)
+    out = big[:n_out].view(n_seq, n_q, n_head, 512)
+    tq = torch.from_numpy(q).to(dev)
+    tk = torch.from_numpy(k).to(dev)
+    tm = None if mask is None else torch.from_numpy(mask).to(dev)
+    binding.forward(tq, tk, 0, tm, scale, out=out, kv_len=kv_len, idx=idx, idx_count=idx_count, **kw)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    assert bool(torch.isnan(big[n_out:]).all()), "write past the end of out"
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("n_seq,n_q,n_head,n_kv", [(1, 1, 16, 300), (4, 1, 128, 3000), (1, 3, 100, 700),
+                                                   (2, 2, 16, 1), (1, 1, 128, 257)])
+def test_dk512_dense_matches_oracle(n_seq, n_q, n_head, n_kv):
+    rng = np.random.default_rng(n_seq * 7 + n_q * 11 + n_head + n_kv)
+    q = rng.standard_normal((n_seq, n_q, n_head, 512)).astype(np.float16)
+    k = (0.5 * rng.standard_normal((n_seq, n_kv, 512))).astype(np.float16)
+    mask = np.where(rng.random((n_seq, n_q, n_kv)) < 0.8, rng.standard_normal((n_seq, n_q, n_kv)),
+                    -np.inf).astype(np.float16)
+    mask[:, :, 0] = 0
+    lens = [n_kv] + [max(1, n_kv - 37 * b) for b in range(1, n_seq)]
+    got = run_dk512(q, k, mask, 0.04, kv_len=lens)
+    for b in range(n_seq):
+        n = lens[b]
+        ref = oracle.attention(q[b], k[b, :n], oracle.KV_F16, mask[b, :, :n], 0.04)
+        assert_parity(got[b].reshape(-1, 512), ref, f"dk512 seq {b}")
+
+
+def test_dk512_index_list_equals_dense_masked():
+    torch = torch_mod()
+    rng = np.random.default_rng(61)
+    n_kv = 5000
+    q = rng.standard_normal((1, 1, 128, 512)).astype(np.float16)
+    k = (0.5 * rng.standard_normal((1, n_kv, 512))).astype(np.float16)
+    keep = rng.random(n_kv) < 0.12
+    mask = np.where(keep, np.float16(0), np.float16(-np.inf)).astype(np.float16)[None, None]
+    lst = np.nonzero(keep)[0].astype(np.int32)
+    idx = torch.full((1, n_kv), -1, dtype=torch.int32, device="cuda")
+    idx[0, : len(lst)] = torch.from_numpy(lst).cuda()
+    cnt = torch.tensor([len(lst)], dtype=torch.int32, device="cuda")
+    got = run_dk512(q, k, mask, 0.04, idx=idx, idx_count=cnt)
+    ref = oracle.attention(q[0], k[0], oracle.KV_F16, mask[0], 0.04)
+    assert_parity(got[0].reshape(-1, 512), ref, "dk512 index list")
+
+
+def test_dk512_with_sinks_and_lse():
+    torch = torch_mod()
+    rng = np.random.default_rng(62)
+    q = rng.standard_normal((2, 1, 16, 512)).astype(np.float16)
+    k = (0.5 * rng.standard_normal((2, 2000, 512))).astype(np.float16)
+    lse = torch.empty((2, 1, 16), device="cuda")
+    got = run_dk512(q, k, None, 0.04, out_lse=lse)
+    for b in range(2):
+        o_ref, l_ref = oracle.attention_lse(q[b], k[b], oracle.KV_F16, None, 0.04)
+        assert_parity(got[b].reshape(-1, 512), o_ref, f"dk512 lse out {b}")
+        assert_lse(lse[b].cpu().numpy(), l_ref, f"dk512 lse {b}")
+    sinks = rng.standard_normal(16).astype(np.float32)
+    got = run_dk512(q, k, None, 0.04, sinks=torch.from_numpy(sinks).cuda())
+    for b in range(2):
+        # a sink is one more logit per head with no value: the row is the plain
+        # attention scaled by its share e^{lse} / (e^{lse} + e^{sink})
+        o_ref, l_ref = oracle.attention_lse(q[b], k[b], oracle.KV_F16, None, 0.04)
+        share = 1.0 / (1.0 + np.exp(np.tile(sinks.astype(np.float64), 1) - l_ref))
+        assert_parity(got[b].reshape(-1, 512), o_ref * share[:, None], f"dk512 sinks {b}")
