@@ -58,7 +58,8 @@ def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
     weights (n_head x 512 x 128 f16) and does 2 x 512 x 128 flops per query row.
     A sparse step reads its mask row and writes then reads the index list; with the
     mask gather there is no list: the mask rows are read once."""
-    row_bytes = 1152 if w.kv_type == W.KV_F16 else W.Q8_ROW_BYTES
+    dk = w.q.shape[-1]  # 576, or 512 for the DK = DV = 512 head shape
+    row_bytes = 2 * dk if w.kv_type == W.KV_F16 else W.Q8_ROW_BYTES
     if kept_cells is None:
         keep = ~np.isneginf(w.mask) if w.mask is not None else None
         kept_cells = []
@@ -80,7 +81,7 @@ def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
     q_bytes = w.q.size * 2
     out_bytes = w.n_seq * w.n_q * w.n_head * (128 if wuv else 512) * 4
     kv_bytes = rows_attended * row_bytes
-    flops = 2.0 * w.n_head * (576 + 512) * pairs
+    flops = 2.0 * w.n_head * (dk + 512) * pairs
     if wuv:
         out_bytes += w.n_head * 512 * 128 * 2
         flops += 2.0 * 512 * 128 * w.n_seq * w.n_q * w.n_head
@@ -93,9 +94,9 @@ def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "c4969cb3127192b8", "bytes": 170689536},
-    "prefill_chunk": {"source": "c4969cb3127192b8", "bytes": 204933376},
-    "sparse_q8_decode": {"source": "c4969cb3127192b8", "bytes": 10393600},
+    "v3_batched_decode": {"source": "a1c2b2b0d122f433", "bytes": 172668672},
+    "prefill_chunk": {"source": "a1c2b2b0d122f433", "bytes": 205501952},
+    "sparse_q8_decode": {"source": "a1c2b2b0d122f433", "bytes": 10392576},
 }
 
 
@@ -114,7 +115,20 @@ def kernel_source_hash():
 def workload_name(args):
     """The workload as the step runs it: the cache geometry plus the fused options."""
     return (args.workload + ("+wuv" if args.wuv else "")
-            + ("+mask_gather" if args.mask_gather else ""))
+            + ("+mask_gather" if args.mask_gather else "")
+            + ("+dk512" if args.head_dim == 512 else ""))
+
+
+def make_workload(args):
+    """The named workload; with --head-dim 512 the same one with the 64 RoPE columns
+    of q and of the cache dropped (the DK = DV = 512 head shape, f16 cache)."""
+    w = W.make(args.workload)
+    if args.head_dim == 512:
+        if w.kv_type != W.KV_F16:
+            raise SystemExit("--head-dim 512 takes an f16-cache workload")
+        w.q = np.ascontiguousarray(w.q[..., :512])
+        w.kcache = np.ascontiguousarray(w.kcache[..., :512])
+    return w
 
 
 def measured_traffic(workload):
@@ -240,7 +254,7 @@ def gpu_arm(args, rank, world):
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     binding.load()
-    w = W.make(args.workload)
+    w = make_workload(args)
     acc = algorithmic(w, wuv=args.wuv, mask_gather=args.mask_gather)
     step = Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather)
     stream = torch.cuda.current_stream()
@@ -521,6 +535,9 @@ def main(argv=None):
     ap.add_argument("--mask-gather", action="store_true",
                     help="masked workloads: sparse attention straight from the mask (the "
                          "compaction fused into the attention kernel, no index list)")
+    ap.add_argument("--head-dim", type=int, default=576, choices=[576, 512],
+                    help="512: the DK = DV = 512 head shape (the workload without its RoPE "
+                         "columns; f16 cache)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0)
@@ -532,6 +549,8 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.wuv and args.impl == "reference":
         ap.error("--wuv applies to --impl ours (the oracle arm times the attention only)")
+    if args.head_dim != 576 and args.impl == "reference":
+        ap.error("--head-dim applies to --impl ours")
     if args.mask_gather and args.impl == "reference":
         ap.error("--mask-gather applies to --impl ours (the oracle arm runs the unfused chain)")
     if args.wuv:
