@@ -637,3 +637,42 @@ def test_dk512_equals_dk576_with_zero_rope_columns_exactly():
     o576, l576 = oracle.attention_lse(pad(q), pad(k), mask=mask, scale=0.07)
     np.testing.assert_array_equal(o512, o576)
     np.testing.assert_array_equal(l512, l576)
+
+
+def test_planted_merge_and_lse_mistakes_are_caught():
+    """Plausible mistakes in the merge and the lse, planted in numpy copies on the CPU:
+    weights exp(lse) without the max shift (overflow), the lse in log2 units, the merge
+    weighting by e^{-lse}, and the lse without the mask. Each must fail a pin above."""
+    rng = np.random.default_rng(45)
+    n = 120
+    q = rand_f16(rng, (2, 3, DK))
+    k = rand_f16(rng, (n, DK))
+    mask = rand_f16(rng, (2, n))
+    o_all, lse_all = oracle.attention_lse(q, k, mask=mask, scale=0.06)
+    parts = [oracle.attention_lse(q, k[a:b], mask=mask[:, a:b], scale=0.06)
+             for a, b in ((0, 50), (50, 120))]
+    o_p = np.stack([p[0] for p in parts])
+    l_p = np.stack([p[1] for p in parts])
+
+    def merge(o, lse, w_of):
+        w = w_of(lse)
+        return (w[:, :, None] * o).sum(0) / w.sum(0)[:, None]
+
+    # the real merge reproduces the whole
+    good, _ = oracle.combine(o_p, l_p)
+    np.testing.assert_allclose(good, o_all, rtol=1e-12, atol=1e-13)
+    # weights by e^{-lse}: wrong result
+    assert np.max(np.abs(merge(o_p, l_p, lambda l: np.exp(-l)) - o_all)) > 1e-3
+    # no max shift: with large lse values the weights overflow to inf and the merge is NaN
+    with np.errstate(over="ignore", invalid="ignore"):
+        assert not np.all(np.isfinite(merge(o_p, l_p + 800.0, np.exp)))
+    shifted, _ = oracle.combine(o_p, l_p + 800.0)  # the real merge is shift invariant
+    np.testing.assert_allclose(shifted, good, rtol=1e-12, atol=1e-13)
+    # lse in log2 units, or without the mask: the one-hot / log(n) pins disagree
+    qz = np.zeros((1, 1, DK), np.float16)
+    _, l_ok = oracle.attention_lse(qz, k[:7], mask=np.zeros((1, 7), np.float16), scale=0.3)
+    assert abs(l_ok[0] - math.log(7)) < 1e-13
+    assert abs(l_ok[0] / math.log(2) - math.log(7)) > 1e-3
+    m1 = np.full((1, 7), np.float16(2.0))
+    _, l_m = oracle.attention_lse(qz, k[:7], mask=m1, scale=0.3)
+    assert abs(l_m[0] - (math.log(7) + 2.0)) < 1e-12 and abs(l_m[0] - math.log(7)) > 1.0
