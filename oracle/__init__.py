@@ -8,12 +8,16 @@ library: the two meet only through the seeded input generators.
 The arithmetic lives in ``mla_oracle.c`` (plain C, fp64, OpenMP over query
 rows). This module compiles it with gcc on first use and wraps it with ctypes.
 What it computes and which page passage each part follows is written at the
-top of ``mla_oracle.c``.
+top of ``mla_oracle.c``. Two definitions are plain numpy here, each with its
+reading in its docstring: ``combine`` (the merge of partial results over
+disjoint key sets) and ``attention_heads`` (a K and a V per KV head, the
+DK = 192 / DV = 128 head shape).
 
 Parity pins (checked by ``tests/test_oracle_pins.py`` against closed forms,
 brute force and invariants, never against the oracle itself):
-  attention / attention_online / attention_split / compact / dequant_q8_0 / project /
-  attention_variants.
+  attention (576- and 512-wide heads) / attention_lse / attention_online /
+  attention_split / compact / dequant_q8_0 / project / attention_variants /
+  combine / attention_heads.
 """
 from __future__ import annotations
 
@@ -221,6 +225,41 @@ def combine(o_parts, lse_parts):
         out[r] = (w[:, None] * o[:, r, :]).sum(axis=0) / w.sum()
         out_lse[r] = M + np.log(w.sum())
     return out, out_lse
+
+
+def attention_heads(q, k, v, mask=None, scale=1.0):
+    """Attention with a K and a V per KV head, the layout of the DK = 192 / DV = 128 head
+    shape (one of the head shapes the llama.cpp tag page lists for the Metal FA kernel,
+    PR #29570): query head h reads KV head h // (n_head / n_kv_head), so n_kv_head =
+    n_head is plain multi-head attention and n_kv_head = 1 shares one head, as the MLA
+    cache does. Per query row, s_j = scale * q . k_j + mask_j, o = sum_j softmax(s)_j v_j;
+    a row with nothing kept gives 0.
+
+    q f16 [n_q][n_head][dk], k f16 [n_kv][n_kv_head][dk], v f16 [n_kv][n_kv_head][dv],
+    mask f16 [n_q][n_kv] or None (shared by the heads of a token). fp64 throughout;
+    returns float64 [n_q * n_head][dv], row t * n_head + h."""
+    qd = np.asarray(q, dtype=np.float16).astype(np.float64)
+    kd = np.asarray(k, dtype=np.float16).astype(np.float64)
+    vd = np.asarray(v, dtype=np.float16).astype(np.float64)
+    n_q, n_head, dk = qd.shape
+    n_kv, n_kv_head, dk2 = kd.shape
+    if dk2 != dk or vd.shape[:2] != (n_kv, n_kv_head) or n_head % n_kv_head:
+        raise ValueError("q [n_q][H][dk], k [n][Hkv][dk], v [n][Hkv][dv], H a multiple of Hkv")
+    group = n_head // n_kv_head
+    md = None if mask is None else np.asarray(mask, dtype=np.float16).astype(np.float64)
+    out = np.zeros((n_q, n_head, vd.shape[2]))
+    for hk in range(n_kv_head):
+        hs = slice(hk * group, (hk + 1) * group)
+        s = scale * np.einsum("thc,nc->thn", qd[:, hs, :], kd[:, hk, :])  # [n_q][group][n_kv]
+        if md is not None:
+            s = s + md[:, None, :]
+        m = s.max(axis=2, keepdims=True)
+        kept = np.isfinite(m)
+        p = np.where(kept, np.exp(s - np.where(kept, m, 0.0)), 0.0)
+        den = p.sum(axis=2, keepdims=True)
+        o = np.einsum("thn,nd->thd", p, vd[:, hk, :])
+        out[:, hs, :] = np.where(den > 0, o / np.where(den > 0, den, 1.0), 0.0)
+    return out.reshape(n_q * n_head, -1)
 
 
 def attention_online(q, kcache, kv_type=KV_F16, mask=None, scale=1.0, tile=64, rows=None,

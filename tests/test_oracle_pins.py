@@ -676,3 +676,74 @@ def test_planted_merge_and_lse_mistakes_are_caught():
     m1 = np.full((1, 7), np.float16(2.0))
     _, l_m = oracle.attention_lse(qz, k[:7], mask=m1, scale=0.3)
     assert abs(l_m[0] - (math.log(7) + 2.0)) < 1e-12 and abs(l_m[0] - math.log(7)) > 1.0
+
+
+# ---- attention with a K and a V per KV head (the DK = 192 / DV = 128 head shape) --------
+
+def _loop_heads(q, k, v, mask, scale):
+    """The same definition by explicit per-row loops (no einsum, no grouping trick)."""
+    n_q, H, _ = q.shape
+    n, Hkv, _ = k.shape
+    out = np.zeros((n_q * H, v.shape[2]))
+    for t in range(n_q):
+        for h in range(H):
+            hk = h // (H // Hkv)
+            s = [scale * float(np.dot(q[t, h].astype(np.float64), k[j, hk].astype(np.float64)))
+                 + (0.0 if mask is None else float(mask[t, j])) for j in range(n)]
+            mx = max(s)
+            if mx == -math.inf:
+                continue
+            w = [math.exp(x - mx) for x in s]
+            tot = math.fsum(w)
+            out[t * H + h] = sum(wj * v[j, hk].astype(np.float64) for j, wj in enumerate(w)) / tot
+    return out
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 4), (4, 2), (6, 1)])
+def test_heads_match_explicit_loops(H, Hkv):
+    rng = np.random.default_rng(70 + H + Hkv)
+    q = rand_f16(rng, (3, H, 192))
+    k = rand_f16(rng, (11, Hkv, 192))
+    v = rand_f16(rng, (11, Hkv, 128))
+    mask = rand_f16(rng, (3, 11))
+    mask[2, :] = NEG  # a token with nothing kept
+    mask[0, 4] = NEG
+    got = oracle.attention_heads(q, k, v, mask, 0.08)
+    np.testing.assert_allclose(got, _loop_heads(q, k, v, mask, 0.08), rtol=1e-12, atol=1e-13)
+    assert np.all(got[2 * H:] == 0)
+
+
+def test_heads_single_key_gives_its_value_row():
+    rng = np.random.default_rng(71)
+    q = rand_f16(rng, (2, 4, 192))
+    k = rand_f16(rng, (1, 2, 192))
+    v = rand_f16(rng, (1, 2, 128))
+    got = oracle.attention_heads(q, k, v, None, 0.3).reshape(2, 4, 128)
+    for h in range(4):
+        np.testing.assert_array_equal(got[:, h], np.broadcast_to(v[0, h // 2].astype(np.float64), (2, 128)))
+
+
+def test_heads_with_one_shared_head_is_the_mla_attention():
+    # one KV head, dk = 576 and V = the first 512 columns of K: the C oracle's MLA
+    # attention, an independent implementation of the same definition
+    rng = np.random.default_rng(72)
+    q = rand_f16(rng, (2, 5, DK))
+    kc = rand_f16(rng, (60, DK))
+    mask = rand_f16(rng, (2, 60))
+    mask[1, 10:20] = NEG
+    got = oracle.attention_heads(q, kc[:, None, :], kc[:, None, :DV], mask, 0.05)
+    np.testing.assert_allclose(got, oracle.attention(q, kc, mask=mask, scale=0.05), rtol=1e-11, atol=1e-12)
+
+
+def test_heads_permuting_kv_heads_with_their_groups_permutes_the_output():
+    rng = np.random.default_rng(73)
+    H, Hkv = 6, 3
+    q = rand_f16(rng, (2, H, 192))
+    k = rand_f16(rng, (20, Hkv, 192))
+    v = rand_f16(rng, (20, Hkv, 128))
+    base = oracle.attention_heads(q, k, v, None, 0.07).reshape(2, H, 128)
+    perm = np.array([2, 0, 1])
+    qperm = np.concatenate([q[:, 2 * p:2 * p + 2] for p in perm], axis=1)
+    got = oracle.attention_heads(qperm, k[:, perm], v[:, perm], None, 0.07).reshape(2, H, 128)
+    want = np.concatenate([base[:, 2 * p:2 * p + 2] for p in perm], axis=1)
+    np.testing.assert_array_equal(got, want)
