@@ -1,4 +1,4 @@
-"""Split-KV decode across ranks, its orchestration on CPU with two and three gloo ranks.
+"""Split-KV decode across ranks, its orchestration on CPU with one, two and three gloo ranks.
 
 The kernels need a GPU; here each rank's attention and the final merge are stand-ins
 built on the oracle (with the same signatures as the library calls), so what runs is
@@ -87,7 +87,7 @@ def _rank_main(rank, world, port, out_dir):
         np.save(os.path.join(out_dir, "ref.npy"), ref)
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [1, 2, 3])
 def test_split_kv_decode_over_gloo_ranks_equals_the_whole_cache(tmp_path, world):
     import torch.multiprocessing as mp
 
