@@ -179,3 +179,19 @@ def test_valid_arguments_reach_the_device_check(lib):
     if torch.cuda.is_available():
         pytest.skip("fake pointers: only meaningful without a GPU")
     assert call_ex(lib, base_args()) in (-6, -8)
+
+
+def test_binding_takes_the_head_width_from_q():
+    # argument marshalling only (CPU tensors, no call into the library's kernels)
+    import torch
+
+    for dk in (576, 512):
+        q = torch.zeros((2, 1, 4, dk), dtype=torch.float16)
+        k = torch.zeros((2, 8, dk), dtype=torch.float16)
+        out = torch.zeros((2, 1, 4, 512), dtype=torch.float32)
+        a, _ = binding.make_args(q, k, 0, None, out, 0.1)
+        assert a.head_dim == dk and a.q_seq_stride == 4 * dk and a.k_seq_stride == 8
+    with pytest.raises(ValueError):
+        binding.make_args(torch.zeros((1, 1, 4, 300), dtype=torch.float16),
+                          torch.zeros((1, 8, 300), dtype=torch.float16), 0, None,
+                          torch.zeros((1, 1, 4, 512)), 0.1)
