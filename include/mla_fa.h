@@ -235,6 +235,13 @@ int mla_fa_forward_noalloc(const mla_fa_args* a, void* stream);
 int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows,
                    float* out, float* out_lse, void* stream);
 
+/* The same plan for a GPU with sm_count SMs, computed on the host alone (no device is
+ * queried, nothing is launched): units, max_splits as mla_fa_query_plan, and the
+ * workspace bytes mla_fa_workspace_size would return on such a GPU. Any pointer may be
+ * NULL. Errors: those of argument validation; sm_count < 1 MLA_ERR_SHAPE. */
+int mla_fa_plan_for_sms(const mla_fa_args* a, int sm_count, int* units, int* max_splits,
+                        size_t* workspace_bytes);
+
 /* How the pass is divided: units = CTA pairs launched, max_splits = largest
  * number of KV splits of one (sequence, 128-row group). For tests and tools. */
 int mla_fa_query_plan(const mla_fa_args* a, int* units, int* max_splits);

@@ -126,6 +126,9 @@ def load(path: str = LIB_PATH):
     lib.mla_profile_begin.restype = I
     lib.mla_profile_end.argtypes = [ctypes.POINTER(mla_profile_entry), I, ctypes.POINTER(I)]
     lib.mla_profile_end.restype = I
+    lib.mla_fa_plan_for_sms.argtypes = [ctypes.POINTER(mla_fa_args), I, ctypes.POINTER(I),
+                                         ctypes.POINTER(I), ctypes.POINTER(Z)]
+    lib.mla_fa_plan_for_sms.restype = I
     lib.mla_fa_combine.argtypes = [P, P, I, ctypes.c_int64, P, P, P]
     lib.mla_fa_combine.restype = I
     _lib = lib
@@ -216,6 +219,14 @@ def mla_fa_query_plan(args):
     _check(load().mla_fa_query_plan(ctypes.byref(args), ctypes.byref(units), ctypes.byref(splits)),
            "mla_fa_query_plan")
     return units.value, splits.value
+
+
+def mla_fa_plan_for_sms(args, sm_count):
+    """Host-only plan for a GPU with sm_count SMs: (units, max_splits, workspace bytes)."""
+    units, splits, ws = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_size_t(0)
+    _check(load().mla_fa_plan_for_sms(ctypes.byref(args), int(sm_count), ctypes.byref(units),
+                                      ctypes.byref(splits), ctypes.byref(ws)), "mla_fa_plan_for_sms")
+    return units.value, splits.value, ws.value
 
 
 def mla_fa_forward_ex(args, workspace=None, stream=None):

@@ -254,15 +254,38 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
     sum_tiles += tiles[b];
   }
   const int64_t total_groups = (int64_t)n * plan->groups;
+  std::vector<int> nsplit(n, 1);
+  if (total_groups < pairs && sum_tiles > 0) {
+    int64_t want_units = 0;
+    for (int b = 0; b < n; ++b) {
+      const double want = (double)pairs * tiles[b] / ((double)sum_tiles * plan->groups);
+      int ns = (int)std::floor(want + 0.5);
+      ns = std::min(ns, std::max(1, tiles[b] / kMinTilesPerSplit));
+      nsplit[b] = std::max(ns, 1);
+      want_units += (int64_t)plan->groups * nsplit[b];
+    }
+    // Rounding can ask for more units than there are SM pairs, and the surplus would
+    // run as a second wave. Take splits back one at a time from the sequence whose
+    // units grow least (in tiles per unit) by losing one.
+    while (want_units > pairs) {
+      int best = -1;
+      int64_t best_load = 0;
+      for (int b = 0; b < n; ++b) {
+        if (nsplit[b] <= 1) continue;
+        const int64_t load = (tiles[b] + nsplit[b] - 2) / (nsplit[b] - 1);  // ceil(t / (ns - 1))
+        if (best < 0 || load < best_load) {
+          best = b;
+          best_load = load;
+        }
+      }
+      if (best < 0) break;
+      --nsplit[best];
+      want_units -= plan->groups;
+    }
+  }
   int units = 0, slots = 0;
   for (int b = 0; b < n; ++b) {
-    int ns = 1;
-    if (total_groups < pairs && sum_tiles > 0) {
-      const double want = (double)pairs * tiles[b] / ((double)sum_tiles * plan->groups);
-      ns = (int)std::floor(want + 0.5);
-      ns = std::min(ns, std::max(1, tiles[b] / kMinTilesPerSplit));
-      ns = std::max(ns, 1);
-    }
+    const int ns = nsplit[b];
     plan->n_split[b] = ns;
     plan->unit_base[b] = units;
     units += plan->groups * ns;
@@ -630,6 +653,20 @@ int mla_fa_query_plan(const mla_fa_args* a, int* units, int* max_splits) {
   rc = current_device(&st);
   if (rc != MLA_OK) return rc;
   workspace_for(r, st->sm_count, units, max_splits);
+  return MLA_OK;
+}
+
+int mla_fa_plan_for_sms(const mla_fa_args* a, int sm_count, int* units, int* max_splits,
+                        size_t* workspace_bytes) {
+  if (sm_count < 1) return MLA_ERR_SHAPE;
+  Resolved r;
+  int rc = validate(a, &r);
+  if (rc != MLA_OK) return rc;
+  int u = 0, m = 0;
+  const size_t need = workspace_for(r, sm_count, &u, &m);
+  if (units) *units = u;
+  if (max_splits) *max_splits = m;
+  if (workspace_bytes) *workspace_bytes = need;
   return MLA_OK;
 }
 

@@ -2,6 +2,8 @@
 include/mla_fa.h declares, and rejects bad arguments on the host before any
 launch (no kernel runs here)."""
 import ctypes
+
+import numpy as np
 import os
 import shutil
 import subprocess
@@ -195,3 +197,66 @@ def test_binding_takes_the_head_width_from_q():
         binding.make_args(torch.zeros((1, 1, 4, 300), dtype=torch.float16),
                           torch.zeros((1, 8, 300), dtype=torch.float16), 0, None,
                           torch.zeros((1, 1, 4, 512)), 0.1)
+
+
+# ---- the split plan, on the host alone (mla_fa_plan_for_sms) -----------------------------
+SLOT_BYTES = 128 * (512 * 2 + 4)  # one partial: 128 rows of f16 O / l and fp32 lse
+
+
+def _plan(sm_count, n_seq, n_q, n_head, lens, **kw):
+    lens_c = (ctypes.c_int32 * n_seq)(*lens)
+    a = base_args(n_seq=n_seq, n_q=n_q, n_head=n_head, n_kv=max(lens),
+                  kv_len=ctypes.cast(lens_c, ctypes.c_void_p), **kw)
+    return binding.mla_fa_plan_for_sms(a, sm_count)
+
+
+def test_plan_never_asks_for_more_units_than_sm_pairs():
+    # the per-sequence split counts are rounded; their sum must still fit one wave of
+    # CTA pairs, or the surplus units would run after the others
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        n_seq = int(rng.integers(1, 30))
+        lens = [int(x) for x in rng.integers(1, 60000, n_seq)]
+        n_q = int(rng.integers(1, 3))
+        sms = int(rng.choice([2, 16, 132, 148]))
+        units, splits, ws = _plan(sms, n_seq, n_q, 128, lens)
+        groups = (n_q * 128 + 127) // 128
+        assert units >= n_seq * groups and splits >= 1
+        if n_seq * groups < sms // 2:
+            assert units <= sms // 2
+        if splits == 1:
+            assert ws == 0
+        else:
+            assert ws > 0 and ws % SLOT_BYTES == 0
+
+
+def test_plan_of_a_batch_that_fills_the_gpu_has_no_splits():
+    units, splits, ws = _plan(148, 100, 1, 128, [5000] * 100)
+    assert (units, splits, ws) == (100, 1, 0)
+
+
+def test_plan_partials_forced_by_sinks_and_lse():
+    for kw in (dict(sinks=FAKE), dict(out_lse=FAKE)):
+        units, splits, ws = _plan(148, 100, 1, 128, [300] * 100, **kw)
+        assert (units, splits) == (100, 1) and ws == 100 * SLOT_BYTES
+
+
+def test_plan_of_the_v3_decode_batch():
+    # lengths of the V3 batched-decode workload (seed 1003): 540 tiles over 74 pairs
+    lens = [12606, 9479, 20813, 11456, 12221, 18279, 28969, 23042]
+    units, splits, ws = _plan(148, 8, 1, 128, lens)
+    assert units == 74 and splits == 16 and ws == 74 * SLOT_BYTES
+
+
+def test_plan_mask_gather_adds_the_cell_lists():
+    units, splits, ws = _plan(148, 1, 1, 128, [131072], mask=FAKE)
+    units_g, splits_g, ws_g = _plan(148, 1, 1, 128, [131072], mask=FAKE, mask_gather=1)
+    assert (units_g, splits_g) == (units, splits)
+    assert ws_g > ws  # the per-CTA lists of kept cells come after the partials
+
+
+def test_plan_rejects_bad_sm_counts_and_arguments(lib):
+    with pytest.raises(binding.MlaError):
+        _plan(0, 1, 1, 16, [100])
+    with pytest.raises(binding.MlaError):
+        binding.mla_fa_plan_for_sms(base_args(n_head=0), 148)
