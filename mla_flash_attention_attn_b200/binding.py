@@ -292,12 +292,12 @@ def combine(o_parts, lse_parts, out=None, out_lse=None, stream=None):
     [rows][512] (allocated if absent); out_lse fp32 [rows] is written if given."""
     import torch
 
-    n_parts = o_parts.shape[0]
-    o = o_parts.reshape(n_parts, -1, DV)
-    rows = o.shape[1]
-    lse = lse_parts.reshape(n_parts, rows)
-    if not (o.is_contiguous() and lse.is_contiguous()):
+    if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
         raise ValueError("o_parts and lse_parts must be contiguous")
+    n_parts = o_parts.shape[0]
+    o = o_parts.view(n_parts, -1, DV)
+    rows = o.shape[1]
+    lse = lse_parts.view(n_parts, rows)
     if out is None:
         out = torch.empty((rows, DV), dtype=torch.float32, device=o_parts.device)
     _check(load().mla_fa_combine(_ptr(o), _ptr(lse), n_parts, rows, _ptr(out), _ptr(out_lse),

@@ -260,3 +260,11 @@ def test_plan_rejects_bad_sm_counts_and_arguments(lib):
         _plan(0, 1, 1, 16, [100])
     with pytest.raises(binding.MlaError):
         binding.mla_fa_plan_for_sms(base_args(n_head=0), 148)
+
+
+def test_combine_binding_rejects_strided_parts():
+    import torch
+
+    o = torch.zeros((2, 8, 1024))[:, :, :512]  # a strided view
+    with pytest.raises(ValueError):
+        binding.combine(o, torch.zeros((2, 8)))
