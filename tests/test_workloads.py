@@ -75,3 +75,19 @@ def test_q8_0_random_value_ranges():
     q = blk[:, :, 2:].view(np.int8)
     assert np.all((d >= 0.5 / 127 - 1e-5) & (d <= 1.5 / 127 + 1e-5))
     assert q.min() >= -127 and q.max() <= 127
+
+
+def test_bench_head_dim_512_drops_the_rope_columns_and_counts_1024_byte_rows():
+    import types
+
+    import bench
+
+    a = types.SimpleNamespace(workload="v3_batched_decode", head_dim=512, wuv=False, mask_gather=False)
+    w5 = bench.make_workload(a)
+    w6 = W.make("v3_batched_decode")
+    assert w5.q.shape[-1] == 512 and w5.kcache.shape[-1] == 512
+    assert np.array_equal(w5.kcache, w6.kcache[..., :512]) and np.array_equal(w5.q, w6.q[..., :512])
+    acc5, acc6 = bench.algorithmic(w5), bench.algorithmic(w6)
+    assert acc5["kv_bytes"] * 1152 == acc6["kv_bytes"] * 1024
+    assert acc5["flops"] * (576 + 512) == acc6["flops"] * (512 + 512)
+    assert bench.workload_name(a) == "v3_batched_decode+dk512"
