@@ -7,18 +7,29 @@ One step = one pass of the workload's whole hot path through the C ABI
 compaction first) over one batch of synthetic inputs resident in HBM. Between
 timed steps L2 is flushed by writing a 256 MiB buffer and then reading another
 (outside the timed events), so a step starts from a cold L2 with no dirty lines
-of the flush left to write back. Each step is timed with CUDA events on the launching stream; with N
-ranks every rank runs its own replica of the batch (weak scaling, no
-collective on the data path) and the time is the max over ranks.
+of the flush left to write back. Each step is timed with CUDA events on the
+launching stream; with N ranks every rank runs its own replica of the batch (weak
+scaling, no collective on the data path) and the time is the max over ranks.
+`--gpus N` without a launcher starts the N ranks itself (torch.distributed.run on
+127.0.0.1, one process per GPU).
 
-Printed (rank 0): one JSON line with the metric, whole-job KV-cache GB/s,
-us/call, the roofline of the dominant kernel (live CUDA-event duration of its
-launches, taken in a second pass of the same steps: events between the launches
-of a step would serialise them, so the step time comes from a pass with only the
-two events around each step), an end-to-end figure through the same C ABI with host buffers
-(pinned host -> device copies of the inputs and device -> host copy of the
-output inside the timed region), the oracle's CPU throughput on a bounded
-sample, SM clocks sampled during the timed region, and the launch count.
+Printed (rank 0): one JSON line. Its headline (`value`, `roofline`, `e2e`,
+`cpu_baseline`) is the V3 batched decode workload, timed over exactly K steps:
+whole-job KV-cache GB/s, us/call, the roofline of the dominant kernel, an
+end-to-end figure through the same C ABI with host buffers (pinned host -> device
+copies of the inputs and device -> host copy of the output inside the timed
+region), the oracle's CPU throughput on a bounded sample, SM clocks sampled during
+the timed passes, and the launch count. `configs` holds the same measurement for
+every other workload of the benchmark definition (tiny decode, V2-Lite decode,
+prefill chunk, sparse q8_0 decode), each in the same process.
+
+Kernel times: the step time comes from a pass with only the two events around each
+step (events between the launches of a step would serialise them); per-kernel
+times come from a second pass of the same steps with the library's per-launch
+events. A roofline takes the dominant kernel's time from the second pass, capped at
+the step time of the first (a kernel cannot take longer than the step holding it;
+the passes may run at different clocks), and for a step of one kernel it is the
+step time itself. The median SM clock of each pass is recorded.
 
 --impl reference times the fp64 CPU oracle as the reference arm (there is no
 runnable reference implementation of this path), on a bounded sample per step.
@@ -150,7 +161,9 @@ def load_peaks():
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+    """Samples SM clock and throttle reasons through NVML while the timed passes run.
+    Each sample is tagged with the pass that was running (set_label), so every pass can
+    report its own median clock."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -159,15 +172,20 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, period=0.002):
         self.index = index
         self.period = period
-        self.samples = []
+        self.samples = []  # (label, MHz)
         self.reasons = set()
         self.max_mhz = None
+        self.label = None
         self._stop = threading.Event()
         self._thread = None
         self.ok = False
+
+    def set_label(self, label):
+        """Samples from now on belong to `label` (None: not a timed pass; not kept)."""
+        self.label = label
 
     def __enter__(self):
         try:
@@ -187,14 +205,17 @@ class ClockSampler:
     def _run(self):
         nv = self._nv
         while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit and bit != 0x1:
-                        self.reasons.add(name)
-            except Exception:  # noqa: BLE001
-                pass
+            label = self.label
+            if label is not None:
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    self.samples.append((label, mhz))
+                    for bit, name in self.REASONS.items():
+                        if mask & bit and bit != 0x1:
+                            self.reasons.add(name)
+                except Exception:  # noqa: BLE001
+                    pass
             time.sleep(self.period)
 
     def __exit__(self, *exc):
@@ -202,10 +223,14 @@ class ClockSampler:
         if self._thread is not None:
             self._thread.join(timeout=2)
 
+    def median(self, prefix=None):
+        xs = [m for lab, m in self.samples if prefix is None or lab.startswith(prefix)]
+        return float(statistics.median(xs)) if xs else None
+
     def summary(self):
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+        return {"sm_mhz": self.median(), "sm_max_mhz": self.max_mhz,
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
@@ -247,14 +272,39 @@ class Step:
         self.b.mla_fa_forward_ex(self.args, self.ws if self.ws_used else None, stream)
 
 
-def gpu_arm(args, rank, world):
-    import torch
+def config_of(w, name, world):
+    """The workload's description as it appears in both arms' JSON lines."""
+    return {"workload": name, "n_seq": w.n_seq, "n_q": w.n_q, "n_head": w.n_head,
+            "n_kv": w.n_kv, "head_dim": int(w.q.shape[-1]),
+            "kv_type": "q8_0" if w.kv_type else "f16",
+            "kv_len": [int(x) for x in w.kv_len][:16],
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed between timed steps (256 MiB written, then 256 MiB read; outside "
+                  "the events)"}
 
-    from mla_flash_attention_attn_b200 import binding
 
-    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    binding.load()
-    w = make_workload(args)
+def roofline_of(kacc, kernel_ms, peaks, peak_kind, traffic):
+    """Roofline of the dominant kernel: algorithmic bytes (or flops) per launch over its
+    time, against the measured peak of the binding roof."""
+    tensor_bound = kacc["flops"] / kacc["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        achieved = kacc["flops"] / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        achieved = kacc["bytes"] / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["traffic"] = traffic
+    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else \
+        "fallback (profiling recipe)"
+    return roof
+
+
+def measure(args, w, name, torch, binding, clocks, world, steps, headline=False):
+    """Time `steps` steps of workload w (after args.warmup untimed ones), then the same
+    steps again with per-kernel events. Returns the measurement and the Step."""
     acc = algorithmic(w, wuv=args.wuv, mask_gather=args.mask_gather)
     step = Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather)
     stream = torch.cuda.current_stream()
@@ -273,102 +323,136 @@ def gpu_arm(args, rank, world):
         step.run()
     torch.cuda.synchronize()
     if binding.mla_get_device_status() != 0:
-        raise RuntimeError("device status after warm-up")
+        raise RuntimeError(f"{name}: device status after warm-up")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clocks:
-        # the step time comes from a pass with nothing but the two events around each
-        # step: per-kernel events between the launches would serialise them (the
-        # combine is a programmatic dependent of the forward kernel) and add their own
-        # cost to the step
-        for i in range(args.steps):
-            l2_flush()
-            starts[i].record(stream)
-            step.run()
-            stops[i].record(stream)
-        torch.cuda.synchronize()
-        # per-kernel device times (roofline, launch counts): a second pass of the same
-        # steps with the library's per-launch events
-        binding.mla_profile_begin()
-        for i in range(args.steps):
-            l2_flush()
-            step.run()
-        torch.cuda.synchronize()
-        prof = binding.mla_profile_end()
+    # pass 1: nothing but the two events around each step (per-kernel events between the
+    # launches would serialise them: the combine is a programmatic dependent of the
+    # forward kernel)
+    clocks.set_label(f"{name}/step")
+    for i in range(steps):
+        l2_flush()
+        starts[i].record(stream)
+        step.run()
+        stops[i].record(stream)
+    torch.cuda.synchronize()
+    # pass 2: per-kernel device times with the library's per-launch events
+    clocks.set_label(f"{name}/kernels")
+    binding.mla_profile_begin()
+    for i in range(steps):
+        l2_flush()
+        step.run()
+    torch.cuda.synchronize()
+    prof = binding.mla_profile_end()
+    clocks.set_label(None)
     barrier(world)
     torch.cuda.synchronize()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, stops)]
-    total_ms = sum(step_ms)
-    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = max_over_ranks(sum(step_ms), world) / steps
     status = binding.mla_get_device_status()
     if status != 0:
-        raise RuntimeError(f"device status {binding.mla_status_string(status)}")
+        raise RuntimeError(f"{name}: device status {binding.mla_status_string(status)}")
+    del flush, flush_rd
 
-    # ---- end to end through the same C ABI with host buffers
-    e2e = None
-    if not args.no_e2e:
-        e2e = e2e_measure(args, w, step, torch, binding, acc, world)
-
-    ms_per_step = total_ms / args.steps
-    kv_gbs = acc["kv_bytes"] * world / (ms_per_step * 1e-3) / 1e9
     peaks, peak_kind = load_peaks()
     dom = max((k for k in prof if k.startswith("mla_fwd")), key=lambda k: prof[k][1])
     launches, dom_ms = prof.get(dom, (0, 0.0))
-    dom_avg_ms = dom_ms / max(launches, 1)
+    dom_prof_ms = dom_ms / max(launches, 1)
+    per_step_launches = sum(v[0] for v in prof.values()) / steps
+    # the kernel's time: its own events, capped at the step that holds it; a step of one
+    # kernel is that kernel
+    kernel_ms = ms_per_step if per_step_launches <= 1 else min(dom_prof_ms, ms_per_step)
     # the roofline is the dominant (attention) kernel's: its own algorithmic bytes and
     # flops, which leave out the W_UV weights and projection of a --wuv step (the
     # combine does those)
     kacc = algorithmic(w, mask_gather=args.mask_gather) if args.wuv else acc
-    tensor_bound = kacc["flops"] / kacc["bytes"] > peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if tensor_bound:
-        achieved = kacc["flops"] / (dom_avg_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
-    else:
-        achieved = kacc["bytes"] / (dom_avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s"}
-    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
-    roof["traffic"] = (args.traffic if args.traffic is not None
-                       else measured_traffic(workload_name(args)))
-    roof["peak_source"] = f"{peak_kind} (MEASURED_PEAKS.json)" if peak_kind == "measured" else \
-        "fallback (profiling recipe)"
+    roof = roofline_of(kacc, kernel_ms, peaks, peak_kind, measured_traffic(
+        name + ("+wuv" if args.wuv else "") + ("+mask_gather" if args.mask_gather else "")
+        + ("+dk512" if args.head_dim == 512 else "")))
     roof["kernel"] = dom
-    roof["kernel_avg_us"] = round(dom_avg_ms * 1e3, 3)
+    roof["kernel_us"] = round(kernel_ms * 1e3, 3)
+    roof["kernel_avg_us_events"] = round(dom_prof_ms * 1e3, 3)
     roof["algorithmic_bytes_per_launch"] = kacc["bytes"]
     roof["algorithmic_flops_per_launch"] = kacc["flops"]
+    res = {
+        "us_per_call": round(ms_per_step * 1e3, 3),
+        "ms_per_step": round(ms_per_step, 6),
+        "kv_gbs": round(acc["kv_bytes"] * world / (ms_per_step * 1e-3) / 1e9, 2),
+        "tokens_per_s": round(w.n_seq * w.n_q * world / (ms_per_step * 1e-3), 1),
+        "steps": steps,
+        "roofline": roof,
+        "kernels": {k: {"launches": v[0], "avg_us": round(1e3 * v[1] / max(v[0], 1), 3)}
+                    for k, v in prof.items()},
+        "gpu_launches": int(sum(v[0] for v in prof.values())),
+        "clocks_mhz": {"step_pass": clocks.median(f"{name}/step"),
+                       "kernel_pass": clocks.median(f"{name}/kernels")},
+    }
+    return res, acc, step
+
+
+def gpu_arm(args, rank, world):
+    import torch
+
+    from mla_flash_attention_attn_b200 import binding
+
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    binding.load()
+    others = [] if (args.only or args.wuv or args.mask_gather or args.head_dim != 576) else \
+        [n for n in W.WORKLOAD_ORDER if n != args.workload]
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        w = make_workload(args)
+        head, acc, step = measure(args, w, args.workload, torch, binding, clocks, world,
+                                  args.steps, headline=True)
+        if args.traffic is not None:
+            head["roofline"]["traffic"] = args.traffic
+        # ---- end to end through the same C ABI with host buffers
+        e2e = None
+        if not args.no_e2e:
+            e2e = e2e_measure(args, w, step, torch, binding, acc, world)
+        del step
+        torch.cuda.empty_cache()
+        cfgs = {}
+        for name in others:
+            wo = W.make(name)
+            # a short step gets the requested step count; a long one (the prefill chunk)
+            # enough steps for the clock sampler to see it under load
+            n = args.steps if name != "prefill_chunk" else max(args.steps, args.prefill_steps)
+            r, acc_o, st = measure(args, wo, name, torch, binding, clocks, world, n)
+            r["config"] = config_of(wo, name, world)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                r["cpu_baseline"] = oracle_throughput(wo, acc_o, args.cpu_budget_configs_s)
+            cfgs[name] = r
+            del st
+            torch.cuda.empty_cache()
+
     result = {
         "metric": METRIC,
-        "value": round(kv_gbs, 2),
+        "value": head["kv_gbs"],
         "unit": "GB/s",
-        "us_per_call": round(ms_per_step * 1e3, 3),
-        "tokens_per_s": round(w.n_seq * w.n_q * world / (ms_per_step * 1e-3), 1),
+        "us_per_call": head["us_per_call"],
+        "tokens_per_s": head["tokens_per_s"],
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 6),
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f16",
         "data": "synthetic (seeded PCG64; DeepSeek-V3/V2-Lite cache geometry, random values)",
-        "config": {"workload": workload_name(args),
-                   "n_seq": w.n_seq, "n_q": w.n_q,
-                   "n_head": w.n_head, "n_kv": w.n_kv,
-                   "kv_type": "q8_0" if w.kv_type else "f16",
-                   "kv_len": [int(x) for x in w.kv_len][:16],
-                   "parallelism": f"replicas x{world}",
-                   "l2": "flushed between timed steps (256 MiB written, then 256 MiB read; outside "
-                         "the events)"},
-        "roofline": roof,
+        "config": config_of(w, workload_name(args), world),
+        "roofline": head["roofline"],
         "e2e": e2e,
-        "gpu_launches": int(sum(v[0] for v in prof.values())),
-        "kernels": {k: {"launches": v[0], "total_ms": round(v[1], 4)} for k, v in prof.items()},
-        "kernel_times": "per-launch CUDA events in a second pass of the same steps",
+        "gpu_launches": head["gpu_launches"],
+        "kernels": head["kernels"],
+        "kernel_times": "per-launch CUDA events in a second pass of the same steps, capped at "
+                        "the step time",
         "clocks": clocks.summary(),
+        "clocks_mhz_by_pass": head["clocks_mhz"],
+        "configs": cfgs,
         "impl": "ours",
     }
     return result, w
@@ -476,9 +560,7 @@ def reference_arm(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded PCG64)",
-        "config": {"workload": args.workload,
-                   "n_seq": w.n_seq, "n_q": w.n_q,
-                   "n_head": w.n_head, "n_kv": w.n_kv, "parallelism": "host cores"},
+        "config": config_of(w, args.workload, world),
         "impl": "reference", "cpu_baseline": cpu,
         "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -521,12 +603,34 @@ def init_ranks(args):
     return rank, world
 
 
+def free_port():
+    import socket
+
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        return sock.getsockname()[1]
+
+
+def launch_ranks(n, argv):
+    """Run this same command as n ranks under torch.distributed.run on 127.0.0.1 (one
+    process per GPU) and return its exit status."""
+    import subprocess
+
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1",
+           "--master-port", str(free_port()), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.WORKLOAD_ORDER)
+    ap.add_argument("--only", action="store_true",
+                    help="time the --workload alone (no per-config measurements)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--wuv", action="store_true",
@@ -539,7 +643,10 @@ def main(argv=None):
                     help="512: the DK = DV = 512 head shape (the workload without its RoPE "
                          "columns; f16 cache)")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--prefill-steps", type=int, default=60,
+                    help="least number of timed steps of the prefill chunk in `configs`")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--cpu-budget-configs-s", type=float, default=3.0)
     ap.add_argument("--ref-budget-s", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic", type=float, default=None,
@@ -547,6 +654,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
     if args.wuv and args.impl == "reference":
         ap.error("--wuv applies to --impl ours (the oracle arm times the attention only)")
     if args.head_dim != 576 and args.impl == "reference":
@@ -555,6 +664,12 @@ def main(argv=None):
         ap.error("--mask-gather applies to --impl ours (the oracle arm runs the unfused chain)")
     if args.wuv:
         args.no_cpu_baseline = True  # the oracle baseline times the attention only
+    if "WORLD_SIZE" not in os.environ:
+        if args.gpus > 1:
+            # one process per GPU: start the ranks under the launcher
+            sys.exit(launch_ranks(args.gpus, argv))
+    elif int(os.environ["WORLD_SIZE"]) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started {os.environ['WORLD_SIZE']} ranks")
     rank, world = init_ranks(args)
     try:
         if args.impl == "reference":

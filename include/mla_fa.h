@@ -211,7 +211,9 @@ int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, vo
  *   MLA_ERR_WORKSPACE before launching anything.
  * - The first call on a device looks up the array's device address once
  *   (cudaGetSymbolAddress) with that device current; make that first call before
- *   any stream capture.
+ *   any stream capture. The address is kept for the life of the process, so do
+ *   not use this call after cudaDeviceReset or from another context on the same
+ *   device (either one reloads the module and moves the array).
  * - All calls share the one array and it keeps the last call's contents. Nothing
  *   in it needs to start at zero: each call writes every partial it reads. Calls
  *   that overlap on the GPU (on different streams, or different host threads

@@ -160,10 +160,82 @@ def _host_i32(arr):
     return (ctypes.c_int32 * len(vals))(*vals)
 
 
+def _check_tensor(t, name, dtype, shape, device, row_contiguous=True):
+    """Raise ValueError unless t is a tensor on `device` with this dtype and shape (None in
+    `shape` matches any size) whose innermost dimension is dense and, with
+    row_contiguous, whose every dimension below the first is dense as well (the C ABI
+    takes one stride per sequence and none inside a sequence)."""
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if t.dim() != len(shape) or any(s is not None and t.shape[i] != s for i, s in enumerate(shape)):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {shape}")
+    if t.numel() == 0:
+        raise ValueError(f"{name} is empty")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name} must be dense in its last dimension")
+    if row_contiguous:
+        expect = 1
+        for i in range(t.dim() - 1, 0, -1):
+            if t.shape[i] != 1 and t.stride(i) != expect:
+                raise ValueError(f"{name} must be contiguous within its first dimension")
+            expect *= t.shape[i]
+
+
+def check_args(q, kcache, kv_type, mask, out, kv_len=None, idx=None, idx_count=None, wv=None,
+               out_proj=None, sinks=None, alibi_slopes=None, out_lse=None):
+    """The checks the C ABI cannot make, since it sees pointers and not buffers: every
+    tensor is a CUDA tensor on q's device, with the dtype and size the header states for
+    it. A host tensor, a wrong dtype or a short buffer would otherwise reach a kernel as a
+    bad address. Raises ValueError."""
+    import torch
+
+    if q.dim() != 4:
+        raise ValueError("q must be [n_seq][n_q][n_head][576 or 512]")
+    if not q.is_cuda:
+        raise ValueError("q must be a CUDA tensor")
+    dev = q.device
+    n_seq, n_q, n_head, dk = q.shape
+    if dk not in (DK, DV):
+        raise ValueError("q must end in 576 (or 512: the DK = DV = 512 head shape)")
+    _check_tensor(q, "q", torch.float16, (n_seq, n_q, n_head, dk), dev)
+    if int(kv_type) == KV_Q8_0:
+        _check_tensor(kcache, "kcache", torch.uint8, (n_seq, None, Q8_ROW_BYTES), dev,
+                      row_contiguous=False)
+    else:
+        _check_tensor(kcache, "kcache", torch.float16, (n_seq, None, dk), dev,
+                      row_contiguous=False)
+    if kcache.stride(1) != kcache.shape[2] or kcache.stride(0) % kcache.stride(1):
+        raise ValueError("kcache rows must be dense and sequences a whole number of rows apart")
+    n_kv = kcache.shape[1]
+    if mask is not None:
+        _check_tensor(mask, "mask", torch.float16, (n_seq, n_q, n_kv), dev, row_contiguous=False)
+    if out is not None:
+        _check_tensor(out, "out", torch.float32, (n_seq, n_q, n_head, DV), dev)
+    if kv_len is not None and len(kv_len) != n_seq:
+        raise ValueError("kv_len must hold one length per sequence")
+    if idx is not None:
+        if idx_count is None:
+            raise ValueError("idx needs idx_count")
+        _check_tensor(idx, "idx", torch.int32, (n_seq, None), dev, row_contiguous=False)
+        _check_tensor(idx_count, "idx_count", torch.int32, (n_seq,), dev)
+    if wv is not None:
+        _check_tensor(wv, "wv", torch.float16, (n_head, DV, None), dev)
+        if out_proj is None:
+            raise ValueError("wv needs out_proj")
+        _check_tensor(out_proj, "out_proj", torch.float32, (n_seq, n_q, n_head, wv.shape[2]), dev)
+    for name, t in (("sinks", sinks), ("alibi_slopes", alibi_slopes)):
+        if t is not None:
+            _check_tensor(t, name, torch.float32, (n_head,), dev)
+    if out_lse is not None:
+        _check_tensor(out_lse, "out_lse", torch.float32, (n_seq, n_q, n_head), dev)
+
+
 def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None,
               wv=None, out_proj=None, sinks=None, alibi_slopes=None, softcap=0.0,
               mask_gather=False, out_lse=None):
-    """Fill mla_fa_args from batched torch tensors.
+    """Fill mla_fa_args from batched torch tensors, after check_args.
 
     q [n_seq][n_q][n_head][576] f16; kcache [n_seq][n_kv][576] f16 (or uint8 [..][612]);
     q [..][512] with kcache [..][512] f16 selects the DK = DV = 512 head shape;
@@ -173,6 +245,17 @@ def make_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_c
     the attention variants; mask_gather=True for sparse attention straight from the mask
     (the kernel compacts it, no index list); out_lse fp32 [n_seq][n_q][n_head] for each
     row's natural log-sum-exp. Returns (args, keepalive)."""
+    check_args(q, kcache, kv_type, mask, out, kv_len=kv_len, idx=idx, idx_count=idx_count,
+               wv=wv, out_proj=out_proj, sinks=sinks, alibi_slopes=alibi_slopes,
+               out_lse=out_lse)
+    return marshal_args(q, kcache, kv_type, mask, out, scale, kv_len, idx, idx_count, wv,
+                        out_proj, sinks, alibi_slopes, softcap, mask_gather, out_lse)
+
+
+def marshal_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, idx_count=None,
+                 wv=None, out_proj=None, sinks=None, alibi_slopes=None, softcap=0.0,
+                 mask_gather=False, out_lse=None):
+    """Pointers, sizes and strides of the tensors, with no checks (make_args checks first)."""
     n_seq, n_q, n_head, dk = q.shape
     if dk not in (DK, DV):
         raise ValueError("q must end in 576 (or 512: the DK = DV = 512 head shape)")
@@ -294,12 +377,28 @@ def combine(o_parts, lse_parts, out=None, out_lse=None, stream=None):
 
     if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
         raise ValueError("o_parts and lse_parts must be contiguous")
+    if not o_parts.is_cuda:
+        raise ValueError("o_parts must be a CUDA tensor")
+    dev = o_parts.device
     n_parts = o_parts.shape[0]
+    if o_parts.dim() < 2 or o_parts.shape[-1] != DV or o_parts.numel() == 0:
+        raise ValueError("o_parts must be [n_parts][...][512]")
     o = o_parts.view(n_parts, -1, DV)
     rows = o.shape[1]
+    _check_tensor(o, "o_parts", torch.float32, (n_parts, rows, DV), dev)
+    if lse_parts.numel() != n_parts * rows:
+        raise ValueError(f"lse_parts must hold n_parts x rows = {n_parts * rows} values")
     lse = lse_parts.view(n_parts, rows)
+    _check_tensor(lse, "lse_parts", torch.float32, (n_parts, rows), dev)
     if out is None:
-        out = torch.empty((rows, DV), dtype=torch.float32, device=o_parts.device)
+        out = torch.empty((rows, DV), dtype=torch.float32, device=dev)
+    if not out.is_contiguous() or out.numel() != rows * DV:
+        raise ValueError(f"out must be contiguous with rows x 512 = {rows * DV} values")
+    _check_tensor(out.view(rows, DV), "out", torch.float32, (rows, DV), dev)
+    if out_lse is not None:
+        if not out_lse.is_contiguous() or out_lse.numel() != rows:
+            raise ValueError(f"out_lse must be contiguous with {rows} values")
+        _check_tensor(out_lse.view(rows), "out_lse", torch.float32, (rows,), dev)
     _check(load().mla_fa_combine(_ptr(o), _ptr(lse), n_parts, rows, _ptr(out), _ptr(out_lse),
                                  _stream_ptr(stream)), "mla_fa_combine")
     return out

@@ -191,12 +191,43 @@ def test_binding_takes_the_head_width_from_q():
         q = torch.zeros((2, 1, 4, dk), dtype=torch.float16)
         k = torch.zeros((2, 8, dk), dtype=torch.float16)
         out = torch.zeros((2, 1, 4, 512), dtype=torch.float32)
-        a, _ = binding.make_args(q, k, 0, None, out, 0.1)
+        a, _ = binding.marshal_args(q, k, 0, None, out, 0.1)
         assert a.head_dim == dk and a.q_seq_stride == 4 * dk and a.k_seq_stride == 8
     with pytest.raises(ValueError):
-        binding.make_args(torch.zeros((1, 1, 4, 300), dtype=torch.float16),
-                          torch.zeros((1, 8, 300), dtype=torch.float16), 0, None,
-                          torch.zeros((1, 1, 4, 512)), 0.1)
+        binding.marshal_args(torch.zeros((1, 1, 4, 300), dtype=torch.float16),
+                             torch.zeros((1, 8, 300), dtype=torch.float16), 0, None,
+                             torch.zeros((1, 1, 4, 512)), 0.1)
+
+
+def test_binding_refuses_host_tensors():
+    # a host pointer handed to a kernel would be a bad device address
+    import torch
+
+    q = torch.zeros((1, 1, 4, 576), dtype=torch.float16)
+    k = torch.zeros((1, 8, 576), dtype=torch.float16)
+    out = torch.zeros((1, 1, 4, 512), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.make_args(q, k, 0, None, out, 0.1)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.combine(torch.zeros((2, 8, 512)), torch.zeros((2, 8)))
+
+
+@pytest.mark.parametrize("bad", ["dtype", "shape", "strided", "device", "empty"])
+def test_binding_tensor_checks(bad):
+    # the per-tensor check that make_args and combine apply (run here on host tensors
+    # against the host device; on a GPU the device is q's)
+    import torch
+
+    cpu = torch.device("cpu")
+    good = torch.zeros((2, 3, 4, 512), dtype=torch.float32)
+    binding._check_tensor(good, "out", torch.float32, (2, 3, 4, 512), cpu)
+    t = {"dtype": good.half(),
+         "shape": torch.zeros((2, 3, 4, 256), dtype=torch.float32),
+         "strided": torch.zeros((2, 3, 8, 512), dtype=torch.float32)[:, :, ::2],
+         "device": torch.zeros((2, 3, 4, 512), dtype=torch.float32, device="meta"),
+         "empty": torch.zeros((2, 0, 4, 512), dtype=torch.float32)}[bad]
+    with pytest.raises(ValueError):
+        binding._check_tensor(t, "out", torch.float32, (2, None, 4, 512), cpu)
 
 
 # ---- the split plan, on the host alone (mla_fa_plan_for_sms) -----------------------------

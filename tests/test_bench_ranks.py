@@ -5,7 +5,9 @@ barrier before and after its timed region and the job's time is the maximum
 over ranks. These tests run that plumbing with two CPU processes over gloo on
 127.0.0.1: the barrier and the max-over-ranks reduction, and the reference arm
 under the torch.distributed launcher, where rank 0 alone prints the JSON line
-and the other rank exits 0 without work.
+and the other rank exits 0 without work. `bench.py --gpus 2` without a launcher
+starts the two ranks itself, and a launcher whose rank count differs from --gpus
+is refused.
 """
 import json
 import os
@@ -76,3 +78,26 @@ def test_reference_arm_under_the_launcher_with_two_ranks():
     assert res["config"]["workload"] == "tiny_decode"
     assert res["value"] > 0 and res["cpu_baseline"]["kind"] == "oracle"
     assert res["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_starts_its_own_ranks_without_a_launcher():
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+           "--warmup", "3", "--workload", "tiny_decode", "--ref-budget-s", "1"]
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    env["OMP_NUM_THREADS"] = "2"
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600, env=env)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    res = json.loads(lines[0])
+    assert res["impl"] == "reference" and res["n_gpus"] == 2
+    assert res["config"]["parallelism"] == "replicas x2"
+
+
+def test_bench_refuses_a_rank_count_other_than_gpus():
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--gpus", "3", "--steps", "1",
+           "--warmup", "3", "--workload", "tiny_decode"]
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert p.returncode != 0 and "--gpus 3" in p.stderr

@@ -3,7 +3,8 @@
 Each test checks the oracle against something other than itself: a closed form,
 an explicit numpy float64 matrix route written here, an invariant of softmax
 attention, or brute force on tiny inputs. The pages print no worked example for
-this computation (see tests/golden/README.md), so these are the pins.
+this computation (the one figure they do print, the size of a dense score
+matrix, is pinned by the golden test), so these are the pins.
 """
 import itertools
 import math
@@ -241,9 +242,7 @@ def test_compaction_brute_force_all_16_cell_masks():
         keep = bits[i]
         row = np.where(keep, np.float16(0), NEG).astype(np.float16)
         got = oracle.compact(row)
-        if i % 4096 == 0 or i in (1, 2, 3, 0xFFFF):
-            assert np.array_equal(got, np.nonzero(keep)[0].astype(np.int32))
-        assert len(got) == int(keep.sum())
+        assert np.array_equal(got, np.nonzero(keep)[0].astype(np.int32)), i
 
 
 def test_compaction_keep_rule_only_minus_inf_dropped():

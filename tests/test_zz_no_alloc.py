@@ -6,8 +6,10 @@ every byte, or a decode loop that cannot take the synchronisation cudaMalloc
 may cause. mla_fa_forward_noalloc serves them by keeping its split-KV partials
 in a static device array. These tests call it through the C ABI and check, on
 two calls in a row with different inputs, that it gives what the allocating
-entry point mla_fa_forward_ex gives, and that a pass needing more scratch than
-the array holds is refused before any launch.
+entry point mla_fa_forward_ex gives and what the fp64 oracle gives, that the
+other users of the array (the mask gather's cell lists and the fused
+projection's partials) survive back-to-back calls of different shapes, and that
+a pass needing more scratch than the array holds is refused before any launch.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes on its own in a fresh process.
@@ -17,6 +19,7 @@ import ctypes
 import numpy as np
 import pytest
 
+import oracle
 from mla_flash_attention_attn_b200 import binding
 from mla_flash_attention_attn_b200 import workloads as W
 
@@ -65,7 +68,54 @@ def test_noalloc_matches_allocating_entry_point_on_two_calls():
         ref = binding.forward(q, k, w.kv_type, m, w.scale, kv_len=w.kv_len)
         torch.cuda.synchronize()
         assert binding.mla_get_device_status() == 0
-        _compare(out_na.cpu().numpy(), ref.cpu().numpy(), f"call {i + 1}")
+        got = out_na.cpu().numpy()
+        _compare(got, ref.cpu().numpy(), f"call {i + 1}")
+        for b in range(w.n_seq):
+            exact = oracle.attention(w.q[b], w.kcache[b], w.kv_type, w.mask[b], w.scale)
+            _compare(got[b].reshape(-1, 512), exact, f"call {i + 1} vs oracle, seq {b}")
+
+
+def test_noalloc_mask_gather_and_projection_back_to_back():
+    # Two more users of the shared array: the mask gather puts each unit's cell list
+    # after the partials, and the fused projection makes every sequence write partials.
+    # Back-to-back calls of different shapes leave stale contents behind; each call must
+    # still read only what it wrote.
+    import torch
+
+    binding.load()
+    dev = torch.device("cuda")
+    # the mask gather on a sparse f16 mask (two sizes, so the lists move)
+    for i, (n_kv, seed) in enumerate(((6000, 5), (2500, 6))):
+        w = W.make("v2lite_decode", seed=seed, n_kv=n_kv, n_head=64, n_pad=0)
+        rng = np.random.default_rng(seed)
+        keep = rng.random(n_kv) < 0.2
+        keep[-3:] = True
+        w.mask[0, 0] = np.where(keep, np.float16(0), np.float16(-np.inf))
+        q, k, m = _inputs(w, torch)
+        out_na = torch.full(w.q.shape[:3] + (512,), float("nan"), dtype=torch.float32, device=dev)
+        args, keep_alive = binding.make_args(q, k, w.kv_type, m, out_na, w.scale, mask_gather=True)
+        assert binding.mla_fa_workspace_size(args) <= binding.NOALLOC_SCRATCH_BYTES
+        binding.mla_fa_forward_noalloc(args)
+        ref = binding.forward(q, k, w.kv_type, m, w.scale, mask_gather=True)
+        torch.cuda.synchronize()
+        assert binding.mla_get_device_status() == 0
+        _compare(out_na.cpu().numpy(), ref.cpu().numpy(), f"mask gather call {i + 1}")
+    # the fused projection (two batch shapes)
+    for i, w in enumerate((W.make("v3_batched_decode", seed=8, n_seq=2, n_head=32, n_kv=2000,
+                                  len_lo=900, len_hi=2000),
+                           W.make("v3_batched_decode", seed=9, n_seq=3, n_head=16, n_kv=1500,
+                                  len_lo=300, len_hi=1500))):
+        q, k, m = _inputs(w, torch)
+        wv = torch.from_numpy(W.wv_random(n_head=w.n_head)).to(dev)
+        op_na = torch.full(w.q.shape[:3] + (128,), float("nan"), dtype=torch.float32, device=dev)
+        args, keep_alive = binding.make_args(q, k, w.kv_type, m, None, w.scale, kv_len=w.kv_len,
+                                             wv=wv, out_proj=op_na)
+        assert binding.mla_fa_workspace_size(args) <= binding.NOALLOC_SCRATCH_BYTES
+        binding.mla_fa_forward_noalloc(args)
+        ref = binding.forward_proj(q, k, w.kv_type, m, w.scale, wv, kv_len=w.kv_len)
+        torch.cuda.synchronize()
+        assert binding.mla_get_device_status() == 0
+        _compare(op_na.cpu().numpy(), ref.cpu().numpy(), f"projection call {i + 1}")
 
 
 def test_noalloc_refuses_a_pass_larger_than_its_scratch():
