@@ -61,6 +61,12 @@ DEFAULT_WORKLOAD = "v3_batched_decode"
 
 # ----------------------------------------------------------------------------- accounting
 def algorithmic(w, kept_cells=None, wuv=False, mask_gather=False):
+    if isinstance(w, W.HeadsWorkload):
+        return algorithmic_heads(w)
+    return algorithmic_mla(w, kept_cells, wuv, mask_gather)
+
+
+def algorithmic_mla(w, kept_cells=None, wuv=False, mask_gather=False):
     """Algorithmic bytes and flops of one step, split partials excluded.
 
     bytes = cache rows attended x row bytes + Q + mask cells read + output;
@@ -127,12 +133,36 @@ def workload_name(args):
     """The workload as the step runs it: the cache geometry plus the fused options."""
     return (args.workload + ("+wuv" if args.wuv else "")
             + ("+mask_gather" if args.mask_gather else "")
-            + ("+dk512" if args.head_dim == 512 else ""))
+            + ("+dk512" if args.head_dim == 512 else ""))  # heads_* names carry their shape
+
+
+HEADS_WORKLOADS = {"heads_prefill": W.heads_prefill, "heads_decode": W.heads_decode}
+
+
+def algorithmic_heads(w):
+    """Algorithmic bytes and flops of one step of the DK = 192 / DV = 128 head shape:
+    bytes = K and V rows attended (every KV head: 384 + 256 bytes per cell) + Q + mask
+    cells read + output; flops = 2 * n_head * (192 + 128) per (query token, kept key)."""
+    keep = ~np.isneginf(w.mask) if w.mask is not None else None
+    rows_attended = pairs = mask_bytes = 0
+    for b in range(w.n_seq):
+        L = int(w.kv_len[b])
+        kept = [L] * w.n_q if keep is None else [int(keep[b, t, :L].sum()) for t in range(w.n_q)]
+        rows_attended += max(kept)
+        pairs += sum(kept)
+        mask_bytes += w.n_q * L * 2 if w.mask is not None else 0
+    kv_bytes = rows_attended * w.n_kv_head * (192 + 128) * 2
+    out_bytes = w.n_seq * w.n_q * w.n_head * 128 * 4
+    return {"kv_bytes": kv_bytes, "bytes": kv_bytes + w.q.size * 2 + mask_bytes + out_bytes,
+            "flops": 2.0 * w.n_head * (192 + 128) * pairs}
 
 
 def make_workload(args):
     """The named workload; with --head-dim 512 the same one with the 64 RoPE columns
-    of q and of the cache dropped (the DK = DV = 512 head shape, f16 cache)."""
+    of q and of the cache dropped (the DK = DV = 512 head shape, f16 cache); the heads_*
+    workloads are the DK = 192 / DV = 128 head shape."""
+    if args.workload in HEADS_WORKLOADS:
+        return HEADS_WORKLOADS[args.workload]()
     w = W.make(args.workload)
     if args.head_dim == 512:
         if w.kv_type != W.KV_F16:
@@ -266,17 +296,52 @@ class Step:
         self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
         self.ws_used = need > 0
 
+    def inputs(self):
+        """(device tensor, host array) of every input a step reads."""
+        ins = [(self.q, self.w.q), (self.k, self.w.kcache)]
+        return ins + ([(self.mask, self.w.mask)] if self.mask is not None else [])
+
     def run(self, stream=None):
         if self.idx is not None:
             self.b.mla_compact_mask_ex(self.mask[:, 0, :], self.idx, self.cnt, self.cws, stream)
         self.b.mla_fa_forward_ex(self.args, self.ws if self.ws_used else None, stream)
 
 
+class HeadsStep:
+    """Device-resident inputs and the hot path of the DK = 192 / DV = 128 head shape."""
+
+    def __init__(self, w, torch, binding):
+        self.w = w
+        self.b = binding
+        dev = torch.device("cuda")
+        self.q = torch.from_numpy(w.q).to(dev)
+        self.k = torch.from_numpy(w.k).to(dev)
+        self.v = torch.from_numpy(w.v).to(dev)
+        self.mask = torch.from_numpy(w.mask).to(dev) if w.mask is not None else None
+        self.out = torch.empty(w.q.shape[:3] + (128,), dtype=torch.float32, device=dev)
+        self.args, self._keep = binding.make_heads_args(self.q, self.k, self.v, self.mask,
+                                                        self.out, w.scale,
+                                                        [int(x) for x in w.kv_len])
+        need = binding.mla_fa_workspace_size(self.args)
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+        self.ws_used = need > 0
+
+    def inputs(self):
+        """(device tensor, host array) of every input a step reads."""
+        ins = [(self.q, self.w.q), (self.k, self.w.k), (self.v, self.w.v)]
+        return ins + ([(self.mask, self.w.mask)] if self.mask is not None else [])
+
+    def run(self, stream=None):
+        self.b.mla_fa_forward_ex(self.args, self.ws if self.ws_used else None, stream)
+
+
 def config_of(w, name, world):
     """The workload's description as it appears in both arms' JSON lines."""
+    heads = isinstance(w, W.HeadsWorkload)
+    extra = {"n_kv_head": w.n_kv_head, "v_head_dim": 128} if heads else {}
     return {"workload": name, "n_seq": w.n_seq, "n_q": w.n_q, "n_head": w.n_head,
-            "n_kv": w.n_kv, "head_dim": int(w.q.shape[-1]),
-            "kv_type": "q8_0" if w.kv_type else "f16",
+            "n_kv": w.n_kv, "head_dim": int(w.q.shape[-1]), **extra,
+            "kv_type": "q8_0" if (not heads and w.kv_type) else "f16",
             "kv_len": [int(x) for x in w.kv_len][:16],
             "parallelism": f"replicas x{world}",
             "l2": "flushed between timed steps (256 MiB written, then 256 MiB read; outside "
@@ -306,7 +371,8 @@ def measure(args, w, name, torch, binding, clocks, world, steps, headline=False)
     """Time `steps` steps of workload w (after args.warmup untimed ones), then the same
     steps again with per-kernel events. Returns the measurement and the Step."""
     acc = algorithmic(w, wuv=args.wuv, mask_gather=args.mask_gather)
-    step = Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather)
+    step = HeadsStep(w, torch, binding) if isinstance(w, W.HeadsWorkload) else \
+        Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather)
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -461,9 +527,7 @@ def gpu_arm(args, rank, world):
 def e2e_measure(args, w, step, torch, binding, acc, world):
     """Same hot path, with the inputs copied from pinned host memory each step and the
     output copied back, all inside the CUDA-event timed region."""
-    hq = torch.from_numpy(w.q).pin_memory()
-    hk = torch.from_numpy(w.kcache).pin_memory()
-    hm = torch.from_numpy(w.mask).pin_memory() if w.mask is not None else None
+    pairs = [(dev_t, torch.from_numpy(host).pin_memory()) for dev_t, host in step.inputs()]
     hout = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
     stream = torch.cuda.current_stream()
     n = max(1, min(args.steps, args.e2e_steps))
@@ -473,17 +537,15 @@ def e2e_measure(args, w, step, torch, binding, acc, world):
         s, e = ev[i - 1] if i else (None, None)
         if s is not None:
             s.record(stream)
-        step.q.copy_(hq, non_blocking=True)
-        step.k.copy_(hk, non_blocking=True)
-        if hm is not None:
-            step.mask.copy_(hm, non_blocking=True)
+        for dev_t, host_t in pairs:
+            dev_t.copy_(host_t, non_blocking=True)
         step.run()
         hout.copy_(step.out, non_blocking=True)
         if e is not None:
             e.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev), world) / n
-    h2d = hq.numel() * 2 + hk.numel() * hk.element_size() + (hm.numel() * 2 if hm is not None else 0)
+    h2d = sum(h.numel() * h.element_size() for _, h in pairs)
     return {"value": round(acc["kv_bytes"] * world / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "us_per_call": round(ms * 1e3, 2), "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(hout.numel() * 4), "steps": n}
@@ -512,7 +574,18 @@ def oracle_throughput(w, acc, budget_s):
 
 
 def _oracle_rows(oracle, w, n):
-    """Compute n query rows spread over the sequences (sparse: over the kept indices)."""
+    """Compute n query rows spread over the sequences (sparse: over the kept indices;
+    the 192 / 128 head shape: whole tokens, every head)."""
+    if isinstance(w, W.HeadsWorkload):
+        toks = max(1, n // w.n_head)
+        per_seq = max(1, toks // w.n_seq)
+        for b in range(w.n_seq):
+            L = int(w.kv_len[b])
+            for t in np.linspace(0, w.n_q - 1, min(per_seq, w.n_q)).astype(int):
+                oracle.attention_heads(w.q[b, t:t + 1], w.k[b, :L], w.v[b, :L],
+                                       w.mask[b, t:t + 1, :L] if w.mask is not None else None,
+                                       w.scale)
+        return
     per_seq = max(1, n // w.n_seq)
     done = 0
     for b in range(w.n_seq):
@@ -628,7 +701,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=W.WORKLOAD_ORDER + list(HEADS_WORKLOADS))
     ap.add_argument("--only", action="store_true",
                     help="time the --workload alone (no per-config measurements)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -639,9 +713,11 @@ def main(argv=None):
     ap.add_argument("--mask-gather", action="store_true",
                     help="masked workloads: sparse attention straight from the mask (the "
                          "compaction fused into the attention kernel, no index list)")
-    ap.add_argument("--head-dim", type=int, default=576, choices=[576, 512],
+    ap.add_argument("--head-dim", type=int, default=576, choices=[576, 512, 192],
                     help="512: the DK = DV = 512 head shape (the workload without its RoPE "
-                         "columns; f16 cache)")
+                         "columns; f16 cache); 192: the DK = 192 / DV = 128 head shape (a K "
+                         "and a V per KV head; the heads_prefill workload unless a heads_* "
+                         "workload is named)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--prefill-steps", type=int, default=60,
                     help="least number of timed steps of the prefill chunk in `configs`")
@@ -664,6 +740,14 @@ def main(argv=None):
         ap.error("--mask-gather applies to --impl ours (the oracle arm runs the unfused chain)")
     if args.wuv:
         args.no_cpu_baseline = True  # the oracle baseline times the attention only
+    if args.head_dim == 192 and args.workload not in HEADS_WORKLOADS:
+        args.workload = "heads_prefill"
+    if args.workload in HEADS_WORKLOADS:
+        if args.impl == "reference":
+            ap.error("the reference arm times the MLA workloads")
+        if args.wuv or args.mask_gather:
+            ap.error("the 192 / 128 head shape takes neither --wuv nor --mask-gather")
+        args.head_dim = 192
     if "WORLD_SIZE" not in os.environ:
         if args.gpus > 1:
             # one process per GPU: start the ranks under the launcher

@@ -51,6 +51,8 @@ extern "C" {
 #define MLA_Q8_0_ROW_BYTES 612 /* q8_0: 18 blocks x {f16 d; int8 q[32]}         */
 #define MLA_MAX_HEADS 128
 #define MLA_PROJ_DIM 128      /* output width of the fused value up-projection   */
+#define MLA_HEADS_DK 192      /* head shape with a K and a V per KV head: K width */
+#define MLA_HEADS_DV 128      /*   ... and V width                                 */
 
 typedef enum {
   MLA_KV_F16 = 0,  /* row = 576 f16 (1152 bytes) */
@@ -130,7 +132,23 @@ typedef enum {
  *         Metal FA kernel, PR #29570): q and the cache rows are 512 wide and V is the
  *         whole row. f16 cache only (else MLA_ERR_UNSUPPORTED); dense or index-list
  *         attention, with sinks, out_lse and wv as above; softcap, ALiBi and mask_gather
- *         MLA_ERR_UNSUPPORTED. Other values MLA_ERR_SHAPE
+ *         MLA_ERR_UNSUPPORTED. MLA_HEADS_DK (192): the DK = 192 / DV = 128 head shape of
+ *         the same list, read as attention with a K and a V per KV head (below).
+ *         Other values MLA_ERR_SHAPE
+ *
+ * The DK = 192 / DV = 128 shape (head_dim = MLA_HEADS_DK): n_kv_head KV heads, query
+ * head h reads KV head h / (n_head / n_kv_head) (n_kv_head = n_head: multi-head
+ * attention; fewer: grouped heads sharing a K and a V); per query row
+ *     S[j] = scale * dot(q[t,h,0:192], k[j,kvh,0:192]) + mask[t,j]
+ *     out[t,h,0:128] = sum_j softmax(S)[j] * v[j,kvh,0:128]
+ * q       f16, element (b, t, h, c) at q[b*q_seq_stride + (t*n_head + h)*192 + c]
+ * kcache  f16 K, element (b, j, kvh, c) at kcache[(b*k_seq_stride + j)*n_kv_head*192 + kvh*192 + c]
+ * v       f16 V, element (b, j, kvh, d) at v[(b*v_seq_stride + j)*n_kv_head*128 + kvh*128 + d]
+ * out     fp32, element (b, t, h, d) at out[b*out_seq_stride + (t*n_head + h)*128 + d]
+ * mask and kv_len as above (the mask shared by the heads of a token). f16 only; idx,
+ * mask_gather, wv, sinks, ALiBi, softcap and out_lse MLA_ERR_UNSUPPORTED. q, kcache, v
+ * and out 16-byte aligned. Other head widths take v = NULL and n_kv_head = 0.
+ * v_seq_stride rows between sequences of v (0 = n_kv); n_kv_head must divide n_head.
  * A stride of 0 means "dense" (the natural value for the given sizes).
  */
 typedef struct mla_fa_args {
@@ -162,7 +180,11 @@ typedef struct mla_fa_args {
   float softcap;            /* > 0 enables the logit softcap                   */
   int mask_gather;          /* 1: gather the mask's kept cells (no idx)        */
   float* out_lse;           /* DEVICE, optional: natural log-sum-exp per row   */
-  int head_dim;             /* 0 / MLA_DK: 576-wide heads; MLA_DV: 512         */
+  int head_dim;             /* 0 / MLA_DK: 576-wide heads; MLA_DV: 512;
+                               MLA_HEADS_DK: 192 (K and V per KV head)          */
+  const void* v;            /* DEVICE f16, head_dim = MLA_HEADS_DK only        */
+  int64_t v_seq_stride;     /* rows; 0 = n_kv                                  */
+  int n_kv_head;            /* head_dim = MLA_HEADS_DK only: KV heads          */
 } mla_fa_args;
 
 /* Forward pass with the sizes of the single-sequence call:

@@ -67,6 +67,9 @@ class mla_fa_args(ctypes.Structure):
         ("mask_gather", ctypes.c_int),
         ("out_lse", ctypes.c_void_p),
         ("head_dim", ctypes.c_int),
+        ("v", ctypes.c_void_p),
+        ("v_seq_stride", ctypes.c_int64),
+        ("n_kv_head", ctypes.c_int),
     ]
 
 
@@ -291,6 +294,74 @@ def marshal_args(q, kcache, kv_type, mask, out, scale, kv_len=None, idx=None, id
         a.idx_count = idx_count.data_ptr()
         a.idx_seq_stride = idx.stride(0)
     return a, keep
+
+
+HEADS_DK = 192
+HEADS_DV = 128
+
+
+def make_heads_args(q, k, v, mask, out, scale, kv_len=None):
+    """mla_fa_args for the DK = 192 / DV = 128 head shape (a K and a V per KV head):
+    q [n_seq][n_q][n_head][192] f16, k [n_seq][n_kv][n_kv_head][192] f16,
+    v [n_seq][n_kv][n_kv_head][128] f16, mask [n_seq][n_q][n_kv] f16 or None,
+    out [n_seq][n_q][n_head][128] fp32. Checks the tensors first (device, dtype, size).
+    Returns (args, keepalive)."""
+    import torch
+
+    if q.dim() != 4 or not q.is_cuda:
+        raise ValueError("q must be a CUDA tensor [n_seq][n_q][n_head][192]")
+    dev = q.device
+    n_seq, n_q, n_head, _ = q.shape
+    _check_tensor(q, "q", torch.float16, (n_seq, n_q, n_head, HEADS_DK), dev)
+    if k.dim() != 4:
+        raise ValueError("k must be [n_seq][n_kv][n_kv_head][192]")
+    n_kv, n_kv_head = k.shape[1], k.shape[2]
+    if n_kv_head < 1 or n_head % n_kv_head:
+        raise ValueError("n_kv_head must divide n_head")
+    for name, t, w in (("k", k, HEADS_DK), ("v", v, HEADS_DV)):
+        _check_tensor(t, name, torch.float16, (n_seq, n_kv, n_kv_head, w), dev, row_contiguous=False)
+        if t.stride(2) != w or t.stride(1) != n_kv_head * w or t.stride(0) % t.stride(1):
+            raise ValueError(f"{name} rows must be dense and sequences a whole number of rows apart")
+    if mask is not None:
+        _check_tensor(mask, "mask", torch.float16, (n_seq, n_q, n_kv), dev, row_contiguous=False)
+    _check_tensor(out, "out", torch.float32, (n_seq, n_q, n_head, HEADS_DV), dev)
+    if kv_len is not None and len(kv_len) != n_seq:
+        raise ValueError("kv_len must hold one length per sequence")
+    a = mla_fa_args()
+    a.q, a.kcache, a.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    a.kcache_type = KV_F16
+    a.mask = None if mask is None else mask.data_ptr()
+    a.out = out.data_ptr()
+    a.n_seq, a.n_q, a.n_head, a.n_kv = n_seq, n_q, n_head, n_kv
+    a.n_kv_head = n_kv_head
+    a.scale = float(scale)
+    a.head_dim = HEADS_DK
+    a.q_seq_stride = q.stride(0)
+    a.k_seq_stride = k.stride(0) // k.stride(1)
+    a.v_seq_stride = v.stride(0) // v.stride(1)
+    if mask is not None:
+        a.mask_seq_stride = mask.stride(0)
+        a.mask_row_stride = mask.stride(1)
+    a.out_seq_stride = out.stride(0)
+    keep = _host_i32(kv_len)
+    a.kv_len = None if keep is None else ctypes.cast(keep, ctypes.c_void_p)
+    return a, keep
+
+
+def forward_heads(q, k, v, mask, scale, out=None, kv_len=None, workspace=None, stream=None):
+    """The DK = 192 / DV = 128 head shape through mla_fa_forward_ex; allocates out and the
+    workspace with torch if absent. Returns out [n_seq][n_q][n_head][128] fp32."""
+    import torch
+
+    if out is None:
+        out = torch.empty(q.shape[:3] + (HEADS_DV,), dtype=torch.float32, device=q.device)
+    args, keep = make_heads_args(q, k, v, mask, out, scale, kv_len)
+    need = mla_fa_workspace_size(args)
+    if need and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    mla_fa_forward_ex(args, workspace if need else None, stream)
+    del keep
+    return out
 
 
 def mla_fa_workspace_size(args) -> int:

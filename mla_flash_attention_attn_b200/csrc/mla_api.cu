@@ -15,6 +15,7 @@
 #include "mla_common.cuh"
 #include "mla_compact.cuh"
 #include "mla_fwd.cuh"
+#include "mla_heads.cuh"
 
 namespace {
 
@@ -30,6 +31,7 @@ struct DeviceState {
   bool supported = false;
   int sm_count = 0;
   bool fwd_attr_set = false;
+  bool heads_attr_set = false;
   void* fwd_ws = nullptr;  // workspace of mla_fa_forward
   size_t fwd_ws_bytes = 0;
   void* cmp_ws = nullptr;  // workspace of mla_compact_mask
@@ -105,11 +107,13 @@ enum KernelId {
   kKernCompact = 4,
   kKernWaitTest = 5,
   kKernMerge = 6,
+  kKernHeads = 7,
+  kKernHeadsCombine = 8,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_fwd_gather_f16", "mla_fwd_q8_0",
                                                "mla_combine", "mla_compact", "mla_wait_timeout",
-                                               "mla_merge"};
+                                               "mla_merge", "mla_fwd_heads", "mla_combine_heads"};
 struct ProfRecord {
   cudaEvent_t start, stop;
   int kernel;
@@ -157,7 +161,8 @@ struct Resolved {
   bool proj;  // fused value up-projection: every sequence writes split partials
   bool sinks; // attention sinks: every sequence writes split partials (the combine adds them)
   bool lse;   // per-row log-sum-exp output: every sequence writes partials (the combine writes it)
-  int dk;     // head width: MLA_DK, or MLA_DV for the DK = DV = 512 shape
+  int dk;     // head width: MLA_DK, MLA_DV for the DK = DV = 512 shape, MLA_HEADS_DK
+  int64_t v_ss;  // DK = 192 shape: rows between sequences of v
 };
 
 int validate(const mla_fa_args* a, Resolved* r) {
@@ -177,9 +182,20 @@ int validate(const mla_fa_args* a, Resolved* r) {
     return MLA_ERR_ALIGN;
   if (a->kcache_type != MLA_KV_F16 && a->kcache_type != MLA_KV_Q8_0) return MLA_ERR_TYPE;
   // head width: 576, or 512 (f16 cache; dense or index-list attention, no softcap,
-  // ALiBi or mask gather)
+  // ALiBi or mask gather), or 192 (a K and a V per KV head; dense, f16)
   const int dk = a->head_dim == 0 ? MLA_DK : a->head_dim;
-  if (dk != MLA_DK && dk != MLA_DV) return MLA_ERR_SHAPE;
+  if (dk != MLA_DK && dk != MLA_DV && dk != MLA_HEADS_DK) return MLA_ERR_SHAPE;
+  if (dk != MLA_HEADS_DK && (a->v != nullptr || a->n_kv_head != 0 || a->v_seq_stride != 0))
+    return MLA_ERR_SHAPE;
+  if (dk == MLA_HEADS_DK) {
+    if (a->v == nullptr) return MLA_ERR_NULL;
+    if (a->n_kv_head < 1 || a->n_head < 1 || a->n_head % a->n_kv_head != 0) return MLA_ERR_SHAPE;
+    if (a->kcache_type != MLA_KV_F16 || a->idx != nullptr || a->mask_gather != 0 || proj ||
+        a->sinks != nullptr || a->alibi_slopes != nullptr || a->softcap > 0.f || a->out_lse != nullptr)
+      return MLA_ERR_UNSUPPORTED;
+    if (a->v_seq_stride < 0) return MLA_ERR_SHAPE;
+    if (!aligned16(a->v)) return MLA_ERR_ALIGN;
+  }
   if (dk == MLA_DV && (a->kcache_type != MLA_KV_F16 || a->softcap > 0.f || a->alibi_slopes != nullptr ||
                        a->mask_gather != 0))
     return MLA_ERR_UNSUPPORTED;
@@ -200,9 +216,12 @@ int validate(const mla_fa_args* a, Resolved* r) {
   r->dk = dk;
   r->q_ss = a->q_seq_stride ? a->q_seq_stride : rows * dk;
   r->k_ss = a->k_seq_stride ? a->k_seq_stride : a->n_kv;
+  r->v_ss = a->v_seq_stride ? a->v_seq_stride : a->n_kv;
+  if (r->v_ss < a->n_kv) return MLA_ERR_SHAPE;
   r->m_rs = a->mask_row_stride ? a->mask_row_stride : a->n_kv;
   r->m_ss = a->mask_seq_stride ? a->mask_seq_stride : (int64_t)a->n_q * r->m_rs;
-  r->o_ss = a->out_seq_stride ? a->out_seq_stride : rows * MLA_DV;
+  const int dv = dk == MLA_HEADS_DK ? MLA_HEADS_DV : MLA_DV;
+  r->o_ss = a->out_seq_stride ? a->out_seq_stride : rows * dv;
   r->idx_ss = a->idx_seq_stride ? a->idx_seq_stride : a->n_kv;
   r->proj = proj;
   r->sinks = a->sinks != nullptr;
@@ -212,7 +231,7 @@ int validate(const mla_fa_args* a, Resolved* r) {
   if (proj && (!aligned16(a->wv) || !aligned16(a->out_proj) || (r->op_ss % 4) != 0))
     return MLA_ERR_ALIGN;
   if (r->q_ss < rows * dk || r->k_ss < a->n_kv || r->m_rs < a->n_kv ||
-      r->m_ss < (int64_t)(a->n_q - 1) * r->m_rs + a->n_kv || r->o_ss < rows * MLA_DV ||
+      r->m_ss < (int64_t)(a->n_q - 1) * r->m_rs + a->n_kv || r->o_ss < rows * dv ||
       r->idx_ss < 0)
     return MLA_ERR_SHAPE;
   if (a->q_seq_stride < 0 || a->k_seq_stride < 0 || a->mask_seq_stride < 0 ||
@@ -321,7 +340,186 @@ size_t gather_bytes(const Resolved& r, const Plan& plan, int slots) {
   return start - head + (size_t)2 * plan.total_units * gather_stride(plan) * sizeof(int32_t);
 }
 
+// ------------------------------------------------ the DK = 192 / DV = 128 head shape
+// Split plan for sequences [s0, s0+n): a unit is (sequence, KV head, 128-row group,
+// split), one CTA each. When the unsplit units do not fill the SMs, each sequence gets
+// splits in proportion to its tiles (all of its KV heads and groups the same number),
+// never more units than SMs. Returns the partial slots it needs.
+int build_heads_plan(const Resolved& r, int s0, int n, int sm_count, mla::heads::Plan* plan) {
+  using namespace mla::heads;
+  std::memset(plan, 0, sizeof(*plan));
+  const mla_fa_args& a = r.a;
+  plan->n_seq = n;
+  plan->seq_offset = s0;
+  plan->n_q = a.n_q;
+  plan->n_head = a.n_head;
+  plan->n_kv_head = a.n_kv_head;
+  plan->group = a.n_head / a.n_kv_head;
+  plan->rows = a.n_q * plan->group;
+  plan->groups = (plan->rows + kRows - 1) / kRows;
+  plan->n_kv = a.n_kv;
+  const int per_seq = a.n_kv_head * plan->groups;  // unsplit units of one sequence
+  const int sms = std::max(1, sm_count);
+  int64_t sum_tiles = 0;
+  std::vector<int> tiles(n);
+  for (int b = 0; b < n; ++b) {
+    plan->kv_len[b] = a.kv_len ? a.kv_len[s0 + b] : a.n_kv;
+    tiles[b] = (plan->kv_len[b] + kTile - 1) / kTile;
+    sum_tiles += tiles[b];
+  }
+  std::vector<int> nsplit(n, 1);
+  if ((int64_t)n * per_seq < sms && sum_tiles > 0) {
+    int64_t units = 0;
+    for (int b = 0; b < n; ++b) {
+      const double want = (double)sms * tiles[b] / ((double)sum_tiles * per_seq);
+      nsplit[b] = std::max(1, std::min((int)std::floor(want + 0.5), std::max(1, tiles[b])));
+      units += (int64_t)per_seq * nsplit[b];
+    }
+    while (units > sms) {  // rounding overshot one wave: take splits back
+      int best = -1;
+      int64_t best_load = 0;
+      for (int b = 0; b < n; ++b) {
+        if (nsplit[b] <= 1) continue;
+        const int64_t load = (tiles[b] + nsplit[b] - 2) / (nsplit[b] - 1);
+        if (best < 0 || load < best_load) {
+          best = b;
+          best_load = load;
+        }
+      }
+      if (best < 0) break;
+      --nsplit[best];
+      units -= per_seq;
+    }
+  }
+  int units = 0, slots = 0;
+  for (int b = 0; b < n; ++b) {
+    plan->n_split[b] = nsplit[b];
+    plan->unit_base[b] = units;
+    units += per_seq * nsplit[b];
+    if (nsplit[b] > 1) {
+      plan->ws_base[b] = slots;
+      slots += per_seq * nsplit[b];
+    } else {
+      plan->ws_base[b] = -1;
+    }
+  }
+  plan->unit_base[n] = units;
+  plan->total_units = units;
+  return slots;
+}
+
+size_t heads_slot_bytes() {
+  return (size_t)mla::heads::kRows * (mla::heads::kHeadDV + 1) * sizeof(float);
+}
+
+size_t heads_workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_splits) {
+  size_t need = 0;
+  int mu = 0, ms = 0;
+  mla::heads::Plan plan;
+  for (int s0 = 0; s0 < r.a.n_seq; s0 += mla::heads::kPlanMaxSeq) {
+    const int n = std::min(mla::heads::kPlanMaxSeq, r.a.n_seq - s0);
+    const int slots = build_heads_plan(r, s0, n, sm_count, &plan);
+    need = std::max(need, (size_t)slots * heads_slot_bytes());
+    mu = std::max(mu, plan.total_units);
+    for (int b = 0; b < n; ++b) ms = std::max(ms, plan.n_split[b]);
+  }
+  if (max_units) *max_units = mu;
+  if (max_splits) *max_splits = ms;
+  return need;
+}
+
+int run_heads(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  using namespace mla::heads;
+  const mla_fa_args& a = r.a;
+  const size_t need = heads_workspace_for(r, st->sm_count, nullptr, nullptr);
+  if (need > 0 && (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)))
+    return MLA_ERR_WORKSPACE;
+  // K: {192 columns, KV heads, keys, sequences}, box {64, 1, 128 keys, 1} -> [key][64]
+  const uint64_t krow = (uint64_t)a.n_kv_head * kHeadDK * 2;
+  CUtensorMap tm_k, tm_v;
+  {
+    cuuint64_t dims[4] = {(cuuint64_t)kHeadDK, (cuuint64_t)a.n_kv_head, (cuuint64_t)a.n_kv, (cuuint64_t)a.n_seq};
+    cuuint64_t strides[3] = {(cuuint64_t)kHeadDK * 2, krow, (cuuint64_t)r.k_ss * krow};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    if (g_encode(&tm_k, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(a.kcache), dims, strides,
+                 box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  // V: {64 columns, keys, 2 column blocks, KV heads, sequences}, box {64, 64 keys, 2, 1, 1}
+  // -> [block][key][64], the MN-major B operand of P.V
+  {
+    const uint64_t vrow = (uint64_t)a.n_kv_head * kHeadDV * 2;
+    cuuint64_t dims[5] = {64, (cuuint64_t)a.n_kv, 2, (cuuint64_t)a.n_kv_head, (cuuint64_t)a.n_seq};
+    cuuint64_t strides[4] = {vrow, 128, (cuuint64_t)kHeadDV * 2, (cuuint64_t)r.v_ss * vrow};
+    cuuint32_t box[5] = {64, 64, 2, 1, 1};
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    if (g_encode(&tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void*>(a.v), dims, strides, box,
+                 es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return MLA_ERR_CUDA;
+  }
+  if (!st->heads_attr_set) {
+    if (cudaFuncSetAttribute(mla::mla_heads_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemAlloc) != cudaSuccess)
+      return MLA_ERR_CUDA;
+    st->heads_attr_set = true;
+  }
+  mla::heads::Params p;
+  p.q = static_cast<const uint16_t*>(a.q);
+  p.mask = static_cast<const uint16_t*>(a.mask);
+  p.out = a.out;
+  p.q_seq_stride = r.q_ss;
+  p.mask_seq_stride = r.m_ss;
+  p.mask_row_stride = r.m_rs;
+  p.out_seq_stride = r.o_ss;
+  p.scale = a.scale;
+  p.mask_vec_ok = (a.mask != nullptr && aligned16(a.mask) && (r.m_ss % 8) == 0 && (r.m_rs % 8) == 0);
+  p.timeout_ns = kDefaultTimeoutNs;
+  mla::heads::Plan plan;
+  for (int s0 = 0; s0 < a.n_seq; s0 += kPlanMaxSeq) {
+    const int n = std::min(kPlanMaxSeq, a.n_seq - s0);
+    const int slots = build_heads_plan(r, s0, n, st->sm_count, &plan);
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                                (size_t)slots * kRows * kHeadDV * sizeof(float))
+                     : nullptr;
+    if (plan.total_units == 0) continue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(plan.total_units);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemAlloc;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    {
+      ProfScope prof(kKernHeads, stream);
+      e = cudaLaunchKernelEx(&cfg, mla::mla_heads_fwd_kernel, tm_k, tm_v, plan, p);
+    }
+    if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (slots > 0) {
+      cudaLaunchConfig_t ccfg = cfg;
+      ccfg.gridDim = dim3((a.n_kv_head * plan.rows + 3) / 4, n);
+      ccfg.blockDim = dim3(128);
+      ccfg.dynamicSmemBytes = 0;
+      {
+        ProfScope prof(kKernHeadsCombine, stream);
+        e = cudaLaunchKernelEx(&ccfg, mla::mla_heads_combine_kernel, plan, (const float*)p.ws_o,
+                               (const float*)p.ws_lse, a.out, (int64_t)r.o_ss);
+      }
+      if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
+  }
+  return MLA_OK;
+}
+
 size_t workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_splits) {
+  if (r.dk == MLA_HEADS_DK) return heads_workspace_for(r, sm_count, max_units, max_splits);
   size_t need = 0;
   int mu = 0, ms = 0;
   Plan plan;
@@ -387,6 +585,7 @@ cudaError_t launch_fwd(cudaLaunchConfig_t cfg, const CUtensorMap& tm_q, const CU
 }
 
 int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (r.dk == MLA_HEADS_DK) return run_heads(r, st, ws, ws_bytes, stream);
   const mla_fa_args& a = r.a;
   const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
   if (need > 0 && (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)))

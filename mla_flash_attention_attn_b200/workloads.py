@@ -185,6 +185,74 @@ def sparse_q8_decode(seed=1005, n_kv=131072, n_head=128, block=64, tail_blocks=1
                     np.array([n_kv], np.int32), SCALE_192, seed, sparse=True)
 
 
+@dataclasses.dataclass
+class HeadsWorkload:
+    """Inputs of the DK = 192 / DV = 128 head shape: a K and a V per KV head."""
+    name: str
+    q: np.ndarray       # f16 [n_seq][n_q][n_head][192]
+    k: np.ndarray       # f16 [n_seq][n_kv][n_kv_head][192]
+    v: np.ndarray       # f16 [n_seq][n_kv][n_kv_head][128]
+    mask: np.ndarray | None
+    kv_len: np.ndarray
+    scale: float
+    seed: int
+
+    @property
+    def n_seq(self):
+        return self.q.shape[0]
+
+    @property
+    def n_q(self):
+        return self.q.shape[1]
+
+    @property
+    def n_head(self):
+        return self.q.shape[2]
+
+    @property
+    def n_kv(self):
+        return self.k.shape[1]
+
+    @property
+    def n_kv_head(self):
+        return self.k.shape[2]
+
+
+def heads_prefill(seed=1007, n_seq=1, n_q=512, n_head=16, n_kv_head=16, n_kv=4096, causal=True,
+                  lengths=None):
+    """The non-absorbed MLA head (DK = 192: 128 nope + 64 rope, DV = 128) with the
+    DeepSeek-V2-Lite head count: n_q new tokens at the end of each sequence, K and V per
+    KV head (n_kv_head = n_head: multi-head attention), Q, K, V ~ N(0,1), causal f16 mask
+    (query i of n_q sees key j iff j <= L - n_q + i), scale 1/sqrt(192). `lengths` (per
+    sequence, <= n_kv) gives ragged sequences; cells past a length are -inf."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens = np.full(n_seq, n_kv, np.int32) if lengths is None else np.asarray(lengths, np.int32)
+    q = _normal_f16(rng, (n_seq, n_q, n_head, 192))
+    k = _normal_f16(rng, (n_seq, n_kv, n_kv_head, 192))
+    v = _normal_f16(rng, (n_seq, n_kv, n_kv_head, 128))
+    j = np.arange(n_kv)[None, None, :]
+    i = np.arange(n_q)[None, :, None]
+    L = lens[:, None, None]
+    keep = np.broadcast_to(j < L, (n_seq, n_q, n_kv))
+    if causal:
+        keep = keep & (j <= L - n_q + i)
+    return HeadsWorkload("heads_prefill", q, k, v, _mask_from_keep(keep), lens, SCALE_192, seed)
+
+
+def heads_decode(seed=1008, n_seq=8, n_head=16, n_kv_head=16, len_lo=1024, len_hi=8192, n_kv=None):
+    """One query token per sequence over a ragged batch of K/V caches (lengths uniform in
+    [len_lo, len_hi], padded cells -inf), the decode step of the same head shape."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens = rng.integers(len_lo, len_hi, size=n_seq, endpoint=True).astype(np.int32)
+    n_kv = int(len_hi if n_kv is None else n_kv)
+    lens = np.minimum(lens, n_kv).astype(np.int32)
+    q = _normal_f16(rng, (n_seq, 1, n_head, 192))
+    k = _normal_f16(rng, (n_seq, n_kv, n_kv_head, 192))
+    v = _normal_f16(rng, (n_seq, n_kv, n_kv_head, 128))
+    keep = np.arange(n_kv)[None, None, :] < lens[:, None, None]
+    return HeadsWorkload("heads_decode", q, k, v, _mask_from_keep(keep), lens, SCALE_192, seed)
+
+
 BUILDERS = {
     "tiny_decode": tiny_decode,
     "v2lite_decode": v2lite_decode,

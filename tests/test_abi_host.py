@@ -114,6 +114,20 @@ def call_ex(lib, a):
     (dict(mask_gather=2, mask=FAKE), -2), (dict(mask_gather=1), -1),
     (dict(mask_gather=1, mask=FAKE, idx=FAKE, idx_count=FAKE), -8),
     (dict(mask_gather=1, mask=FAKE, alibi_slopes=FAKE), -8),
+    # the DK = 192 / DV = 128 shape: needs v and a KV head count dividing n_head; dense f16
+    # attention only; other widths take no v and no KV head count
+    (dict(head_dim=192, n_kv_head=4), -1), (dict(head_dim=192, v=FAKE), -2),
+    (dict(head_dim=192, v=FAKE, n_kv_head=3), -2), (dict(head_dim=192, v=FAKE, n_kv_head=32), -2),
+    (dict(head_dim=192, v=FAKE + 8, n_kv_head=4), -4),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, kcache_type=1), -8),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, idx=FAKE, idx_count=FAKE), -8),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, sinks=FAKE), -8),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, out_lse=FAKE), -8),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, softcap=2.0), -8),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, mask=FAKE, mask_gather=1), -8),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, v_seq_stride=100, n_seq=2), -2),
+    (dict(head_dim=192, v=FAKE, n_kv_head=4, out_seq_stride=16 * 128 - 4, n_seq=2), -2),
+    (dict(v=FAKE), -2), (dict(n_kv_head=4), -2), (dict(head_dim=512, v=FAKE, n_kv_head=1), -2),
 ])
 def test_argument_errors_are_returned_before_any_launch(lib, kw, expect):
     assert call_ex(lib, base_args(**kw)) == expect
@@ -299,3 +313,17 @@ def test_combine_binding_rejects_strided_parts():
     o = torch.zeros((2, 8, 1024))[:, :, :512]  # a strided view
     with pytest.raises(ValueError):
         binding.combine(o, torch.zeros((2, 8)))
+
+
+def test_plan_of_the_192_head_shape():
+    # one CTA per (sequence, KV head, 128-row group, split); splits only while the unsplit
+    # units leave SMs idle, never more units than SMs
+    lens_c = (ctypes.c_int32 * 1)(30000)
+    a = base_args(head_dim=192, v=FAKE, n_kv_head=4, n_head=4, n_kv=30000,
+                  kv_len=ctypes.cast(lens_c, ctypes.c_void_p))
+    units, splits, ws = binding.mla_fa_plan_for_sms(a, 148)
+    assert units <= 148 and units == 4 * splits and splits >= 16
+    assert ws == units * 128 * 129 * 4  # fp32 O rows and lse per slot
+    b = base_args(head_dim=192, v=FAKE, n_kv_head=16, n_head=16, n_seq=10, n_q=1)
+    units, splits, ws = binding.mla_fa_plan_for_sms(b, 148)
+    assert (units, splits, ws) == (160, 1, 0)
