@@ -132,6 +132,7 @@ def kernel_source_hash():
 def workload_name(args):
     """The workload as the step runs it: the cache geometry plus the fused options."""
     return (args.workload + ("+wuv" if args.wuv else "")
+            + ("+no_kv_len" if getattr(args, "no_kv_len", False) else "")
             + ("+mask_gather" if args.mask_gather else "")
             + ("+dk512" if args.head_dim == 512 else ""))  # heads_* names carry their shape
 
@@ -268,7 +269,7 @@ class ClockSampler:
 class Step:
     """Device-resident inputs and the hot path of one workload."""
 
-    def __init__(self, w, torch, binding, wuv=False, mask_gather=False):
+    def __init__(self, w, torch, binding, wuv=False, mask_gather=False, lengths=True):
         self.w = w
         self.torch = torch
         self.b = binding
@@ -280,7 +281,8 @@ class Step:
         self.wv = torch.from_numpy(W.wv_random(n_head=w.n_head)).to(dev) if wuv else None
         self.out = torch.empty(w.q.shape[:3] + ((128 if wuv else 512),), dtype=torch.float32,
                                device=dev)
-        self.kv_len = [int(x) for x in w.kv_len]
+        # without lengths the mask alone says which cells (and tiles) are kept
+        self.kv_len = [int(x) for x in w.kv_len] if lengths else None
         self.idx = self.cnt = None
         if w.sparse and not mask_gather:
             # the step starts from the mask row: compaction, then attention over the kept rows
@@ -372,7 +374,8 @@ def measure(args, w, name, torch, binding, clocks, world, steps, headline=False)
     steps again with per-kernel events. Returns the measurement and the Step."""
     acc = algorithmic(w, wuv=args.wuv, mask_gather=args.mask_gather)
     step = HeadsStep(w, torch, binding) if isinstance(w, W.HeadsWorkload) else \
-        Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather)
+        Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather,
+             lengths=not getattr(args, "no_kv_len", False))
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -466,7 +469,8 @@ def gpu_arm(args, rank, world):
 
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     binding.load()
-    others = [] if (args.only or args.wuv or args.mask_gather or args.head_dim != 576) else \
+    others = [] if (args.only or args.wuv or args.mask_gather or args.head_dim != 576 or
+                    args.no_kv_len) else \
         [n for n in W.WORKLOAD_ORDER if n != args.workload]
     with ClockSampler(torch.cuda.current_device()) as clocks:
         w = make_workload(args)
@@ -718,6 +722,9 @@ def main(argv=None):
                          "columns; f16 cache); 192: the DK = 192 / DV = 128 head shape (a K "
                          "and a V per KV head; the heads_prefill workload unless a heads_* "
                          "workload is named)")
+    ap.add_argument("--no-kv-len", action="store_true",
+                    help="pass no host lengths: the kept tiles come from the mask alone "
+                         "(scanned on the device)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--prefill-steps", type=int, default=60,
                     help="least number of timed steps of the prefill chunk in `configs`")

@@ -109,11 +109,14 @@ enum KernelId {
   kKernMerge = 6,
   kKernHeads = 7,
   kKernHeadsCombine = 8,
+  kKernScan = 9,
+  kKernDevPlan = 10,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_fwd_gather_f16", "mla_fwd_q8_0",
                                                "mla_combine", "mla_compact", "mla_wait_timeout",
-                                               "mla_merge", "mla_fwd_heads", "mla_combine_heads"};
+                                               "mla_merge", "mla_fwd_heads", "mla_combine_heads",
+                                               "mla_scan", "mla_device_plan"};
 struct ProfRecord {
   cudaEvent_t start, stop;
   int kernel;
@@ -518,8 +521,63 @@ int run_heads(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cud
   return MLA_OK;
 }
 
+// ------------------------------------------------ the device plan (tile ranges from the mask)
+// Used by dense f16 calls with a mask that either give no lengths or have several query
+// tokens (a causal prefill chunk ends each token's keys at a different tile): the mask
+// decides each group's tiles. Calls with lengths and one query token keep the host plan.
+bool use_device_plan(const Resolved& r) {
+  const mla_fa_args& a = r.a;
+  return a.mask != nullptr && (a.kv_len == nullptr || a.n_q > 1) && a.kcache_type == MLA_KV_F16 &&
+         a.idx == nullptr && !a.mask_gather && !r.proj && !r.sinks && !r.lse;
+}
+
+struct DevLayout {
+  int n_groups, grid_units, slots;
+  size_t off_ranges, off_units, off_gsplit, bytes;
+};
+
+// Workspace of one launch of the device plan: partial slots (at most one per SM pair, and
+// only when there are fewer groups than pairs), then the ranges, unit descriptors and the
+// per-group split table.
+DevLayout dev_layout(int n_seq, int groups, int sm_count) {
+  DevLayout l;
+  const int pairs = std::max(1, sm_count / 2);
+  l.n_groups = n_seq * groups;
+  const bool split = l.n_groups < pairs && l.n_groups <= mla::kDevPlanMaxGroups;
+  l.grid_units = l.n_groups >= pairs ? l.n_groups : pairs;
+  l.slots = split ? pairs : 0;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  l.off_ranges = up((size_t)l.slots * slot_bytes());
+  l.off_units = up(l.off_ranges + (size_t)l.n_groups * sizeof(int2));
+  l.off_gsplit = up(l.off_units + (size_t)l.grid_units * sizeof(mla::DevUnit));
+  l.bytes = l.off_gsplit + (size_t)l.n_groups * sizeof(int2);
+  return l;
+}
+
+// Splits one group may take in the device plan: with three groups or more at most 16, so
+// the combine reads a row's partials in one round trip (an even share is at most a third
+// of the SM pairs); with fewer groups as many as the SM pairs, for the wide combine.
+int dev_max_split(const DevLayout& l) { return l.n_groups >= 3 ? 16 : std::max(1, l.slots); }
+
 size_t workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_splits) {
   if (r.dk == MLA_HEADS_DK) return heads_workspace_for(r, sm_count, max_units, max_splits);
+  if (use_device_plan(r)) {
+    // the split counts are decided on the device: report the launch shape and the most
+    // splits a group can take
+    size_t need = 0;
+    int mu = 0, ms = 1;
+    const int groups = (r.rows + mla::kRowsPerGroup - 1) / mla::kRowsPerGroup;
+    for (int s0 = 0; s0 < r.a.n_seq; s0 += mla::kPlanMaxSeq) {
+      const int n = std::min(mla::kPlanMaxSeq, r.a.n_seq - s0);
+      const DevLayout l = dev_layout(n, groups, sm_count);
+      need = std::max(need, l.bytes);
+      mu = std::max(mu, l.grid_units);
+      if (l.slots > 0) ms = std::max(ms, dev_max_split(l));
+    }
+    if (max_units) *max_units = mu;
+    if (max_splits) *max_splits = ms;
+    return need;
+  }
   size_t need = 0;
   int mu = 0, ms = 0;
   Plan plan;
@@ -674,7 +732,45 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   Plan plan;
   for (int s0 = 0; s0 < a.n_seq; s0 += mla::kPlanMaxSeq) {
     const int n = std::min(mla::kPlanMaxSeq, a.n_seq - s0);
-    const int slots = build_plan(r, s0, n, st->sm_count, &plan);
+    const bool dev = use_device_plan(r);
+    int slots = build_plan(r, s0, n, st->sm_count, &plan);
+    DevLayout dl = {};
+    p.units = nullptr;
+    int2* d_gsplit = nullptr;
+    if (dev) {
+      // the grid and the partial slots are sized for the device plan, which the scan and
+      // plan kernels fill in before the attention kernel reads them
+      dl = dev_layout(n, plan.groups, st->sm_count);
+      slots = dl.slots;
+      plan.total_units = dl.grid_units;
+      int2* d_ranges = reinterpret_cast<int2*>(static_cast<char*>(ws) + dl.off_ranges);
+      p.units = reinterpret_cast<const mla::DevUnit*>(static_cast<char*>(ws) + dl.off_units);
+      d_gsplit = reinterpret_cast<int2*>(static_cast<char*>(ws) + dl.off_gsplit);
+      cudaLaunchConfig_t scfg = {};
+      scfg.gridDim = dim3(dl.n_groups);
+      scfg.blockDim = dim3(256);
+      scfg.stream = stream;
+      cudaLaunchAttribute sattr[1];
+      sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      sattr[0].val.programmaticStreamSerializationAllowed = 1;
+      scfg.attrs = sattr;
+      scfg.numAttrs = 1;
+      cudaError_t se;
+      {
+        ProfScope prof(kKernScan, stream);
+        se = cudaLaunchKernelEx(&scfg, mla::mla_scan_kernel, plan, static_cast<const uint16_t*>(a.mask),
+                                (int64_t)r.m_ss, (int64_t)r.m_rs, p.mask_vec_ok, d_ranges);
+      }
+      if (se != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+      scfg.gridDim = dim3(1);
+      {
+        ProfScope prof(kKernDevPlan, stream);
+        se = cudaLaunchKernelEx(&scfg, mla::mla_device_plan_kernel, plan, (const int2*)d_ranges,
+                                std::max(1, st->sm_count / 2), dev_max_split(dl), dl.grid_units,
+                                const_cast<mla::DevUnit*>(p.units), d_gsplit);
+      }
+      if (se != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
     p.ws_o = static_cast<uint16_t*>(ws);
     p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                 (size_t)slots * mla::kRowsPerGroup * mla::kDV * 2)
@@ -738,7 +834,8 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       // (one round trip); more: one CTA per (row, quarter of the value columns)
       int ns_max = 1;
       for (int b = 0; b < n; ++b) ns_max = std::max(ns_max, plan.n_split[b]);
-      const bool wide = ns_max > 16;
+      // the device plan's splits are known only on the device: at most dev_max_split
+      const bool wide = dev ? dev_max_split(dl) > 16 : ns_max > 16;
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = wide ? dim3(r.rows, 4, n) : dim3(r.rows, n);
       cfg.blockDim = dim3(128);
@@ -766,10 +863,12 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
                                   a.out_proj, (int64_t)r.op_ss, a.sinks);
         else if (wide)
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_wide_kernel, plan, (const uint16_t*)p.ws_o,
-                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks, a.out_lse);
+                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks, a.out_lse,
+                                  (const int2*)d_gsplit);
         else
           ce = cudaLaunchKernelEx(&cfg, mla::mla_combine_kernel, plan, (const uint16_t*)p.ws_o,
-                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks, a.out_lse);
+                                  (const float*)p.ws_lse, a.out, (int64_t)r.o_ss, a.sinks, a.out_lse,
+                                  (const int2*)d_gsplit);
       }
       if (ce != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }

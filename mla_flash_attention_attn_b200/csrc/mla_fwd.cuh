@@ -44,6 +44,7 @@
 #include <cuda_fp16.h>
 
 #include "mla_common.cuh"
+#include "mla_plan.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mla {
@@ -82,6 +83,9 @@ struct MlaFwdParams {
   int mask_gather;
   int32_t* gather_list;
   int64_t gather_stride;
+  // device plan (tile ranges found from the mask on the device): unit u's descriptor;
+  // nullptr: the host plan
+  const DevUnit* units;
 };
 
 // How K/V tiles reach shared memory.
@@ -316,11 +320,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   // visible from here on; a launch without the programmatic attribute returns at once
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- work unit
-  int b, g, s;
-  decode_unit(plan, blockIdx.x >> 1, b, g, s);
+  // ---- work unit: from the host plan, or from the device plan's descriptor (an idle
+  // descriptor leaves the unit without tiles and without output)
+  int b, g, s, n_split;
+  bool idle = false;
+  DevUnit du = {0, 0, 0, 1, 0, 0, -1, 0};
+  if (p.units != nullptr) {
+    du = p.units[blockIdx.x >> 1];
+    idle = du.b < 0;
+    b = idle ? 0 : du.b;
+    g = du.g;
+    s = du.s;
+    n_split = du.n_split;
+  } else {
+    decode_unit(plan, blockIdx.x >> 1, b, g, s);
+    n_split = plan.n_split[b];
+  }
   const int b_abs = plan.seq_offset + b;
-  const int n_split = plan.n_split[b];
   const int row0 = g * kRowsPerGroup;
   constexpr bool gather = kManual && kGather;
   const bool sparse = p.idx != nullptr || gather;
@@ -399,11 +415,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     key_end = len;
   } else {
     len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
-    const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
-    tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
-    const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
-    n_tiles = tile_end - tile_begin;
-    key_end = min(len, tile_end * kTileKeys);
+    if (p.units != nullptr) {
+      // tiles the mask leaves something in (dense mode; the range is within the length)
+      tile_begin = du.tile_begin;
+      n_tiles = idle ? 0 : du.n_tiles;
+      key_end = min(len, (tile_begin + n_tiles) * kTileKeys);
+    } else {
+      const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
+      tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
+      const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
+      n_tiles = tile_end - tile_begin;
+      key_end = min(len, tile_end * kTileKeys);
+    }
   }
   bool failed = false;
 
@@ -745,7 +768,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     const int kh = L >> 6;                    // which 64 keys of a tile this lane holds
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = row0 + kRowsPerCta * (int)rank + r;  // row within the sequence
-    const bool row_valid = row < plan.rows;
+    const bool row_valid = row < plan.rows && !idle;
     const int tok = row / plan.n_head;
     const uint16_t* mrow = (p.mask != nullptr && row_valid)
                                ? p.mask + (int64_t)b_abs * p.mask_seq_stride +
@@ -1004,7 +1027,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     named_bar_sync(1, 128);
     const float l_tot = l_part + xl[L ^ 64];
     const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
-    const int ws_slot = plan.ws_base[b] >= 0 ? plan.ws_base[b] + g * n_split + s : -1;
+    const int ws_slot = p.units != nullptr ? du.slot
+                        : (plan.ws_base[b] >= 0 ? plan.ws_base[b] + g * n_split + s : -1);
     // O / l goes out through shared memory: each warp stages its 32 rows as eight
     // 32 x 32 fp32 boxes, or for a split partial four 32 x 64 f16 boxes (128-byte rows,
     // 16-byte chunks XOR-swizzled by row, the layout of a 128-byte-swizzle tensor map),
@@ -1131,16 +1155,26 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __grid_constant_
                                                           float* __restrict__ out,
                                                           int64_t out_seq_stride,
                                                           const float* __restrict__ sinks,
-                                                          float* __restrict__ out_lse) {
+                                                          float* __restrict__ out_lse,
+                                                          const int2* __restrict__ gsplit) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.y;
   const int row = blockIdx.x;
-  if (plan.ws_base[b] < 0 || row >= plan.rows) return;
-  const int ns = min(plan.n_split[b], 32);
-  const int lane = threadIdx.x & 31;
+  if (row >= plan.rows) return;
   const int g = row / kRowsPerGroup;
+  // the group's first partial slot and splits: the host plan's, or the device plan's table
+  int slot0, ns;
+  if (gsplit != nullptr) {
+    const int2 gs = gsplit[b * plan.groups + g];
+    slot0 = gs.x;
+    ns = min(gs.y, 32);
+  } else {
+    slot0 = plan.ws_base[b] >= 0 ? plan.ws_base[b] + g * plan.n_split[b] : -1;
+    ns = min(plan.n_split[b], 32);
+  }
+  if (slot0 < 0) return;  // written by the attention kernel itself
+  const int lane = threadIdx.x & 31;
   const int rin = row % kRowsPerGroup;
-  const int slot0 = plan.ws_base[b] + g * plan.n_split[b];
   const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
   constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // 4-value groups per slot
   const uint2* src0 =
@@ -1206,19 +1240,28 @@ __global__ void __launch_bounds__(128)
     mla_combine_wide_kernel(const __grid_constant__ Plan plan, const uint16_t* __restrict__ ws_o,
                             const float* __restrict__ ws_lse, float* __restrict__ out,
                             int64_t out_seq_stride, const float* __restrict__ sinks,
-                            float* __restrict__ out_lse) {
+                            float* __restrict__ out_lse, const int2* __restrict__ gsplit) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 red[4][32];
   const int b = blockIdx.z;
   const int row = blockIdx.x;
   const int qtr = blockIdx.y;
-  if (plan.ws_base[b] < 0 || row >= plan.rows) return;  // the whole CTA leaves
-  const int ns = plan.n_split[b];
+  if (row >= plan.rows) return;  // the whole CTA leaves
+  const int g = row / kRowsPerGroup;
+  // the group's first partial slot and splits: the host plan's, or the device plan's table
+  int ns, slot0;
+  if (gsplit != nullptr) {
+    const int2 gs = gsplit[b * plan.groups + g];
+    slot0 = gs.x;
+    ns = gs.y;
+  } else {
+    ns = plan.n_split[b];
+    slot0 = plan.ws_base[b] >= 0 ? plan.ws_base[b] + g * ns : -1;
+  }
+  if (slot0 < 0) return;  // written by the attention kernel itself
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int g = row / kRowsPerGroup;
   const int rin = row % kRowsPerGroup;
-  const int slot0 = plan.ws_base[b] + g * ns;
   const float* lse_col = ws_lse + (int64_t)slot0 * kRowsPerGroup + rin;
   constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;  // 4-value groups per slot
   const uint2* src0 = reinterpret_cast<const uint2*>(ws_o + ((int64_t)slot0 * kRowsPerGroup + rin) * kDV) +

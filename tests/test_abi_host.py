@@ -327,3 +327,25 @@ def test_plan_of_the_192_head_shape():
     b = base_args(head_dim=192, v=FAKE, n_kv_head=16, n_head=16, n_seq=10, n_q=1)
     units, splits, ws = binding.mla_fa_plan_for_sms(b, 148)
     assert (units, splits, ws) == (160, 1, 0)
+
+
+def test_plan_of_mask_derived_ranges():
+    # with a mask and no lengths (or with several query tokens) the tile ranges come from
+    # the mask on the device: the launch has one unit per SM pair while there are fewer
+    # groups than pairs (the device decides the splits: at most 16 per group with three
+    # groups or more, else up to the pairs), else one unit per group
+    a = base_args(n_seq=8, n_q=1, n_head=128, n_kv=32768, mask=FAKE)
+    units, splits, ws = binding.mla_fa_plan_for_sms(a, 148)
+    assert units == 74 and splits == 16 and ws > 74 * SLOT_BYTES
+    units, splits, ws = binding.mla_fa_plan_for_sms(base_args(n_kv=32768, n_head=128, mask=FAKE), 148)
+    assert units == 74 and splits == 74
+    lens_c = (ctypes.c_int32 * 1)(16384)
+    b = base_args(n_seq=1, n_q=512, n_head=128, n_kv=16384, mask=FAKE,
+                  kv_len=ctypes.cast(lens_c, ctypes.c_void_p))
+    units, splits, ws = binding.mla_fa_plan_for_sms(b, 148)
+    assert (units, splits) == (512, 1) and 0 < ws < SLOT_BYTES  # descriptors only
+    # lengths and one query token: the host plan, as before
+    lens8 = (ctypes.c_int32 * 8)(*[12606, 9479, 20813, 11456, 12221, 18279, 28969, 23042])
+    c = base_args(n_seq=8, n_q=1, n_head=128, n_kv=32768, mask=FAKE,
+                  kv_len=ctypes.cast(lens8, ctypes.c_void_p))
+    assert binding.mla_fa_plan_for_sms(c, 148) == (74, 16, 74 * SLOT_BYTES)

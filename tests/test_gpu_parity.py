@@ -855,3 +855,48 @@ def test_dk512_with_sinks_and_lse():
         o_ref, l_ref = oracle.attention_lse(q[b], k[b], oracle.KV_F16, None, 0.04)
         share = 1.0 / (1.0 + np.exp(np.tile(sinks.astype(np.float64), 1) - l_ref))
         assert_parity(got[b].reshape(-1, 512), o_ref * share[:, None], f"dk512 sinks {b}")
+
+
+# ------------------------------------------------------------------ tile ranges from the mask
+def _launches(fn):
+    binding.mla_profile_begin()
+    fn()
+    torch_mod().cuda.synchronize()
+    return {k: v[0] for k, v in binding.mla_profile_end().items()}
+
+
+def test_mask_derived_ranges_skip_leading_and_trailing_tiles():
+    # a window of kept cells in the middle of each sequence, no host lengths: the scan
+    # finds each group's first and last kept tile and the device plan spreads those tiles
+    # over the SM pairs
+    w = W.make("v3_batched_decode", seed=21, n_seq=3, n_kv=6000, len_lo=6000, len_hi=6000)
+    windows = [(1000, 1777), (0, 300), (4100, 6000)]
+    for b, (lo, hi) in enumerate(windows):
+        w.mask[b, 0, :] = np.float16(-np.inf)
+        w.mask[b, 0, lo:hi] = 0
+    got = run_gpu(w, kv_len=None)
+    check_all_rows(w, got, what="window")
+
+
+def test_mask_derived_ranges_fully_masked_sequence_and_group():
+    w = W.make("v3_batched_decode", seed=22, n_seq=2, n_head=100, n_kv=1500, len_lo=1500,
+               len_hi=1500)
+    w.q = np.ascontiguousarray(np.repeat(w.q, 3, axis=1))  # 3 tokens: groups span tokens
+    w.mask = np.ascontiguousarray(np.repeat(w.mask, 3, axis=1))
+    w.mask[0] = np.float16(-np.inf)        # a whole sequence masked
+    w.mask[1, 1, :] = np.float16(-np.inf)  # one token of the other
+    got = run_gpu(w, kv_len=None)
+    assert np.all(got[0] == 0.0) and np.all(got[1, 1] == 0.0)
+    check_all_rows(w, got, what="masked groups")
+
+
+def test_mask_derived_ranges_are_the_path_taken():
+    torch = torch_mod()
+    w = W.make("v3_batched_decode", seed=23, n_seq=2, n_kv=3000, len_lo=1000, len_hi=3000)
+    dev = torch.device("cuda")
+    q, k, m = (torch.from_numpy(x).to(dev) for x in (w.q, w.kcache, w.mask))
+    no_len = _launches(lambda: binding.forward(q, k, w.kv_type, m, w.scale))
+    with_len = _launches(lambda: binding.forward(q, k, w.kv_type, m, w.scale, kv_len=w.kv_len))
+    assert no_len.get("mla_scan") == 1 and no_len.get("mla_device_plan") == 1
+    assert "mla_scan" not in with_len and "mla_device_plan" not in with_len
+    assert binding.mla_get_device_status() == 0
