@@ -132,6 +132,7 @@ def kernel_source_hash():
 def workload_name(args):
     """The workload as the step runs it: the cache geometry plus the fused options."""
     return (args.workload + ("+wuv" if args.wuv else "")
+            + (f"+split_kv{args.split_kv}" if getattr(args, "split_kv", 0) > 1 else "")
             + ("+no_kv_len" if getattr(args, "no_kv_len", False) else "")
             + ("+mask_gather" if args.mask_gather else "")
             + ("+dk512" if args.head_dim == 512 else ""))  # heads_* names carry their shape
@@ -337,6 +338,46 @@ class HeadsStep:
         self.b.mla_fa_forward_ex(self.args, self.ws if self.ws_used else None, stream)
 
 
+class SplitKVStep:
+    """The ranks' calls of a split-KV decode (the cache split into `parts` ranges), made
+    one after another on one GPU: each attends over its range with each row's lse,
+    writing O and lse into its slice of the packed buffer the all-gather would fill,
+    and the merge (mla_fa_combine_strided) combines them. The all-gather itself is not
+    part of this step (one GPU)."""
+
+    def __init__(self, w, torch, binding, parts):
+        from mla_flash_attention_attn_b200 import split_kv
+
+        self.w = w
+        self.b = binding
+        dev = torch.device("cuda")
+        self.q = torch.from_numpy(w.q).to(dev)
+        self.rows = w.n_seq * w.n_q * w.n_head
+        self.packed = torch.empty((parts, binding.packed_width(self.rows)), dtype=torch.float32,
+                                  device=dev)
+        self.out = torch.empty((self.rows, 512), dtype=torch.float32, device=dev)
+        self.shards = []
+        for r, (lo, hi) in enumerate(split_kv.shard_bounds(w.n_kv, parts)):
+            k = torch.from_numpy(np.ascontiguousarray(w.kcache[:, lo:hi])).to(dev)
+            m = torch.from_numpy(np.ascontiguousarray(w.mask[:, :, lo:hi])).to(dev)
+            o = self.packed[r, : self.rows * 512].view(w.n_seq, w.n_q, w.n_head, 512)
+            lse = self.packed[r, self.rows * 512:].view(w.n_seq, w.n_q, w.n_head)
+            args, keep = binding.make_args(self.q, k, w.kv_type, m, o, w.scale,
+                                           kv_len=split_kv.shard_lengths(w.kv_len, lo, hi),
+                                           out_lse=lse)
+            need = binding.mla_fa_workspace_size(args)
+            ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+            self.shards.append((args, keep, ws, k, m))
+
+    def inputs(self):
+        return [(self.q, self.w.q)]
+
+    def run(self, stream=None):
+        for args, _, ws, _, _ in self.shards:
+            self.b.mla_fa_forward_ex(args, ws, stream)
+        self.b.combine_packed(self.packed, self.rows, out=self.out, stream=stream)
+
+
 def config_of(w, name, world):
     """The workload's description as it appears in both arms' JSON lines."""
     heads = isinstance(w, W.HeadsWorkload)
@@ -373,9 +414,13 @@ def measure(args, w, name, torch, binding, clocks, world, steps, headline=False)
     """Time `steps` steps of workload w (after args.warmup untimed ones), then the same
     steps again with per-kernel events. Returns the measurement and the Step."""
     acc = algorithmic(w, wuv=args.wuv, mask_gather=args.mask_gather)
-    step = HeadsStep(w, torch, binding) if isinstance(w, W.HeadsWorkload) else \
-        Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather,
-             lengths=not getattr(args, "no_kv_len", False))
+    if isinstance(w, W.HeadsWorkload):
+        step = HeadsStep(w, torch, binding)
+    elif getattr(args, "split_kv", 0) > 1:
+        step = SplitKVStep(w, torch, binding, args.split_kv)
+    else:
+        step = Step(w, torch, binding, wuv=args.wuv, mask_gather=args.mask_gather,
+                    lengths=not getattr(args, "no_kv_len", False))
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -431,9 +476,11 @@ def measure(args, w, name, torch, binding, clocks, world, steps, headline=False)
     launches, dom_ms = prof.get(dom, (0, 0.0))
     dom_prof_ms = dom_ms / max(launches, 1)
     per_step_launches = sum(v[0] for v in prof.values()) / steps
-    # the kernel's time: its own events, capped at the step that holds it; a step of one
-    # kernel is that kernel
-    kernel_ms = ms_per_step if per_step_launches <= 1 else min(dom_prof_ms, ms_per_step)
+    # the kernel's time in a step: its own events (all its launches of the step: the
+    # emulated split-KV step launches it once per cache range), capped at the step that
+    # holds it; a step of one kernel is that kernel
+    dom_step_ms = dom_ms / steps
+    kernel_ms = ms_per_step if per_step_launches <= 1 else min(dom_step_ms, ms_per_step)
     # the roofline is the dominant (attention) kernel's: its own algorithmic bytes and
     # flops, which leave out the W_UV weights and projection of a --wuv step (the
     # combine does those)
@@ -443,6 +490,7 @@ def measure(args, w, name, torch, binding, clocks, world, steps, headline=False)
         + ("+dk512" if args.head_dim == 512 else "")))
     roof["kernel"] = dom
     roof["kernel_us"] = round(kernel_ms * 1e3, 3)
+    roof["kernel_launches_per_step"] = round(launches / steps, 3)
     roof["kernel_avg_us_events"] = round(dom_prof_ms * 1e3, 3)
     roof["algorithmic_bytes_per_launch"] = kacc["bytes"]
     roof["algorithmic_flops_per_launch"] = kacc["flops"]
@@ -470,7 +518,7 @@ def gpu_arm(args, rank, world):
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     binding.load()
     others = [] if (args.only or args.wuv or args.mask_gather or args.head_dim != 576 or
-                    args.no_kv_len) else \
+                    args.no_kv_len or args.split_kv > 1) else \
         [n for n in W.WORKLOAD_ORDER if n != args.workload]
     with ClockSampler(torch.cuda.current_device()) as clocks:
         w = make_workload(args)
@@ -725,6 +773,10 @@ def main(argv=None):
     ap.add_argument("--no-kv-len", action="store_true",
                     help="pass no host lengths: the kept tiles come from the mask alone "
                          "(scanned on the device)")
+    ap.add_argument("--split-kv", type=int, default=0,
+                    help="R >= 2: the calls of a split-KV decode over R cache ranges, made one "
+                         "after another on this GPU (R shard forwards with the lse, then the "
+                         "merge of the packed parts; the all-gather between GPUs is left out)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--prefill-steps", type=int, default=60,
                     help="least number of timed steps of the prefill chunk in `configs`")
@@ -747,6 +799,12 @@ def main(argv=None):
         ap.error("--mask-gather applies to --impl ours (the oracle arm runs the unfused chain)")
     if args.wuv:
         args.no_cpu_baseline = True  # the oracle baseline times the attention only
+    if args.split_kv > 1 and (args.impl == "reference" or args.wuv or args.mask_gather or
+                              args.head_dim != 576 or args.workload in HEADS_WORKLOADS or
+                              args.gpus > 1):
+        ap.error("--split-kv emulates the ranks on one GPU, for the MLA decode workloads")
+    if args.split_kv > 1:
+        args.no_e2e = True  # the emulated ranks' step reads shards no host copy would fill
     if args.head_dim == 192 and args.workload not in HEADS_WORKLOADS:
         args.workload = "heads_prefill"
     if args.workload in HEADS_WORKLOADS:

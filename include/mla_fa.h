@@ -259,6 +259,16 @@ int mla_fa_forward_noalloc(const mla_fa_args* a, void* stream);
 int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows,
                    float* out, float* out_lse, void* stream);
 
+/* The same merge with the parts at any spacing: part p's O rows start at
+ * o_parts + p*o_part_stride and its lse at lse_parts + p*lse_part_stride (floats), so the
+ * parts can travel as one packed buffer each (rows x 512 values of O, then the rows'
+ * lse), gathered across devices by a single all-gather. o_part_stride >= rows*512 and a
+ * multiple of 4, lse_part_stride >= rows (else MLA_ERR_SHAPE / MLA_ERR_ALIGN); the rest as
+ * mla_fa_combine, which is this call with o_part_stride = rows*512, lse_part_stride = rows. */
+int mla_fa_combine_strided(const float* o_parts, int64_t o_part_stride, const float* lse_parts,
+                           int64_t lse_part_stride, int n_parts, int64_t rows, float* out,
+                           float* out_lse, void* stream);
+
 /* The same plan for a GPU with sm_count SMs, computed on the host alone (no device is
  * queried, nothing is launched): units, max_splits as mla_fa_query_plan, and the
  * workspace bytes mla_fa_workspace_size would return on such a GPU. Any pointer may be

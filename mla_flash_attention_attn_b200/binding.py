@@ -134,6 +134,9 @@ def load(path: str = LIB_PATH):
     lib.mla_fa_plan_for_sms.restype = I
     lib.mla_fa_combine.argtypes = [P, P, I, ctypes.c_int64, P, P, P]
     lib.mla_fa_combine.restype = I
+    lib.mla_fa_combine_strided.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, I, ctypes.c_int64,
+                                           P, P, P]
+    lib.mla_fa_combine_strided.restype = I
     _lib = lib
     return lib
 
@@ -472,6 +475,39 @@ def combine(o_parts, lse_parts, out=None, out_lse=None, stream=None):
         _check_tensor(out_lse.view(rows), "out_lse", torch.float32, (rows,), dev)
     _check(load().mla_fa_combine(_ptr(o), _ptr(lse), n_parts, rows, _ptr(out), _ptr(out_lse),
                                  _stream_ptr(stream)), "mla_fa_combine")
+    return out
+
+
+def packed_width(rows):
+    """Floats of one packed part: rows x 512 of O, then the rows' lse."""
+    return rows * DV + rows
+
+
+def combine_packed(parts, rows, out=None, out_lse=None, stream=None):
+    """mla_fa_combine_strided over packed parts: parts fp32 [n_parts][rows*512 + rows],
+    each part its O rows then its rows' lse (natural log). Returns out fp32 [rows][512]."""
+    import torch
+
+    if not parts.is_cuda:
+        raise ValueError("parts must be a CUDA tensor")
+    width = packed_width(rows)
+    if parts.dim() != 2 or parts.shape[1] != width:
+        raise ValueError(f"parts must be [n_parts][{width}]")
+    _check_tensor(parts, "parts", torch.float32, (parts.shape[0], width), parts.device)
+    if out is None:
+        out = torch.empty((rows, DV), dtype=torch.float32, device=parts.device)
+    if not out.is_contiguous() or out.numel() != rows * DV:
+        raise ValueError(f"out must be contiguous with rows x 512 = {rows * DV} values")
+    _check_tensor(out.view(rows, DV), "out", torch.float32, (rows, DV), parts.device)
+    if out_lse is not None:
+        if not out_lse.is_contiguous() or out_lse.numel() != rows:
+            raise ValueError(f"out_lse must be contiguous with {rows} values")
+        _check_tensor(out_lse.view(rows), "out_lse", torch.float32, (rows,), parts.device)
+    base = parts.data_ptr()
+    _check(load().mla_fa_combine_strided(ctypes.c_void_p(base), width,
+                                         ctypes.c_void_p(base + rows * DV * 4), width,
+                                         parts.shape[0], rows, _ptr(out), _ptr(out_lse),
+                                         _stream_ptr(stream)), "mla_fa_combine_strided")
     return out
 
 

@@ -1071,12 +1071,15 @@ int mla_compact_mask_ex(const void* mask, int n_rows, int64_t mask_row_stride, i
   return MLA_OK;
 }
 
-int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows,
-                   float* out, float* out_lse, void* stream) {
+int mla_fa_combine_strided(const float* o_parts, int64_t o_part_stride, const float* lse_parts,
+                           int64_t lse_part_stride, int n_parts, int64_t rows, float* out,
+                           float* out_lse, void* stream) {
   if (o_parts == nullptr || lse_parts == nullptr || out == nullptr) return MLA_ERR_NULL;
   if (n_parts < 1 || n_parts > MLA_COMBINE_MAX_PARTS || rows < 1) return MLA_ERR_SHAPE;
+  if (o_part_stride < rows * MLA_DV || lse_part_stride < rows) return MLA_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(o_parts) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
-      (reinterpret_cast<uintptr_t>(lse_parts) & 3) || (reinterpret_cast<uintptr_t>(out_lse) & 3))
+      (reinterpret_cast<uintptr_t>(lse_parts) & 3) || (reinterpret_cast<uintptr_t>(out_lse) & 3) ||
+      (o_part_stride % 4) != 0)
     return MLA_ERR_ALIGN;
   DeviceState* st = nullptr;
   int rc = current_device(&st);
@@ -1084,11 +1087,17 @@ int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, in
   const unsigned grid = (unsigned)std::min<int64_t>(rows, (int64_t)1 << 30);
   {
     ProfScope prof(kKernMerge, static_cast<cudaStream_t>(stream));
-    mla::mla_merge_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(o_parts, lse_parts, n_parts,
-                                                                               rows, out, out_lse);
+    mla::mla_merge_kernel<<<grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        o_parts, o_part_stride, lse_parts, lse_part_stride, n_parts, rows, out, out_lse);
   }
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
+}
+
+int mla_fa_combine(const float* o_parts, const float* lse_parts, int n_parts, int64_t rows,
+                   float* out, float* out_lse, void* stream) {
+  return mla_fa_combine_strided(o_parts, rows * MLA_DV, lse_parts, rows, n_parts, rows, out, out_lse,
+                                stream);
 }
 
 int mla_compact_mask(const void* mask_row, int n_kv, int32_t* idx_out, int32_t* count_out,

@@ -3,11 +3,12 @@
 // compaction": contiguous segments, a count per segment, one scan over the
 // counts giving each segment its output offset; the list stays ascending).
 //
-// Mapping: a thread's segment is 16 consecutive cells (two 16-byte loads); a CTA
-// covers 1024 segments = 16384 cells, so a row of 131072 cells takes 8 CTAs and
-// every look-back fits in one window. The scan over segment counts is done in one
-// pass: warp shuffle scan, then a scan of the 32 warp totals, then a decoupled
-// look-back across CTAs (one warp reads 32 predecessor flags per round trip). CTAs take their tile in ticket order
+// Mapping: a thread's segment is 8 consecutive cells (one 16-byte load); a CTA covers
+// 256 segments = 2048 cells, so a row of 131072 cells is read by 64 CTAs on as many SMs
+// (8 CTAs of 16384 cells left the row's latency on a few SMs). The scan over segment
+// counts is done in one pass: warp shuffle scan, then a scan of the 8 warp totals, then
+// a decoupled look-back across CTAs (one warp reads 32 predecessor flags per round trip,
+// so the last tile of such a row needs two). CTAs take their tile in ticket order
 // (atomicAdd), so every tile a CTA waits on belongs to a CTA that is already
 // running; each wait is bounded and reports MLA_ERR_TIMEOUT instead of hanging.
 // Look-back flags carry a per-call epoch, so stale flags from an earlier call
@@ -21,9 +22,9 @@
 namespace mla {
 
 namespace compact {
-constexpr int kThreads = 1024;
-constexpr int kCellsPerThread = 16;
-constexpr int kTileCells = kThreads * kCellsPerThread;  // 16384
+constexpr int kThreads = 256;
+constexpr int kCellsPerThread = 8;
+constexpr int kTileCells = kThreads * kCellsPerThread;  // 2048
 constexpr uint32_t kStateAggregate = 1;
 constexpr uint32_t kStateInclusive = 2;
 constexpr uint16_t kNegInfBits = 0xFC00;
@@ -62,14 +63,14 @@ __global__ void __launch_bounds__(compact::kThreads)
   const uint16_t* mrow = mask + (int64_t)row * mask_row_stride;
   const int64_t cell0 = (int64_t)tile * kTileCells + (int64_t)tid * kCellsPerThread;
 
-  // keep bits of this thread's 8 cells
+  // keep bits of this thread's cells
+  static_assert(kCellsPerThread == 8, "one 16-byte load per segment");
   uint32_t keep = 0;
   if (cell0 + kCellsPerThread <= n_kv && ((reinterpret_cast<uintptr_t>(mrow + cell0) & 15) == 0)) {
-    const uint4* src = reinterpret_cast<const uint4*>(mrow + cell0);
-    const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(mrow + cell0));
+    const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
+    for (int h = 0; h < 4; ++h) {
       keep |= (uint32_t)((w[h] & 0xFFFFu) != kNegInfBits) << (2 * h);
       keep |= (uint32_t)((w[h] >> 16) != kNegInfBits) << (2 * h + 1);
     }

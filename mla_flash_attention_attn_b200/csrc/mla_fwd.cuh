@@ -807,11 +807,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // A row past the sequence's rows is computed but never stored: it takes the vector
     // path with a zero mask, so that its lanes follow the same path as their warp's
     // valid rows.
+    // A ragged tile (the unit's keys end inside it) takes the vector path too while its
+    // mask loads stay inside the mask row, and then drops the cells past the unit's last
+    // key; otherwise it goes key by key.
     auto mask_vec_ok = [&](int t) {
       if ((kManual && sparse) || !row_valid) return true;
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
-      if (k0 + kHalf > key_end) return false;  // ragged: per-key path
-      return mrow == nullptr || p.mask_vec_ok;  // no mask: zeros
+      if (mrow == nullptr) return true;  // no mask: zeros
+      return p.mask_vec_ok && (k0 + kHalf <= key_end || k0 + kHalf <= p.n_kv);
     };
     auto load_mask = [&](int t) {
       const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
@@ -890,7 +893,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             mv = (mrow != nullptr && key < key_end) ? __half2float(__ushort_as_half(__ldg(mrow + key))) : 0.f;
           }
           const float xv = fmaf(slope, (float)(key - alibi_ref), sv + mv);
-          x[j] = (vec_mask || key < key_end) ? xv : -INFINITY;
+          x[j] = key < key_end ? xv : -INFINITY;
         }
       } else {
         if (vec_mask) {
@@ -905,6 +908,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               x[j] = fmaf(__uint_as_float(sr[j]), p.scale, f.x);
               x[j + 1] = fmaf(__uint_as_float(sr[j + 1]), p.scale, f.y);
             }
+          }
+          if (key0 + kHalf > key_end) {  // ragged tile: cells past the unit's keys drop out
+#pragma unroll
+            for (int j = 0; j < kHalf; ++j)
+              if (key0 + j >= key_end) x[j] = -INFINITY;
           }
         } else {
 #pragma unroll
@@ -1350,23 +1358,25 @@ __global__ void __launch_bounds__(128)
 // (mla_fa_combine): the log-sum-exp combine across calls, with natural-log lse.
 // One CTA of 128 threads per row (grid-stride over the rows), thread i owning value
 // columns 4i..4i+3; every thread reads the parts' lse (the same addresses across the
-// CTA), then sums the weighted parts.
+// CTA), then sums the weighted parts. Part p's rows start o_stride (and lse_stride)
+// floats after part p - 1's, so the parts may sit in one packed buffer per part.
 __global__ void __launch_bounds__(128)
-    mla_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts,
-                     int n_parts, int64_t rows, float* __restrict__ out, float* __restrict__ out_lse) {
+    mla_merge_kernel(const float* __restrict__ o_parts, int64_t o_stride, const float* __restrict__ lse_parts,
+                     int64_t lse_stride, int n_parts, int64_t rows, float* __restrict__ out,
+                     float* __restrict__ out_lse) {
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     float mx = -INFINITY;
-    for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, __ldg(lse_parts + (int64_t)p * rows + r));
+    for (int p = 0; p < n_parts; ++p) mx = fmaxf(mx, __ldg(lse_parts + (int64_t)p * lse_stride + r));
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float wsum = 0.f;
     if (mx != -INFINITY) {
 #pragma unroll 4
       for (int p = 0; p < n_parts; ++p) {
-        const float l = __ldg(lse_parts + (int64_t)p * rows + r);
+        const float l = __ldg(lse_parts + (int64_t)p * lse_stride + r);
         const float w = l == -INFINITY ? 0.f : ex2_approx((l - mx) * kLog2e);
         if (w == 0.f) continue;  // the same in every thread of the CTA
         const float4 x =
-            __ldg(reinterpret_cast<const float4*>(o_parts + ((int64_t)p * rows + r) * kDV) + threadIdx.x);
+            __ldg(reinterpret_cast<const float4*>(o_parts + (int64_t)p * o_stride + r * kDV) + threadIdx.x);
         acc.x = fmaf(w, x.x, acc.x);
         acc.y = fmaf(w, x.y, acc.y);
         acc.z = fmaf(w, x.z, acc.z);

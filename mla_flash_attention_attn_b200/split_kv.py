@@ -37,26 +37,27 @@ def decode(q, kcache_shard, kv_type, mask_shard, scale, kv_len_shard=None, group
     mask_shard: the mask's columns for those cells, f16 [n_seq][n_q][cells] or None;
     kv_len_shard: valid cells of each sequence in the shard (host ints), or None for all.
     Returns the merged out, fp32 [n_seq][n_q][n_head][512], on every rank.
-    `forward` and `combine` default to this library's calls (binding.forward,
-    binding.combine); tests of the orchestration on CPU pass stand-ins with the same
-    signatures."""
+
+    The rank writes its O rows and their lse straight into one packed buffer
+    (binding.packed_width(rows) floats: O, then lse), and a single all-gather brings the
+    ranks' buffers together in rank order: rows x (512 + 1) x 4 bytes sent per rank and
+    step. `forward` and `combine` default to this library's calls (binding.forward,
+    binding.combine_packed); tests of the orchestration on CPU pass stand-ins with the
+    same signatures."""
     import torch
     import torch.distributed as dist
 
     forward = forward or binding.forward
-    combine = combine or binding.combine
+    combine = combine or binding.combine_packed
     world = dist.get_world_size(group)
     n_seq, n_q, n_head = q.shape[:3]
     rows = n_seq * n_q * n_head
-    # the ranks' results land in one buffer each for O and lse: part r = rank r
-    o_all = torch.empty((world, rows, DV), dtype=torch.float32, device=q.device)
-    lse_all = torch.empty((world, rows), dtype=torch.float32, device=q.device)
-    me = dist.get_rank(group)
-    o_mine = o_all[me].view(n_seq, n_q, n_head, DV)
-    lse_mine = lse_all[me].view(n_seq, n_q, n_head)
-    forward(q, kcache_shard, kv_type, mask_shard, scale, out=o_mine, kv_len=kv_len_shard,
-            out_lse=lse_mine)
-    dist.all_gather(list(o_all.unbind(0)), o_all[me].clone(), group=group)
-    dist.all_gather(list(lse_all.unbind(0)), lse_all[me].clone(), group=group)
-    out = combine(o_all, lse_all)
+    width = binding.packed_width(rows)
+    mine = torch.empty((width,), dtype=torch.float32, device=q.device)
+    forward(q, kcache_shard, kv_type, mask_shard, scale,
+            out=mine[: rows * DV].view(n_seq, n_q, n_head, DV), kv_len=kv_len_shard,
+            out_lse=mine[rows * DV:].view(n_seq, n_q, n_head))
+    parts = torch.empty((world * width,), dtype=torch.float32, device=q.device)
+    dist.all_gather_into_tensor(parts, mine, group=group)
+    out = combine(parts.view(world, width), rows)
     return out.view(n_seq, n_q, n_head, DV)

@@ -167,9 +167,9 @@ def test_compaction_argument_errors(lib):
     assert lib.mla_compact_mask_ex(FAKE + 1, 1, 10, 10, FAKE, 10, FAKE, FAKE, 4096, None) == -4
     assert lib.mla_compact_mask_ex(FAKE, 1, 10, 10, FAKE, 10, FAKE, None, 0, None) == -5
     assert lib.mla_compact_mask_ex(FAKE, 1, 5, 10, FAKE, 10, FAKE, FAKE, 4096, None) == -2
-    # 256 bytes of row tickets, then 8 bytes of look-back state per 16384-cell tile
-    assert lib.mla_compact_workspace_size(1, 131072) == 256 + 8 * 8
-    assert lib.mla_compact_workspace_size(3, 16385) == 256 + 3 * 2 * 8
+    # 256 bytes of row tickets, then 8 bytes of look-back state per 2048-cell tile
+    assert lib.mla_compact_workspace_size(1, 131072) == 256 + 64 * 8
+    assert lib.mla_compact_workspace_size(3, 2049) == 256 + 3 * 2 * 8
     assert lib.mla_compact_workspace_size(0, 10) == 0
 
 
@@ -185,6 +185,18 @@ def test_combine_argument_errors(lib):
     assert f(FAKE, FAKE, 2, 10, FAKE + 8, None, None) == -4
     assert f(FAKE, FAKE + 2, 2, 10, FAKE, None, None) == -4
     assert f(FAKE, FAKE, 2, 10, FAKE, FAKE + 1, None) == -4
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, 5 * 512, FAKE, 5, 2, 5, FAKE, None), -1),
+    ((FAKE, 5 * 512 - 4, FAKE, 5, 2, 5, FAKE, None), -2),   # parts overlap
+    ((FAKE, 5 * 512, FAKE, 4, 2, 5, FAKE, None), -2),
+    ((FAKE, 5 * 512 + 2, FAKE, 5, 2, 5, FAKE, None), -4),   # O rows of a part misaligned
+    ((FAKE, 5 * 513, FAKE, 5 * 513, 0, 5, FAKE, None), -2),
+])
+def test_strided_combine_argument_errors(lib, args, expect):
+    o, os_, l, ls, n, rows, out, out_lse = args
+    assert lib.mla_fa_combine_strided(o, os_, l, ls, n, rows, out, out_lse, None) == expect
 
 
 def test_valid_arguments_reach_the_device_check(lib):

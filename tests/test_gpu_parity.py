@@ -267,8 +267,8 @@ def compact_gpu(row_np, lib_ws=True):
     return idx_h[:c]
 
 
-@pytest.mark.parametrize("n", [1, 7, 8, 9, 15, 16, 17, 2047, 2049, 5000, 16383, 16384, 16385,
-                               40000, 65537])
+@pytest.mark.parametrize("n", [1, 7, 8, 9, 15, 16, 17, 2047, 2048, 2049, 5000, 16383, 16384, 16385,
+                               40000, 65537, 100000])
 @pytest.mark.parametrize("p_keep", [0.0, 0.1, 0.5, 1.0])
 def test_compaction_bit_exact(n, p_keep):
     rng = np.random.default_rng(n + int(p_keep * 100))
@@ -733,20 +733,21 @@ def test_split_kv_decode_emulated_on_one_gpu(world):
     torch = torch_mod()
     from mla_flash_attention_attn_b200 import split_kv
 
+    # (the packed layout split_kv.decode gathers: each rank's O rows, then their lse)
     w = W.make("v3_batched_decode", n_kv=4096, len_lo=100, len_hi=4096)
     dev = torch.device("cuda")
     q = torch.from_numpy(w.q).to(dev)
     rows = w.n_seq * w.n_q * w.n_head
-    o_all = torch.empty((world, rows, 512), device=dev)
-    lse_all = torch.empty((world, rows), device=dev)
+    parts = torch.empty((world, binding.packed_width(rows)), device=dev)
     for r, (lo, hi) in enumerate(split_kv.shard_bounds(w.n_kv, world)):
         k = torch.from_numpy(w.kcache[:, lo:hi].copy()).to(dev)
         m = torch.from_numpy(w.mask[:, :, lo:hi].copy()).to(dev)
-        binding.forward(q, k, w.kv_type, m, w.scale, out=o_all[r].view(w.n_seq, 1, w.n_head, 512),
+        binding.forward(q, k, w.kv_type, m, w.scale,
+                        out=parts[r, : rows * 512].view(w.n_seq, 1, w.n_head, 512),
                         kv_len=split_kv.shard_lengths(w.kv_len, lo, hi),
-                        out_lse=lse_all[r].view(w.n_seq, 1, w.n_head))
+                        out_lse=parts[r, rows * 512:].view(w.n_seq, 1, w.n_head))
     lse_out = torch.empty((rows,), device=dev)
-    out = binding.combine(o_all, lse_all, out_lse=lse_out)
+    out = binding.combine_packed(parts, rows, out_lse=lse_out)
     torch.cuda.synchronize()
     assert binding.mla_get_device_status() == 0
     got = out.cpu().numpy().reshape(w.n_seq, -1, 512)

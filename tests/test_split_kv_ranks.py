@@ -40,12 +40,15 @@ def _oracle_forward(q, k, kv_type, mask, scale, out=None, kv_len=None, out_lse=N
         out_lse[b].copy_(torch.from_numpy(lse.reshape(out_lse[b].shape)))
 
 
-def _oracle_combine(o_all, lse_all):
+def _oracle_combine(parts, rows):
     import torch
 
     import oracle
 
-    o, _ = oracle.combine(o_all.numpy(), lse_all.numpy())
+    p = parts.numpy()
+    o_all = p[:, : rows * 512].reshape(p.shape[0], rows, 512)
+    lse_all = p[:, rows * 512:]
+    o, _ = oracle.combine(o_all, lse_all)
     return torch.from_numpy(o).float()
 
 
