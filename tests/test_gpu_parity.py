@@ -268,7 +268,7 @@ def compact_gpu(row_np, lib_ws=True):
 
 
 @pytest.mark.parametrize("n", [1, 7, 8, 9, 15, 16, 17, 2047, 2048, 2049, 5000, 16383, 16384, 16385,
-                               40000, 65537, 100000])
+                               40000, 65537, 100000, 262144, 262145, 600001])
 @pytest.mark.parametrize("p_keep", [0.0, 0.1, 0.5, 1.0])
 def test_compaction_bit_exact(n, p_keep):
     rng = np.random.default_rng(n + int(p_keep * 100))
