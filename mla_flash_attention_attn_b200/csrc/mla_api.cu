@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <utility>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -22,7 +23,7 @@ namespace {
 using mla::Plan;
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per bounded wait
-constexpr int kMinTilesPerSplit = 1;
+constexpr int kMinKeysPerSplit = 256;  // a KV split holds at least this many keys (one 256-key tile)
 
 thread_local cudaStream_t t_stream = nullptr;
 
@@ -254,9 +255,23 @@ int validate(const mla_fa_args* a, Resolved* r) {
 }
 
 // Split plan for sequences [s0, s0+n). Returns the partial slots it needs.
+// Keys per pipeline step of the attention kernel, which is also the plan's tile. The TMA
+// mode (dense f16 cache) takes steps of 128 keys when a sequence's keys are read by a
+// single 128-row group: the cache then streams from DRAM once, and 128-key steps
+// double-buffer S and P in TMEM, so that the K stream and Q.K^T run on while the softmax
+// and P.V work on the previous step. With several groups per sequence (a prefill chunk)
+// the keys come back from L2 and the MMAs bound the kernel: steps of 256 keys issue half
+// as many MMAs and softmax rounds per key. The gather and q8_0 modes take 256.
+int kernel_step(const Resolved& r) {
+  const mla_fa_args& a = r.a;
+  const bool tma = a.kcache_type != MLA_KV_Q8_0 && a.idx == nullptr && !a.mask_gather;
+  return tma && r.rows <= mla::kRowsPerGroup ? 128 : 256;
+}
+
 int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
   std::memset(plan, 0, sizeof(Plan));
   const mla_fa_args& a = r.a;
+  plan->tile_keys = kernel_step(r);
   plan->n_seq = n;
   plan->seq_offset = s0;
   plan->rows = r.rows;
@@ -272,7 +287,7 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
     int len = a.kv_len ? a.kv_len[s0 + b] : a.n_kv;
     if (a.idx != nullptr) len = (int)std::min<int64_t>(len, r.idx_ss);
     plan->kv_len[b] = len;
-    tiles[b] = (len + mla::kTileKeys - 1) / mla::kTileKeys;
+    tiles[b] = (len + plan->tile_keys - 1) / plan->tile_keys;
     sum_tiles += tiles[b];
   }
   const int64_t total_groups = (int64_t)n * plan->groups;
@@ -282,7 +297,7 @@ int build_plan(const Resolved& r, int s0, int n, int sm_count, Plan* plan) {
     for (int b = 0; b < n; ++b) {
       const double want = (double)pairs * tiles[b] / ((double)sum_tiles * plan->groups);
       int ns = (int)std::floor(want + 0.5);
-      ns = std::min(ns, std::max(1, tiles[b] / kMinTilesPerSplit));
+      ns = std::min(ns, std::max(1, tiles[b] / (kMinKeysPerSplit / plan->tile_keys)));
       nsplit[b] = std::max(ns, 1);
       want_units += (int64_t)plan->groups * nsplit[b];
     }
@@ -632,15 +647,18 @@ int make_part_map(CUtensorMap* m, void* base, uint64_t rows) {
   return res == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// One instance of the attention kernel, with its block size (cfg has the rest).
-template <int kMode, bool kVariant, bool kGather, int kNC = 9>
+// One instance of the attention kernel, with its block size and shared memory (cfg has
+// the rest).
+template <int kMode, bool kVariant, bool kGather, int kNC = 9, int kTK = 256>
 cudaError_t launch_fwd(cudaLaunchConfig_t cfg, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                        const CUtensorMap& tm_v, const CUtensorMap& tm_o, const CUtensorMap& tm_w,
                        const mla::Plan& plan, const mla::MlaFwdParams& p) {
   cfg.blockDim = dim3(mla::FwdCfg<kMode>::kThreads);
-  return cudaLaunchKernelEx(&cfg, mla::mla_fwd_kernel<kMode, kVariant, kGather, kNC>, tm_q, tm_k, tm_v,
-                            tm_o, tm_w, plan, p);
+  cfg.dynamicSmemBytes = mla::fwd::Geo<kTK>::kSmemAlloc;
+  return cudaLaunchKernelEx(&cfg, mla::mla_fwd_kernel<kMode, kVariant, kGather, kNC, kTK>, tm_q, tm_k,
+                            tm_v, tm_o, tm_w, plan, p);
 }
+
 
 int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, cudaStream_t stream) {
   if (r.dk == MLA_HEADS_DK) return run_heads(r, st, ws, ws_bytes, stream);
@@ -655,7 +673,7 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   int rc = make_map(&tm_q, a.q, r.dk, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
   if (rc == MLA_OK && mode == mla::kModeTma) {
     rc = make_map(&tm_k, a.kcache, r.dk, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
-                  64, mla::kTileKeys / 2);
+                  64, (uint32_t)kernel_step(r) / 2);
     if (rc == MLA_OK) {
       // value view: {64 columns, keys, 8 column blocks, sequences}; a box of
       // {64, 64, 2, 1} lands as [column block][key][64 columns]
@@ -686,23 +704,27 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   }
   if (rc != MLA_OK) return rc;
   if (!st->fwd_attr_set) {
-    const void* fwd_kernels[] = {
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, true, false, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, false, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, true, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, true, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, false, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, false, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, true, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, true, 9>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 8>,
-        (const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false, 8>};
+    constexpr int kSmem256 = mla::fwd::Geo<256>::kSmemAlloc, kSmem128 = mla::fwd::Geo<128>::kSmemAlloc;
+    const std::pair<const void*, int> fwd_kernels[] = {
+        {(const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeTma, true, false, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 9, 128>, kSmem128},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeTma, true, false, 9, 128>, kSmem128},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, false, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, true, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, true, true, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, false, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, false, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeQ8, false, true, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeQ8, true, true, 9, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 8, 256>, kSmem256},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeTma, false, false, 8, 128>, kSmem128},
+        {(const void*)mla::mla_fwd_kernel<mla::kModeGatherF16, false, false, 8, 256>, kSmem256}};
     bool ok = true;
-    for (const void* k : fwd_kernels)
-      ok = ok && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      mla::fwd::kSmemAlloc) == cudaSuccess;
+    for (const auto& k : fwd_kernels)
+      ok = ok && cudaFuncSetAttribute(k.first, cudaFuncAttributeMaxDynamicSharedMemorySize, k.second) ==
+                     cudaSuccess;
     if (!ok ||
         cudaFuncSetAttribute(mla::mla_combine_proj_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -793,7 +815,6 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     // every read of its inputs
     cudaLaunchConfig_t fcfg = {};
     fcfg.gridDim = dim3(2 * plan.total_units);
-    fcfg.dynamicSmemBytes = mla::fwd::kSmemAlloc;
     fcfg.stream = stream;
     cudaLaunchAttribute fattr[1];
     fattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -808,10 +829,15 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     {
       ProfScope prof(mode == mla::kModeTma ? kKernFwdF16
                      : mode == mla::kModeGatherF16 ? kKernFwdGather : kKernFwdQ8, stream);
+      const bool step128 = mode == mla::kModeTma && plan.tile_keys == 128;
       if (r.dk != MLA_DK)  // the DK = DV = 512 shape: dense or index-list, f16 cache
         fe = mode == mla::kModeTma
-                 ? launch_fwd<mla::kModeTma, false, false, 8>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                 ? (step128 ? launch_fwd<mla::kModeTma, false, false, 8, 128>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                            : launch_fwd<mla::kModeTma, false, false, 8>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p))
                  : launch_fwd<mla::kModeGatherF16, false, false, 8>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
+      else if (mode == mla::kModeTma && step128)
+        fe = variant ? launch_fwd<mla::kModeTma, true, false, 9, 128>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
+                     : launch_fwd<mla::kModeTma, false, false, 9, 128>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);
       else if (mode == mla::kModeTma)
         fe = variant ? launch_fwd<mla::kModeTma, true, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p)
                      : launch_fwd<mla::kModeTma, false, false>(fcfg, tm_q, tm_k, tm_v, tm_o, tm_w, plan, p);

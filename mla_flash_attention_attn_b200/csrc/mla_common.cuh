@@ -9,7 +9,6 @@ constexpr int kDK = 576;             // cache row / query width (512 latent + 64
 constexpr int kDV = 512;             // value width: first 512 columns of the row
 constexpr int kRowsPerGroup = 128;   // M of the 2-SM MMA (64 rows in each CTA)
 constexpr int kRowsPerCta = 64;
-constexpr int kTileKeys = 256;       // N of one Q.K^T MMA: keys per tile
 constexpr int kPlanMaxSeq = 128;     // sequences per launch (larger batches are chunked)
 constexpr int kQ8RowBytes = 612;     // q8_0: 18 blocks of {f16 d; int8 q[32]}
 constexpr float kLog2e = 1.4426950408889634f;
@@ -35,6 +34,7 @@ struct Plan {
   int n_split[kPlanMaxSeq];          // KV splits of each sequence
   int kv_len[kPlanMaxSeq];           // dense: cells read for each sequence
   int ws_base[kPlanMaxSeq];          // first partial slot (-1: no split, direct output)
+  int tile_keys;                     // keys of a plan tile: the attention kernel's step (128 or 256)
 };
 
 }  // namespace mla

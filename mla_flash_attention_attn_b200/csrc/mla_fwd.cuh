@@ -97,56 +97,74 @@ enum FwdMode {
 
 namespace fwd {
 
-constexpr int kKStages = 4;      // ring of Q.K^T operand stages (K chunks, from DRAM)
-constexpr int kVStages = 3;      // ring of P.V operand stages (V columns, L2-resident)
 constexpr int kChunkBytes = 8192;                 // 64 rows x 64 f16 (one swizzle tile)
-constexpr int kKChunkBytes = 2 * kChunkBytes;     // 128 keys x 64 columns
 constexpr int kQBytes = 9 * kChunkBytes;          // this CTA's 64 query rows x 576, resident
-constexpr int kKStageBytes = kKChunkBytes;
 constexpr int kVStageBytes = 2 * kChunkBytes;     // V stage: 64 keys x 128 value columns
-constexpr int kXRounds = 1;                       // P exchange rounds per tile (1 or 2)
-constexpr int kXWords = 64 / kXRounds;            // f16 pairs per lane and round
-constexpr int kXBytes = 128 * kXWords * 4;        // P exchange buffer
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKStages * kKStageBytes;
-constexpr int kOffX = kOffV + kVStages * kVStageBytes;
-constexpr int kOffBar = kOffX + kXBytes;
-constexpr int kBarBytes = 8 * (2 * kKStages + 2 * kVStages + 1 + 1 + 2 + 2 + 1);
-constexpr int kOffTmemSlot = kOffBar + kBarBytes;
-constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
-constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
-constexpr int kSmemBytes = kOffXl + 128 * 4;
-constexpr int kSmemAlloc = kSmemBytes + 1024;                   // 1024-byte alignment slack
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S (fp32 scores of 128 keys per lane), P (f16 pairs of the tile's 256
-// keys per lane), O (256 fp32 columns: 128 values of each value half per lane)
-constexpr uint32_t kTmemS = 0;
-constexpr uint32_t kTmemP = 128;
-constexpr uint32_t kTmemO = 256;
-constexpr float kRescaleThreshold = 5.5451774f;                 // 8 ln 2 (natural units)
+constexpr float kRescaleThreshold = 5.5451774f;   // 8 ln 2 (natural units)
 
-static_assert(kSmemAlloc <= 232448, "shared memory beyond the 227 KB per-CTA limit");
-static_assert(kTmemO + 256 <= kTmemCols, "S, P and O exceed the TMEM allocation");
-static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
-              "128-byte swizzle needs 1 KB alignment");
-static_assert(kOffBar >= 128 * 1024, "the epilogue stages O in the first 128 KB");
+// Layout of the pipeline for steps of kTK keys (one Q.K^T MMA has N = kTK; CTA c
+// loads keys [c kTK/2, (c+1) kTK/2) of a step):
+//  * kTK = 256: one S buffer and one P buffer of 128 TMEM columns; the K ring holds 4
+//    stages of 128 keys x 64 columns (16 KB).
+//  * kTK = 128: two S buffers and two P buffers of 64 columns (step i uses buffer
+//    i % 2), so that Q.K^T of step i+1 runs while the softmax reads S(i), and the
+//    softmax writes P(i) while P.V(i-1) still reads P(i-1); the K ring holds 10 stages
+//    of 64 keys x 64 columns (8 KB), more than a step's 9 chunks.
+// TMEM columns: S buffers from 0, P buffers from 128 (f16 pairs of all kTK keys of the
+// step, in both lanes of a row), O from 256 (256 fp32 columns: 128 values of each value
+// half per lane).
+template <int kTK>
+struct Geo {
+  static_assert(kTK == 128 || kTK == 256, "steps of 128 or 256 keys");
+  static constexpr int kBufs = kTK == 128 ? 2 : 1;        // S buffers and P buffers
+  static constexpr int kKStages = kTK == 128 ? 10 : 4;    // ring of Q.K^T operand stages
+  static constexpr int kVStages = 3;                      // ring of P.V operand stages (L2-resident V)
+  static constexpr int kKStageBytes = kTK * 64;           // kTK/2 keys x 64 columns, f16
+  static constexpr int kXWords = kTK / 4;                 // f16 pairs a lane swaps per step
+  static constexpr int kXBytes = 128 * kXWords * 4;       // P exchange buffer
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKStageBytes;
+  static constexpr int kOffX = kOffV + kVStages * kVStageBytes;
+  static constexpr int kOffBar = kOffX + kXBytes;
+  static constexpr int kBarBytes = 8 * (2 * kKStages + 2 * kVStages + 2 * kBufs + 2 + 2 + 1);
+  static constexpr int kOffTmemSlot = kOffBar + kBarBytes;
+  static constexpr int kOffXmax = ((kOffTmemSlot + 4 + 15) / 16) * 16;  // float[2][128]
+  static constexpr int kOffXl = kOffXmax + 2 * 128 * 4;                  // float[128]
+  static constexpr int kSmemBytes = kOffXl + 128 * 4;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;                   // 1024-byte alignment slack
+  static constexpr uint32_t kSCols = kTK / 2;   // TMEM columns of one S or one P buffer
+  static constexpr uint32_t kTmemS = 0;
+  static constexpr uint32_t kTmemP = 128;
+  static constexpr uint32_t kTmemO = 256;
+  static constexpr uint32_t kIdescQK = idesc_f16_f32(128, kTK, 0, 0);  // K-major A and B
+  static constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);  // A (P, TMEM) K-major, B (V) MN-major
 
-constexpr uint32_t kIdescQK = idesc_f16_f32(128, 256, 0, 0);    // K-major A and B
-constexpr uint32_t kIdescPV = idesc_f16_f32(128, 256, 0, 1);    // A (P, TMEM) K-major, B (V) MN-major
+  static_assert(kSmemAlloc <= 232448, "shared memory beyond the 227 KB per-CTA limit");
+  static_assert(kBufs * kSCols <= kTmemP && kTmemP + kBufs * kSCols <= kTmemO && kTmemO + 256 <= kTmemCols,
+                "S, P and O exceed the TMEM allocation");
+  static_assert(kOffQ % 1024 == 0 && kOffK % 1024 == 0 && kOffV % 1024 == 0,
+                "128-byte swizzle needs 1 KB alignment");
+  static_assert(kOffBar >= 128 * 1024, "the epilogue stages O in the first 128 KB");
+};
 
-struct Bars {
-  uint64_t k_full[kKStages];     // leader: both CTAs' K chunk bytes landed
-  uint64_t k_empty[kKStages];    // both: the Q.K^T MMAs reading a stage are done
-  uint64_t v_full[kVStages];     // leader: both CTAs' V chunk bytes landed
-  uint64_t v_empty[kVStages];    // both: the P.V MMAs reading a V stage are done
-  uint64_t s_full;               // both: S written by Q.K^T
-  uint64_t s_free;               // leader: S read out by the softmax (8 warp arrivals)
+template <int kKS, int kVS, int kB>
+struct BarsT {
+  uint64_t k_full[kKS];          // leader: both CTAs' K chunk bytes landed
+  uint64_t k_empty[kKS];         // both: the Q.K^T MMAs reading a stage are done
+  uint64_t v_full[kVS];          // leader: both CTAs' V chunk bytes landed
+  uint64_t v_empty[kVS];         // both: the P.V MMAs reading a V stage are done
+  uint64_t s_full[kB];           // both: S buffer written by Q.K^T
+  uint64_t s_free[kB];           // leader: S buffer read out by the softmax (8 warp arrivals)
   uint64_t p_full[2];            // leader: P written to TMEM (8 warp arrivals, both CTAs)
-  uint64_t o_done[2];            // both: P.V of a tile (parity-indexed) complete
+  uint64_t o_done[2];            // both: P.V of a step (parity-indexed) complete
   uint64_t q_full;               // leader, gather modes: both CTAs' Q rows landed (TMA)
 };
-static_assert(sizeof(Bars) == kBarBytes, "barrier block size");
+template <int kTK>
+using BarsOf = BarsT<Geo<kTK>::kKStages, Geo<kTK>::kVStages, Geo<kTK>::kBufs>;
+static_assert(sizeof(BarsOf<256>) == Geo<256>::kBarBytes && sizeof(BarsOf<128>) == Geo<128>::kBarBytes,
+              "barrier block size");
 
 }  // namespace fwd
 
@@ -246,8 +264,9 @@ __device__ __forceinline__ void block_values(const RawBlock<kMode>& rb, uint32_t
 // that compacts the mask itself (gather modes only). The host launches them only when a
 // call asks for them, so the common path carries none of that code. kNC: 64-column
 // chunks of the head width, 9 (576: 512 latent + 64 RoPE) or 8 (the DK = DV = 512
-// shape, f16 cache, V the whole row).
-template <int kMode, bool kVariant, bool kGather, int kNC>
+// shape, f16 cache, V the whole row). kTK: keys of a pipeline step (128 or 256; the
+// gather modes take 256).
+template <int kMode, bool kVariant, bool kGather, int kNC, int kTK>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThreads, 1)
     mla_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k,
@@ -256,27 +275,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                    const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ Plan plan,
                    const __grid_constant__ MlaFwdParams p) {
   using namespace fwd;
+  using G = Geo<kTK>;
   constexpr bool kManual = FwdCfg<kMode>::kManual;
   static_assert(kNC == 9 || (kNC == 8 && kMode != kModeQ8), "head width 576, or 512 with an f16 cache");
+  static_assert(kTK == 256 || !kManual, "the gather modes' producers fill 256-key steps");
+  constexpr int kKStages = G::kKStages;
+  constexpr int kKStageBytes = G::kKStageBytes;
+  constexpr int kVStages = G::kVStages;
+  constexpr int kXRounds = 1;                   // P exchange rounds per step
+  constexpr int kXWords = G::kXWords;
+  constexpr int kBufs = G::kBufs;
+  constexpr uint32_t kSCols = G::kSCols;
+  constexpr uint32_t kTmemS = G::kTmemS, kTmemP = G::kTmemP, kTmemO = G::kTmemO;
+  constexpr uint32_t kIdescQK = G::kIdescQK, kIdescPV = G::kIdescPV;
+  using Bars = BarsOf<kTK>;
   // bytes of a cache row: q8_0 rows are 612 bytes; f16 rows 2 x the head width
   constexpr int kRowBytes = kMode == kModeQ8 ? kQ8RowBytes : 128 * kNC;
   extern __shared__ uint8_t smem_raw[];
   // a launch with too little dynamic shared memory reports and returns (every CTA takes
   // this branch, so no cluster barrier is left waiting)
-  if (dynamic_smem_bytes() < (uint32_t)fwd::kSmemAlloc) {
+  if (dynamic_smem_bytes() < (uint32_t)G::kSmemAlloc) {
     if (threadIdx.x == 0) record_status(kStatusLaunch);
     return;
   }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem + kOffQ;
-  uint8_t* sK = smem + kOffK;
-  uint8_t* sV = smem + kOffV;
-  uint4* sX = reinterpret_cast<uint4*>(smem + kOffX);
-  Bars& bars = *reinterpret_cast<Bars*>(smem + kOffBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
-  float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
-  float* xl = reinterpret_cast<float*>(smem + kOffXl);
+  uint8_t* sQ = smem + G::kOffQ;
+  uint8_t* sK = smem + G::kOffK;
+  uint8_t* sV = smem + G::kOffV;
+  uint4* sX = reinterpret_cast<uint4*>(smem + G::kOffX);
+  Bars& bars = *reinterpret_cast<Bars*>(smem + G::kOffBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + G::kOffTmemSlot);
+  float* xmax = reinterpret_cast<float*>(smem + G::kOffXmax);
+  float* xl = reinterpret_cast<float*>(smem + G::kOffXl);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -295,8 +326,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       mbar_init(&bars.v_full[i], kManual ? 4 : 1);
       mbar_init(&bars.v_empty[i], 1);
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_free, 8);
+    for (int i = 0; i < kBufs; ++i) {
+      mbar_init(&bars.s_full[i], 1);
+      mbar_init(&bars.s_free[i], 8);
+    }
     mbar_init(&bars.q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.p_full[i], 8);
@@ -411,7 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     __syncthreads();  // the list is complete and visible to every thread of this CTA
     len = base;
     tile_begin = 0;
-    n_tiles = (len + kTileKeys - 1) / kTileKeys;
+    n_tiles = (len + kTK - 1) / kTK;
     key_end = len;
   } else {
     len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
@@ -419,15 +452,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       // tiles the mask leaves something in (dense mode; the range is within the length)
       tile_begin = du.tile_begin;
       n_tiles = idle ? 0 : du.n_tiles;
-      key_end = min(len, (tile_begin + n_tiles) * kTileKeys);
+      key_end = min(len, (tile_begin + n_tiles) * kTK);
     } else {
-      const int n_tiles_total = (len + kTileKeys - 1) / kTileKeys;
+      const int n_tiles_total = (len + kTK - 1) / kTK;
       tile_begin = (int)((int64_t)s * n_tiles_total / n_split);
       const int tile_end = (int)((int64_t)(s + 1) * n_tiles_total / n_split);
       n_tiles = tile_end - tile_begin;
-      key_end = min(len, tile_end * kTileKeys);
+      key_end = min(len, tile_end * kTK);
     }
   }
+  // the plan's tiles are the pipeline's steps of kTK keys (the host plans in steps of
+  // the instance it launches), over [key_start, key_end)
+  const int key_start = tile_begin * kTK;
+  const int n_steps = n_tiles;
   bool failed = false;
 
   if constexpr (kManual) {
@@ -438,13 +475,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
   if (warp == 0) {
     // ================= producer (TMA mode): K chunks; the first tile's stages also
     // bring the matching chunk of this CTA's 64 query rows, which stay resident
-    if (!kManual && n_tiles > 0 && elect_one()) {
-      // this CTA's 128 keys of each tile, 9 chunks of 64 columns, as far ahead as the
+    if (!kManual && n_steps > 0 && elect_one()) {
+      // this CTA's kTK/2 keys of each step, 9 chunks of 64 columns, as far ahead as the
       // ring allows (only Q.K^T consumption frees stages)
       int stage = 0;
       uint32_t ephase = 0;
-      for (int i = 0; i < n_tiles && !failed; ++i) {
-        const int key0 = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
+      for (int i = 0; i < n_steps && !failed; ++i) {
+        const int key0 = key_start + i * kTK + (kTK / 2) * (int)rank;
         for (int c = 0; c < kNC; ++c) {
           if (!mbar_wait(&bars.k_empty[stage], ephase ^ 1, to)) {
             // stop issuing: a stage may still be in use, and the copies already in
@@ -465,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       }
     }
     // gather modes: this CTA's Q rows by TMA (the producers gather K and V)
-    if (kManual && n_tiles > 0 && elect_one()) {
+    if (kManual && n_steps > 0 && elect_one()) {
       if (rank == 0) mbar_arrive_expect_tx(&bars.q_full, 2 * kNC * kChunkBytes);
       const uint32_t fq = mapa_shared(smem_u32(&bars.q_full), 0);
       for (int c = 0; c < kNC; ++c)
@@ -474,12 +511,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     __syncwarp();
   } else if (warp == 2) {
     // ================= V producer (TMA mode): value columns of each tile, own ring
-    if (!kManual && n_tiles > 0 && elect_one()) {
+    if (!kManual && n_steps > 0 && elect_one()) {
       int stage = 0;
       uint32_t ephase = 0;
-      for (int j = 0; j < n_tiles && !failed; ++j) {
-        const int key0 = (tile_begin + j) * kTileKeys;
-        for (int kg = 0; kg < kTileKeys / 64 && !failed; ++kg)
+      for (int j = 0; j < n_steps && !failed; ++j) {
+        const int key0 = key_start + j * kTK;
+        for (int kg = 0; kg < kTK / 64 && !failed; ++kg)
           for (int nb = 0; nb < 2; ++nb) {
             if (!mbar_wait(&bars.v_empty[stage], ephase ^ 1, to)) {
               failed = true;  // stop issuing (see the K producer)
@@ -503,7 +540,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // waiting on a barrier would leave the pipe idle; with Q.K^T and P.V on separate
     // threads one thread's wait is covered by the other's MMAs. A commit tracks the
     // MMAs of the thread that issues it.
-    if (rank == 0 && n_tiles > 0 && elect_one()) {
+    if (rank == 0 && n_steps > 0 && elect_one()) {
       // Descriptor bases; an operand at byte offset `off` within a region is the base
       // plus off/16 (the start address field is the low 14 bits, no carry possible
       // below 256 KB).
@@ -521,14 +558,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       }
       // On a timeout the issuer stops (no further MMAs or commits); the waits that
       // depend on its commits then time out in turn and the kernel winds down.
-      for (int t = 0; t < n_tiles && !failed; ++t) {
-        // S is free once the softmax has read the scores of tile t - 1
-        if (t >= 1 && !mbar_wait_cluster(&bars.s_free, (t - 1) & 1, to)) {
+      for (int t = 0; t < n_steps && !failed; ++t) {
+        // S buffer t % kBufs is free once the softmax has read the scores of step t - kBufs
+        const int sb = t % kBufs;
+        if (t >= kBufs && !mbar_wait_cluster(&bars.s_free[sb], ((t - kBufs) / kBufs) & 1, to)) {
           failed = true;
           record_status(kStatusTimeout);
           break;
         }
-        const uint32_t d_s = tmem + kTmemS;
+        const uint32_t d_s = tmem + kTmemS + sb * kSCols;
         for (int c = 0; c < kNC; ++c) {
           const bool ok = kManual ? mbar_wait_cluster(&bars.k_full[kst], kph, to)
                                   : mbar_wait(&bars.k_full[kst], kph, to);
@@ -548,7 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           if (++kst == kKStages) { kst = 0; kph ^= 1; }
         }
         if (failed) break;
-        mma_commit_2sm_mc(&bars.s_full, 0x3);
+        mma_commit_2sm_mc(&bars.s_full[sb], 0x3);
       }
     }
     __syncwarp();
@@ -556,18 +594,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // ================= P.V issuer (leader CTA, one thread): per tile, wait for P, then
     // consume the V stages (64 keys x one 256-column half each) in the producer's order.
     // A (P) is read from TMEM: 16 keys per MMA are 8 columns of the P buffer.
-    if (rank == 0 && n_tiles > 0 && elect_one()) {
+    if (rank == 0 && n_steps > 0 && elect_one()) {
       const uint64_t dv = smem_desc_sw128(smem_u32(sV), 8192, 1024);
       constexpr uint32_t kVUnits = kVStageBytes >> 4;   // V stage stride
       int vst = 0;
       uint32_t vph = 0;
-      for (int t = 0; t < n_tiles && !failed; ++t) {  // stops on a timeout, as above
+      for (int t = 0; t < n_steps && !failed; ++t) {  // stops on a timeout, as above
         if (!mbar_wait_cluster(&bars.p_full[t & 1], (t >> 1) & 1, to)) {
           failed = true;
           record_status(kStatusTimeout);
           break;
         }
-        for (int kg = 0; kg < kTileKeys / 64 && !failed; ++kg)
+        const uint32_t p_buf = tmem + kTmemP + (t % kBufs) * kSCols;
+        for (int kg = 0; kg < kTK / 64 && !failed; ++kg)
           for (int nb = 0; nb < 2; ++nb) {
             const bool ok = kManual ? mbar_wait_cluster(&bars.v_full[vst], vph, to)
                                     : mbar_wait(&bars.v_full[vst], vph, to);
@@ -577,7 +616,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
               break;
             }
             tc_fence_after();
-            const uint32_t a0 = tmem + kTmemP + (uint32_t)(kg * 32);
+            const uint32_t a0 = p_buf + (uint32_t)(kg * 32);
             const uint64_t b0 = dv + (uint32_t)(vst * kVUnits);
             const uint32_t d = tmem + kTmemO + nb * 128;
             mma_f16_ts_2sm(d, a0, b0, kIdescPV, (t > 0 || kg > 0) ? 1u : 0u);
@@ -656,8 +695,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         // batch of kLoadBatch blocks go out before the previous batch is converted and
         // stored, so a chunk's load latency overlaps the previous chunk's work.
         constexpr int kBpc = 4 / kLoadBatch;  // batches per stage
-        for (int i = 0; i < n_tiles; ++i) {
-          const int kbase = (tile_begin + i) * kTileKeys + (kTileKeys / 2) * (int)rank;
+        for (int i = 0; i < n_steps; ++i) {
+          const int kbase = key_start + i * kTK + (kTK / 2) * (int)rank;
           const int half = pt & 1;
           int keys[4];
 #pragma unroll
@@ -711,18 +750,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         // one group ahead.
         const int q4 = pt & 3, box = q4 >> 1, half = q4 & 1;
         constexpr int kBpc = 4 / kLoadBatch;  // batches per stage
-        for (int j = 0; j < n_tiles; ++j) {
-          const int kbase = (tile_begin + j) * kTileKeys;
+        for (int j = 0; j < n_steps; ++j) {
+          const int kbase = key_start + j * kTK;
           int kc[4], kn[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) kc[q] = resolve(kbase + (pt >> 2) + 16 * q);
           RawBlock<kMode> cur[kLoadBatch];
 #pragma unroll
           for (int q = 0; q < kLoadBatch; ++q) load32(kc[q], 4 * (int)rank + q4, cur[q]);
-          for (int kg = 0; kg < kTileKeys / 64; ++kg) {
+          for (int kg = 0; kg < kTK / 64; ++kg) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              kn[q] = kg + 1 < kTileKeys / 64 ? resolve(kbase + 64 * (kg + 1) + (pt >> 2) + 16 * q) : -1;
+              kn[q] = kg + 1 < kTK / 64 ? resolve(kbase + 64 * (kg + 1) + (pt >> 2) + 16 * q) : -1;
 #pragma unroll
             for (int nb = 0; nb < 2; ++nb) {
               uint8_t* st = nullptr;
@@ -737,7 +776,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll
                 for (int q = 0; q < kLoadBatch; ++q) {
                   const int key = next_group ? kn[nq0 + q] : kc[nq0 + q];
-                  if (!next_group || kg + 1 < kTileKeys / 64) load32(key, 8 * nnb + 4 * (int)rank + q4, nxt[q]);
+                  if (!next_group || kg + 1 < kTK / 64) load32(key, 8 * nnb + 4 * (int)rank + q4, nxt[q]);
                   else { nxt[q].valid = false; nxt[q].odd = false; }
                 }
                 if (bq == 0) {
@@ -774,7 +813,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
                                ? p.mask + (int64_t)b_abs * p.mask_seq_stride +
                                      (int64_t)tok * p.mask_row_stride
                                : nullptr;
-    const uint32_t s_free_l = mapa_shared(smem_u32(&bars.s_free), 0);
+    const uint32_t s_free_l0 = mapa_shared(smem_u32(&bars.s_free[0]), 0);
+    const uint32_t s_free_l1 = mapa_shared(smem_u32(&bars.s_free[kBufs - 1]), 0);
     // variants: the ALiBi bias is slope * (key - position of the query), the query
     // tokens being the last n_q positions of the sequence (with sinks the softmax is no
     // longer shift invariant, so this position is the defined one)
@@ -795,7 +835,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     float m_ref = -INFINITY;  // reference max (natural units) used for exponentiation
     float l_part = 0.f;       // this lane's half of the row sum, relative to m_ref
 
-    constexpr int kHalf = kTileKeys / 2;  // keys of one lane (128)
+    constexpr int kHalf = kTK / 2;  // keys of one lane in a step
     // The mask loads of a tile are issued while the previous tile is still being
     // processed (after its exponentials), so their latency is hidden. Full tiles take
     // this vector path (zeros without a mask); a ragged last tile goes key by key.
@@ -812,18 +852,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     // key; otherwise it goes key by key.
     auto mask_vec_ok = [&](int t) {
       if ((kManual && sparse) || !row_valid) return true;
-      const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
+      const int k0 = key_start + t * kTK + kHalf * kh;
       if (mrow == nullptr) return true;  // no mask: zeros
       return p.mask_vec_ok && (k0 + kHalf <= key_end || k0 + kHalf <= p.n_kv);
     };
     auto load_mask = [&](int t) {
-      const int k0 = (tile_begin + t) * kTileKeys + kHalf * kh;
+      const int k0 = key_start + t * kTK + kHalf * kh;
       if (!row_valid) {
 #pragma unroll
         for (int c = 0; c < kHalf / 8; ++c) mvec[c] = make_uint4(0u, 0u, 0u, 0u);
       } else if (kManual && sparse) {
         const int32_t* ix = list_ptr();
         uint32_t* mw = reinterpret_cast<uint32_t*>(mvec);
+        static_assert(!kManual || kHalf == 128, "index-list steps of 256 keys");
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           int cl[64];
@@ -852,28 +893,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
       }
     };
-    bool vec_next = n_tiles > 0 && mask_vec_ok(0);
+    bool vec_next = n_steps > 0 && mask_vec_ok(0);
     if (vec_next) load_mask(0);
 
-    for (int i = 0; i < n_tiles; ++i) {
+    for (int i = 0; i < n_steps; ++i) {
       const int sb = i & 1;          // max-exchange slot and p_full barrier
-      const int key0 = (tile_begin + i) * kTileKeys + kHalf * kh;
+      const int buf = i % kBufs;     // S and P buffers of this step
+      const int key0 = key_start + i * kTK + kHalf * kh;
       const bool vec_mask = vec_next;
-      wait_local(&bars.s_full, i & 1);
+      wait_local(&bars.s_full[buf], (i / kBufs) & 1);
       tc_fence_after();
       // scores x = scale * s + mask (natural units); cells beyond the unit's keys are
-      // dropped. 128 values per lane, read from TMEM with 4 loads and one wait.
+      // dropped. kHalf values per lane, read from TMEM with kHalf / 32 loads and one wait.
       uint32_t sr[kHalf];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tmem_ld32(tmem + lane_base + kTmemS + 32 * q,
+      for (int q = 0; q < kHalf / 32; ++q)
+        tmem_ld32(tmem + lane_base + kTmemS + buf * kSCols + 32 * q,
                   *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * q));
       tmem_wait_ld();
-      // the scores are in registers: Q.K^T of the next tile may overwrite S (the loads
-      // are complete, so a relaxed arrive suffices)
+      // the scores are in registers: Q.K^T may overwrite this S buffer (the loads are
+      // complete, so a relaxed arrive suffices)
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster_relaxed(s_free_l);
+      if (lane == 0) mbar_arrive_cluster_relaxed(buf ? s_free_l1 : s_free_l0);
       float x[kHalf];
       if constexpr (kVariant) {
         // softcapped (or plainly scaled) score, then the mask, then the ALiBi bias
@@ -925,7 +967,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
           }
         }
       }
-      // row max over this lane's 128 keys (8 independent chains), then over the pair
+      // row max over this lane's kHalf keys (8 independent chains), then over the pair
       float m8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) m8[u] = x[u];
@@ -961,19 +1003,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       l_part = l_part * alpha + lsum;
       // next tile's mask: its loads overlap the rest of this tile (the scores are dead)
-      vec_next = i + 1 < n_tiles && mask_vec_ok(i + 1);
+      vec_next = i + 1 < n_steps && mask_vec_ok(i + 1);
       if (vec_next) load_mask(i + 1);
 
       // P goes to TMEM as the A operand of P.V. That MMA reads A for the value columns
       // of the first N half from lanes 0-63 and for the second half from lanes 64-127,
-      // so each of a row's two lanes needs all 256 keys: the lanes of a row swap their
-      // 128 keys through shared memory (the previous tile's reads of the exchange
+      // so each of a row's two lanes needs all kTK keys: the lanes of a row swap their
+      // kHalf keys through shared memory (the previous step's reads of the exchange
       // buffer finished before the max exchange barrier above).
       {
-        // keys 0..127 of the tile in columns 0..63, keys 128..255 in columns 64..127;
-        // kXRounds rounds of kXWords f16 pairs
-        const uint32_t a = tmem + lane_base + kTmemP;
-        const uint32_t a_own = a + 64 * kh, a_peer = a + 64 * (kh ^ 1);
+        // keys 0..kHalf-1 of the step in the buffer's first kHalf/2 columns, the other
+        // kHalf keys in the next kHalf/2; kXRounds rounds of kXWords f16 pairs
+        const uint32_t a = tmem + lane_base + kTmemP + buf * kSCols;
+        const uint32_t a_own = a + (kHalf / 2) * kh, a_peer = a + (kHalf / 2) * (kh ^ 1);
 #pragma unroll
         for (int rd = 0; rd < kXRounds; ++rd) {
           const int w0 = rd * kXWords;
@@ -990,8 +1032,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
             pw[4 * gq] = v.x; pw[4 * gq + 1] = v.y; pw[4 * gq + 2] = v.z; pw[4 * gq + 3] = v.w;
           }
           if (rd == 0) {
-            // the P buffer (and O) are free once P.V of the previous tile has completed
-            if (i > 0) wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
+            // this P buffer is free once P.V of step i - kBufs has completed (with one
+            // buffer that also leaves O free)
+            if (i >= kBufs) wait_local(&bars.o_done[(i - kBufs) & 1], ((i - kBufs) >> 1) & 1);
             tc_fence_after();
           }
 #pragma unroll
@@ -1003,9 +1046,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         }
         tmem_wait_st();
       }
-      // rescale O (only when some row of this warp raised its reference max); P.V(i-1)
-      // has completed (waited above)
+      // rescale O (only when some row of this warp raised its reference max), once
+      // P.V(i-1) has completed (P.V(i) waits for this step's P)
       if (__any_sync(0xffffffffu, need && i > 0)) {
+        if (kBufs > 1) {
+          wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
+          tc_fence_after();
+        }
 #pragma unroll 1
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t v[32];
@@ -1027,7 +1074,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     }
 
     // ---- epilogue
-    if (n_tiles > 0) wait_local(&bars.o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
+    if (n_steps > 0) wait_local(&bars.o_done[(n_steps - 1) & 1], ((n_steps - 1) >> 1) & 1);
     // a dependent (combine) launch may start scheduling; it waits for this grid's end
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_after();
@@ -1059,7 +1106,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
 #pragma unroll 1
       for (int g0 = 0; g0 < 8; g0 += kEpi) {
         uint32_t v[kEpi][32];
-        if (n_tiles > 0) {
+        if (n_steps > 0) {
 #pragma unroll
           for (int u = 0; u < kEpi; ++u) tmem_ld32(tmem + lane_base + kTmemO + 32 * (g0 + u), v[u]);
           tmem_wait_ld();

@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(256)
       first = min(first, red[0][w]);
       last = max(last, red[1][w]);
     }
-    ranges[bg] = last < 0 ? make_int2(0, 0) : make_int2(first / kTileKeys, last / kTileKeys + 1);
+    ranges[bg] = last < 0 ? make_int2(0, 0) : make_int2(first / plan.tile_keys, last / plan.tile_keys + 1);
   }
 }
 

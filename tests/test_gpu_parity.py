@@ -147,6 +147,25 @@ def test_large_finite_mask_values_and_shift():
     check_all_rows(w, run_gpu(w), what="large mask")
 
 
+def test_rising_scores_rescale_every_few_steps():
+    """One 128-row sequence of 2048 keys whose mask rises by 60 from the first key to the
+    last: its rows' running maximum passes the rescale threshold every one or two 128-key
+    steps. 74 one-key sequences beside it leave the plan unsplit (as many groups as SM
+    pairs), so one unit takes all 16 steps and rescales O in TMEM while the P.V of the
+    previous step may still be running."""
+    n_seq, n_kv = 75, 2048
+    w = W.make("v3_batched_decode", n_seq=n_seq, n_kv=n_kv, len_lo=1, len_hi=1)
+    w.kv_len[0] = n_kv
+    w.mask[0, 0] = np.linspace(0.0, 60.0, n_kv).astype(np.float16)
+    got = run_gpu(w)
+    for b in range(n_seq):
+        # cells past a sequence's length are -inf in its mask and add nothing: the oracle
+        # takes the valid prefix
+        n = int(w.kv_len[b])
+        ref = oracle.attention(w.q[b], w.kcache[b][:n], w.kv_type, w.mask[b][:, :n], w.scale)
+        assert_parity(got[b].reshape(-1, 512), ref, f"rising scores seq {b}")
+
+
 def test_zero_length_sequence_and_strided_cache():
     w = W.make("v3_batched_decode", n_seq=3, n_head=16, n_kv=700, len_lo=0, len_hi=700)
     w.kv_len[:] = [0, 1, 700]
