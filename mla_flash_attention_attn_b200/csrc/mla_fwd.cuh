@@ -893,6 +893,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
         for (int c = 0; c < kHalf / 8; ++c) mvec[c] = __ldg(mv + c);
       }
     };
+    // The mask cells of a step are a fresh DRAM read (a decode reads each once), and their
+    // load for step i+1 is issued during step i: too late to hide the latency of a loaded
+    // DRAM. Each lane's slice is therefore brought into L2 kMaskAhead steps ahead (dense
+    // steps whose slice lies inside the mask row).
+    constexpr int kMaskAhead = 4;
+    auto prefetch_mask = [&](int t) {
+      if ((kManual && sparse) || mrow == nullptr) return;
+      const int k0 = key_start + t * kTK + kHalf * kh;
+      if (k0 + kHalf > p.n_kv) return;
+#pragma unroll
+      for (int c = 0; c < kHalf * 2; c += 128) prefetch_l2(reinterpret_cast<const uint8_t*>(mrow + k0) + c);
+    };
+    for (int t = 0; t < kMaskAhead && t < n_steps; ++t) prefetch_mask(t);
     bool vec_next = n_steps > 0 && mask_vec_ok(0);
     if (vec_next) load_mask(0);
 
@@ -1005,6 +1018,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       // next tile's mask: its loads overlap the rest of this tile (the scores are dead)
       vec_next = i + 1 < n_steps && mask_vec_ok(i + 1);
       if (vec_next) load_mask(i + 1);
+      if (i + kMaskAhead < n_steps) prefetch_mask(i + kMaskAhead);
 
       // P goes to TMEM as the A operand of P.V. That MMA reads A for the value columns
       // of the first N half from lanes 0-63 and for the second half from lanes 64-127,
