@@ -16,6 +16,7 @@
 #include "mla_common.cuh"
 #include "mla_compact.cuh"
 #include "mla_fwd.cuh"
+#include "mla_gather.cuh"
 #include "mla_heads.cuh"
 
 namespace {
@@ -112,12 +113,13 @@ enum KernelId {
   kKernHeadsCombine = 8,
   kKernScan = 9,
   kKernDevPlan = 10,
+  kKernGatherRows = 11,
   kNumKernels
 };
 const char* const kKernelNames[kNumKernels] = {"mla_fwd_f16", "mla_fwd_gather_f16", "mla_fwd_q8_0",
                                                "mla_combine", "mla_compact", "mla_wait_timeout",
                                                "mla_merge", "mla_fwd_heads", "mla_combine_heads",
-                                               "mla_scan", "mla_device_plan"};
+                                               "mla_scan", "mla_device_plan", "mla_gather_rows"};
 struct ProfRecord {
   cudaEvent_t start, stop;
   int kernel;
@@ -262,9 +264,31 @@ int validate(const mla_fa_args* a, Resolved* r) {
 // and P.V work on the previous step. With several groups per sequence (a prefill chunk)
 // the keys come back from L2 and the MMAs bound the kernel: steps of 256 keys issue half
 // as many MMAs and softmax rounds per key. The gather and q8_0 modes take 256.
+// Index-list calls of a single 128-row group (a decode): the listed rows are first
+// gathered into a dense f16 buffer in the workspace (mla_gather_rows_kernel, every SM at
+// once), and the TMA-mode kernel streams that buffer. With more groups per sequence each
+// group would re-read the list's rows, so those calls keep the gather modes.
+bool gathered_rows(const Resolved& r) {
+  return r.a.idx != nullptr && !r.a.mask_gather && r.rows <= mla::kRowsPerGroup && r.dk != MLA_HEADS_DK;
+}
+
+// Rows per sequence in the gathered buffer: the most any sequence's list can use.
+int64_t gathered_cap(const Resolved& r) {
+  int64_t m = 0;
+  for (int b = 0; b < r.a.n_seq; ++b) m = std::max<int64_t>(m, r.a.kv_len ? r.a.kv_len[b] : r.a.n_kv);
+  return std::max<int64_t>(1, std::min<int64_t>(m, r.idx_ss));
+}
+int64_t gathered_mask_stride(const Resolved& r) { return (gathered_cap(r) + 63) / 64 * 64; }
+// Bytes of the gathered rows and of their mask values (every sequence of the call).
+size_t gathered_bytes(const Resolved& r) {
+  if (!gathered_rows(r)) return 0;
+  const size_t rows = (size_t)r.a.n_seq * gathered_cap(r) * r.dk * 2;
+  return (rows + 255) / 256 * 256 + (size_t)r.a.n_seq * r.a.n_q * gathered_mask_stride(r) * 2;
+}
+
 int kernel_step(const Resolved& r) {
   const mla_fa_args& a = r.a;
-  const bool tma = a.kcache_type != MLA_KV_Q8_0 && a.idx == nullptr && !a.mask_gather;
+  const bool tma = gathered_rows(r) || (a.kcache_type != MLA_KV_Q8_0 && a.idx == nullptr && !a.mask_gather);
   return tma && r.rows <= mla::kRowsPerGroup ? 128 : 256;
 }
 
@@ -605,7 +629,21 @@ size_t workspace_for(const Resolved& r, int sm_count, int* max_units, int* max_s
   }
   if (max_units) *max_units = mu;
   if (max_splits) *max_splits = ms;
+  // gathered rows: after the partials (the same offset for every launch of the call)
+  if (gathered_rows(r)) need = (need + 255) / 256 * 256 + gathered_bytes(r);
   return need;
+}
+
+// Offset of the gathered rows in the workspace (256-aligned, after every launch's partials).
+size_t gathered_offset(const Resolved& r, int sm_count) {
+  size_t need = 0;
+  Plan plan;
+  for (int s0 = 0; s0 < r.a.n_seq; s0 += mla::kPlanMaxSeq) {
+    const int n = std::min(mla::kPlanMaxSeq, r.a.n_seq - s0);
+    const int slots = build_plan(r, s0, n, sm_count, &plan);
+    need = std::max(need, (size_t)slots * slot_bytes() + gather_bytes(r, plan, slots));
+  }
+  return (need + 255) / 256 * 256;
 }
 
 int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
@@ -666,22 +704,40 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   const size_t need = workspace_for(r, st->sm_count, nullptr, nullptr);
   if (need > 0 && (ws == nullptr || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255)))
     return MLA_ERR_WORKSPACE;
-  const int mode = a.kcache_type == MLA_KV_Q8_0 ? mla::kModeQ8
+  // index lists of a single group: the rows are gathered into the workspace first, and
+  // the TMA mode streams them (gathered_rows)
+  const bool gat = gathered_rows(r);
+  const int mode = gat ? mla::kModeTma
+                   : a.kcache_type == MLA_KV_Q8_0 ? mla::kModeQ8
                    : (a.idx != nullptr || a.mask_gather ? mla::kModeGatherF16 : mla::kModeTma);
+  const int64_t g_cap = gat ? gathered_cap(r) : 0;
+  const int64_t g_mstride = gat ? gathered_mask_stride(r) : 0;
+  uint16_t* g_rows = nullptr;
+  uint16_t* g_mask = nullptr;
+  if (gat) {
+    const size_t off = gathered_offset(r, st->sm_count);
+    g_rows = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + off);
+    g_mask = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + off +
+                                         ((size_t)a.n_seq * g_cap * r.dk * 2 + 255) / 256 * 256);
+  }
+  // the cells the TMA mode streams: the cache, or the gathered rows
+  const void* k_base = gat ? static_cast<const void*>(g_rows) : a.kcache;
+  const uint64_t k_rows = gat ? (uint64_t)g_cap : (uint64_t)a.n_kv;
   CUtensorMap tm_q, tm_k, tm_v;
   const uint64_t row_bytes = (uint64_t)r.dk * 2;
+  const uint64_t k_seq_bytes = gat ? (uint64_t)g_cap * row_bytes : (uint64_t)r.k_ss * row_bytes;
   int rc = make_map(&tm_q, a.q, r.dk, r.rows, a.n_seq, row_bytes, (uint64_t)r.q_ss * 2, 64, 64);
   if (rc == MLA_OK && mode == mla::kModeTma) {
-    rc = make_map(&tm_k, a.kcache, r.dk, a.n_kv, a.n_seq, row_bytes, (uint64_t)r.k_ss * row_bytes,
-                  64, (uint32_t)kernel_step(r) / 2);
+    rc = make_map(&tm_k, k_base, r.dk, k_rows, a.n_seq, row_bytes, k_seq_bytes, 64,
+                  (uint32_t)kernel_step(r) / 2);
     if (rc == MLA_OK) {
       // value view: {64 columns, keys, 8 column blocks, sequences}; a box of
       // {64, 64, 2, 1} lands as [column block][key][64 columns]
-      cuuint64_t dims[4] = {64, (cuuint64_t)a.n_kv, 8, (cuuint64_t)a.n_seq};
-      cuuint64_t strides[3] = {row_bytes, 128, (cuuint64_t)r.k_ss * row_bytes};
+      cuuint64_t dims[4] = {64, (cuuint64_t)k_rows, 8, (cuuint64_t)a.n_seq};
+      cuuint64_t strides[3] = {row_bytes, 128, k_seq_bytes};
       cuuint32_t box[4] = {64, 64, 2, 1};
       cuuint32_t es[4] = {1, 1, 1, 1};
-      CUresult res = g_encode(&tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(a.kcache),
+      CUresult res = g_encode(&tm_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void*>(k_base),
                               dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -748,6 +804,16 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   p.n_kv = a.n_kv;
   p.idx = a.idx;
   p.idx_count = a.idx_count;
+  if (gat) {
+    // the kernel streams the gathered rows, with their gathered mask values, up to each
+    // list's count
+    p.idx = nullptr;
+    p.mask = g_mask;
+    p.mask_seq_stride = (int64_t)a.n_q * g_mstride;
+    p.mask_row_stride = g_mstride;
+    p.mask_vec_ok = 1;
+    p.n_kv = (int)g_mstride;
+  }
   p.idx_seq_stride = r.idx_ss;
   p.softcap = a.softcap;
   p.slopes = a.alibi_slopes;
@@ -809,6 +875,47 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     if (slots > 0) {
       rc = make_part_map(&tm_w, ws, (uint64_t)slots * mla::kRowsPerGroup);
       if (rc != MLA_OK) return rc;
+    }
+    if (gat) {
+      // the lists' rows (and mask values) into the dense buffer, every SM at once; a
+      // programmatic dependent of the kernel that wrote the lists
+      mla::GatherParams gp;
+      gp.idx = a.idx;
+      gp.idx_count = a.idx_count;
+      gp.idx_seq_stride = r.idx_ss;
+      gp.kcache = static_cast<const uint8_t*>(a.kcache);
+      gp.k_seq_stride = r.k_ss;
+      gp.n_kv = a.n_kv;
+      gp.mask = static_cast<const uint16_t*>(a.mask);
+      gp.mask_seq_stride = r.m_ss;
+      gp.mask_row_stride = r.m_rs;
+      gp.n_q = a.n_q;
+      gp.rows = g_rows;
+      gp.gmask = g_mask;
+      gp.cap = g_cap;
+      gp.gmask_stride = g_mstride;
+      const int64_t items = g_cap * (r.dk / 32);
+      const int per_seq = std::max(1, (st->sm_count * 2 + n - 1) / n);  // two CTAs of 256 per SM
+      cudaLaunchConfig_t gcfg = {};
+      gcfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((items + 1023) / 1024, per_seq)), n);
+      gcfg.blockDim = dim3(256);
+      gcfg.stream = stream;
+      cudaLaunchAttribute gattr[1];
+      gattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      gattr[0].val.programmaticStreamSerializationAllowed = 1;
+      gcfg.attrs = gattr;
+      gcfg.numAttrs = 1;
+      cudaError_t ge;
+      {
+        ProfScope prof(kKernGatherRows, stream);
+        if (a.kcache_type == MLA_KV_Q8_0)
+          ge = cudaLaunchKernelEx(&gcfg, mla::mla_gather_rows_kernel<mla::kModeQ8, 9>, plan, gp);
+        else if (r.dk == MLA_DK)
+          ge = cudaLaunchKernelEx(&gcfg, mla::mla_gather_rows_kernel<mla::kModeGatherF16, 9>, plan, gp);
+        else
+          ge = cudaLaunchKernelEx(&gcfg, mla::mla_gather_rows_kernel<mla::kModeGatherF16, 8>, plan, gp);
+      }
+      if (ge != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     }
     // launched as a programmatic dependent of the stream's previous kernel: its setup
     // overlaps that kernel's tail, and griddepcontrol.wait in the kernel precedes

@@ -71,7 +71,9 @@ struct MlaFwdParams {
   // query rows read by the manual producers: row r of sequence b at q + b*q_seq_stride + r*576
   const uint16_t* q;
   int64_t q_seq_stride;      // elements
-  // sparse: sequence b attends to rows idx[b*idx_seq_stride + i], i < idx_count[b]
+  // sparse: sequence b attends to rows idx[b*idx_seq_stride + i], i < idx_count[b]; in
+  // TMA mode with idx == nullptr, idx_count (when set) bounds the rows of sequence b
+  // (rows gathered from an index list)
   const int32_t* idx;
   const int32_t* idx_count;
   int64_t idx_seq_stride;
@@ -447,7 +449,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     n_tiles = (len + kTK - 1) / kTK;
     key_end = len;
   } else {
-    len = sparse ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b]) : plan.kv_len[b];
+    // an index list (or, in TMA mode, the rows gathered from one) ends at its count
+    len = (sparse || p.idx_count != nullptr) ? min(max(__ldg(p.idx_count + b_abs), 0), plan.kv_len[b])
+                                             : plan.kv_len[b];
     if (p.units != nullptr) {
       // tiles the mask leaves something in (dense mode; the range is within the length)
       tile_begin = du.tile_begin;
