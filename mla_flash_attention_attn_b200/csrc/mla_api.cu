@@ -894,10 +894,10 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       gp.gmask = g_mask;
       gp.cap = g_cap;
       gp.gmask_stride = g_mstride;
-      const int64_t items = g_cap * (r.dk / 32);
-      const int per_seq = std::max(1, (st->sm_count * 2 + n - 1) / n);  // two CTAs of 256 per SM
+      const int64_t rows_per_cta = a.kcache_type == MLA_KV_Q8_0 ? 32 : 16;  // 8 warps x positions in flight
+      const int per_seq = std::max(1, (st->sm_count * 4 + n - 1) / n);
       cudaLaunchConfig_t gcfg = {};
-      gcfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((items + 1023) / 1024, per_seq)), n);
+      gcfg.gridDim = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>((g_cap + rows_per_cta - 1) / rows_per_cta, per_seq)), n);
       gcfg.blockDim = dim3(256);
       gcfg.stream = stream;
       cudaLaunchAttribute gattr[1];
