@@ -264,27 +264,52 @@ int validate(const mla_fa_args* a, Resolved* r) {
 // and P.V work on the previous step. With several groups per sequence (a prefill chunk)
 // the keys come back from L2 and the MMAs bound the kernel: steps of 256 keys issue half
 // as many MMAs and softmax rounds per key. The gather and q8_0 modes take 256.
-// Index-list calls of a single 128-row group (a decode): the listed rows are first
-// gathered into a dense f16 buffer in the workspace (mla_gather_rows_kernel, every SM at
-// once), and the TMA-mode kernel streams that buffer. With more groups per sequence each
-// group would re-read the list's rows, so those calls keep the gather modes.
+// Sparse calls of a single 128-row group (a decode): an index list (the caller's, or
+// with the mask gather one built here from the mask by mla_compact_union_kernel) has its
+// rows gathered into a dense f16 buffer in the workspace (mla_gather_rows_kernel, every
+// SM at once), and the TMA-mode kernel streams that buffer. With more groups per
+// sequence each group would re-read the list's rows, so those calls keep the gather
+// modes.
 bool gathered_rows(const Resolved& r) {
-  return r.a.idx != nullptr && !r.a.mask_gather && r.rows <= mla::kRowsPerGroup && r.dk != MLA_HEADS_DK;
+  return (r.a.idx != nullptr || r.a.mask_gather) && r.rows <= mla::kRowsPerGroup && r.dk != MLA_HEADS_DK;
 }
+// The list is built here (mask gather) rather than passed in.
+bool internal_list(const Resolved& r) { return gathered_rows(r) && r.a.mask_gather; }
 
 // Rows per sequence in the gathered buffer: the most any sequence's list can use.
 int64_t gathered_cap(const Resolved& r) {
   int64_t m = 0;
   for (int b = 0; b < r.a.n_seq; ++b) m = std::max<int64_t>(m, r.a.kv_len ? r.a.kv_len[b] : r.a.n_kv);
-  return std::max<int64_t>(1, std::min<int64_t>(m, r.idx_ss));
+  if (r.a.idx != nullptr) m = std::min<int64_t>(m, r.idx_ss);
+  return std::max<int64_t>(1, m);
 }
 int64_t gathered_mask_stride(const Resolved& r) { return (gathered_cap(r) + 63) / 64 * 64; }
-// Bytes of the gathered rows and of their mask values (every sequence of the call).
-size_t gathered_bytes(const Resolved& r) {
-  if (!gathered_rows(r)) return 0;
-  const size_t rows = (size_t)r.a.n_seq * gathered_cap(r) * r.dk * 2;
-  return (rows + 255) / 256 * 256 + (size_t)r.a.n_seq * r.a.n_q * gathered_mask_stride(r) * 2;
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+// Layout of the gathered region (offsets from its start): rows, mask values, and for an
+// internal list the list, its counts, and the compaction's tickets and look-back flags
+// (one launch's sequences at a time, cleared before each launch).
+struct GatheredLayout {
+  size_t mask, list, count, tickets, flags, bytes;
+  int tiles;  // compaction tiles of the longest list
+};
+GatheredLayout gathered_layout(const Resolved& r) {
+  GatheredLayout l = {};
+  if (!gathered_rows(r)) return l;
+  const int64_t cap = gathered_cap(r);
+  l.mask = align256((size_t)r.a.n_seq * cap * r.dk * 2);
+  l.list = l.mask + align256((size_t)r.a.n_seq * r.a.n_q * gathered_mask_stride(r) * 2);
+  l.bytes = l.list;
+  if (internal_list(r)) {
+    l.tiles = (int)((cap + mla::compact::kTileCells - 1) / mla::compact::kTileCells);
+    l.count = l.list + align256((size_t)r.a.n_seq * cap * 4);
+    l.tickets = l.count + align256((size_t)r.a.n_seq * 4);
+    l.flags = l.tickets + align256((size_t)mla::kPlanMaxSeq * 4);
+    l.bytes = l.flags + align256((size_t)mla::kPlanMaxSeq * l.tiles * 8);
+  }
+  return l;
 }
+// Bytes of the gathered region (every sequence of the call).
+size_t gathered_bytes(const Resolved& r) { return gathered_layout(r).bytes; }
 
 int kernel_step(const Resolved& r) {
   const mla_fa_args& a = r.a;
@@ -376,7 +401,7 @@ int64_t gather_stride(const Plan& plan) {
   return std::max<int64_t>(64, (m + 63) / 64 * 64);
 }
 size_t gather_bytes(const Resolved& r, const Plan& plan, int slots) {
-  if (!r.a.mask_gather) return 0;
+  if (!r.a.mask_gather || gathered_rows(r)) return 0;
   const size_t head = (size_t)slots * slot_bytes();
   const size_t start = (head + 255) / 256 * 256;
   return start - head + (size_t)2 * plan.total_units * gather_stride(plan) * sizeof(int32_t);
@@ -714,11 +739,21 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
   const int64_t g_mstride = gat ? gathered_mask_stride(r) : 0;
   uint16_t* g_rows = nullptr;
   uint16_t* g_mask = nullptr;
+  const GatheredLayout gl = gathered_layout(r);
+  char* g_base = nullptr;
   if (gat) {
-    const size_t off = gathered_offset(r, st->sm_count);
-    g_rows = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + off);
-    g_mask = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + off +
-                                         ((size_t)a.n_seq * g_cap * r.dk * 2 + 255) / 256 * 256);
+    g_base = static_cast<char*>(ws) + gathered_offset(r, st->sm_count);
+    g_rows = reinterpret_cast<uint16_t*>(g_base);
+    g_mask = reinterpret_cast<uint16_t*>(g_base + gl.mask);
+  }
+  // the list the rows are gathered from: the caller's, or the one built here
+  const int32_t* list = a.idx;
+  const int32_t* list_count = a.idx_count;
+  int64_t list_stride = r.idx_ss;
+  if (internal_list(r)) {
+    list = reinterpret_cast<const int32_t*>(g_base + gl.list);
+    list_count = reinterpret_cast<const int32_t*>(g_base + gl.count);
+    list_stride = g_cap;
   }
   // the cells the TMA mode streams: the cache, or the gathered rows
   const void* k_base = gat ? static_cast<const void*>(g_rows) : a.kcache;
@@ -808,6 +843,7 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     // the kernel streams the gathered rows, with their gathered mask values, up to each
     // list's count
     p.idx = nullptr;
+    p.idx_count = list_count;
     p.mask = g_mask;
     p.mask_seq_stride = (int64_t)a.n_q * g_mstride;
     p.mask_row_stride = g_mstride;
@@ -863,10 +899,10 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
     p.ws_lse = slots ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                 (size_t)slots * mla::kRowsPerGroup * mla::kDV * 2)
                      : nullptr;
-    p.mask_gather = a.mask_gather;
+    p.mask_gather = gat ? 0 : a.mask_gather;
     p.gather_list = nullptr;
     p.gather_stride = 0;
-    if (a.mask_gather) {
+    if (p.mask_gather) {
       const size_t head = (size_t)slots * slot_bytes();
       p.gather_list = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + (head + 255) / 256 * 256);
       p.gather_stride = gather_stride(plan);
@@ -876,13 +912,44 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       rc = make_part_map(&tm_w, ws, (uint64_t)slots * mla::kRowsPerGroup);
       if (rc != MLA_OK) return rc;
     }
+    if (internal_list(r)) {
+      // the list of each sequence: the cells its query tokens keep (mask gather)
+      int* tickets = reinterpret_cast<int*>(g_base + gl.tickets);
+      auto* flags = reinterpret_cast<unsigned long long*>(g_base + gl.flags);
+      if (cudaMemsetAsync(g_base + gl.tickets, 0, gl.bytes - gl.tickets, stream) != cudaSuccess)
+        return MLA_ERR_CUDA;
+      uint32_t epoch;
+      {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        epoch = st->cmp_epoch;
+        st->cmp_epoch = (st->cmp_epoch + 1) & 0x3FFFFFFFu;
+        if (st->cmp_epoch == 0) st->cmp_epoch = 1;
+      }
+      cudaLaunchConfig_t ccfg = {};
+      ccfg.gridDim = dim3(gl.tiles, n);
+      ccfg.blockDim = dim3(mla::compact::kThreads);
+      ccfg.stream = stream;
+      cudaLaunchAttribute cattr[1];
+      cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      cattr[0].val.programmaticStreamSerializationAllowed = 1;
+      ccfg.attrs = cattr;
+      ccfg.numAttrs = 1;
+      cudaError_t ce;
+      {
+        ProfScope prof(kKernCompact, stream);
+        ce = cudaLaunchKernelEx(&ccfg, mla::mla_compact_union_kernel, plan, static_cast<const uint16_t*>(a.mask),
+                                (int64_t)r.m_ss, (int64_t)r.m_rs, const_cast<int32_t*>(list), list_stride,
+                                const_cast<int32_t*>(list_count), tickets, flags, epoch, kDefaultTimeoutNs);
+      }
+      if (ce != cudaSuccess || cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    }
     if (gat) {
       // the lists' rows (and mask values) into the dense buffer, every SM at once; a
       // programmatic dependent of the kernel that wrote the lists
       mla::GatherParams gp;
-      gp.idx = a.idx;
-      gp.idx_count = a.idx_count;
-      gp.idx_seq_stride = r.idx_ss;
+      gp.idx = list;
+      gp.idx_count = list_count;
+      gp.idx_seq_stride = list_stride;
       gp.kcache = static_cast<const uint8_t*>(a.kcache);
       gp.k_seq_stride = r.k_ss;
       gp.n_kv = a.n_kv;

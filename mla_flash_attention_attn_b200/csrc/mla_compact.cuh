@@ -39,45 +39,34 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   return v;
 }
 
-// Grid: (tiles_per_row, n_rows). Workspace per row: one ticket counter (int) and
-// tiles_per_row look-back flags (u64 = tag<<32 | value, tag = epoch*4 + state).
-__global__ void __launch_bounds__(compact::kThreads)
-    mla_compact_kernel(const uint16_t* __restrict__ mask, int64_t mask_row_stride, int n_kv,
-                       int32_t* __restrict__ idx_out, int64_t idx_row_stride,
-                       int32_t* __restrict__ count_out, int* __restrict__ tickets,
-                       unsigned long long* __restrict__ flags, uint32_t epoch,
-                       uint64_t timeout_ns) {
+// One tile of one row: keep bits of the tile's cells from keep_of(cell0, n) (bit k:
+// cell cell0 + k kept, n cells of the segment in range), then the scan, the look-back
+// and the ascending writes. Workspace per row: one ticket counter (int) and n_tiles
+// look-back flags (u64 = tag<<32 | value, tag = epoch*4 + state).
+template <class KeepOf>
+__device__ __forceinline__ void compact_row_tile(int row, int n_tiles, int n_cells, KeepOf keep_of,
+                                                 int32_t* __restrict__ idx_out, int64_t idx_row_stride,
+                                                 int32_t* __restrict__ count_out, int* __restrict__ tickets,
+                                                 unsigned long long* __restrict__ flags, uint32_t epoch,
+                                                 uint64_t timeout_ns) {
   using namespace compact;
   __shared__ int s_tile;
   __shared__ int s_warp_tot[kThreads / 32];
   __shared__ int s_excl;
-  const int row = blockIdx.y;
-  const int n_tiles = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) s_tile = atomicAdd(&tickets[row], 1);
-  // the attention kernel that follows may start its setup now; it waits for this grid
-  // to complete before it reads the index lists
+  // the kernel that follows may start its setup now; it waits for this grid to
+  // complete before it reads the index lists
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __syncthreads();
   const int tile = s_tile;
-  const uint16_t* mrow = mask + (int64_t)row * mask_row_stride;
   const int64_t cell0 = (int64_t)tile * kTileCells + (int64_t)tid * kCellsPerThread;
 
   // keep bits of this thread's cells
   static_assert(kCellsPerThread == 8, "one 16-byte load per segment");
-  uint32_t keep = 0;
-  if (cell0 + kCellsPerThread <= n_kv && ((reinterpret_cast<uintptr_t>(mrow + cell0) & 15) == 0)) {
-    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(mrow + cell0));
-    const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      keep |= (uint32_t)((w[h] & 0xFFFFu) != kNegInfBits) << (2 * h);
-      keep |= (uint32_t)((w[h] >> 16) != kNegInfBits) << (2 * h + 1);
-    }
-  } else {
-    for (int k = 0; k < kCellsPerThread; ++k)
-      if (cell0 + k < n_kv && __ldg(mrow + cell0 + k) != kNegInfBits) keep |= 1u << k;
-  }
+  const int64_t left = (int64_t)n_cells - cell0;
+  const int n_in = left <= 0 ? 0 : (left < kCellsPerThread ? (int)left : kCellsPerThread);
+  const uint32_t keep = n_in > 0 ? keep_of(cell0, n_in) : 0u;
   const int cnt = __popc(keep);
 
   // warp inclusive scan of the segment counts
@@ -162,6 +151,66 @@ __global__ void __launch_bounds__(compact::kThreads)
   int32_t* orow = idx_out + (int64_t)row * idx_row_stride;
   for (int k = 0; k < kCellsPerThread; ++k)
     if (keep & (1u << k)) orow[pos++] = (int32_t)(cell0 + k);
+}
+
+// Keep bits of n cells from cell0 of an f16 mask row: one 16-byte load when the 8 cells
+// are whole and aligned, else cell by cell.
+__device__ __forceinline__ uint32_t keep_bits(const uint16_t* mrow, int64_t cell0, int n) {
+  using namespace compact;
+  uint32_t keep = 0;
+  if (n == kCellsPerThread && ((reinterpret_cast<uintptr_t>(mrow + cell0) & 15) == 0)) {
+    const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(mrow + cell0));
+    const uint32_t w[4] = {v0.x, v0.y, v0.z, v0.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      keep |= (uint32_t)((w[h] & 0xFFFFu) != kNegInfBits) << (2 * h);
+      keep |= (uint32_t)((w[h] >> 16) != kNegInfBits) << (2 * h + 1);
+    }
+  } else {
+    for (int k = 0; k < n; ++k)
+      if (__ldg(mrow + cell0 + k) != kNegInfBits) keep |= 1u << k;
+  }
+  return keep;
+}
+
+// Grid: (tiles_per_row, n_rows): the kept cells of each mask row.
+__global__ void __launch_bounds__(compact::kThreads)
+    mla_compact_kernel(const uint16_t* __restrict__ mask, int64_t mask_row_stride, int n_kv,
+                       int32_t* __restrict__ idx_out, int64_t idx_row_stride,
+                       int32_t* __restrict__ count_out, int* __restrict__ tickets,
+                       unsigned long long* __restrict__ flags, uint32_t epoch,
+                       uint64_t timeout_ns) {
+  const int row = blockIdx.y;
+  const uint16_t* mrow = mask + (int64_t)row * mask_row_stride;
+  compact_row_tile(
+      row, gridDim.x, n_kv, [&](int64_t cell0, int n) { return keep_bits(mrow, cell0, n); }, idx_out,
+      idx_row_stride, count_out, tickets, flags, epoch, timeout_ns);
+}
+
+// Grid: (tiles of the longest sequence, sequences of the launch): the cells of sequence
+// b's first plan.kv_len[b] that any of its n_q query tokens keeps (the union of the
+// token rows' masks), as one list per sequence. A programmatic dependent of the kernel
+// before it.
+__global__ void __launch_bounds__(compact::kThreads)
+    mla_compact_union_kernel(const __grid_constant__ Plan plan, const uint16_t* __restrict__ mask,
+                             int64_t mask_seq_stride, int64_t mask_row_stride,
+                             int32_t* __restrict__ idx_out, int64_t idx_row_stride,
+                             int32_t* __restrict__ count_out, int* __restrict__ tickets,
+                             unsigned long long* __restrict__ flags, uint32_t epoch,
+                             uint64_t timeout_ns) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int b = blockIdx.y;
+  const uint16_t* mseq = mask + (int64_t)(plan.seq_offset + b) * mask_seq_stride;
+  const int n_q = plan.n_q;
+  compact_row_tile(
+      b, gridDim.x, plan.kv_len[b],
+      [&](int64_t cell0, int n) {
+        uint32_t keep = 0;
+        for (int t = 0; t < n_q; ++t) keep |= keep_bits(mseq + (int64_t)t * mask_row_stride, cell0, n);
+        return keep;
+      },
+      idx_out + (int64_t)plan.seq_offset * idx_row_stride, idx_row_stride, count_out + plan.seq_offset,
+      tickets, flags, epoch, timeout_ns);
 }
 
 }  // namespace mla
