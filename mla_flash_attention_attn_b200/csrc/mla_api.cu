@@ -169,6 +169,7 @@ struct Resolved {
   bool lse;   // per-row log-sum-exp output: every sequence writes partials (the combine writes it)
   int dk;     // head width: MLA_DK, MLA_DV for the DK = DV = 512 shape, MLA_HEADS_DK
   int64_t v_ss;  // DK = 192 shape: rows between sequences of v
+  bool no_gathered_rows = false;  // sparse calls keep the gather modes (a scratch too small for the rows)
 };
 
 int validate(const mla_fa_args* a, Resolved* r) {
@@ -271,7 +272,8 @@ int validate(const mla_fa_args* a, Resolved* r) {
 // sequence each group would re-read the list's rows, so those calls keep the gather
 // modes.
 bool gathered_rows(const Resolved& r) {
-  return (r.a.idx != nullptr || r.a.mask_gather) && r.rows <= mla::kRowsPerGroup && r.dk != MLA_HEADS_DK;
+  return (r.a.idx != nullptr || r.a.mask_gather) && r.rows <= mla::kRowsPerGroup && r.dk != MLA_HEADS_DK &&
+         !r.no_gathered_rows;
 }
 // The list is built here (mask gather) rather than passed in.
 bool internal_list(const Resolved& r) { return gathered_rows(r) && r.a.mask_gather; }
@@ -1188,6 +1190,10 @@ int mla_fa_forward_noalloc(const mla_fa_args* a, void* stream) {
   if (rc != MLA_OK) return rc;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MLA_ERR_CUDA;
+  // a sparse pass whose gathered rows do not fit the scratch takes the gather modes,
+  // which need only the partials
+  if (workspace_for(r, st->sm_count, nullptr, nullptr) > (size_t)MLA_NOALLOC_SCRATCH_BYTES)
+    r.no_gathered_rows = true;
   if (workspace_for(r, st->sm_count, nullptr, nullptr) > (size_t)MLA_NOALLOC_SCRATCH_BYTES)
     return MLA_ERR_WORKSPACE;
   void* scratch = nullptr;

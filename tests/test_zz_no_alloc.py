@@ -8,8 +8,10 @@ in a static device array. These tests call it through the C ABI and check, on
 two calls in a row with different inputs, that it gives what the allocating
 entry point mla_fa_forward_ex gives and what the fp64 oracle gives, that the
 other users of the array (the mask gather's cell lists and the fused
-projection's partials) survive back-to-back calls of different shapes, and that
-a pass needing more scratch than the array holds is refused before any launch.
+projection's partials) survive back-to-back calls of different shapes, that an
+index list whose gathered rows would not fit the array is attended with the
+in-kernel gather instead, and that a pass needing more scratch than the array
+holds is refused before any launch.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes on its own in a fresh process.
@@ -116,6 +118,32 @@ def test_noalloc_mask_gather_and_projection_back_to_back():
         torch.cuda.synchronize()
         assert binding.mla_get_device_status() == 0
         _compare(op_na.cpu().numpy(), ref.cpu().numpy(), f"projection call {i + 1}")
+
+
+def test_noalloc_index_list_larger_than_its_scratch_takes_the_gather_modes():
+    # The allocating entry point gathers an index list's rows into its workspace (here
+    # 32768 rows of 1152 bytes, more than the scratch holds); the no-alloc entry point
+    # then attends over the list with the in-kernel gather, which needs only the partials.
+    import torch
+
+    binding.load()
+    dev = torch.device("cuda")
+    w = W.make("sparse_q8_decode", n_kv=32768, n_head=128, tail_blocks=4)
+    q, k, m = _inputs(w, torch)
+    idx = torch.full((1, w.n_kv), -1, dtype=torch.int32, device=dev)
+    cnt = torch.zeros((1,), dtype=torch.int32, device=dev)
+    cws = torch.zeros(binding.mla_compact_workspace_size(1, w.n_kv), dtype=torch.uint8, device=dev)
+    binding.mla_compact_mask_ex(m[:, 0, :], idx, cnt, cws)
+    out_na = torch.full(w.q.shape[:3] + (512,), float("nan"), dtype=torch.float32, device=dev)
+    args, keep_alive = binding.make_args(q, k, w.kv_type, m, out_na, w.scale, idx=idx, idx_count=cnt)
+    assert binding.mla_fa_workspace_size(args) > binding.NOALLOC_SCRATCH_BYTES
+    binding.mla_fa_forward_noalloc(args)
+    torch.cuda.synchronize()
+    assert binding.mla_get_device_status() == 0
+    ref_idx = oracle.compact(w.mask[0, 0])
+    assert int(cnt[0]) == len(ref_idx)
+    ref = oracle.attention(w.q[0], w.kcache[0], oracle.KV_Q8_0, w.mask[0], w.scale, idx=ref_idx)
+    _compare(out_na[0].reshape(-1, 512).cpu().numpy(), ref, "no-alloc index list, gather modes")
 
 
 def test_noalloc_refuses_a_pass_larger_than_its_scratch():
