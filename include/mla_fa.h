@@ -115,12 +115,15 @@ typedef enum {
  * (the variants are named for the Metal FA kernel of the llama.cpp tag page, PR
  * #29570; these formulas are this library's reading of them)
  * mask_gather 1: sparse attention straight from the mask, without an index list
- *         (the compaction fused into the attention, for any n_q): the cells, in
- *         chunks of 8, are dealt round-robin to a sequence's KV splits; every work
- *         unit compacts its chunks and gathers only the cache rows that some query
- *         row of its 128-row group keeps (mask != -inf); each row still applies its
- *         own mask. Requires mask, excludes idx and alibi_slopes. The workspace then
- *         also holds the units' cell lists
+ *         (for any n_q): only the cache rows that some query row of a 128-row group
+ *         keeps (mask != -inf) are attended, and each row still applies its own mask.
+ *         When a sequence has a single 128-row group (n_q * n_head <= 128), its list
+ *         of such cells is built in the workspace (the union of its tokens' masks,
+ *         one compaction) and attended as an index list (below); with more groups the
+ *         cells, in chunks of 8, are dealt round-robin to a sequence's KV splits and
+ *         every work unit compacts its chunks inside the attention kernel. Requires
+ *         mask, excludes idx and alibi_slopes. The workspace then also holds the cell
+ *         lists
  * out_lse DEVICE fp32 [n_seq][n_q][n_head] or NULL: each row's natural log-sum-exp of
  *         its scores, lse = log sum_j exp(scale q.k_j + mask_j) (-inf for a row with
  *         nothing kept), next to out. With it, partial results of the same rows over
@@ -201,7 +204,11 @@ int mla_fa_forward(const void* q, const void* kcache, int kcache_type, const voi
 int mla_set_stream(void* cuda_stream);
 
 /* Bytes of workspace mla_fa_forward_ex needs for these arguments (0 when the
- * pass needs no split-KV partials). Returns 0 as well for invalid arguments. */
+ * pass needs no split-KV partials). Returns 0 as well for invalid arguments.
+ * A sparse pass (idx, or mask_gather) whose sequences have a single 128-row group
+ * also keeps in the workspace the rows it attends, gathered into a dense f16 buffer
+ * (head width x 2 bytes per row, for as many rows per sequence as its list can hold:
+ * the smaller of idx_seq_stride and its length), and their mask values. */
 size_t mla_fa_workspace_size(const mla_fa_args* a);
 
 /* Batched / sparse forward pass into caller-owned workspace (device memory of
@@ -228,9 +235,11 @@ int mla_fa_forward_ex(const mla_fa_args* a, void* workspace, size_t ws_bytes, vo
  * Every GPU that loads the library holds that array until the process exits.
  * The caller still passes q, kcache, mask and out.
  *
- * - If the pass needs more scratch than MLA_NOALLOC_SCRATCH_BYTES
- *   (mla_fa_workspace_size(a) > MLA_NOALLOC_SCRATCH_BYTES), it returns
- *   MLA_ERR_WORKSPACE before launching anything.
+ * - A sparse pass whose gathered rows (see mla_fa_workspace_size) do not fit the
+ *   scratch attends over its list with the gather inside the attention kernel,
+ *   which keeps only the partials in the scratch.
+ * - If the pass needs more scratch than MLA_NOALLOC_SCRATCH_BYTES even so, it
+ *   returns MLA_ERR_WORKSPACE before launching anything.
  * - The first call on a device looks up the array's device address once
  *   (cudaGetSymbolAddress) with that device current; make that first call before
  *   any stream capture. The address is kept for the life of the process, so do
