@@ -431,15 +431,56 @@ def test_sparse_count_zero_and_partial_lists():
         assert_parity(got[b].reshape(-1, 512), ref, f"sparse list {b}")
 
 
-def test_sparse_out_of_range_index_is_reported_not_read():
-    w = W.make("tiny_decode", n_kv=300)
+@pytest.mark.parametrize("kv", ["f16", "q8_0"])
+def test_sparse_out_of_range_index_is_reported_not_read(kv):
+    if kv == "f16":
+        w = W.make("tiny_decode", n_kv=300)
+    else:
+        w = W.make("sparse_q8_decode", n_kv=300, n_head=16, block=8, tail_blocks=1)
     w.mask[:] = 0
-    lst = np.array([3, 10, 299, 300 + 5, 17], np.int32)  # one index beyond n_kv
-    got, _, _, status = run_sparse_gpu(w, idx_rows=[lst], counts=[5], use_gpu_compaction=False)
-    assert status == -9  # MLA_ERR_INDEX recorded; the bad row is treated as dropped
-    ok = np.array([3, 10, 299, 17], np.int32)
-    ref = oracle.attention(w.q[0], w.kcache[0], 0, w.mask[0], w.scale, idx=ok)
-    assert_parity(got[0].reshape(-1, 512), ref, "bad index dropped")
+    # one index beyond n_kv, one negative: both dropped (zero row, -inf score)
+    lst = np.array([3, 10, 299, 300 + 5, 17, -2, 250], np.int32)
+    got, _, _, status = run_sparse_gpu(w, idx_rows=[lst], counts=[len(lst)], use_gpu_compaction=False)
+    assert status == -9  # MLA_ERR_INDEX recorded; the bad rows are treated as dropped
+    ok = np.array([3, 10, 299, 17, 250], np.int32)
+    ref = oracle.attention(w.q[0], w.kcache[0], w.kv_type, w.mask[0], w.scale, idx=ok)
+    assert_parity(got[0].reshape(-1, 512), ref, f"bad index dropped ({kv})")
+
+
+@pytest.mark.parametrize("kv", ["f16", "q8_0"])
+def test_index_list_paths_by_group_count(kv):
+    # A sequence with a single 128-row group gathers its list's rows into a dense buffer
+    # for the TMA-mode kernel; with several groups (3 query tokens x 128 heads) the list
+    # is read by the gather modes inside the attention kernel. Both against the oracle,
+    # and the kernels each path launches.
+    torch = torch_mod()
+    rng = np.random.default_rng(71 if kv == "f16" else 72)
+    n_kv = 2600
+    for n_q, n_head in ((1, 128), (3, 128)):
+        if kv == "f16":
+            w = W.make("prefill_chunk", seed=81, n_q=n_q, n_head=n_head, n_kv=n_kv)
+        else:
+            w = W.make("sparse_q8_decode", seed=82, n_kv=n_kv, n_head=n_head, block=8, tail_blocks=2)
+            w.q = rng.standard_normal((1, n_q, n_head, 576)).astype(np.float16)
+        w.mask = np.where(rng.random((1, n_q, n_kv)) < 0.9, rng.standard_normal((1, n_q, n_kv)),
+                          -np.inf).astype(np.float16)
+        lst = np.sort(rng.choice(n_kv, 700, replace=False)).astype(np.int32)
+        dev = torch.device("cuda")
+        q, k, m = (torch.from_numpy(x).to(dev) for x in (w.q, w.kcache, w.mask))
+        idx = torch.full((1, n_kv), -1, dtype=torch.int32, device=dev)
+        idx[0, : len(lst)] = torch.from_numpy(lst).to(dev)
+        cnt = torch.tensor([len(lst)], dtype=torch.int32, device=dev)
+        out = torch.full((1, n_q, n_head, 512), float("nan"), dtype=torch.float32, device=dev)
+        ran = _launches(lambda: binding.forward(q, k, w.kv_type, m, w.scale, out=out, idx=idx, idx_count=cnt))
+        assert binding.mla_get_device_status() == 0
+        if n_q * n_head <= 128:
+            assert ran.get("mla_gather_rows") == 1 and "mla_fwd_f16" in ran, ran
+        else:
+            assert "mla_gather_rows" not in ran, ran
+            assert ("mla_fwd_q8_0" if kv == "q8_0" else "mla_fwd_gather_f16") in ran, ran
+        kref = q8_f16_rounded(w.kcache[0]) if kv == "q8_0" else w.kcache[0]
+        ref = oracle.attention(w.q[0], kref, oracle.KV_F16, w.mask[0], w.scale, idx=lst)
+        assert_parity(out[0].reshape(-1, 512).cpu().numpy(), ref, f"index list {kv} n_q={n_q}")
 
 
 # ---- fused value up-projection (out_proj = O . W_UV per head) ---------------------
