@@ -1088,9 +1088,11 @@ int ensure_ws(void** ptr, size_t* have, size_t need) {
   return MLA_OK;
 }
 
-// Scratch of mla_fa_forward_noalloc: the split-KV partials of one call (f16 O rows,
-// then fp32 lse; with mask_gather, the units' cell lists after them), in static
-// device memory so that the call allocates nothing.
+// Scratch of mla_fa_forward_noalloc: the workspace of one call (the split-KV
+// partials: f16 O rows, then fp32 lse; with the in-kernel mask gather, the units' cell
+// lists after them; for a single-group sparse call whose rows fit, the gathered rows,
+// their mask values and the internal list), in static device memory so that the call
+// allocates nothing.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_noalloc_mutex;
