@@ -208,6 +208,27 @@ def test_batch_larger_than_one_launch():
     check_all_rows(w, run_gpu(w), what="130 sequences")
 
 
+def test_sparse_batch_larger_than_one_launch():
+    # 130 single-group sequences with sparse masks, through the two sparse routes that
+    # gather rows into the workspace (indexed by the sequence's place in the whole batch,
+    # over two launches of the plan): the mask gather (an internal list per sequence) and
+    # caller index lists from the compaction
+    w = W.make("v3_batched_decode", seed=41, n_seq=130, n_head=16, n_kv=600, len_lo=1, len_hi=600)
+    rng = np.random.default_rng(41)
+    keep = (rng.random((130, 1, 600)) < 0.3) & (np.arange(600)[None, None, :] < w.kv_len[:, None, None])
+    keep[:, 0, 0] = True
+    w.mask = np.where(keep, rng.standard_normal((130, 1, 600)), -np.inf).astype(np.float16)
+    check_all_rows(w, run_gpu(w, mask_gather=True), what="130 sequences, mask gather")
+    w.sparse = True
+    got, idx, cnt, status = run_sparse_gpu(w)
+    assert status == 0
+    for b in range(w.n_seq):
+        lst = oracle.compact(w.mask[b, 0])
+        assert cnt[b] == len(lst)
+        ref = oracle.attention(w.q[b], w.kcache[b], w.kv_type, w.mask[b], w.scale, idx=lst)
+        assert_parity(got[b].reshape(-1, 512), ref, f"130 sequences, index list {b}")
+
+
 def test_many_splits_of_one_long_sequence():
     # one 16-head sequence of 20000 keys: 79 tiles over the 74 SM pairs, so its rows are
     # combined from 74 partials by the multi-group combine
