@@ -1,37 +1,39 @@
 // MLA flash attention forward on sm_100a: one 2-CTA cluster per work unit.
 //
 // Per unit (sequence b, 128-row group g, KV split s) the pair computes, for
-// its 128 query rows (row = token*n_head + head) and its range of key tiles,
-//   S = scale * Q K^T + mask      (Q: 128 x 576, K tile: 128 keys x 576)
+// its 128 query rows (row = token*n_head + head) and its range of keys,
+//   S = scale * Q K^T + mask      (Q: 128 x 576, a step of kTK keys x 576)
 //   online softmax with running max m and running sum l per row
 //   O += P V                      (V = first 512 columns of the same K rows)
-// tile by tile, with S, P and O never leaving the SM pair (Vulkan FA for
+// step by step, with S, P and O never leaving the SM pair (Vulkan FA for
 // DeepSeek MLA article, sections 2.1-2.2; V taken from the K row per the
 // ik_llama.cpp -mla guide, section "-mla四檔語義").
 //
 // Hardware mapping (cta_group::2, M = 128 rows, 64 rows in each CTA):
 //  * Each CTA keeps its 64 Q rows in shared memory (9 chunks of 64 columns,
-//    128-byte swizzle) for the whole unit; they arrive with the first tile's K.
-//  * Q.K^T: N = 256 keys (a tile); CTA c loads keys [128c, 128c+128) of each
-//    tile, so the pair reads every K byte once. In TMEM, lane r holds keys
-//    0..127 of row r and lane r+64 keys 128..255 (128 columns of S).
+//    128-byte swizzle) for the whole unit; they arrive with the first step's K.
+//  * Q.K^T: N = kTK keys (a step of 128 or 256, fwd::Geo); CTA c loads keys
+//    [c kTK/2, (c+1) kTK/2) of each step, so the pair reads every K byte once. In
+//    TMEM, lane r holds the first kTK/2 keys of row r and lane r+64 the others.
 //  * P.V: N = 256 value columns per MMA (one value half), K = 16 keys; CTA c
-//    loads value columns [256j+128c, +128) of the tile's rows. A (P) is read from
+//    loads value columns [256j+128c, +128) of the step's rows. A (P) is read from
 //    TMEM and O accumulates in TMEM (256 columns per CTA: lane r holds 128 of row
 //    r's values per value half).
-//  * TMEM: S (128 columns), P (128 columns: f16 pairs of all 256 keys of the tile
-//    in both lanes of a row), O (256 columns). The softmax frees S as soon as the
-//    scores are in registers, so Q.K^T of the next tile overlaps the softmax.
-//  * K stages (16 KB: 128 keys x 64 columns) and V stages (16 KB: 64 keys x 128
-//    value columns) stream through two rings of shared-memory stages; every
-//    stage is 4 MMAs and one tcgen05.commit releases it.
+//  * TMEM: S buffers, P buffers (f16 pairs of all keys of the step in both lanes
+//    of a row), O (256 columns). With 128-key steps two S and two P buffers let
+//    Q.K^T of the next step run while the softmax reads S and the softmax write P
+//    while P.V of the previous step reads the other P; with 256-key steps there is
+//    one of each, and the softmax frees S as soon as the scores are in registers.
+//  * K stages (kTK/2 keys x 64 columns) and V stages (16 KB: 64 keys x 128 value
+//    columns) stream through two rings of shared-memory stages; every stage is
+//    4 MMAs and one tcgen05.commit releases it.
 //  * Two threads issue MMAs: one for Q.K^T, one for P.V. An issuing thread
 //    cannot run ahead of the tensor pipe, so the cycles it spends waiting on a
 //    barrier would idle the pipe; with two issuers one's wait is covered by the
 //    other's MMAs.
 //  * Softmax warpgroup: thread = TMEM lane; the two lanes of a row exchange
-//    their tile maximum and their P halves through shared memory. The reference
-//    max is raised only when a tile's max exceeds it by more than 2^8, so O is
+//    their step maximum and their P halves through shared memory. The reference
+//    max is raised only when a step's max exceeds it by more than 2^8, so O is
 //    rescaled in TMEM rarely.
 //  * Epilogue: O / l is staged in shared memory and written by TMA stores.
 //
@@ -477,7 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 96;");
   }
   if (warp == 0) {
-    // ================= producer (TMA mode): K chunks; the first tile's stages also
+    // ================= producer (TMA mode): K chunks; the first step's stages also
     // bring the matching chunk of this CTA's 64 query rows, which stay resident
     if (!kManual && n_steps > 0 && elect_one()) {
       // this CTA's kTK/2 keys of each step, 9 chunks of 64 columns, as far ahead as the
@@ -554,7 +556,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       constexpr uint32_t kQUnits = kChunkBytes >> 4;       // Q chunk stride
       int kst = 0;
       uint32_t kph = 0;
-      // Q chunk c is resident once the first tile's stage c has landed (TMA mode) or
+      // Q chunk c is resident once the first step's stage c has landed (TMA mode) or
       // once q_full completes (gather modes)
       if (kManual && !mbar_wait(&bars.q_full, 0, to)) {
         failed = true;
@@ -595,7 +597,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     }
     __syncwarp();
   } else if (warp == 3) {
-    // ================= P.V issuer (leader CTA, one thread): per tile, wait for P, then
+    // ================= P.V issuer (leader CTA, one thread): per step, wait for P, then
     // consume the V stages (64 keys x one 256-column half each) in the producer's order.
     // A (P) is read from TMEM: 16 keys per MMA are 8 columns of the P buffer.
     if (rank == 0 && n_steps > 0 && elect_one()) {
@@ -808,7 +810,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     if constexpr (kManual) asm volatile("setmaxnreg.inc.sync.aligned.u32 256;");
     const int L = threadIdx.x - 128;          // TMEM lane
     const int r = L & 63;                     // row within this CTA
-    const int kh = L >> 6;                    // which 64 keys of a tile this lane holds
+    const int kh = L >> 6;                    // which half of a step's keys this lane holds
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = row0 + kRowsPerCta * (int)rank + r;  // row within the sequence
     const bool row_valid = row < plan.rows && !idle;
@@ -840,7 +842,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
     float l_part = 0.f;       // this lane's half of the row sum, relative to m_ref
 
     constexpr int kHalf = kTK / 2;  // keys of one lane in a step
-    // The mask loads of a tile are issued while the previous tile is still being
+    // The mask loads of a step are issued while the previous step is still being
     // processed (after its exponentials), so their latency is hidden. Full tiles take
     // this vector path (zeros without a mask); a ragged last tile goes key by key.
     uint4 mvec[kHalf / 8];
@@ -1019,7 +1021,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(FwdCfg<kMode>::kThre
       }
       const float lsum = ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       l_part = l_part * alpha + lsum;
-      // next tile's mask: its loads overlap the rest of this tile (the scores are dead)
+      // next step's mask: its loads overlap the rest of this step (the scores are dead)
       vec_next = i + 1 < n_steps && mask_vec_ok(i + 1);
       if (vec_next) load_mask(i + 1);
       if (i + kMaskAhead < n_steps) prefetch_mask(i + kMaskAhead);
