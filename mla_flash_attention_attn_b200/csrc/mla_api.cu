@@ -436,28 +436,38 @@ int build_heads_plan(const Resolved& r, int s0, int n, int sm_count, mla::heads:
     tiles[b] = (plan->kv_len[b] + kTile - 1) / kTile;
     sum_tiles += tiles[b];
   }
+  // When the unsplit units do not fill the SMs, splits go one at a time to the sequence
+  // whose units are longest (in tiles), within one, two or three waves of units; the
+  // wave count kept is the one with the shortest estimate: the larger of the longest
+  // unit and the average work per SM, plus each wave's fixed cost (set-up, first loads,
+  // epilogue: about kWaveCostTiles tiles). A decode batch of ragged lengths with many
+  // KV heads per sequence (16 units per split) otherwise leaves its longest sequences
+  // unsplit, each on one SM.
+  constexpr double kWaveCostTiles = 3.0;
   std::vector<int> nsplit(n, 1);
   if ((int64_t)n * per_seq < sms && sum_tiles > 0) {
-    int64_t units = 0;
-    for (int b = 0; b < n; ++b) {
-      const double want = (double)sms * tiles[b] / ((double)sum_tiles * per_seq);
-      nsplit[b] = std::max(1, std::min((int)std::floor(want + 0.5), std::max(1, tiles[b])));
-      units += (int64_t)per_seq * nsplit[b];
-    }
-    while (units > sms) {  // rounding overshot one wave: take splits back
-      int best = -1;
-      int64_t best_load = 0;
-      for (int b = 0; b < n; ++b) {
-        if (nsplit[b] <= 1) continue;
-        const int64_t load = (tiles[b] + nsplit[b] - 2) / (nsplit[b] - 1);
-        if (best < 0 || load < best_load) {
-          best = b;
-          best_load = load;
-        }
+    double best_est = 0.0;
+    std::vector<int> ns(n);
+    for (int waves = 1; waves <= 3; ++waves) {
+      std::fill(ns.begin(), ns.end(), 1);
+      int64_t units = (int64_t)n * per_seq;
+      auto load = [&](int b) { return (double)tiles[b] / ns[b]; };
+      while (units + per_seq <= (int64_t)waves * sms) {
+        int arg = -1;
+        for (int b = 0; b < n; ++b)
+          if (ns[b] < tiles[b] && (arg < 0 || load(b) > load(arg))) arg = b;
+        if (arg < 0) break;
+        ++ns[arg];
+        units += per_seq;
       }
-      if (best < 0) break;
-      --nsplit[best];
-      units -= per_seq;
+      double max_load = 0.0;
+      for (int b = 0; b < n; ++b) max_load = std::max(max_load, load(b));
+      const double avg = (double)sum_tiles * per_seq / sms;
+      const double est = std::max(max_load, avg) + kWaveCostTiles * (double)((units + sms - 1) / sms);
+      if (waves == 1 || est < best_est) {
+        best_est = est;
+        nsplit = ns;
+      }
     }
   }
   int units = 0, slots = 0;
