@@ -17,7 +17,11 @@
 //  * P.V: N = 128 value columns, K = 16 keys per MMA; A (P) from TMEM, B (V) from V stages
 //    {64 keys x 128 columns} loaded by TMA from the V tensor.
 //  * TMEM (cta_group::1, M = 128: lane = row): S 128 columns, P 64 columns (f16 pairs), O
-//    128 columns. Each lane holds its whole row, so the softmax needs no exchange.
+//    128 columns. Each lane holds its whole row.
+//  * Two softmax warpgroups share each tile: warpgroup w takes keys [64w, 64w+64) of
+//    every row (S columns, P columns, and O columns [64w, 64w+64) for the rescale and the
+//    epilogue); the two swap their row maxima through shared memory, so both raise the
+//    reference max at the same tiles, and their row sums add up at the end.
 //  * The softmax frees S as soon as the scores are in registers, so Q.K^T of the next
 //    tile overlaps it; P is written once P.V of the previous tile has completed.
 // Every wait is bounded (params.timeout_ns); a timeout records MLA_ERR_TIMEOUT and the
@@ -48,9 +52,11 @@ constexpr int kOffV = kOffK + kKStages * kChunkBytes;
 constexpr int kOffBar = kOffV + kVStages * kVStageBytes;
 constexpr int kBarBytes = 8 * (2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1);
 constexpr int kOffTmemSlot = kOffBar + kBarBytes;
-constexpr int kSmemBytes = kOffTmemSlot + 16;
+constexpr int kOffXmax = kOffTmemSlot + 16;                 // float[2 tile parities][2 warpgroups][128]
+constexpr int kOffXl = kOffXmax + 2 * 2 * kRows * 4;        // float[2 warpgroups][128]
+constexpr int kSmemBytes = kOffXl + 2 * kRows * 4;
 constexpr int kSmemAlloc = kSmemBytes + 1024;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;        // roles in warps 0-3, two softmax warpgroups
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemS = 0;
 constexpr uint32_t kTmemP = 128;
@@ -69,8 +75,8 @@ struct Bars {
   uint64_t v_full[kVStages];
   uint64_t v_empty[kVStages];
   uint64_t s_full;
-  uint64_t s_free;      // 4 softmax warps
-  uint64_t p_full[2];   // 4 softmax warps
+  uint64_t s_free;      // 8 softmax warps
+  uint64_t p_full[2];   // 8 softmax warps
   uint64_t o_done[2];
   uint64_t q_full;      // 4 softmax warps: Q staged in shared memory
 };
@@ -150,9 +156,9 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
       mbar_init(&bars.v_empty[i], 1);
     }
     mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_free, 4);
+    mbar_init(&bars.s_free, 8);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars.p_full[i], 4);
+      mbar_init(&bars.p_full[i], 8);
       mbar_init(&bars.o_done[i], 1);
     }
     mbar_init(&bars.q_full, 4);
@@ -292,8 +298,12 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ================= softmax / correction / epilogue warpgroup: thread = TMEM lane = row
-    const int r = threadIdx.x - 128;
+    // ================= softmax / correction / epilogue warpgroups: thread = TMEM lane = row;
+    // warpgroup kw takes keys [64 kw, 64 kw + 64) of each tile
+    const int kw = warp >= 8 ? 1 : 0;
+    const int r = (threadIdx.x - 128) & 127;
+    float* xmax = reinterpret_cast<float*>(smem + kOffXmax);
+    float* xl = reinterpret_cast<float*>(smem + kOffXl);
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int rho = g * kRows + r;                  // row within the KV head
     const bool row_valid = rho < plan.rows;
@@ -310,7 +320,7 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
         if (lane == 0) record_status(kStatusTimeout);
       }
     };
-    if (n_tiles > 0) {
+    if (n_tiles > 0 && kw == 0) {
       // this row of Q into the three swizzled chunks (rows past the unit's rows: zeros)
       const uint4* qsrc = reinterpret_cast<const uint4*>(
           p.q + (int64_t)b_abs * p.q_seq_stride + ((int64_t)tok * plan.n_head + head) * kHeadDK);
@@ -328,25 +338,49 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
     float m_ref = -INFINITY;
     float l_sum = 0.f;
     const bool vec_ok = mrow == nullptr || p.mask_vec_ok;
+    constexpr int kKeys = kTile / 2;  // keys of a tile per warpgroup
+    // The mask of a tile (each row its own token's) is loaded into registers during the
+    // previous tile, after its exponentials, and brought into L2 kMaskAhead tiles ahead,
+    // so that its latency stays off the softmax's path (half tiles inside the mask row
+    // take this path; a ragged half tile goes key by key).
+    constexpr int kMaskAhead = 4;
+    auto half_key0 = [&](int t) { return (tile_begin + t) * kTile + kKeys * kw; };
+    auto vec_half = [&](int t) { return vec_ok && half_key0(t) + kKeys <= key_end; };
+    auto prefetch_mask = [&](int t) {
+      if (mrow != nullptr && half_key0(t) + kKeys <= plan.n_kv) {
+        prefetch_l2(mrow + half_key0(t));
+        prefetch_l2(reinterpret_cast<const uint8_t*>(mrow + half_key0(t)) + 2 * kKeys - 2);  // its last cell
+      }
+    };
+    uint4 mvec[kKeys / 8];
+    auto load_mask = [&](int t) {
+#pragma unroll
+      for (int c = 0; c < kKeys / 8; ++c)
+        mvec[c] = mrow ? __ldg(reinterpret_cast<const uint4*>(mrow + half_key0(t)) + c) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    for (int t = 0; t < kMaskAhead && t < n_tiles; ++t) prefetch_mask(t);
+    bool vec_next = n_tiles > 0 && vec_half(0);
+    if (vec_next) load_mask(0);
     for (int i = 0; i < n_tiles; ++i) {
-      const int key0 = (tile_begin + i) * kTile;
+      const int key0 = half_key0(i);  // this warpgroup's first key
+      const bool vec_mask = vec_next;
       wait_local(&bars.s_full, i & 1);
       tc_fence_after();
-      uint32_t sr[kTile];
+      uint32_t sr[kKeys];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        tmem_ld32(tmem + lane_base + kTmemS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * q));
+      for (int q = 0; q < kKeys / 32; ++q)
+        tmem_ld32(tmem + lane_base + kTmemS + kKeys * kw + 32 * q,
+                  *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * q));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free);
-      float x[kTile];
-      if (vec_ok && key0 + kTile <= key_end) {
-        // full tile: 16-byte mask loads (zeros without a mask)
+      float x[kKeys];
+      if (vec_mask) {
+        // whole half tile: the mask loaded during the previous tile (zeros without a mask)
 #pragma unroll
-        for (int c = 0; c < kTile / 8; ++c) {
-          const uint4 mv = mrow ? __ldg(reinterpret_cast<const uint4*>(mrow + key0) + c)
-                                : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < kKeys / 8; ++c) {
+          const uint4 mv = mvec[c];
           const uint32_t w[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
@@ -357,7 +391,7 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < kTile; ++j) {
+        for (int j = 0; j < kKeys; ++j) {
           const int key = key0 + j;
           float mv = 0.f;
           if (mrow != nullptr && key < key_end) mv = __half2float(__ushort_as_half(__ldg(mrow + key)));
@@ -368,9 +402,15 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
 #pragma unroll
       for (int u = 0; u < 8; ++u) m8[u] = x[u];
 #pragma unroll
-      for (int j = 8; j < kTile; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
-      const float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      for (int j = 8; j < kKeys; ++j) m8[j & 7] = fmaxf(m8[j & 7], x[j]);
+      float mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      // the row's max over the whole tile: swap halves with the other warpgroup (a slot
+      // per tile parity: the other warpgroup may write the next tile's before this one
+      // reads)
+      xmax[((i & 1) * 2 + kw) * kRows + r] = mt;
+      named_bar_sync(1, 256);
+      mt = fmaxf(mt, xmax[((i & 1) * 2 + (kw ^ 1)) * kRows + r]);
       const bool need = mt > m_ref + kRescaleThreshold;
       float alpha = 1.f;
       if (need) {
@@ -378,12 +418,12 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
         m_ref = mt;
       }
       const float nb = (m_ref == -INFINITY) ? 0.f : -m_ref * kLog2e;
-      uint32_t pk[kTile / 2];
+      uint32_t pk[kKeys / 2];
       float ls8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) ls8[u] = 0.f;
 #pragma unroll
-      for (int j = 0; j < kTile / 2; ++j) {
+      for (int j = 0; j < kKeys / 2; ++j) {
         const float e0 = ex2_approx(fmaf(x[2 * j], kLog2e, nb));
         const float e1 = ex2_approx(fmaf(x[2 * j + 1], kLog2e, nb));
         __half2 h2 = __floats2half2_rn(e0, e1);
@@ -392,14 +432,18 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
       }
       l_sum = l_sum * alpha +
               (((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7])));
+      // next tile's mask (the scores are dead)
+      vec_next = i + 1 < n_tiles && vec_half(i + 1);
+      if (vec_next) load_mask(i + 1);
+      if (i + kMaskAhead < n_tiles) prefetch_mask(i + kMaskAhead);
       // P (and O) are free once P.V of the previous tile has completed
       if (i > 0) wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
       tc_fence_after();
-      tmem_st32(tmem + lane_base + kTmemP, *reinterpret_cast<uint32_t(*)[32]>(pk));
-      tmem_st32(tmem + lane_base + kTmemP + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+      tmem_st32(tmem + lane_base + kTmemP + (kKeys / 2) * kw, *reinterpret_cast<uint32_t(*)[32]>(pk));
       if (__any_sync(0xffffffffu, need && i > 0)) {
+        // this warpgroup's half of the row's O columns
 #pragma unroll 1
-        for (int cc = 0; cc < kHeadDV / 32; ++cc) {
+        for (int cc = 2 * kw; cc < 2 * kw + 2; ++cc) {
           uint32_t v[32];
           const uint32_t a = tmem + lane_base + kTmemO + cc * 32;
           tmem_ld32(a, v);
@@ -414,11 +458,15 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.p_full[i & 1]);
     }
-    // ---- epilogue: O / l to the output row, or a split partial and its lse
+    // ---- epilogue: O / l to the output row, or a split partial and its lse; each
+    // warpgroup writes its half of the row's columns
     if (n_tiles > 0) wait_local(&bars.o_done[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     tc_fence_after();
-    const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+    xl[kw * kRows + r] = l_sum;
+    named_bar_sync(1, 256);
+    const float l_tot = xl[r] + xl[kRows + r];
+    const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
     const int slot = plan.ws_base[b] >= 0 ? plan.ws_base[b] + (kvh * plan.groups + g) * n_split + s : -1;
     float4* dst = nullptr;
     if (row_valid)
@@ -426,7 +474,7 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
                       : reinterpret_cast<float4*>(p.out + (int64_t)b_abs * p.out_seq_stride +
                                                   ((int64_t)tok * plan.n_head + head) * kHeadDV);
 #pragma unroll 1
-    for (int cc = 0; cc < kHeadDV / 32; ++cc) {
+    for (int cc = 2 * kw; cc < 2 * kw + 2; ++cc) {
       uint32_t v[32];
       if (n_tiles > 0) {
         tmem_ld32(tmem + lane_base + kTmemO + cc * 32, v);
@@ -442,8 +490,8 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
                                         __uint_as_float(v[4 * j + 2]) * inv_l, __uint_as_float(v[4 * j + 3]) * inv_l);
       }
     }
-    if (slot >= 0 && row_valid)
-      p.ws_lse[(int64_t)slot * kRows + r] = l_sum > 0.f ? m_ref * kLog2e + __log2f(l_sum) : -INFINITY;
+    if (kw == 0 && slot >= 0 && row_valid)
+      p.ws_lse[(int64_t)slot * kRows + r] = l_tot > 0.f ? m_ref * kLog2e + __log2f(l_tot) : -INFINITY;
   }
 
   if (failed) sleep_at_least_ns(100000);
