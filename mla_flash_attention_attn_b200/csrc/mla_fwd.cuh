@@ -1470,16 +1470,16 @@ __global__ void __launch_bounds__(128)
 // column, so CTA q reads only its quarter of the partial rows: warp w combines row w of
 // the batch (lane l: columns 4l..4l+3 of the quarter), with the lse of up to 96 splits
 // and the first 16 partial rows loaded together. Then thread (warp w, lane l) multiplies
-// latent columns 16w..16w+15 of the quarter into output columns 8 (l % 16) .. +7 of rows
-// 4 (l / 16) .. +3; the 8 warps' sums meet in shared memory, and the 4 CTAs' sums over
-// distributed shared memory (CTA q adds up rows 2q, 2q+1). Launched as a programmatic
-// dependent of the forward kernel.
+// the quarter's 128 latent columns of row l / 4 into output columns 16 w + 4 (l % 4) .. +3
+// (each warp its own 16 output columns, so no sum across warps), and the 4 CTAs' sums
+// meet over distributed shared memory (CTA q adds up rows 2q, 2q+1). Launched as a
+// programmatic dependent of the forward kernel; the weight slice, which the forward
+// does not write, is requested before the wait for the forward's partials.
 constexpr int kProjRows = 8;
 constexpr int kProjDim = 128;
 constexpr int kProjWBytes = 128 * kProjDim * 2;                       // W slice: 32 KB
 constexpr int kProjORow = 132;                                        // padded o_s row
 constexpr int kProjSmem = kProjWBytes + kProjRows * kProjORow * 4 +   // W, o_s
-                          8 * kProjRows * kProjDim * 4 +              // warps' sums
                           kProjRows * kProjDim * 4 + 16;              // CTA sum, barrier
 
 __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
@@ -1487,7 +1487,6 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
                             const float* __restrict__ ws_lse, const uint16_t* __restrict__ wv,
                             float* __restrict__ out_proj, int64_t op_seq_stride,
                             const float* __restrict__ sinks) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ __align__(128) uint8_t proj_smem[];
   // a launch with too little dynamic shared memory reports and returns (every CTA takes
   // this branch, so no cluster barrier is left waiting)
@@ -1497,25 +1496,25 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
   }
   const uint16_t* w_s = reinterpret_cast<const uint16_t*>(proj_smem);               // [128 d][128 n]
   float (*o_s)[kProjORow] = reinterpret_cast<float (*)[kProjORow]>(proj_smem + kProjWBytes);
-  float (*red)[kProjRows][kProjDim] =
-      reinterpret_cast<float (*)[kProjRows][kProjDim]>(proj_smem + kProjWBytes + kProjRows * kProjORow * 4);
-  float (*part)[kProjDim] = reinterpret_cast<float (*)[kProjDim]>(
-      proj_smem + kProjWBytes + kProjRows * kProjORow * 4 + 8 * kProjRows * kProjDim * 4);
-  uint64_t* wbar = reinterpret_cast<uint64_t*>(
-      proj_smem + kProjWBytes + kProjRows * kProjORow * 4 + 8 * kProjRows * kProjDim * 4 + kProjRows * kProjDim * 4);
+  float (*part)[kProjDim] =
+      reinterpret_cast<float (*)[kProjDim]>(proj_smem + kProjWBytes + kProjRows * kProjORow * 4);
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(proj_smem + kProjWBytes + kProjRows * kProjORow * 4 +
+                                               kProjRows * kProjDim * 4);
   const int h = blockIdx.x;
   const uint32_t qtr = cluster_ctarank();
   const int j0 = (int)(blockIdx.y >> 2) * kProjRows;
   const int nrows = plan.n_seq * plan.n_q;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int64_t kSplitStride4 = (int64_t)kRowsPerGroup * kDV / 4;
-  // this CTA's slice of W_h first (it does not depend on the combine)
+  // this CTA's slice of W_h first: it is an input of the call, not written by the
+  // forward kernel, so it is requested before the wait for the forward's partials
   if (threadIdx.x == 0) {
     mbar_init(wbar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(wbar, kProjWBytes);
     bulk_load(proj_smem, wv + ((int64_t)h * kDV + 128 * qtr) * kProjDim, kProjWBytes, wbar);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   {
     // ---- combine columns 128 qtr + 4 lane .. +3 of row j0 + warp
     const int j = j0 + warp;
@@ -1590,46 +1589,24 @@ __global__ void __cluster_dims__(1, 4, 1) __launch_bounds__(256, 2)
   }
   __syncthreads();  // o_s complete; the barrier init is visible to every thread
   if (!mbar_wait(wbar, 0, 2000000000ull)) record_status(kStatusTimeout);
-  // ---- project this quarter: latent columns 16 warp .. +15, output columns 8 ng .. +7,
-  //      rows 4 rg .. +3
-  const int ng = lane & 15, rg = lane >> 4;
-  float a[4][8];
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) a[r][c] = 0.f;
-#pragma unroll 4
-  for (int d = 0; d < 16; ++d) {
-    const int dl = 16 * warp + d;  // latent column within the quarter
-    const uint4 w4 = *reinterpret_cast<const uint4*>(w_s + dl * kProjDim + 8 * ng);
-    const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
-    float wf[8];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[c]));
-      wf[2 * c] = f.x;
-      wf[2 * c + 1] = f.y;
+  // ---- project this quarter: row l / 4, output columns 16 warp + 4 (l % 4) .. +3, over
+  //      the quarter's 128 latent columns (o_s rows are padded: the 8 rows of a warp's
+  //      loads fall in different banks; the W loads of a warp are 4 distinct words)
+  {
+    const int pr = lane >> 2, pc = 16 * warp + 4 * (lane & 3);
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 8
+    for (int d = 0; d < 128; ++d) {
+      const uint2 w2 = *reinterpret_cast<const uint2*>(w_s + d * kProjDim + pc);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w2.x));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w2.y));
+      const float o = o_s[pr][d];
+      a0 = fmaf(o, f0.x, a0);
+      a1 = fmaf(o, f0.y, a1);
+      a2 = fmaf(o, f1.x, a2);
+      a3 = fmaf(o, f1.y, a3);
     }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float o = o_s[4 * rg + r][dl];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) a[r][c] = fmaf(o, wf[c], a[r][c]);
-    }
-  }
-#pragma unroll
-  for (int r = 0; r < 4; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) red[warp][4 * rg + r][8 * ng + c] = a[r][c];
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < kProjRows * kProjDim / 256; ++k) {
-    const int e = threadIdx.x + 256 * k;
-    const int r = e / kProjDim, n = e % kProjDim;
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) sum += red[w][r][n];
-    part[r][n] = sum;
+    *reinterpret_cast<float4*>(&part[pr][pc]) = make_float4(a0, a1, a2, a3);
   }
   // ---- the cluster's 4 quarters: CTA qtr adds up rows 2 qtr, 2 qtr + 1
   cluster_sync();
