@@ -111,9 +111,9 @@ def algorithmic_mla(w, kept_cells=None, wuv=False, mask_gather=False):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "4bfeb267b4a95262", "bytes": 172668672},
-    "prefill_chunk": {"source": "4bfeb267b4a95262", "bytes": 205501952},
-    "sparse_q8_decode": {"source": "4bfeb267b4a95262", "bytes": 10392576},
+    "v3_batched_decode": {"source": "73d2bc745c0a2b5e", "bytes": 166982400},
+    "prefill_chunk": {"source": "73d2bc745c0a2b5e", "bytes": 203892480},
+    "sparse_q8_decode": {"source": "73d2bc745c0a2b5e", "bytes": 19130880},
 }
 
 
