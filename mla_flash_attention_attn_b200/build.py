@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmla_fa.so")
 SOURCES = ["mla_api.cu"]
-DEPS = ["mla_api.cu", "mla_fwd.cuh", "mla_compact.cuh", "mla_common.cuh", "sm100_ptx.cuh"]
+# every source of the translation unit: the .cu and all the headers it includes
+DEPS = sorted(f for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h")))
 HEADER = os.path.join(ROOT, "include", "mla_fa.h")
 
 NVCC_FLAGS = [

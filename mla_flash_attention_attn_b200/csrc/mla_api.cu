@@ -964,6 +964,8 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       gp.idx_seq_stride = list_stride;
       gp.kcache = static_cast<const uint8_t*>(a.kcache);
       gp.k_seq_stride = r.k_ss;
+      const int64_t cache_row = a.kcache_type == MLA_KV_Q8_0 ? (int64_t)mla::kQ8RowBytes : (int64_t)r.dk * 2;
+      gp.kcache_bytes = ((int64_t)(a.n_seq - 1) * r.k_ss + a.n_kv) * cache_row;
       gp.n_kv = a.n_kv;
       gp.mask = static_cast<const uint16_t*>(a.mask);
       gp.mask_seq_stride = r.m_ss;
@@ -973,6 +975,7 @@ int run_forward(const Resolved& r, DeviceState* st, void* ws, size_t ws_bytes, c
       gp.gmask = g_mask;
       gp.cap = g_cap;
       gp.gmask_stride = g_mstride;
+      gp.timeout_ns = kDefaultTimeoutNs;
       const int64_t rows_per_cta = a.kcache_type == MLA_KV_Q8_0 ? 32 : 16;  // 8 warps x positions in flight
       const int per_seq = std::max(1, (st->sm_count * 4 + n - 1) / n);
       cudaLaunchConfig_t gcfg = {};

@@ -504,6 +504,42 @@ def test_index_list_paths_by_group_count(kv):
         assert_parity(out[0].reshape(-1, 512).cpu().numpy(), ref, f"index list {kv} n_q={n_q}")
 
 
+@pytest.mark.parametrize("pad", [0, 3])
+def test_q8_gathered_rows_at_the_cache_ends(pad):
+    # The row gather copies each q8_0 row's 16-byte-aligned span (612-byte rows start 4
+    # bytes apart modulo 16); a span that would reach past the end of the cache is read
+    # word by word instead. Lists holding the first and last rows of every sequence, two
+    # sequences, a contiguous cache and one with `pad` rows between sequences; the last
+    # row of the cache starts 4 and 0 bytes past a 16-byte boundary in the two cases.
+    torch = torch_mod()
+    rng = np.random.default_rng(91 + pad)
+    n_kv, n_seq, n_head = 1001, 2, 128
+    k = W.q8_0_random(np.random.Generator(np.random.PCG64(92 + pad)), (n_seq, n_kv + pad))
+    q = rng.standard_normal((n_seq, 1, n_head, 576)).astype(np.float16)
+    mask = np.where(rng.random((n_seq, 1, n_kv)) < 0.95, rng.standard_normal((n_seq, 1, n_kv)),
+                    -np.inf).astype(np.float16)
+    lists = [np.unique(np.concatenate([[0, 1, 2, 3, n_kv - 2, n_kv - 1], rng.choice(n_kv, 240)])),
+             np.array([0, n_kv - 1], dtype=np.int64)]
+    dev = torch.device("cuda")
+    kt = torch.from_numpy(k).to(dev)[:, :n_kv]  # sequences n_kv + pad rows apart
+    qt, mt = torch.from_numpy(q).to(dev), torch.from_numpy(mask).to(dev)
+    idx = torch.full((n_seq, n_kv), -1, dtype=torch.int32, device=dev)
+    for b, lst in enumerate(lists):
+        idx[b, : len(lst)] = torch.from_numpy(lst.astype(np.int32)).to(dev)
+    cnt = torch.tensor([len(x) for x in lists], dtype=torch.int32, device=dev)
+    out = torch.full((n_seq, 1, n_head, 512), float("nan"), dtype=torch.float32, device=dev)
+    ran = _launches(lambda: binding.forward(qt, kt, binding.KV_Q8_0, mt, W.SCALE_192, out=out, idx=idx,
+                                            idx_count=cnt))
+    assert binding.mla_get_device_status() == 0
+    assert ran.get("mla_gather_rows") == 1, ran
+    last = (n_seq - 1) * (n_kv + pad) + n_kv - 1
+    assert (612 * last) % 16 != 12  # the last row's span would pass the cache's end
+    for b, lst in enumerate(lists):
+        ref = oracle.attention(q[b], q8_f16_rounded(k[b, :n_kv]), oracle.KV_F16, mask[b], W.SCALE_192,
+                               idx=lst.astype(np.int32))
+        assert_parity(out[b].reshape(-1, 512).cpu().numpy(), ref, f"q8_0 gathered rows pad={pad} seq {b}")
+
+
 # ---- fused value up-projection (out_proj = O . W_UV per head) ---------------------
 
 # ---- mask gather: sparse attention straight from the mask (the compaction fused in) ----
