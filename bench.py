@@ -111,9 +111,9 @@ def algorithmic_mla(w, kept_cells=None, wuv=False, mask_gather=False):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "73d2bc745c0a2b5e", "bytes": 166982400},
-    "prefill_chunk": {"source": "73d2bc745c0a2b5e", "bytes": 203892480},
-    "sparse_q8_decode": {"source": "73d2bc745c0a2b5e", "bytes": 19130880},
+    "v3_batched_decode": {"source": "f085e43eef0e420e", "bytes": 165794816},
+    "prefill_chunk": {"source": "f085e43eef0e420e", "bytes": 204983296},
+    "sparse_q8_decode": {"source": "f085e43eef0e420e", "bytes": 19130624},
 }
 
 
