@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
     const bool vec_ok = mrow == nullptr || p.mask_vec_ok;
     constexpr int kKeys = kTile / 2;  // keys of a tile per warpgroup
     // The mask of a tile (each row its own token's) is loaded into registers during the
-    // previous tile, after its exponentials, and brought into L2 kMaskAhead tiles ahead,
+    // previous tile, once that tile's mask is used, and brought into L2 kMaskAhead tiles ahead,
     // so that its latency stays off the softmax's path (half tiles inside the mask row
     // take this path; a ragged half tile goes key by key).
     constexpr int kMaskAhead = 4;
@@ -398,6 +398,11 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
           x[j] = key < key_end ? fmaf(__uint_as_float(sr[j]), p.scale, mv) : -INFINITY;
         }
       }
+      // next tile's mask, as soon as this tile's is used: the load has the rest of the
+      // tile to land
+      vec_next = i + 1 < n_tiles && vec_half(i + 1);
+      if (vec_next) load_mask(i + 1);
+      if (i + kMaskAhead < n_tiles) prefetch_mask(i + kMaskAhead);
       float m8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) m8[u] = x[u];
@@ -432,10 +437,6 @@ __global__ void __launch_bounds__(heads::kThreads, 1)
       }
       l_sum = l_sum * alpha +
               (((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7])));
-      // next tile's mask (the scores are dead)
-      vec_next = i + 1 < n_tiles && vec_half(i + 1);
-      if (vec_next) load_mask(i + 1);
-      if (i + kMaskAhead < n_tiles) prefetch_mask(i + kMaskAhead);
       // P (and O) are free once P.V of the previous tile has completed
       if (i > 0) wait_local(&bars.o_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
       tc_fence_after();
