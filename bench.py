@@ -111,9 +111,9 @@ def algorithmic_mla(w, kept_cells=None, wuv=False, mask_gather=False):
 # hash of the kernel sources the capture ran. Any change to those sources makes the
 # figure stale, and the roofline then reports traffic as null.
 MEASURED_TRAFFIC = {
-    "v3_batched_decode": {"source": "f085e43eef0e420e", "bytes": 165794816},
-    "prefill_chunk": {"source": "f085e43eef0e420e", "bytes": 204983296},
-    "sparse_q8_decode": {"source": "f085e43eef0e420e", "bytes": 19130624},
+    "v3_batched_decode": {"source": "a3f8efe4f21d1aa1", "bytes": 164443392},
+    "prefill_chunk": {"source": "a3f8efe4f21d1aa1", "bytes": 203976704},
+    "sparse_q8_decode": {"source": "a3f8efe4f21d1aa1", "bytes": 19130880},
 }
 
 
