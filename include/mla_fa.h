@@ -79,7 +79,10 @@ typedef enum {
  * q       f16, element (b, t, h, c) at q[b*q_seq_stride + (t*n_head + h)*dk + c], dk the
  *         head width (576, or 512 with head_dim = 512)
  * kcache  row (b, j) at byte offset (b*k_seq_stride + j) * row_bytes, where
- *         row_bytes = 2*dk (MLA_KV_F16: 1152, or 1024) or 612 (MLA_KV_Q8_0)
+ *         row_bytes = 2*dk (MLA_KV_F16: 1152, or 1024) or 612 (MLA_KV_Q8_0); the
+ *         bytes from kcache to the end of row (n_seq - 1, n_kv - 1) must be one
+ *         readable buffer (a gather of listed q8_0 rows copies each row's 16-byte
+ *         aligned span, up to 12 bytes next to the row, inside that range)
  * mask    f16 or NULL, element (b, t, j) at mask[b*mask_seq_stride + t*mask_row_stride + j];
  *         0 keeps a cell, -inf drops it, any finite value is added to the score;
  *         shared by all heads of a token
