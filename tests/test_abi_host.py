@@ -19,6 +19,13 @@ def lib():
     return binding.load()
 
 
+def test_build_tracks_every_source_of_the_library():
+    # the library is rebuilt when any file the translation unit includes is newer
+    srcs = sorted(f for f in os.listdir(build.CSRC) if f.endswith((".cu", ".cuh", ".h")))
+    assert build.DEPS == srcs
+    assert "mla_gather.cuh" in srcs and "mla_heads.cuh" in srcs
+
+
 def test_header_declares_the_boundary():
     names = binding.header_functions()
     for required in ("mla_fa_forward", "mla_fa_forward_ex", "mla_fa_workspace_size",
